@@ -1,0 +1,381 @@
+"""Pins the CPU oracle to facts fixed outside itself (no GPU needed).
+
+* published SplitMix64 outputs (start-slot hash),
+* a hand-worked table walkthrough (wrap-around windows, tie-breaks, refresh
+  before insert, ascending insert order, dropped write, first occurrence),
+* textbook special cases: P = C with one id per step is an LRU cache, P = 1 is
+  a direct-mapped cache,
+* a brute-force simulator (whole-array search, literal insert rule) on tiny
+  tables, and table invariants after every step,
+* hand-worked binary32 Writeback cases and the Writeback error bound,
+* exact rational recomputation of the int8 quantiser and its error bound,
+* first-occurrence dedup against numpy.unique, gather against torch.where.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import OracleTable
+import pyref
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def load(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- hash
+def test_splitmix64_published_outputs():
+    g = load("splitmix64_seed0.json")
+    gamma = int(g["gamma"], 16)
+    for i, want in enumerate(g["outputs_seed0"]):
+        state = (i * gamma) & ((1 << 64) - 1)
+        assert oracle.splitmix64(state) == int(want, 16)
+        assert pyref.splitmix64(state) == int(want, 16)
+
+
+def test_home_slot_matches_independent_hash():
+    rng = np.random.default_rng(0)
+    keys = rng.integers(0, 2**63 - 1, size=2000, dtype=np.int64)
+    for C in (1, 7, 4096, 1 << 20, (1 << 31) - 1):
+        for k in keys[:300]:
+            assert oracle.home_slot(int(k), C) == pyref.home(int(k), C)
+
+
+# ---------------------------------------------------------------- walkthrough
+def e_rule(t, n, d):
+    i = np.arange(n, dtype=np.float32)[:, None]
+    dd = np.arange(d, dtype=np.float32)[None, :]
+    return (100 * t + 10 * i + dd + 1).astype(np.float32)
+
+
+def test_hand_worked_walkthrough():
+    g = load("table_c8_p3_walkthrough.json")
+    C, D, P = g["capacity"], g["dim"], g["probes"]
+    for k, s in g["home_slots"].items():
+        assert oracle.home_slot(int(k), C) == s
+    T = OracleTable(C, D, P)
+    for st in g["steps"]:
+        ids = np.array(st["ids"], np.int64)
+        rc, rows, hit = T.lookup(ids)
+        assert rc == 0
+        assert rows.tolist() == st["lookup_rows"], st["why"]
+        assert hit.tolist() == [int(r >= 0) for r in st["lookup_rows"]]
+        e = e_rule(st["t"], ids.size, D)
+        rc, stats = T.writeback(ids, e, st["t"])
+        assert rc == 0
+        keys, last, ls = T.state()
+        assert keys.tolist() == st["keys"], st["why"]
+        assert last.tolist() == st["last"], st["why"]
+        assert ls == st["t"]
+        assert stats == st["stats"], st["why"]
+        for r, (tt, i) in st["rows_written"].items():
+            np.testing.assert_array_equal(T.row(int(r)), e_rule(tt, i + 1, D)[i])
+    fl = g["final_lookup"]
+    rc, rows, _ = T.lookup(np.array(fl["ids"], np.int64))
+    assert rows.tolist() == fl["rows"]
+    assert T.select_written_since(3).tolist() == g["select_since_3"]
+    for r, v in g["final_values"].items():
+        np.testing.assert_array_equal(T.row(int(r)), np.array(v, np.float32))
+    for r in range(4, C):
+        np.testing.assert_array_equal(T.row(r), np.zeros(D, np.float32))
+
+
+def test_step_must_increase():
+    T = OracleTable(16, 4, 2)
+    e = np.zeros((1, 4), np.float32)
+    assert T.writeback(np.array([3]), e, 5)[0] == 0
+    assert T.writeback(np.array([3]), e, 5)[0] == oracle.ORC_EINVAL
+    assert T.writeback(np.array([3]), e, 4)[0] == oracle.ORC_EINVAL
+    assert T.writeback(np.array([3]), e, 6)[0] == 0
+
+
+def test_negative_id_is_reported_and_skipped():
+    T = OracleTable(16, 4, 2)
+    e = np.ones((2, 4), np.float32)
+    rc, st = T.writeback(np.array([-5, 3]), e, 0)
+    assert rc == oracle.ORC_EBADKEY
+    assert st["n_unique"] == 1
+    rc, rows, hit = T.lookup(np.array([-1, 3]))
+    assert rc == oracle.ORC_EBADKEY and rows[0] == -1 and hit[1] == 1
+
+
+# ---------------------------------------------------------------- textbook special cases
+@pytest.mark.parametrize("C,n_keys,seed", [(16, 40, 0), (32, 50, 1), (5, 9, 2)])
+def test_full_window_is_textbook_lru(C, n_keys, seed):
+    """P = C and one id per step: step-granular recency is exact recency and
+    no two occupied rows share a last-access step, so hits and victims are
+    those of an LRU cache of capacity C."""
+    rng = np.random.default_rng(seed)
+    T = OracleTable(C, 4, C)
+    lru = pyref.TextbookLRU(C)
+    for t in range(600):
+        k = int(rng.zipf(1.3) % n_keys)
+        _, rows, hit = T.lookup(np.array([k]))
+        keys_before, _, _ = T.state()
+        want_hit, victim = lru.access(k)
+        assert bool(hit[0]) == want_hit, t
+        rc, st = T.writeback(np.array([k]), np.zeros((1, 4), np.float32), t)
+        keys_after, _, _ = T.state()
+        gone = (set(keys_before.tolist()) - set(keys_after.tolist())) - {-1}
+        assert gone == ({victim} if victim is not None else set()), t
+        assert st["n_evicted"] == (victim is not None)
+
+
+@pytest.mark.parametrize("C,seed", [(64, 0), (13, 1)])
+def test_single_probe_is_textbook_direct_mapped(C, seed):
+    rng = np.random.default_rng(seed)
+    T = OracleTable(C, 4, 1)
+    dm = pyref.TextbookDirectMapped(C, lambda k: pyref.home(k, C))
+    for t in range(800):
+        k = int(rng.integers(0, 3 * C))
+        _, _, hit = T.lookup(np.array([k]))
+        assert bool(hit[0]) == dm.access(k), t
+        T.writeback(np.array([k]), np.zeros((1, 4), np.float32), t)
+
+
+# ---------------------------------------------------------------- brute force + invariants
+def check_invariants(T, t, prev_live, stats):
+    keys, last, _ = T.state()
+    live = keys[keys >= 0]
+    assert len(set(live.tolist())) == live.size, "duplicate live key"
+    for r in np.nonzero(keys >= 0)[0]:
+        k = int(keys[r])
+        h = pyref.home(k, T.capacity)
+        assert (r - h) % T.capacity < T.probes, "live key outside its window"
+    assert (last <= t).all()
+    assert ((keys >= 0) == (last >= 0)).all()
+    assert live.size >= prev_live
+    assert stats["n_inserted"] - stats["n_evicted"] == live.size - prev_live
+    assert stats["n_unique"] == stats["n_hit_unique"] + stats["n_inserted"]
+    return live.size
+
+
+@pytest.mark.parametrize("C,P,D,B,n_keys,seed", [
+    (16, 3, 8, 10, 40, 0), (16, 16, 4, 12, 30, 1), (17, 5, 4, 9, 60, 2),
+    (64, 8, 8, 40, 300, 3), (8, 8, 4, 20, 12, 4), (31, 1, 4, 16, 50, 5),
+])
+def test_oracle_matches_brute_force(C, P, D, B, n_keys, seed):
+    rng = np.random.default_rng(seed)
+    T = OracleTable(C, D, P)
+    Bt = pyref.BruteTable(C, D, P)
+    live = 0
+    for t in range(60):
+        ids = (rng.zipf(1.2, size=B) % n_keys).astype(np.int64)
+        e = rng.standard_normal((B, D)).astype(np.float32)
+        rc, rows, hit = T.lookup(ids)
+        brows, bhit = Bt.lookup(ids)
+        np.testing.assert_array_equal(rows, brows)
+        np.testing.assert_array_equal(hit, bhit)
+        rc, st = T.writeback(ids, e, t)
+        bst = Bt.writeback(ids, e, t)
+        assert st == bst, t
+        keys, last, _ = T.state()
+        assert keys.tolist() == Bt.keys
+        assert last.tolist() == Bt.last
+        np.testing.assert_array_equal(T.values(), Bt.M)
+        live = check_invariants(T, t, live, st)
+
+
+# ---------------------------------------------------------------- writeback arithmetic
+def _val(s):
+    s = s.strip()
+    if "^" in s:
+        if "*" in s:
+            a, b = s.split("*")
+            return float(a) * 2.0 ** int(b.split("^")[1])
+        return 2.0 ** int(s.split("^")[1])
+    return float(s)
+
+
+def test_writeback_hand_worked_binary32_cases():
+    g = load("writeback_fp32_cases.json")
+    for case in g["cases"]:
+        e_hat, e, want = (np.float32(_val(case[k])) for k in ("e_hat", "e", "expect"))
+        T = OracleTable(8, 4, 8)
+        k = np.array([11])
+        T.writeback(k, np.zeros((1, 4), np.float32), 0)  # insert key 11 into a zero row
+        r = int(T.lookup(k)[1][0])
+        T.set_row(r, np.full(4, e_hat, np.float32))
+        T.writeback(k, np.full((1, 4), e, np.float32), 1)
+        got = T.row(r)
+        assert got.view(np.uint32).tolist() == [np.float32(want).view(np.uint32)] * 4, case["why"]
+
+
+def test_writeback_from_empty_table_is_exact_and_first_occurrence():
+    rng = np.random.default_rng(7)
+    T = OracleTable(1024, 16, 8)
+    ids = rng.integers(0, 300, size=500).astype(np.int64)
+    e = rng.standard_normal((500, 16)).astype(np.float32)
+    T.writeback(ids, e, 0)
+    uk, first = np.unique(ids, return_index=True)
+    _, rows, hit = T.lookup(uk)
+    keys, _, _ = T.state()
+    for k, i, r, h in zip(uk, first, rows, hit):
+        if h:  # not dropped by a later insert of this same step
+            np.testing.assert_array_equal(T.row(r), e[i])
+
+
+def test_writeback_error_bound_and_float32_recompute():
+    rng = np.random.default_rng(8)
+    T = OracleTable(256, 32, 4)
+    prev = {}
+    for t in range(30):
+        ids = rng.integers(0, 120, size=64).astype(np.int64)
+        e = (rng.standard_normal((64, 32)) * rng.choice([1e-3, 1, 1e3], size=(64, 1))).astype(np.float32)
+        _, rows_before, hit_before = T.lookup(ids)
+        ehat = {int(r): T.row(r) for r in set(rows_before[hit_before == 1].tolist())}
+        T.writeback(ids, e, t)
+        uk, first = np.unique(ids, return_index=True)
+        _, rows, hit = T.lookup(uk)
+        for k, i, r, h in zip(uk, first, rows, hit):
+            if not h or int(r) not in ehat:
+                continue
+            eh = ehat[int(r)]
+            got = T.row(r)
+            want = (eh - (eh - e[i])).astype(np.float32)
+            np.testing.assert_array_equal(got, want)
+            bound = 2.0 ** -22 * np.maximum(np.abs(eh), np.abs(e[i]))
+            assert (np.abs(got.astype(np.float64) - e[i]) <= bound).all()
+
+
+# ---------------------------------------------------------------- dedup / gather / select
+def test_dedup_first_occurrence_matches_numpy_unique():
+    rng = np.random.default_rng(3)
+    for n in (0, 1, 7, 1000, 5000):
+        ids = (rng.zipf(1.1, size=n) % 997).astype(np.int64)
+        uniq, pos = oracle.dedup(ids)
+        uk, first = np.unique(ids, return_index=True)
+        order = np.argsort(pos)
+        np.testing.assert_array_equal(np.sort(uniq), uk)
+        np.testing.assert_array_equal(pos[order], np.sort(first))
+        assert (np.diff(pos) > 0).all()  # first-occurrence order
+        np.testing.assert_array_equal(ids[pos], uniq)
+
+
+def test_gather_fused_matches_torch_where():
+    rng = np.random.default_rng(4)
+    T = OracleTable(512, 8, 4)
+    for t in range(5):
+        ids = rng.integers(0, 900, size=200).astype(np.int64)
+        T.writeback(ids, rng.standard_normal((200, 8)).astype(np.float32), t)
+    q = rng.integers(0, 900, size=333).astype(np.int64)
+    _, rows, hit = T.lookup(q)
+    ao = rng.standard_normal((64, 12)).astype(np.float32)
+    ao_rows = rng.integers(0, 64, size=333).astype(np.int32)
+    out = T.gather_fused(rows, hit, ao, ao_rows)
+    M = torch.from_numpy(T.values())
+    h = torch.from_numpy(hit.astype(bool))
+    cached = torch.where(h[:, None], M[torch.from_numpy(np.where(hit == 1, rows, 0)).long()],
+                         torch.zeros(1, 8))
+    want = torch.cat([cached, torch.from_numpy(ao)[torch.from_numpy(ao_rows).long()]], dim=1)
+    np.testing.assert_array_equal(out, want.numpy())
+    assert (out[hit == 0, :8].view(np.uint32) == 0).all()  # +0.0, not -0.0
+    out2 = T.gather_fused(rows, hit)
+    np.testing.assert_array_equal(out2, want.numpy()[:, :8])
+
+
+def test_select_written_since_matches_numpy():
+    rng = np.random.default_rng(5)
+    T = OracleTable(300, 4, 6)
+    for t in range(20):
+        ids = rng.integers(0, 700, size=50).astype(np.int64)
+        T.writeback(ids, np.zeros((50, 4), np.float32), t)
+    keys, last, _ = T.state()
+    for s in (0, 10, 19, 20):
+        want = np.nonzero((keys != -1) & (last >= s))[0]
+        np.testing.assert_array_equal(T.select_written_since(s), want)
+
+
+# ---------------------------------------------------------------- int8
+def test_quantize_hand_worked_rows():
+    g = load("int8_rows.json")
+    for row in g["rows"]:
+        x = np.array(row["x"], np.float32)
+        q, s = oracle.quantize_row(x)
+        if "scale" in row:
+            assert s == np.float32(row["scale"]), row["why"]
+        else:
+            assert s == np.float32(np.abs(x).max()) / np.float32(127.0)
+        assert q.tolist() == row["q"], row["why"]
+
+
+def test_quantize_matches_exact_rational_rounding():
+    rng = np.random.default_rng(6)
+    for trial in range(60):
+        d = int(rng.integers(1, 40))
+        x = (rng.standard_normal(d) * 10.0 ** rng.integers(-6, 6)).astype(np.float32)
+        if trial % 7 == 0:
+            x[rng.integers(0, d)] *= -1
+        q, s = oracle.quantize_row(x)
+        qe, se = pyref.quantize_exact(x)
+        assert s.view(np.uint32) == se.view(np.uint32)
+        np.testing.assert_array_equal(q, qe)
+        # dequantisation error: scale/2 plus the two binary32 roundings
+        deq = q.astype(np.float32) * s
+        ulp = lambda v: np.spacing(np.abs(v).astype(np.float32))
+        slack = s / 2 + 2 * ulp(x) + ulp(np.float32(s * 127))
+        assert (np.abs(deq.astype(np.float64) - x) <= slack).all()
+        assert np.abs(q).max() <= 127
+
+
+def test_export_int8_uses_table_rows_and_keys():
+    rng = np.random.default_rng(9)
+    T = OracleTable(128, 16, 4)
+    ids = rng.integers(0, 400, size=60).astype(np.int64)
+    T.writeback(ids, rng.standard_normal((60, 16)).astype(np.float32), 0)
+    rows = T.select_written_since(0)
+    q, s, k = T.export_int8(rows)
+    keys, _, _ = T.state()
+    np.testing.assert_array_equal(k, keys[rows])
+    for i, r in enumerate(rows):
+        qq, ss = pyref.quantize_exact(T.row(r))
+        np.testing.assert_array_equal(q[i], qq)
+        assert s[i] == ss
+
+
+def test_serve_gather_matches_numpy():
+    rng = np.random.default_rng(10)
+    C, P, D = 97, 5, 12
+    snap_keys = np.full(C, -1, np.int64)
+    for k in rng.choice(10_000, size=60, replace=False):
+        h = pyref.home(int(k), C)
+        for j in range(P):
+            if snap_keys[(h + j) % C] == -1:
+                snap_keys[(h + j) % C] = k
+                break
+    q = rng.integers(-127, 128, size=(C, D)).astype(np.int8)
+    sc = rng.random(C).astype(np.float32)
+    ids = np.concatenate([snap_keys[snap_keys >= 0], rng.integers(0, 10_000, size=40)]).astype(np.int64)
+    rc, rows, hit, out = oracle.serve_gather(snap_keys, C, P, q, sc, D, ids)
+    assert rc == 0
+    for i, k in enumerate(ids):
+        where = [r for r in range(C) if snap_keys[r] == k]
+        if where:
+            r = where[0]
+            assert rows[i] == r and hit[i] == 1
+            np.testing.assert_array_equal(out[i], q[r].astype(np.float32) * sc[r])
+        else:
+            assert rows[i] == -1 and hit[i] == 0
+            assert (out[i].view(np.uint32) == 0).all()
+
+
+# ---------------------------------------------------------------- input generator self-check
+@pytest.mark.parametrize("alpha,n", [(0.9, 60), (1.05, 40), (1.2, 80)])
+def test_zipf_sampler_matches_exact_pmf(alpha, n):
+    from hashed_sparse_table_b200 import inputs
+    rng = np.random.Generator(np.random.PCG64([42, n]))
+    s = inputs.zipf_ranks(rng, alpha, n, 400_000)
+    assert s.min() >= 1 and s.max() <= n
+    p = inputs.math_zipf_pmf(alpha, n)
+    f = np.bincount(s, minlength=n + 1)[1:]
+    chi2 = (((f - p * s.size) ** 2) / (p * s.size)).sum()
+    # n-1 degrees of freedom: mean n-1, sd sqrt(2(n-1)); 6 sd is a generous gate
+    assert chi2 < (n - 1) + 6 * np.sqrt(2 * (n - 1)), chi2
