@@ -1,0 +1,386 @@
+"""Benchmark of the Memory Layer hot path on B200.
+
+Workload: the multi-table training step (1M rows x 512-d fp32 table, 8 probes;
+per step a labeled batch of 32,768 ids and an unlabeled candidate-pool batch of
+131,072 ids, both Zipf(0.9) over 5M keys, merged labeled-first).  One step =
+MPZCH lookup of the labeled ids -> fused gather (cached row or zeros, plus the
+128-d author embedding from a 1M-row always-on table) -> Writeback of the
+merged batch (dedup, refresh, ascending-key insert/evict, exact row write).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is unique rows per second through
+lookup + gather + Writeback with inputs resident in HBM; `e2e` is the same
+metric with each step's inputs copied from pinned host memory and the step's
+counters copied back inside the timed region.  Multi-GPU runs are independent
+replicas (one table per GPU, each with its own id stream): no collective is on
+the data path.  `--impl reference` times the CPU oracle on the host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hashed_sparse_table_b200 import inputs  # noqa: E402
+
+W = inputs.CFG3_MULTI
+METRIC = "unique rows/s through lookup+gather+writeback"
+UNIT = "unique rows/s"
+PREFILL = 20  # untimed steps that bring the table to its steady state
+REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--prefill", type=int, default=PREFILL)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def config_dict(extra=None):
+    d = {"workload": W.name, "capacity": W.capacity, "dim": W.dim, "probes": W.probes,
+         "labeled_ids_per_step": W.labeled, "pool_ids_per_step": W.pool,
+         "zipf_alpha": W.zipf_alpha, "zipf_keys": W.zipf_keys, "author_table": [W.ao_rows, W.ao_dim],
+         "l2": "inputs larger than L2 (e is 320 MiB per step, M is 2 GiB)",
+         "parallelism": "independent replicas, one table per GPU"}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(local_rank: int) -> str:
+    cvd = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if cvd:
+        items = [x.strip() for x in cvd.split(",") if x.strip()]
+        if local_rank < len(items):
+            return items[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------------ host-side inputs
+def host_step(t: int, rank: int):
+    tt = t + rank * REPLICA_STRIDE
+    ids = inputs.step_ids(W, tt)
+    aor = inputs.author_rows(W, ids[:W.labeled])
+    return ids, aor
+
+
+def oracle_sample(steps: int, prefill: int):
+    """Times the CPU oracle on `steps` steps after `prefill` untimed ones."""
+    import oracle
+    orc = oracle.OracleTable(W.capacity, W.dim, W.probes)
+    ao = inputs.author_table(W)
+    e_pool = {}
+    total_u = 0
+    elapsed = 0.0
+    for t in range(prefill + steps):
+        ids, aor = host_step(t, 0)
+        k = t % inputs.E_POOL
+        if k not in e_pool:
+            e_pool[k] = inputs.step_e(W, t)
+        e = e_pool[k]
+        t0 = time.perf_counter()
+        _, rows, hit = orc.lookup(ids[:W.labeled])
+        orc.gather_fused(rows, hit, ao, aor)
+        _, st = orc.writeback(ids, e, t)
+        dt = time.perf_counter() - t0
+        if t >= prefill:
+            elapsed += dt
+            total_u += st["n_unique"]
+    orc.close()
+    return total_u / elapsed, total_u, elapsed
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    steps = args.steps
+    prefill = min(args.prefill, 10)
+    # bounded sample: at most 20 timed oracle steps, so the run ends within minutes
+    k = max(1, min(steps, 20))
+    v, tot, el = oracle_sample(k, prefill + args.warmup)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": k, "warmup": args.warmup,
+            "ms_per_step": el / k * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_dict({"prefill_steps": prefill}),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{k} steps of the multi-table workload after "
+                                       f"{prefill + args.warmup} untimed steps, one host thread"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from hashed_sparse_table_b200 import binding
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    K, Wm, Pf = args.steps, args.warmup, args.prefill
+    total = Pf + Wm + K
+    stream = torch.cuda.current_stream()
+
+    # inputs: ids / author rows per step (device resident), e pool (device resident)
+    host = [host_step(t, rank) for t in range(total)]
+    ids_d = [torch.from_numpy(h[0]).to(dev) for h in host]
+    aor_d = [torch.from_numpy(h[1]).to(dev) for h in host]
+    e_host = [torch.from_numpy(inputs.step_e(W, t)) for t in range(inputs.E_POOL)]
+    e_d = [x.to(dev) for x in e_host]
+    ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
+    lab = W.labeled
+    rows = torch.empty(lab, dtype=torch.int32, device=dev)
+    hits = torch.empty((total, lab), dtype=torch.uint8, device=dev)
+    out = torch.empty((lab, W.dim + W.ao_dim), dtype=torch.float32, device=dev)
+    stats = torch.zeros((total, 7), dtype=torch.int64, device=dev)
+
+    tbl = binding.MpzchTable(W.capacity, W.dim, W.probes)
+    binding.mpzch_reserve(tbl.h, W.batch)
+
+    def step(t):
+        binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])
+        binding.mpzch_gather_fused(tbl.h, rows, hits[t], out, ao_d, aor_d[t])
+        binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % inputs.E_POOL], t, stats[t])
+
+    for t in range(Pf):
+        step(t)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.1)
+    for t in range(Pf, Pf + Wm):
+        step(t)
+    binding.mpzch_trace_read(tbl.h)  # drop warm-up records
+    binding.mpzch_trace_enable(tbl.h, True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = binding.mpzch_launch_count()
+    ev0.record(stream)
+    for t in range(Pf + Wm, total):
+        step(t)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    launches = binding.mpzch_launch_count() - l0
+    if world > 1:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    trace = binding.mpzch_trace_read(tbl.h)
+    binding.mpzch_trace_enable(tbl.h, False)
+    clk = clocks.stop() if clocks else None
+
+    st = stats[Pf + Wm:].cpu().numpy()
+    n_unique = int(st[:, 1].sum())
+    n_written = int((st[:, 1] - st[:, 5]).sum())
+    n_hit_lab = int(hits[Pf + Wm:].sum().item())
+    t_units = torch.tensor([float(n_unique), ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        u = t_units[:1].clone()
+        m = t_units[1:].clone()
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+        dist.all_reduce(m, op=dist.ReduceOp.MAX)
+        tot_units, max_ms = float(u.item()), float(m.item())
+    else:
+        tot_units, max_ms = float(n_unique), ms
+
+    # roofline of the dominant kernel (the Writeback row update)
+    D, A = W.dim, W.ao_dim
+    wb_ms, wb_launches = trace["writeback"]
+    wb_bytes = n_written * 12 * D + n_unique * 24  # e + M read, M write; 24 B of index data per id
+    g_ms, _ = trace["gather"]
+    g_bytes = n_hit_lab * 4 * D + K * lab * (4 * A + 4 * (D + A) + 9)
+    peak, peak_kind = load_peaks()
+    wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
+    gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
+
+    # end to end: host inputs (pinned) -> device -> step -> counters back to host
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host)
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, tot, el = oracle_sample(10, args.prefill)
+            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                   "sample": f"10 steps of the same workload after {args.prefill} untimed "
+                             f"steps ({tot} unique rows, {el:.1f} s), one host thread"}
+        result = {
+            "metric": METRIC, "value": tot_units / (max_ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": max_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded Zipf id streams, N(0,1) item-tower targets)",
+            "config": config_dict({"prefill_steps": Pf}),
+            "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "kernel": "k_writeback", "achieved": wb_gbs,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": wb_gbs / peak, "traffic": None,
+                         "bytes_per_launch": wb_bytes / max(1, wb_launches),
+                         "avg_launch_us": wb_ms * 1e3 / max(1, wb_launches)},
+            "gather_writeback_gbs": gw_gbs,
+            "gather_writeback_frac_of_peak": gw_gbs / peak,
+            "gather_writeback_frac_of_8tbs": gw_gbs / 8000.0,
+            "phase_ms_per_step": {k: v[0] / K for k, v in trace.items() if v[1]},
+            "unique_rows_per_step": n_unique / K,
+            "hit_rate_labeled": n_hit_lab / (K * lab),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+        }
+    tbl.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host):
+    """Same steps (continuing the stream) with host inputs copied in every step."""
+    import torch.distributed as dist
+    lab = W.labeled
+    n0 = total
+    host = [host_step(t, rank) for t in range(n0, n0 + K)]
+    ids_h = [torch.from_numpy(h[0]).pin_memory() for h in host]
+    aor_h = [torch.from_numpy(h[1]).pin_memory() for h in host]
+    e_h = [x.pin_memory() for x in e_host]
+    ids_d = torch.empty(W.batch, dtype=torch.int64, device=dev)
+    aor_d = torch.empty(lab, dtype=torch.int32, device=dev)
+    e_d = torch.empty((W.batch, W.dim), dtype=torch.float32, device=dev)
+    rows = torch.empty(lab, dtype=torch.int32, device=dev)
+    hit = torch.empty(lab, dtype=torch.uint8, device=dev)
+    out = torch.empty((lab, W.dim + W.ao_dim), dtype=torch.float32, device=dev)
+    ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
+    st_d = torch.zeros(7, dtype=torch.int64, device=dev)
+    st_h = torch.zeros((K, 7), dtype=torch.int64).pin_memory()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for j in range(K):
+        t = n0 + j
+        ids_d.copy_(ids_h[j], non_blocking=True)
+        aor_d.copy_(aor_h[j], non_blocking=True)
+        e_d.copy_(e_h[t % inputs.E_POOL], non_blocking=True)
+        binding.mpzch_lookup(tbl.h, ids_d[:lab], rows, hit)
+        binding.mpzch_gather_fused(tbl.h, rows, hit, out, ao_d, aor_d)
+        binding.mpzch_writeback(tbl.h, ids_d, e_d, t, st_d)
+        st_h[j].copy_(st_d, non_blocking=True)
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    units = float(st_h[:, 1].sum().item())
+    if world > 1:
+        u = torch.tensor([units], dtype=torch.float64, device=dev)
+        m = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(u, op=dist.ReduceOp.SUM)
+        dist.all_reduce(m, op=dist.ReduceOp.MAX)
+        units, ms = float(u.item()), float(m.item())
+    h2d = W.batch * 8 + lab * 4 + W.batch * W.dim * 4
+    return {"value": units / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": 7 * 8, "ms_per_step": ms / K}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

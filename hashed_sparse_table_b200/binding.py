@@ -1,0 +1,330 @@
+"""Thin ctypes binding of libmpzch.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls (see
+``include/mpzch.h``), takes torch CUDA tensors where the C call takes device
+pointers, passes the current CUDA stream unless one is given, and raises
+``MpzchError`` on a negative return code.  All table work runs in the CUDA
+kernels of the library; there is no other implementation behind this module.
+If the built library is missing, importing this module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmpzch.so")
+
+MPZCH_OK = 0
+MPZCH_EINVAL = -1
+MPZCH_ENOMEM = -2
+MPZCH_ECUDA = -3
+MPZCH_ECAPTURE = -5
+MPZCH_STATUS_BADKEY = 1
+MPZCH_STATUS_BADROW = 2
+MPZCH_STATUS_BADAO = 4
+MPZCH_STATUS_INTERNAL = 8
+MPZCH_NPHASES = 7
+MPZCH_OPT_WIDE_ROUNDS = 1
+PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
+STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
+                "n_rounds")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libmpzch.so is not built ({LIB_PATH}); run "
+                      "`python -m hashed_sparse_table_b200.build`")
+
+_lib = C.CDLL(LIB_PATH)
+_p, _i64, _i32 = C.c_void_p, C.c_int64, C.c_int32
+_SIGS = {
+    "mpzch_create": [_i64, _i32, _i32, _p, C.POINTER(_p)],
+    "mpzch_destroy": [_p],
+    "mpzch_reserve": [_p, _i64, _p],
+    "mpzch_lookup": [_p, _p, _i64, _p, _p, _p],
+    "mpzch_gather_fused": [_p, _p, _p, _i64, _p, _i64, _i32, _p, _p, _p],
+    "mpzch_dedup": [_p, _p, _i64, _p, _p, _p, _p],
+    "mpzch_writeback": [_p, _p, _p, _i64, _i64, _p, _p],
+    "mpzch_select_written_since": [_p, _i64, _p, _p, _p],
+    "mpzch_export_int8": [_p, _p, _i64, _p, _p, _p, _p, _p],
+    "mpzch_serve_gather": [_p, _i64, _i32, _p, _p, _i32, _p, _i64, _p, _p, _p, _p, _p],
+    "mpzch_state_views": [_p, C.POINTER(_p), C.POINTER(_p), C.POINTER(_p)],
+    "mpzch_get_last_step": [_p, C.POINTER(_i64)],
+    "mpzch_set_last_step": [_p, _i64],
+    "mpzch_get_status": [_p, C.POINTER(_i32), _p],
+    "mpzch_trace_enable": [_p, _i32],
+    "mpzch_trace_read": [_p, C.POINTER(C.c_double), C.POINTER(_i64), _i32],
+    "mpzch_set_option": [_p, _i32, _i64],
+    "mpzch_debug_fail_allocs": [_i32],
+}
+for _name, _args in _SIGS.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = C.c_int
+_lib.mpzch_launch_count.argtypes = []
+_lib.mpzch_launch_count.restype = _i64
+
+
+class MpzchError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} failed with code {code}")
+        self.code = code
+
+
+def _check(fn: str, rc: int) -> None:
+    if rc != MPZCH_OK:
+        raise MpzchError(fn, rc)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> C.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def _need(t: torch.Tensor, dtype, name: str):
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
+                         f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+
+
+def lib() -> C.CDLL:
+    return _lib
+
+
+# ------------------------------------------------------------------ entry points
+def mpzch_create(capacity: int, dim: int, probes: int, stream=None) -> C.c_void_p:
+    h = C.c_void_p()
+    _check("mpzch_create", _lib.mpzch_create(capacity, dim, probes, _stream(stream), C.byref(h)))
+    return h
+
+
+def mpzch_destroy(h) -> None:
+    _check("mpzch_destroy", _lib.mpzch_destroy(h))
+
+
+def mpzch_reserve(h, max_batch: int, stream=None) -> None:
+    _check("mpzch_reserve", _lib.mpzch_reserve(h, max_batch, _stream(stream)))
+
+
+def mpzch_lookup(h, ids, rows, hit, stream=None) -> None:
+    _need(ids, torch.int64, "ids")
+    _need(rows, torch.int32, "rows")
+    _need(hit, torch.uint8, "hit")
+    n = ids.numel()
+    assert rows.numel() >= n and hit.numel() >= n
+    _check("mpzch_lookup", _lib.mpzch_lookup(h, _ptr(ids), n, _ptr(rows), _ptr(hit), _stream(stream)))
+
+
+def mpzch_gather_fused(h, rows, hit, out, ao_table=None, ao_rows=None, stream=None, n=None) -> None:
+    n = rows.numel() if n is None else n
+    _need(rows, torch.int32, "rows")
+    _need(hit, torch.uint8, "hit")
+    _need(out, torch.float32, "out")
+    ao_n, ao_dim = 0, 0
+    if ao_table is not None:
+        _need(ao_table, torch.float32, "ao_table")
+        _need(ao_rows, torch.int32, "ao_rows")
+        ao_n, ao_dim = ao_table.shape
+    _check("mpzch_gather_fused", _lib.mpzch_gather_fused(
+        h, _ptr(rows), _ptr(hit), n, _ptr(ao_table), ao_n, ao_dim, _ptr(ao_rows), _ptr(out),
+        _stream(stream)))
+
+
+def mpzch_dedup(h, ids, uniq, pos, count, stream=None) -> None:
+    _need(ids, torch.int64, "ids")
+    _need(uniq, torch.int64, "uniq")
+    _need(pos, torch.int32, "pos")
+    _need(count, torch.int64, "count")
+    _check("mpzch_dedup", _lib.mpzch_dedup(h, _ptr(ids), ids.numel(), _ptr(uniq), _ptr(pos),
+                                           _ptr(count), _stream(stream)))
+
+
+def mpzch_writeback(h, ids, e, step: int, stats=None, stream=None) -> None:
+    _need(ids, torch.int64, "ids")
+    _need(e, torch.float32, "e")
+    if stats is not None:
+        _need(stats, torch.int64, "stats")
+        assert stats.numel() >= 7
+    n = ids.numel()
+    assert e.dim() == 2 and e.shape[0] >= n
+    _check("mpzch_writeback", _lib.mpzch_writeback(h, _ptr(ids), _ptr(e), n, step, _ptr(stats),
+                                                   _stream(stream)))
+
+
+def mpzch_select_written_since(h, since: int, rows_out, count, stream=None) -> None:
+    _need(rows_out, torch.int32, "rows_out")
+    _need(count, torch.int64, "count")
+    _check("mpzch_select_written_since", _lib.mpzch_select_written_since(
+        h, since, _ptr(rows_out), _ptr(count), _stream(stream)))
+
+
+def mpzch_export_int8(h, rows, q, scale, keys_out, n=None, dev_n=None, stream=None) -> None:
+    _need(rows, torch.int32, "rows")
+    _need(q, torch.int8, "q")
+    _need(scale, torch.float32, "scale")
+    _need(keys_out, torch.int64, "keys_out")
+    if dev_n is not None:
+        _need(dev_n, torch.int64, "dev_n")
+    n = rows.numel() if n is None else n
+    _check("mpzch_export_int8", _lib.mpzch_export_int8(
+        h, _ptr(rows), n, _ptr(dev_n), _ptr(q), _ptr(scale), _ptr(keys_out), _stream(stream)))
+
+
+def mpzch_serve_gather(snap_keys, probes: int, snap_q, snap_scale, ids, rows, hit, out,
+                       status=None, stream=None) -> None:
+    _need(snap_keys, torch.int64, "snap_keys")
+    _need(snap_q, torch.int8, "snap_q")
+    _need(snap_scale, torch.float32, "snap_scale")
+    _need(ids, torch.int64, "ids")
+    _need(rows, torch.int32, "rows")
+    _need(hit, torch.uint8, "hit")
+    _need(out, torch.float32, "out")
+    if status is not None:
+        _need(status, torch.int32, "status")
+    cap, dim = snap_q.shape
+    _check("mpzch_serve_gather", _lib.mpzch_serve_gather(
+        _ptr(snap_keys), cap, probes, _ptr(snap_q), _ptr(snap_scale), dim, _ptr(ids), ids.numel(),
+        _ptr(rows), _ptr(hit), _ptr(out), _ptr(status), _stream(stream)))
+
+
+def mpzch_state_views(h):
+    k, l, m = C.c_void_p(), C.c_void_p(), C.c_void_p()
+    _check("mpzch_state_views", _lib.mpzch_state_views(h, C.byref(k), C.byref(l), C.byref(m)))
+    return k.value, l.value, m.value
+
+
+def mpzch_get_last_step(h) -> int:
+    s = C.c_int64()
+    _check("mpzch_get_last_step", _lib.mpzch_get_last_step(h, C.byref(s)))
+    return s.value
+
+
+def mpzch_set_last_step(h, step: int) -> None:
+    _check("mpzch_set_last_step", _lib.mpzch_set_last_step(h, step))
+
+
+def mpzch_get_status(h, stream=None) -> int:
+    s = C.c_int32()
+    _check("mpzch_get_status", _lib.mpzch_get_status(h, C.byref(s), _stream(stream)))
+    return s.value
+
+
+def mpzch_trace_enable(h, on: bool) -> None:
+    _check("mpzch_trace_enable", _lib.mpzch_trace_enable(h, 1 if on else 0))
+
+
+def mpzch_trace_read(h):
+    ms = (C.c_double * MPZCH_NPHASES)()
+    ln = (C.c_int64 * MPZCH_NPHASES)()
+    _check("mpzch_trace_read", _lib.mpzch_trace_read(h, ms, ln, MPZCH_NPHASES))
+    return {p: (ms[i], ln[i]) for i, p in enumerate(PHASES)}
+
+
+def mpzch_set_option(h, option: int, value: int) -> None:
+    _check("mpzch_set_option", _lib.mpzch_set_option(h, option, value))
+
+
+def mpzch_debug_fail_allocs(count: int) -> None:
+    _check("mpzch_debug_fail_allocs", _lib.mpzch_debug_fail_allocs(count))
+
+
+def mpzch_launch_count() -> int:
+    return int(_lib.mpzch_launch_count())
+
+
+# ------------------------------------------------------------------ handle helper
+def _view(addr: int, shape, dtype, device) -> torch.Tensor:
+    """A torch tensor over library-owned device memory (no copy, no ownership)."""
+    numel = 1
+    for s in shape:
+        numel *= s
+    itemsize = torch.empty((), dtype=dtype).element_size()
+
+    class _Iface:
+        __cuda_array_interface__ = {
+            "shape": tuple(shape), "typestr": {torch.int64: "<i8", torch.float32: "<f4"}[dtype],
+            "data": (addr, False), "version": 3, "strides": None,
+        }
+    t = torch.as_tensor(_Iface(), device=device)
+    assert t.numel() == numel and t.element_size() == itemsize
+    return t
+
+
+class MpzchTable:
+    """Owns one table handle; methods forward to the entry points above."""
+
+    def __init__(self, capacity: int, dim: int, probes: int, stream=None):
+        self.capacity, self.dim, self.probes = capacity, dim, probes
+        self.device = torch.device("cuda", torch.cuda.current_device())
+        self.h = mpzch_create(capacity, dim, probes, stream)
+
+    def close(self):
+        if getattr(self, "h", None):
+            mpzch_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def state(self):
+        """(keys, last, M) as torch views of the table's own device memory."""
+        k, l, m = mpzch_state_views(self.h)
+        return (_view(k, (self.capacity,), torch.int64, self.device),
+                _view(l, (self.capacity,), torch.int64, self.device),
+                _view(m, (self.capacity, self.dim), torch.float32, self.device))
+
+    def lookup(self, ids, rows=None, hit=None, stream=None):
+        n = ids.numel()
+        rows = torch.empty(n, dtype=torch.int32, device=ids.device) if rows is None else rows
+        hit = torch.empty(n, dtype=torch.uint8, device=ids.device) if hit is None else hit
+        mpzch_lookup(self.h, ids, rows, hit, stream)
+        return rows, hit
+
+    def gather_fused(self, rows, hit, ao_table=None, ao_rows=None, out=None, stream=None):
+        n = rows.numel()
+        w = self.dim + (0 if ao_table is None else ao_table.shape[1])
+        out = torch.empty((n, w), dtype=torch.float32, device=rows.device) if out is None else out
+        mpzch_gather_fused(self.h, rows, hit, out, ao_table, ao_rows, stream)
+        return out
+
+    def dedup(self, ids, stream=None):
+        n = ids.numel()
+        uniq = torch.empty(n, dtype=torch.int64, device=ids.device)
+        pos = torch.empty(n, dtype=torch.int32, device=ids.device)
+        cnt = torch.empty(1, dtype=torch.int64, device=ids.device)
+        mpzch_dedup(self.h, ids, uniq, pos, cnt, stream)
+        return uniq, pos, cnt
+
+    def writeback(self, ids, e, step, stats=None, stream=None):
+        mpzch_writeback(self.h, ids, e, step, stats, stream)
+
+    def select_written_since(self, since, stream=None):
+        rows = torch.empty(self.capacity, dtype=torch.int32, device=self.device)
+        cnt = torch.empty(1, dtype=torch.int64, device=self.device)
+        mpzch_select_written_since(self.h, since, rows, cnt, stream)
+        return rows, cnt
+
+    def export_int8(self, rows, n=None, dev_n=None, stream=None):
+        n = rows.numel() if n is None else n
+        q = torch.empty((n, self.dim), dtype=torch.int8, device=self.device)
+        scale = torch.empty(n, dtype=torch.float32, device=self.device)
+        keys = torch.empty(n, dtype=torch.int64, device=self.device)
+        mpzch_export_int8(self.h, rows, q, scale, keys, n=n, dev_n=dev_n, stream=stream)
+        return q, scale, keys
+
+    def status(self, stream=None) -> int:
+        return mpzch_get_status(self.h, stream)

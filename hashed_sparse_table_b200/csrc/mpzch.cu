@@ -1,0 +1,554 @@
+// libmpzch: C ABI, table handle and launch orchestration for the Memory Layer
+// table kernels (see include/mpzch.h for the contract of every entry point).
+#include "mpzch.h"
+#include "mpzch_kernels.cuh"
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+using namespace mpzch;
+
+namespace {
+
+std::atomic<int> g_fail_allocs{0};
+std::atomic<int64_t> g_launches{0};
+
+int dev_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return MPZCH_OK;
+  if (g_fail_allocs.load() > 0) {
+    g_fail_allocs.fetch_sub(1);
+    return MPZCH_ENOMEM;
+  }
+  if (cudaMalloc(p, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return MPZCH_ENOMEM;
+  }
+  return MPZCH_OK;
+}
+
+void dev_free(void* p) {
+  if (p) cudaFree(p);
+}
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Grid for a grid-stride kernel: enough blocks for `work` threads, at most
+// `per_sm` resident blocks on every SM.
+unsigned grid_for(int64_t work_threads, int block, int per_sm = 8) {
+  int64_t g = (work_threads + block - 1) / block;
+  const int64_t cap = (int64_t)sm_count() * per_sm;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (unsigned)g;
+}
+
+int after_launch() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return cudaGetLastError() == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
+}
+
+uint64_t pow2_at_least(uint64_t x) {
+  uint64_t p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+Geo make_geo(int64_t C, int32_t P) {
+  Geo g;
+  g.C = C;
+  g.pow2 = (C & (C - 1)) == 0;
+  g.mask = g.pow2 ? (uint64_t)(C - 1) : 0;
+  g.P = P;
+  return g;
+}
+
+enum Phase { PH_LOOKUP = 0, PH_GATHER, PH_DEDUP, PH_INSERT, PH_WRITEBACK, PH_SELECT, PH_EXPORT };
+
+}  // namespace
+
+struct mpzch_table {
+  int64_t C = 0;
+  int32_t D = 0, P = 0;
+  int device = 0;
+  Geo geo{};
+  // table state (row-indexed arrays)
+  long long* keys = nullptr;
+  long long* last = nullptr;
+  float* M = nullptr;
+  // insert scratch: three claim arrays of C slots
+  unsigned long long* claims[3] = {nullptr, nullptr, nullptr};
+  // per-batch scratch, sized for `cap` ids
+  int64_t cap = 0;
+  uint64_t hmask = 0;
+  unsigned long long* hkey = nullptr;
+  uint32_t* hpos = nullptr;
+  int32_t* slot_of = nullptr;
+  int32_t* bcount = nullptr;
+  long long* ukey = nullptr;
+  int32_t* upos = nullptr;
+  int32_t* urow = nullptr;
+  int32_t* lists[3] = {nullptr, nullptr, nullptr};
+  // small device words
+  StepCtr* ctr = nullptr;
+  WbStats* stats = nullptr;  // used when the caller passes no stats buffer
+  int32_t* status = nullptr;
+  int32_t* sel_bcount = nullptr;
+  int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
+  int64_t last_step = -1;
+  int wide_rounds = 3;
+  // tracing
+  bool trace = false;
+  struct Rec {
+    cudaEvent_t a, b;
+    int phase;
+  };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  double ms[MPZCH_NPHASES] = {0};
+  int64_t launches[MPZCH_NPHASES] = {0};
+};
+
+namespace {
+
+void free_batch_scratch(mpzch_table* t) {
+  dev_free(t->hkey);
+  dev_free(t->hpos);
+  dev_free(t->slot_of);
+  dev_free(t->bcount);
+  dev_free(t->ukey);
+  dev_free(t->upos);
+  dev_free(t->urow);
+  for (auto& l : t->lists) dev_free(l), l = nullptr;
+  t->hkey = nullptr;
+  t->hpos = nullptr;
+  t->slot_of = t->bcount = t->upos = t->urow = nullptr;
+  t->ukey = nullptr;
+  t->cap = 0;
+  t->hmask = 0;
+}
+
+void free_all(mpzch_table* t) {
+  free_batch_scratch(t);
+  dev_free(t->keys);
+  dev_free(t->last);
+  dev_free(t->M);
+  for (auto& c : t->claims) dev_free(c), c = nullptr;
+  dev_free(t->ctr);
+  dev_free(t->stats);
+  dev_free(t->status);
+  dev_free(t->sel_bcount);
+  if (t->h_status) cudaFreeHost(t->h_status);
+  for (auto& r : t->pending) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (auto e : t->pool) cudaEventDestroy(e);
+}
+
+// Grow the per-batch scratch to hold batches of n ids.
+int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
+  if (n <= t->cap) return MPZCH_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MPZCH_ECUDA;
+  if (cs != cudaStreamCaptureStatusNone) return MPZCH_ECAPTURE;
+  int64_t cap = n < 4096 ? 4096 : n;
+  // The old scratch may still be in use by queued work.
+  if (t->cap > 0 && cudaDeviceSynchronize() != cudaSuccess) return MPZCH_ECUDA;
+  free_batch_scratch(t);
+  const uint64_t H = pow2_at_least((uint64_t)cap * 2);
+  const int64_t tiles = (cap + kTile - 1) / kTile + 1;
+  int rc = MPZCH_OK;
+  if (!rc) rc = dev_alloc((void**)&t->hkey, H * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->hpos, H * sizeof(uint32_t));
+  if (!rc) rc = dev_alloc((void**)&t->slot_of, cap * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->bcount, tiles * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
+  if (!rc) rc = dev_alloc((void**)&t->upos, cap * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->urow, cap * sizeof(int32_t));
+  for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lists[i], cap * sizeof(int32_t));
+  if (rc) {
+    free_batch_scratch(t);
+    return rc;
+  }
+  // Scratch hash: empty key (-1) and empty position (all ones).
+  if (cudaMemsetAsync(t->hkey, 0xFF, H * sizeof(unsigned long long), st) != cudaSuccess ||
+      cudaMemsetAsync(t->hpos, 0xFF, H * sizeof(uint32_t), st) != cudaSuccess) {
+    free_batch_scratch(t);
+    return MPZCH_ECUDA;
+  }
+  t->cap = cap;
+  t->hmask = H - 1;
+  return MPZCH_OK;
+}
+
+bool on_device(const mpzch_table* t) {
+  int d = -1;
+  return cudaGetDevice(&d) == cudaSuccess && d == t->device;
+}
+
+cudaEvent_t take_event(mpzch_table* t) {
+  if (!t->pool.empty()) {
+    cudaEvent_t e = t->pool.back();
+    t->pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets the launches of one phase with events when tracing is on.
+struct PhaseScope {
+  mpzch_table* t;
+  int phase;
+  cudaStream_t st;
+  cudaEvent_t a = nullptr;
+  int64_t start_launches;
+  PhaseScope(mpzch_table* t_, int ph, cudaStream_t s) : t(t_), phase(ph), st(s) {
+    start_launches = g_launches.load();
+    if (t->trace) {
+      a = take_event(t);
+      cudaEventRecord(a, st);
+    }
+  }
+  ~PhaseScope() {
+    t->launches[phase] += g_launches.load() - start_launches;
+    if (t->trace && a) {
+      cudaEvent_t b = take_event(t);
+      cudaEventRecord(b, st);
+      t->pending.push_back({a, b, phase});
+    }
+  }
+};
+
+// The three dedup phases; with `wb` the compaction also re-probes the table,
+// refreshes resident rows and opens insert round 0.
+int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, int32_t* pos,
+              long long* dev_count, bool wb, int64_t step, WbStats* stats, cudaStream_t st) {
+  const long long* id = reinterpret_cast<const long long*>(ids);
+  const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
+  k_dedup_insert<<<grid_for(n, kBlock), kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask,
+                                                         t->slot_of, t->ctr, stats, t->status);
+  if (after_launch()) return MPZCH_ECUDA;
+  k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
+  if (after_launch()) return MPZCH_ECUDA;
+  k_dedup_compact<<<tiles, kBlock, 0, st>>>(
+      id, n, t->slot_of, t->hkey, t->hpos, t->bcount, uniq, pos, dev_count,
+      wb ? t->keys : nullptr, t->last, t->geo, (long long)step, t->urow, t->lists[0],
+      t->claims[0], t->ctr, stats);
+  return after_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mpzch_table** out) {
+  if (!out) return MPZCH_EINVAL;
+  *out = nullptr;
+  if (capacity < 1 || capacity > 0x7FFFFFFFLL || dim <= 0 || dim % 4 != 0 || probes < 1 ||
+      (int64_t)probes > capacity)
+    return MPZCH_EINVAL;
+  mpzch_table* t = new (std::nothrow) mpzch_table;
+  if (!t) return MPZCH_ENOMEM;
+  t->C = capacity;
+  t->D = dim;
+  t->P = probes;
+  t->geo = make_geo(capacity, probes);
+  cudaStream_t st = S(stream);
+  int rc = MPZCH_OK;
+  if (!rc) rc = dev_alloc((void**)&t->keys, capacity * sizeof(long long));
+  if (!rc) rc = dev_alloc((void**)&t->last, capacity * sizeof(long long));
+  if (!rc) rc = dev_alloc((void**)&t->M, (size_t)capacity * dim * sizeof(float));
+  for (int i = 0; i < 3 && !rc; ++i)
+    rc = dev_alloc((void**)&t->claims[i], capacity * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
+  if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
+  if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
+  if (!rc)
+    rc = dev_alloc((void**)&t->sel_bcount, ((capacity + kSelTile - 1) / kSelTile) * sizeof(int32_t));
+  if (!rc && cudaHostAlloc((void**)&t->h_status, sizeof(int32_t), cudaHostAllocDefault) != cudaSuccess) {
+    t->h_status = nullptr;
+    rc = MPZCH_ENOMEM;
+  }
+  if (!rc && cudaGetDevice(&t->device) != cudaSuccess) rc = MPZCH_ECUDA;
+  if (!rc) {
+    bool ok = cudaMemsetAsync(t->keys, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
+              cudaMemsetAsync(t->last, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
+              cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) == cudaSuccess &&
+              cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
+              cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
+              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
+    for (int i = 0; i < 3 && ok; ++i)
+      ok = cudaMemsetAsync(t->claims[i], 0xFF, capacity * sizeof(unsigned long long), st) ==
+           cudaSuccess;
+    if (!ok) rc = MPZCH_ECUDA;
+  }
+  if (rc) {
+    if (rc == MPZCH_ECUDA) cudaGetLastError();
+    free_all(t);
+    delete t;
+    return rc;
+  }
+  *out = t;
+  return MPZCH_OK;
+}
+
+int mpzch_destroy(mpzch_table* t) {
+  if (!t) return MPZCH_OK;
+  cudaDeviceSynchronize();
+  free_all(t);
+  delete t;
+  return MPZCH_OK;
+}
+
+int mpzch_reserve(mpzch_table* t, int64_t max_batch, void* stream) {
+  if (!t || max_batch < 0 || max_batch > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  if (!on_device(t)) return MPZCH_EINVAL;
+  return ensure_batch(t, max_batch, S(stream));
+}
+
+int mpzch_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit,
+                 void* stream) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!ids || !rows || !hit || !on_device(t)) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  PhaseScope ps(t, PH_LOOKUP, st);
+  int G = (int)pow2_at_least((uint64_t)t->P);
+  if (G > 32) G = 32;
+  k_lookup<<<grid_for(n * G, kBlock), kBlock, 0, st>>>(
+      reinterpret_cast<const long long*>(ids), n, t->keys, t->geo, G, rows, hit, t->status);
+  return after_launch();
+}
+
+int mpzch_gather_fused(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
+                       const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
+                       const int32_t* ao_rows, float* out, void* stream) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  const bool has_ao = ao_table != nullptr;
+  if (has_ao && (ao_dim <= 0 || ao_dim % 4 != 0 || ao_nrows <= 0 || !ao_rows)) return MPZCH_EINVAL;
+  if (!has_ao && (ao_dim != 0 || ao_rows)) return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!rows || !hit || !out || !on_device(t)) return MPZCH_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (has_ao && (reinterpret_cast<uintptr_t>(ao_table) & 15)))
+    return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  PhaseScope ps(t, PH_GATHER, st);
+  k_gather_fused<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+      rows, hit, n, reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
+      reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0, ao_rows,
+      reinterpret_cast<float4*>(out), t->status);
+  return after_launch();
+}
+
+int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
+                int64_t* dev_count, void* stream) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL || !dev_count) return MPZCH_EINVAL;
+  if (n > 0 && (!ids || !uniq || !pos)) return MPZCH_EINVAL;
+  if (!on_device(t)) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  if (n == 0) return cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
+  int rc = ensure_batch(t, n, st);
+  if (rc) return rc;
+  PhaseScope ps(t, PH_DEDUP, st);
+  return run_dedup(t, ids, n, reinterpret_cast<long long*>(uniq), pos,
+                   reinterpret_cast<long long*>(dev_count), false, 0, nullptr, st);
+}
+
+int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
+                    mpzch_wb_stats* dev_stats, void* stream) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  if (step <= t->last_step) return MPZCH_EINVAL;
+  if (n > 0 && (!ids || !e)) return MPZCH_EINVAL;
+  if (!on_device(t)) return MPZCH_EINVAL;
+  if (reinterpret_cast<uintptr_t>(e) & 15) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  WbStats* stats = dev_stats ? reinterpret_cast<WbStats*>(dev_stats) : t->stats;
+  if (n == 0) {
+    if (cudaMemsetAsync(stats, 0, sizeof(WbStats), st) != cudaSuccess) return MPZCH_ECUDA;
+    t->last_step = step;
+    return MPZCH_OK;
+  }
+  int rc = ensure_batch(t, n, st);
+  if (rc) return rc;
+  {
+    PhaseScope ps(t, PH_DEDUP, st);
+    rc = run_dedup(t, ids, n, t->ukey, t->upos, nullptr, true, step, stats, st);
+    if (rc) return rc;
+  }
+  {
+    PhaseScope ps(t, PH_INSERT, st);
+    const unsigned grid = grid_for(n, kBlock, 4);
+    const int R = t->wide_rounds;
+    for (int r = 0; r < R; ++r) {
+      k_insert_round<<<grid, kBlock, 0, st>>>(
+          r, t->ukey, t->keys, t->last, t->geo, (long long)step, t->urow, t->lists[(r + 2) % 3],
+          t->lists[r % 3], t->lists[(r + 1) % 3], t->claims[(r + 2) % 3], t->claims[r % 3],
+          t->claims[(r + 1) % 3], t->ctr, stats);
+      if (after_launch()) return MPZCH_ECUDA;
+    }
+    k_insert_finish<<<1, 1024, 0, st>>>(R, t->ukey, t->keys, t->last, t->geo, (long long)step,
+                                        t->urow, t->lists[0], t->lists[1], t->lists[2],
+                                        t->claims[0], t->claims[1], t->claims[2], t->ctr, stats,
+                                        t->status);
+    if (after_launch()) return MPZCH_ECUDA;
+  }
+  {
+    PhaseScope ps(t, PH_WRITEBACK, st);
+    k_writeback<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+        t->ukey, t->upos, t->urow, &stats->n_unique, t->keys, reinterpret_cast<float4*>(t->M),
+        reinterpret_cast<const float4*>(e), t->D / 4, stats);
+    if (after_launch()) return MPZCH_ECUDA;
+  }
+  t->last_step = step;
+  return MPZCH_OK;
+}
+
+int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows_out,
+                               int64_t* dev_count, void* stream) {
+  if (!t || !rows_out || !dev_count || !on_device(t)) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  PhaseScope ps(t, PH_SELECT, st);
+  const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
+  k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
+                                           t->sel_bcount);
+  if (after_launch()) return MPZCH_ECUDA;
+  k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
+                                             t->sel_bcount, rows_out,
+                                             reinterpret_cast<long long*>(dev_count));
+  return after_launch();
+}
+
+int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n,
+                      int8_t* q, float* scale, int64_t* keys_out, void* stream) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!rows || !q || !scale || !keys_out || !on_device(t)) return MPZCH_EINVAL;
+  if (reinterpret_cast<uintptr_t>(q) & 3) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  PhaseScope ps(t, PH_EXPORT, st);
+  k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+      rows, n, reinterpret_cast<const long long*>(dev_n), reinterpret_cast<const float4*>(t->M),
+      t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale,
+      reinterpret_cast<long long*>(keys_out), t->status);
+  return after_launch();
+}
+
+int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probes,
+                       const int8_t* snap_q, const float* snap_scale, int32_t dim,
+                       const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit, float* out,
+                       int32_t* dev_status, void* stream) {
+  if (capacity < 1 || capacity > 0x7FFFFFFFLL || probes < 1 || (int64_t)probes > capacity ||
+      dim <= 0 || dim % 4 != 0 || n < 0 || n > 0x7FFFFFFFLL)
+    return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!snap_keys || !snap_q || !snap_scale || !ids || !rows || !hit || !out) return MPZCH_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(snap_q) & 3))
+    return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  k_serve_gather<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+      reinterpret_cast<const long long*>(snap_keys), make_geo(capacity, probes),
+      reinterpret_cast<const char4*>(snap_q), snap_scale, dim / 4,
+      reinterpret_cast<const long long*>(ids), n, rows, hit, reinterpret_cast<float4*>(out),
+      dev_status);
+  return after_launch();
+}
+
+int mpzch_state_views(mpzch_table* t, int64_t** keys, int64_t** last, float** M) {
+  if (!t) return MPZCH_EINVAL;
+  if (keys) *keys = reinterpret_cast<int64_t*>(t->keys);
+  if (last) *last = reinterpret_cast<int64_t*>(t->last);
+  if (M) *M = t->M;
+  return MPZCH_OK;
+}
+
+int mpzch_get_last_step(mpzch_table* t, int64_t* step) {
+  if (!t || !step) return MPZCH_EINVAL;
+  *step = t->last_step;
+  return MPZCH_OK;
+}
+
+int mpzch_set_last_step(mpzch_table* t, int64_t step) {
+  if (!t || step < -1) return MPZCH_EINVAL;
+  t->last_step = step;
+  return MPZCH_OK;
+}
+
+int mpzch_get_status(mpzch_table* t, int32_t* status, void* stream) {
+  if (!t || !status || !on_device(t)) return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  if (cudaMemcpyAsync(t->h_status, t->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MPZCH_ECUDA;
+  *status = *t->h_status;
+  return MPZCH_OK;
+}
+
+int mpzch_trace_enable(mpzch_table* t, int32_t on) {
+  if (!t) return MPZCH_EINVAL;
+  t->trace = on != 0;
+  return MPZCH_OK;
+}
+
+int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t nphases) {
+  if (!t || nphases < 0) return MPZCH_EINVAL;
+  for (auto& r : t->pending) {
+    float x = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&x, r.a, r.b) != cudaSuccess)
+      return MPZCH_ECUDA;
+    t->ms[r.phase] += x;
+    t->pool.push_back(r.a);
+    t->pool.push_back(r.b);
+  }
+  t->pending.clear();
+  for (int i = 0; i < nphases && i < MPZCH_NPHASES; ++i) {
+    if (ms) ms[i] = t->ms[i];
+    if (launches) launches[i] = t->launches[i];
+  }
+  for (int i = 0; i < MPZCH_NPHASES; ++i) {
+    t->ms[i] = 0;
+    t->launches[i] = 0;
+  }
+  return MPZCH_OK;
+}
+
+int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
+  if (!t) return MPZCH_EINVAL;
+  if (option == MPZCH_OPT_WIDE_ROUNDS) {
+    if (value < 0 || value > kMaxRounds) return MPZCH_EINVAL;
+    t->wide_rounds = (int)value;
+    return MPZCH_OK;
+  }
+  return MPZCH_EINVAL;
+}
+
+int mpzch_debug_fail_allocs(int32_t count) {
+  if (count < 0) return MPZCH_EINVAL;
+  g_fail_allocs.store(count);
+  return MPZCH_OK;
+}
+
+int64_t mpzch_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,713 @@
+// Device code of libmpzch: the Memory Layer table kernels for sm_100a.
+//
+// All kernels are HBM/L2-bound hashing, scanning and row-copy work; nothing
+// here is a dense contraction, so no tensor-core path is used.  Rows are moved
+// as 16-byte vectors by whole warps (one 2 KiB row = 4 x 512 B coalesced
+// requests at D = 512).  Every loop has a static bound; no kernel waits on a
+// flag written by another block, and no kernel traps.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace mpzch {
+
+constexpr unsigned long long kEmptyKey = 0xFFFFFFFFFFFFFFFFull;  // key -1
+constexpr unsigned long long kNoClaim = 0xFFFFFFFFFFFFFFFFull;   // larger than any key
+constexpr uint32_t kNoPos = 0xFFFFFFFFu;
+constexpr int kBlock = 256;
+constexpr int kTile = 1024;  // ids per block in the ordered compactions (4 per thread)
+constexpr int kSelTile = 4096;  // rows per block in select (16 per thread)
+constexpr int kMaxRounds = 16;
+
+// Status bits (mirror of the MPZCH_STATUS_* values of the public header).
+constexpr int kStBadKey = 1, kStBadRow = 2, kStBadAo = 4, kStInternal = 8;
+
+struct Geo {
+  int64_t C;
+  uint64_t mask;  // C - 1 when C is a power of two
+  int32_t pow2;
+  int32_t P;
+};
+
+// Device counters of one Writeback.
+struct StepCtr {
+  int32_t nlist[kMaxRounds + 2];  // unresolved missing keys entering each insert round
+  uint32_t done_blocks;           // completion ticket of the last kernel's blocks
+  int32_t pad;
+};
+
+// Per-Writeback counters; same layout as mpzch_wb_stats.
+struct WbStats {
+  long long n_ids, n_unique, n_hit_unique, n_inserted, n_evicted, n_dropped, n_rounds;
+};
+
+// SplitMix64 generator output for state x (Steele, Lea, Flood, OOPSLA 2014):
+// add the golden gamma, two xor-shift-multiply rounds, a final xor-shift.
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__device__ __forceinline__ int64_t home_slot(int64_t k, const Geo& g) {
+  const uint64_t h = splitmix64((uint64_t)k);
+  return g.pow2 ? (int64_t)(h & g.mask) : (int64_t)(h % (uint64_t)g.C);
+}
+
+// Slot h + j of a window (h < C, j < P <= C, so one subtraction wraps it).
+__device__ __forceinline__ int64_t wslot(int64_t h, int32_t j, const Geo& g) {
+  int64_t s = h + j;
+  return s >= g.C ? s - g.C : s;
+}
+
+__device__ __forceinline__ long long ld_cg(const long long* p) { return __ldcg(p); }
+__device__ __forceinline__ unsigned long long ld_cg(const unsigned long long* p) {
+  return __ldcg(p);
+}
+
+// 64-bit signed add through the unsigned atomic (two's complement).
+__device__ __forceinline__ void atomic_add_ll(long long* p, long long v) {
+  atomicAdd(reinterpret_cast<unsigned long long*>(p), (unsigned long long)v);
+}
+
+__device__ __forceinline__ void set_status(int32_t* st, int bits) {
+  if (st) atomicOr(st, bits);
+}
+
+// Row of `k` by one thread scanning the whole window (first match in probe
+// order; the identity map holds at most one).  -1 if absent.
+__device__ __forceinline__ int64_t find_row_thread(const long long* __restrict__ keys, int64_t k,
+                                                   int64_t h, const Geo& g) {
+  int64_t found = -1;
+  for (int32_t j = 0; j < g.P; ++j) {
+    const int64_t s = wslot(h, j, g);
+    if (found < 0 && ld_cg(keys + s) == k) found = s;
+  }
+  return found;
+}
+
+// ---------------------------------------------------------------------------
+// Lookup: G lanes cooperate on one id (G = next power of two >= P, at most 32),
+// so the P keys of a window are fetched by one coalesced request.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_lookup(const long long* __restrict__ ids, int64_t n,
+                                                   const long long* __restrict__ keys, Geo g,
+                                                   int G, int32_t* __restrict__ rows,
+                                                   uint8_t* __restrict__ hit, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & (G - 1);
+  const unsigned gmask = (G == 32) ? 0xFFFFFFFFu : (((1u << G) - 1u) << (lane & ~(G - 1)));
+  const int64_t groups_per_grid = ((int64_t)gridDim.x * blockDim.x) / G;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / G; i < n;
+       i += groups_per_grid) {
+    const long long k = ids[i];
+    int32_t best = 0x7FFFFFFF;
+    if (k >= 0) {
+      const int64_t h = home_slot(k, g);
+      for (int32_t j = sub; j < g.P; j += G)
+        if (__ldg(keys + wslot(h, j, g)) == k && j < best) best = j;
+    }
+    for (int off = G >> 1; off > 0; off >>= 1) {
+      const int32_t o = __shfl_xor_sync(gmask, best, off, G);
+      best = o < best ? o : best;
+    }
+    if (sub == 0) {
+      int32_t r = -1;
+      if (k < 0)
+        set_status(status, kStBadKey);
+      else if (best != 0x7FFFFFFF)
+        r = (int32_t)wslot(home_slot(k, g), best, g);
+      rows[i] = r;
+      hit[i] = r >= 0 ? 1 : 0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Fused gather: out[i] = [hit ? M[rows[i]] : +0] ++ ao[ao_rows[i]], one warp per
+// output row, 16-byte vectors, all loads of a chunk issued before its stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_gather_fused(
+    const int32_t* __restrict__ rows, const uint8_t* __restrict__ hit, int64_t n,
+    const float4* __restrict__ M, int64_t C, int D4, const float4* __restrict__ ao,
+    int64_t ao_n, int A4, const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
+    int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int W4 = D4 + A4;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += warps) {
+    int32_t r = rows[i];
+    bool h = hit[i] != 0;
+    if (h && (r < 0 || (int64_t)r >= C)) {
+      if (lane == 0) set_status(status, kStBadRow);
+      h = false;
+    }
+    int32_t a = 0;
+    bool has_a = A4 > 0;
+    if (has_a) {
+      a = ao_rows[i];
+      if (a < 0 || (int64_t)a >= ao_n) {
+        if (lane == 0) set_status(status, kStBadAo);
+        has_a = false;
+      }
+    }
+    const float4* src = M + (int64_t)(h ? r : 0) * D4;
+    const float4* asrc = ao + (int64_t)a * A4;
+    float4* dst = out + i * (int64_t)W4;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < W4; base += 4 * 32) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        v[u] = z;
+        if (c < D4) {
+          if (h) v[u] = __ldg(src + c);
+        } else if (c < W4 && has_a) {
+          v[u] = __ldg(asrc + (c - D4));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        if (c < W4) __stcs(dst + c, v[u]);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dedup, phase 1: insert every id into an open-addressing scratch hash (key,
+// smallest position).  Lanes of a warp holding the same id elect the lowest
+// lane first, so a hot id costs one atomic per warp instead of one per copy.
+// Block 0 also clears the step counters used by the later phases.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_dedup_insert(
+    const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
+    uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
+    WbStats* stats, int32_t* status) {
+  if (blockIdx.x == 0 && threadIdx.x < sizeof(StepCtr) / 4)
+    reinterpret_cast<int32_t*>(ctr)[threadIdx.x] = 0;
+  if (stats && blockIdx.x == 0 && threadIdx.x < 7) reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // Whole warps iterate together so that __match_any_sync sees all lanes.
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n;
+       base += stride) {
+    const int64_t i = base + (threadIdx.x & 31);
+    const bool valid = i < n;
+    const long long k = valid ? ids[i] : -1;
+    const unsigned active = __ballot_sync(0xFFFFFFFFu, valid);
+    const unsigned same = __match_any_sync(0xFFFFFFFFu, (unsigned long long)k) & active;
+    if (!valid) continue;
+    if (k < 0) {
+      slot_of[i] = -1;
+      set_status(status, kStBadKey);
+      continue;
+    }
+    const int leader = __ffs(same) - 1;
+    int64_t s = (int64_t)(splitmix64((uint64_t)k ^ 0xD6E8FEB86659FD93ull) & hmask);
+    if ((int)(threadIdx.x & 31) == leader) {
+      bool placed = false;
+      for (uint64_t probe = 0; probe <= hmask && !placed; ++probe) {
+        unsigned long long cur = __ldcg(hkey + s);
+        if (cur == kEmptyKey) cur = atomicCAS(hkey + s, kEmptyKey, (unsigned long long)k);
+        if (cur == kEmptyKey || cur == (unsigned long long)k) {
+          if (__ldcg(hpos + s) > (uint32_t)i) atomicMin(hpos + s, (uint32_t)i);
+          placed = true;
+        } else {
+          s = (s + 1) & (int64_t)hmask;
+        }
+      }
+      if (!placed) set_status(status, kStInternal);  // scratch hash sized >= 2n: never expected
+    }
+    // Every copy learns the slot from its leader.
+    s = __shfl_sync(same, s, leader);
+    slot_of[i] = (int32_t)s;
+  }
+}
+
+// Block-wide exclusive scan of one int per thread; returns the block total.
+__device__ __forceinline__ int block_excl_scan(int v, int* smem /* >= 33 ints */, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) smem[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? smem[lane] : 0;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, w, off);
+      if (lane >= off) w += y;
+    }
+    if (lane < nw) smem[lane] = w;
+    if (lane == nw - 1) smem[32] = w;
+  }
+  __syncthreads();
+  const int before = (warp ? smem[warp - 1] : 0) + x - v;
+  total = smem[32];
+  __syncthreads();
+  return before;
+}
+
+__device__ __forceinline__ long long block_sum_ll(long long v, long long* smem /* >= 32 */) {
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane == 0) smem[warp] = v;
+  __syncthreads();
+  long long t = 0;
+  if (threadIdx.x == 0)
+    for (int w = 0; w < nw; ++w) t += smem[w];
+  __syncthreads();
+  if (threadIdx.x == 0) smem[0] = t;
+  __syncthreads();
+  t = smem[0];
+  __syncthreads();
+  return t;
+}
+
+// Sum of cnt[0 .. upto) by the whole block.
+__device__ __forceinline__ long long block_prefix_of_counts(const int32_t* cnt, int64_t upto,
+                                                            long long* smem) {
+  long long acc = 0;
+  for (int64_t b = threadIdx.x; b < upto; b += blockDim.x) acc += cnt[b];
+  return block_sum_ll(acc, smem);
+}
+
+// Dedup, phase 2: per tile of kTile positions, count first occurrences.
+__global__ void __launch_bounds__(kBlock) k_dedup_count(const int32_t* __restrict__ slot_of,
+                                                        const uint32_t* __restrict__ hpos,
+                                                        int64_t n, int32_t* __restrict__ bcount) {
+  __shared__ long long sm[33];
+  const int64_t base = (int64_t)blockIdx.x * kTile + threadIdx.x * 4;
+  int c = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = base + u;
+    if (i < n) {
+      const int32_t s = slot_of[i];
+      c += (s >= 0 && __ldcg(hpos + s) == (uint32_t)i);
+    }
+  }
+  const long long t = block_sum_ll(c, sm);
+  if (threadIdx.x == 0) bcount[blockIdx.x] = (int32_t)t;
+}
+
+// Dedup, phase 3: ordered compaction of first occurrences into (uniq, pos), and
+// reset of the scratch hash slots for the next call.  With `keys` non-null
+// (Writeback) each distinct id is also re-probed in the table: a resident id
+// refreshes last[row] = step; a missing id joins insert round 0 and claims its
+// window in claims0.
+__global__ void __launch_bounds__(kBlock) k_dedup_compact(
+    const long long* __restrict__ ids, int64_t n, const int32_t* __restrict__ slot_of,
+    unsigned long long* __restrict__ hkey, uint32_t* __restrict__ hpos,
+    const int32_t* __restrict__ bcount, long long* __restrict__ ukey, int32_t* __restrict__ upos,
+    long long* dev_count,
+    // Writeback extras (keys == nullptr for plain dedup)
+    const long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
+    int32_t* __restrict__ urow, int32_t* __restrict__ list0, unsigned long long* __restrict__ claims0,
+    StepCtr* ctr, WbStats* stats) {
+  __shared__ long long sm[33];
+  __shared__ int smi[33];
+  const long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
+  const int64_t base = (int64_t)blockIdx.x * kTile + threadIdx.x * 4;
+  int flags = 0, c = 0, nvalid = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t i = base + u;
+    if (i < n) {
+      const int32_t s = slot_of[i];
+      nvalid += s >= 0;
+      if (s >= 0 && __ldcg(hpos + s) == (uint32_t)i) {
+        flags |= 1 << u;
+        ++c;
+      }
+    }
+  }
+  int total = 0;
+  int rank = block_excl_scan(c, smi, total);
+  int hits = 0;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (!(flags & (1 << u))) continue;
+    const int64_t i = base + u;
+    const int64_t uidx = offset + rank++;
+    const long long k = ids[i];
+    const int32_t s = slot_of[i];
+    ukey[uidx] = k;
+    upos[uidx] = (int32_t)i;
+    hkey[s] = kEmptyKey;  // only this thread owns slot s now
+    hpos[s] = kNoPos;
+    if (keys) {
+      const int64_t h = home_slot(k, g);
+      const int64_t r = find_row_thread(keys, k, h, g);
+      if (r >= 0) {
+        urow[uidx] = (int32_t)r;
+        last[r] = step;
+        ++hits;
+      } else {
+        urow[uidx] = -1;
+        const int m = atomicAdd(&ctr->nlist[0], 1);
+        list0[m] = (int32_t)uidx;
+        for (int32_t j = 0; j < g.P; ++j) atomicMin(claims0 + wslot(h, j, g), (unsigned long long)k);
+      }
+    }
+  }
+  if (stats) {
+    const long long bh = block_sum_ll(hits, sm);
+    const long long bv = block_sum_ll(nvalid, sm);
+    if (threadIdx.x == 0) {
+      if (bh) atomic_add_ll(&stats->n_hit_unique, bh);
+      if (bv) atomic_add_ll(&stats->n_ids, bv);
+    }
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    const long long U = offset + total;
+    if (dev_count) *dev_count = U;
+    if (stats) stats->n_unique = U;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Insert of missing keys in conflict rounds.
+//
+// Sequential rule: missing keys are inserted one at a time in ascending key
+// order, each into the row of its window with the smallest (last, row).  A key
+// k may be placed as soon as no smaller missing key that is still unplaced has
+// a window overlapping W(k): then the rows of W(k) already hold their final
+// state with respect to every smaller key, and no larger key can touch them
+// before k in the sequential order.  Each round every unplaced key writes
+// atomicMin(claim[s], k) on its window; a key that finds its own value in all
+// of its P claim slots is the smallest unplaced key over every overlapping
+// window, so it commits.  Keys committing in the same round have disjoint
+// windows (a shared slot would hold the smaller key), so they write the table
+// independently.  The smallest unplaced key always commits, so rounds end.
+//
+// Round r checks claims[r % 3], makes round-(r+1) claims in claims[(r+1) % 3]
+// and clears round-(r-1) claims in claims[(r-1) % 3]: the three uses never
+// touch the same array inside one launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool try_commit(int64_t uidx, const long long* __restrict__ ukey,
+                                           const unsigned long long* claims,
+                                           long long* __restrict__ keys,
+                                           long long* __restrict__ last, const Geo& g,
+                                           long long step, int32_t* __restrict__ urow,
+                                           long long& evicted) {
+  const long long k = ukey[uidx];
+  const int64_t h = home_slot(k, g);
+  for (int32_t j = 0; j < g.P; ++j)
+    if (ld_cg(claims + wslot(h, j, g)) != (unsigned long long)k) return false;
+  int64_t best = -1;
+  long long best_last = 0;
+  for (int32_t j = 0; j < g.P; ++j) {
+    const int64_t s = wslot(h, j, g);
+    const long long l = ld_cg(last + s);
+    if (best < 0 || l < best_last || (l == best_last && s < best)) {
+      best = s;
+      best_last = l;
+    }
+  }
+  if (ld_cg(keys + best) != -1) ++evicted;
+  keys[best] = k;
+  last[best] = step;
+  urow[uidx] = (int32_t)best;
+  return true;
+}
+
+__device__ __forceinline__ void claim_window(unsigned long long* claims, long long k, const Geo& g) {
+  const int64_t h = home_slot(k, g);
+  for (int32_t j = 0; j < g.P; ++j) atomicMin(claims + wslot(h, j, g), (unsigned long long)k);
+}
+
+__device__ __forceinline__ void clear_window(unsigned long long* claims, long long k, const Geo& g) {
+  const int64_t h = home_slot(k, g);
+  for (int32_t j = 0; j < g.P; ++j) claims[wslot(h, j, g)] = kNoClaim;
+}
+
+__global__ void __launch_bounds__(kBlock) k_insert_round(
+    int r, const long long* __restrict__ ukey, long long* __restrict__ keys,
+    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
+    int32_t* list_prev, int32_t* list_cur, int32_t* list_next, unsigned long long* claims_prev,
+    unsigned long long* claims_cur, unsigned long long* claims_next, StepCtr* ctr,
+    WbStats* stats) {
+  __shared__ long long sm[33];
+  const int32_t nprev = r > 0 ? ctr->nlist[r - 1] : 0;
+  const int32_t ncur = ctr->nlist[r];
+  const int32_t nmax = nprev > ncur ? nprev : ncur;
+  long long evicted = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t first = (int64_t)blockIdx.x * blockDim.x;
+  // Whole blocks iterate together (block_sum below needs every thread).
+  for (int64_t base = first; base < nmax; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    if (i < nprev) clear_window(claims_prev, ukey[list_prev[i]], g);
+    if (i < ncur) {
+      const int32_t u = list_cur[i];
+      if (!try_commit(u, ukey, claims_cur, keys, last, g, step, urow, evicted)) {
+        const int m = atomicAdd(&ctr->nlist[r + 1], 1);
+        list_next[m] = u;
+        claim_window(claims_next, ukey[u], g);
+      }
+    }
+  }
+  if (first < nmax) {
+    const long long ev = block_sum_ll(evicted, sm);
+    if (threadIdx.x == 0 && ev && stats) atomic_add_ll(&stats->n_evicted, ev);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0 && stats) atomic_add_ll(&stats->n_rounds, 1LL);
+}
+
+// Remaining rounds in one block (block barriers only).  Lists and claims
+// rotate exactly as in k_insert_round; the list buffers come from the caller.
+__global__ void __launch_bounds__(1024) k_insert_finish(
+    int r0, const long long* __restrict__ ukey, long long* __restrict__ keys,
+    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
+    int32_t* lists0, int32_t* lists1, int32_t* lists2, unsigned long long* claims0,
+    unsigned long long* claims1, unsigned long long* claims2, StepCtr* ctr, WbStats* stats,
+    int32_t* status) {
+  __shared__ int32_t s_cnt[2];  // next-list counters, alternating by iteration parity
+  __shared__ long long sm[33];
+  int32_t* lists[3] = {lists0, lists1, lists2};
+  unsigned long long* claims[3] = {claims0, claims1, claims2};
+  int32_t nprev = r0 > 0 ? ctr->nlist[r0 - 1] : 0;
+  int32_t ncur = ctr->nlist[r0];
+  const int32_t bound = ncur + 2;  // each round commits at least one key
+  long long evicted = 0, rounds = 0;
+  int r = r0;
+  for (int32_t it = 0; it <= bound; ++it) {
+    // s_cnt[it & 1] was last read right after the barrier that ended iteration
+    // it - 2, before every thread passed the first barrier of iteration it - 1.
+    int32_t* s_next = &s_cnt[it & 1];
+    if (threadIdx.x == 0) *s_next = 0;
+    __syncthreads();
+    const int32_t nmax = nprev > ncur ? nprev : ncur;
+    int32_t* lp = lists[(r + 2) % 3];
+    int32_t* lc = lists[r % 3];
+    int32_t* ln = lists[(r + 1) % 3];
+    for (int32_t i = threadIdx.x; i < nmax; i += blockDim.x) {
+      if (i < nprev) clear_window(claims[(r + 2) % 3], ukey[lp[i]], g);
+      if (i < ncur) {
+        const int32_t u = lc[i];
+        if (!try_commit(u, ukey, claims[r % 3], keys, last, g, step, urow, evicted)) {
+          const int m = atomicAdd(s_next, 1);
+          ln[m] = u;
+          claim_window(claims[(r + 1) % 3], ukey[u], g);
+        }
+      }
+    }
+    rounds += ncur > 0;
+    __threadfence();
+    __syncthreads();
+    nprev = ncur;
+    ncur = *s_next;
+    ++r;
+    if (nprev == 0 && ncur == 0) break;
+    if (it == bound && threadIdx.x == 0) set_status(status, kStInternal);
+  }
+  const long long ev = block_sum_ll(evicted, sm);
+  if (threadIdx.x == 0 && stats) {
+    if (ev) atomic_add_ll(&stats->n_evicted, ev);
+    if (rounds) atomic_add_ll(&stats->n_rounds, rounds);
+    stats->n_inserted = ctr->nlist[0];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Writeback: M[r] <- fl(e_hat - fl(e_hat - e)) for every distinct id still owning
+// its row; one warp per row, 16-byte vectors, loads of a chunk before stores.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_writeback(
+    const long long* __restrict__ ukey, const int32_t* __restrict__ upos,
+    const int32_t* __restrict__ urow, const long long* U_ptr, const long long* __restrict__ keys,
+    float4* __restrict__ M, const float4* __restrict__ e, int D4, WbStats* stats) {
+  __shared__ long long sm[33];
+  const int lane = threadIdx.x & 31;
+  const long long U = *U_ptr;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  long long dropped = 0;
+  for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
+    const int32_t r = urow[u];
+    if (r < 0) {  // every distinct id gets a row; never expected
+      dropped += lane == 0;
+      continue;
+    }
+    if (__ldcg(keys + r) != ukey[u]) {
+      dropped += lane == 0;
+      continue;
+    }
+    float4* m = M + (int64_t)r * D4;
+    const float4* ev = e + (int64_t)upos[u] * D4;
+    for (int base = 0; base < D4; base += 4 * 32) {
+      float4 a[4], b[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = base + q * 32 + lane;
+        if (c < D4) {
+          a[q] = __ldcg(m + c);
+          b[q] = __ldcs(ev + c);
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = base + q * 32 + lane;
+        if (c < D4) {
+          float4 o;
+          o.x = __fsub_rn(a[q].x, __fsub_rn(a[q].x, b[q].x));
+          o.y = __fsub_rn(a[q].y, __fsub_rn(a[q].y, b[q].y));
+          o.z = __fsub_rn(a[q].z, __fsub_rn(a[q].z, b[q].z));
+          o.w = __fsub_rn(a[q].w, __fsub_rn(a[q].w, b[q].w));
+          m[c] = o;
+        }
+      }
+    }
+  }
+  if (stats) {
+    const long long d = block_sum_ll(dropped, sm);
+    if (threadIdx.x == 0 && d) atomic_add_ll(&stats->n_dropped, d);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Select rows written at or after `since`, ascending (ordered compaction).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_select_count(const long long* __restrict__ keys,
+                                                         const long long* __restrict__ last,
+                                                         int64_t C, long long since,
+                                                         int32_t* __restrict__ bcount) {
+  __shared__ long long sm[33];
+  const int64_t base = (int64_t)blockIdx.x * kSelTile + threadIdx.x;
+  int c = 0;
+#pragma unroll 4
+  for (int u = 0; u < kSelTile / kBlock; ++u) {
+    const int64_t r = base + (int64_t)u * kBlock;
+    if (r < C) c += keys[r] != -1 && last[r] >= since;
+  }
+  const long long t = block_sum_ll(c, sm);
+  if (threadIdx.x == 0) bcount[blockIdx.x] = (int32_t)t;
+}
+
+__global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __restrict__ keys,
+                                                           const long long* __restrict__ last,
+                                                           int64_t C, long long since,
+                                                           const int32_t* __restrict__ bcount,
+                                                           int32_t* __restrict__ rows_out,
+                                                           long long* dev_count) {
+  __shared__ long long sm[33];
+  __shared__ int smi[33];
+  long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
+  // kSelTile rows in kSelTile/kBlock passes of kBlock consecutive rows (coalesced).
+  for (int u = 0; u < kSelTile / kBlock; ++u) {
+    const int64_t r = (int64_t)blockIdx.x * kSelTile + (int64_t)u * kBlock + threadIdx.x;
+    const int f = (r < C) && keys[r] != -1 && last[r] >= since;
+    int total = 0;
+    const int before = block_excl_scan(f, smi, total);
+    if (f) rows_out[offset + before] = (int32_t)r;
+    offset += total;
+  }
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) *dev_count = offset;
+}
+
+// ---------------------------------------------------------------------------
+// int8 export: one warp per row.  a = max|x| (exact), scale = a/127 and x/scale
+// as IEEE divisions, round-half-even, clamp to +-127.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_export_int8(
+    const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
+    const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C, int D4,
+    char4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
+    int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  int64_t nn = n;
+  if (dev_n) {
+    const long long d = *dev_n;
+    nn = d < nn ? d : nn;
+  }
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nn; i += warps) {
+    const int32_t r = rows[i];
+    char4* qo = q + i * (int64_t)D4;
+    if (r < 0 || (int64_t)r >= C) {
+      if (lane == 0) {
+        set_status(status, kStBadRow);
+        scale[i] = 0.f;
+        keys_out[i] = -1;
+      }
+      for (int c = lane; c < D4; c += 32) qo[c] = make_char4(0, 0, 0, 0);
+      continue;
+    }
+    const float4* x = M + (int64_t)r * D4;
+    float a = 0.f;
+    for (int c = lane; c < D4; c += 32) {
+      const float4 v = x[c];
+      a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+    for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+    const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
+    for (int c = lane; c < D4; c += 32) {
+      const float4 v = x[c];
+      char4 o = make_char4(0, 0, 0, 0);
+      if (a != 0.f) {
+        auto qz = [s](float xv) -> signed char {
+          int t = __float2int_rn(__fdiv_rn(xv, s));
+          t = t > 127 ? 127 : (t < -127 ? -127 : t);
+          return (signed char)t;
+        };
+        o = make_char4(qz(v.x), qz(v.y), qz(v.z), qz(v.w));
+      }
+      qo[c] = o;
+    }
+    if (lane == 0) {
+      scale[i] = s;
+      keys_out[i] = keys[r];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Serving gather from an int8 snapshot: one warp per id; lanes j < P probe the
+// window, the first matching probe offset wins; then out = hit ? q*scale : +0.
+// Lane l stores the 16-byte vector l + 32*c, so every store request covers a
+// contiguous 512 B of the output row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_serve_gather(
+    const long long* __restrict__ snap_keys, Geo g, const char4* __restrict__ q,
+    const float* __restrict__ scale, int D4, const long long* __restrict__ ids, int64_t n,
+    int32_t* __restrict__ rows, uint8_t* __restrict__ hit, float4* __restrict__ out,
+    int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += warps) {
+    const long long k = ids[i];
+    int32_t best = 0x7FFFFFFF;
+    int64_t h = 0;
+    if (k >= 0) {
+      h = home_slot(k, g);
+      for (int32_t j = lane; j < g.P; j += 32)
+        if (__ldg(snap_keys + wslot(h, j, g)) == k && j < best) best = j;
+    }
+    for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xFFFFFFFFu, best, off));
+    const int64_t r = (k >= 0 && best != 0x7FFFFFFF) ? wslot(h, best, g) : -1;
+    if (lane == 0) {
+      if (k < 0) set_status(status, kStBadKey);
+      rows[i] = (int32_t)r;
+      hit[i] = r >= 0;
+    }
+    float4* o = out + i * (int64_t)D4;
+    if (r >= 0) {
+      const float s = __ldg(scale + r);
+      const char4* qr = q + r * (int64_t)D4;
+      for (int c = lane; c < D4; c += 32) {
+        const char4 v = __ldg(qr + c);
+        __stcs(o + c, make_float4(__fmul_rn((float)v.x, s), __fmul_rn((float)v.y, s),
+                                  __fmul_rn((float)v.z, s), __fmul_rn((float)v.w, s)));
+      }
+    } else {
+      for (int c = lane; c < D4; c += 32) __stcs(o + c, make_float4(0.f, 0.f, 0.f, 0.f));
+    }
+  }
+}
+
+}  // namespace mpzch

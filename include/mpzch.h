@@ -1,0 +1,215 @@
+/*
+ * mpzch.h -- C ABI of libmpzch.so, the B200 (sm_100a) hot path of the Memory
+ * Layer trainable in-model embedding cache.
+ *
+ * Source: "Memory Layer: Train the In-Model Cache for Recommendation Models"
+ * (cited below as "Memory Layer"), section 2 (method) and section 5
+ * (limitations: int8 row quantisation at serving time).  The table M maps an
+ * item id to a dense D-dim item-tower vector.  A Multi-Probe Zero-Collision
+ * Hashing (MPZCH) identity map sends raw ids to rows without collisions,
+ * per-row metadata shares the row index, capacity is bounded and eviction is
+ * LRU.  Training reads e_hat = M[i]; Writeback applies g = e_hat - e with an
+ * exact SGD step of learning rate 1, i.e. M[i] <- e_hat - (e_hat - e), once
+ * per row after in-batch dedup.  On a miss the cached branch is zeroed and the
+ * always-on (author id) features remain.
+ *
+ * Fixed rules of this implementation (the page leaves them open):
+ *   start slot   h(k) = splitmix64(k) mod C   (SplitMix64 generator output for state k)
+ *   window       W(k) = { (h(k) + j) mod C : j = 0..P-1 }; lookups scan all P slots
+ *   empty row    key -1, last-write step -1
+ *   victim       the row of W(k) with the smallest (last-write step, row index)
+ *   order        resident keys are refreshed first, then missing keys are
+ *                inserted one at a time in ascending key order
+ *   dedup        the first occurrence of an id in the batch supplies e
+ *   export       a = max|x|, scale = a/127 (binary32), q = clamp(rne(x/scale), +-127)
+ * Valid item ids are 0 <= k < 2^63.  Negative ids are skipped and raise
+ * MPZCH_STATUS_BADKEY in the sticky device status.
+ *
+ * Conventions for every call:
+ *  - Pointers named dev_* or documented as "device" are device pointers on the
+ *    device that was current at mpzch_create; they are owned by the caller and
+ *    must stay valid until the stream work completes.  The table's own storage
+ *    (keys, last-write steps, values, scratch) is owned by the handle.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on it unless stated otherwise.
+ *  - The return value is MPZCH_OK or a negative MPZCH_E* code for errors the
+ *    host can see (bad arguments, allocation, CUDA launch errors).  Errors the
+ *    device sees (bad ids, rows out of range) set bits of a sticky device status
+ *    word, read and cleared by mpzch_get_status.  No kernel traps or spins.
+ *  - Calls must be issued with the table's device current.  A handle is not
+ *    thread-safe; calls on one handle must be ordered on one stream.
+ */
+#ifndef MPZCH_H
+#define MPZCH_H
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MPZCH_API __attribute__((visibility("default")))
+#else
+#define MPZCH_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MPZCH_OK 0
+#define MPZCH_EINVAL (-1)  /* bad argument (null pointer, size, step order, device) */
+#define MPZCH_ENOMEM (-2)  /* device allocation failed */
+#define MPZCH_ECUDA (-3)   /* a CUDA runtime call or launch failed */
+#define MPZCH_ECAPTURE (-5) /* would allocate while the stream is being captured */
+
+/* Sticky device status bits (mpzch_get_status). */
+#define MPZCH_STATUS_BADKEY 1   /* a negative item id was given */
+#define MPZCH_STATUS_BADROW 2   /* a row index outside [0, C) was given to gather/export */
+#define MPZCH_STATUS_BADAO 4    /* an always-on row outside [0, ao_nrows) was given */
+#define MPZCH_STATUS_INTERNAL 8 /* an internal bound was hit (never expected) */
+
+typedef struct mpzch_table mpzch_table;
+
+/* Per-Writeback counters, written to device memory by mpzch_writeback. */
+typedef struct {
+  int64_t n_ids;        /* valid (non-negative) ids in the batch */
+  int64_t n_unique;     /* distinct ids */
+  int64_t n_hit_unique; /* distinct ids resident before the step */
+  int64_t n_inserted;   /* distinct ids inserted (missing before the step) */
+  int64_t n_evicted;    /* inserts that replaced a live key */
+  int64_t n_dropped;    /* distinct ids evicted again later in the same step (no write) */
+  int64_t n_rounds;     /* insert conflict rounds executed */
+} mpzch_wb_stats;
+
+/* Create a table with `capacity` rows (1 <= C <= 2^31-1) of `dim` fp32 values
+ * (dim > 0, dim % 4 == 0 so rows are 16-byte vectors) and a `probes`-slot
+ * window (1 <= P <= C).  Allocates keys[C] int64 = -1, last[C] int64 = -1,
+ * M[C][dim] fp32 = +0 and insert scratch (3*C*8 bytes) on the current device,
+ * initialised on `stream`.  Memory layout: keys, last and M are separate
+ * row-indexed arrays (the metadata shares the row index with the vectors,
+ * Memory Layer section 2).  Returns MPZCH_EINVAL for bad sizes or a null
+ * `out`, MPZCH_ENOMEM if an allocation fails (nothing is leaked). */
+MPZCH_API int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mpzch_table** out);
+
+/* Free all device memory of the table (synchronises the device). NULL is a no-op. */
+MPZCH_API int mpzch_destroy(mpzch_table* t);
+
+/* Pre-size the per-batch scratch for batches of up to `max_batch` ids so that
+ * later calls never allocate (growth otherwise happens on demand inside
+ * mpzch_writeback / mpzch_dedup, synchronises the device, and is refused with
+ * MPZCH_ECAPTURE while `stream` is being captured). */
+MPZCH_API int mpzch_reserve(mpzch_table* t, int64_t max_batch, void* stream);
+
+/* MPZCH lookup (Memory Layer section 2: the identity map sends a raw id to its
+ * row).  ids: device int64[n].  rows: device int32[n], the row holding the id
+ * or -1.  hit: device uint8[n], 1 iff rows[i] >= 0.  Read-only on the table;
+ * never refreshes LRU metadata.  n == 0 is a no-op. */
+MPZCH_API int mpzch_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit,
+                 void* stream);
+
+/* Fused cached read with the always-on fallback (Memory Layer section 2: the
+ * loss uses e_hat = M[i]; on a miss the cached branch is zeroed and the
+ * always-on author embedding remains).  For i < n:
+ *   out[i][0:dim]          = hit[i] ? M[rows[i]][:] : +0.0
+ *   out[i][dim:dim+ao_dim] = ao_table[ao_rows[i]][:]
+ * rows/hit: device, as produced by mpzch_lookup.  ao_table: device fp32
+ * [ao_nrows][ao_dim] (ao_dim % 4 == 0), ao_rows: device int32[n]; pass
+ * ao_table = NULL, ao_nrows = 0, ao_dim = 0, ao_rows = NULL for no concat.
+ * out: device fp32 [n][dim + ao_dim], 16-byte aligned.  Out-of-range rows set
+ * MPZCH_STATUS_BADROW / BADAO and produce zeros. */
+MPZCH_API int mpzch_gather_fused(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
+                       const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
+                       const int32_t* ao_rows, float* out, void* stream);
+
+/* In-batch dedup (Memory Layer section 2, Writeback paragraph: duplicate ids
+ * of a batch are removed first so each row gets one exact write).  ids: device
+ * int64[n].  uniq: device int64[n] and pos: device int32[n] receive the
+ * distinct ids and the index of their first occurrence, in first-occurrence
+ * order; dev_count: device int64, receives the number of distinct ids.
+ * Negative ids are skipped (MPZCH_STATUS_BADKEY).  Uses the table's scratch. */
+MPZCH_API int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
+                int64_t* dev_count, void* stream);
+
+/* One training step of the table (Memory Layer section 2, MPZCH and Writeback
+ * paragraphs).  ids: device int64[n]; e: device fp32 [n][dim], the item-tower
+ * targets, row i belonging to ids[i].  step must exceed every earlier step of
+ * this table (host-checked; MPZCH_EINVAL otherwise).  In order:
+ *   1. dedup (first occurrence supplies e);
+ *   2. resident ids: last[row] = step;
+ *   3. missing ids, ascending: victim = argmin over W(k) of (last, row);
+ *      keys[victim] = k, last[victim] = step;
+ *   4. every id still owning its row r: M[r] <- fl(e_hat - fl(e_hat - e)),
+ *      e_hat = the row's content before this step.
+ * dev_stats: nullable device mpzch_wb_stats, written before the call's work
+ * completes on `stream`.  Call order within a step: lookup -> gather_fused ->
+ * writeback (a gather issued after writeback sees the new values). */
+MPZCH_API int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
+                    mpzch_wb_stats* dev_stats, void* stream);
+
+/* Rows written recently (Memory Layer section 2, RES paragraph: fresh rows are
+ * streamed to the predictors): rows_out (device int32[C]) receives, in
+ * ascending order, every row r with keys[r] != -1 and last[r] >= since_step;
+ * dev_count (device int64) receives their number. */
+MPZCH_API int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows_out,
+                               int64_t* dev_count, void* stream);
+
+/* Per-row int8 export of the serving snapshot (Memory Layer section 2, RES:
+ * rows are quantised before the push; section 5: serving uses int8 row
+ * quantisation).  For i < min(n, *dev_n): with x = M[rows[i]],
+ *   a = max|x|, scale[i] = a / 127 (binary32), q[i][d] = clamp(rne(x[d]/scale[i]), -127, 127),
+ *   a == 0 gives scale 0 and q 0;  keys_out[i] = keys[rows[i]].
+ * rows: device int32[n]; q: device int8[n][dim]; scale: device fp32[n];
+ * keys_out: device int64[n]; dev_n: nullable device int64 count (e.g. the
+ * dev_count of mpzch_select_written_since), NULL = n. */
+MPZCH_API int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n,
+                      int8_t* q, float* scale, int64_t* keys_out, void* stream);
+
+/* Serving read from an int8 snapshot (Memory Layer section 2, RES: predictors
+ * receive vectors + identity map; section 5: int8 rows).  The snapshot is a
+ * table image: snap_keys device int64[capacity] (-1 = empty), snap_q device
+ * int8[capacity][dim], snap_scale device fp32[capacity].  For each ids[i]
+ * (device int64[n]): rows[i] = the snapshot row holding it or -1 (all `probes`
+ * window slots scanned), hit[i] = rows[i] >= 0, and
+ *   out[i][:] = hit ? fl((float)q * scale) : +0.0      (out: device fp32 [n][dim]).
+ * dev_status: nullable device int32, OR-ed with MPZCH_STATUS_BADKEY for
+ * negative ids.  Needs no table handle and allocates nothing. */
+MPZCH_API int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probes,
+                       const int8_t* snap_q, const float* snap_scale, int32_t dim,
+                       const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit, float* out,
+                       int32_t* dev_status, void* stream);
+
+/* Device pointers to the table's state (for checkpoint/resume and tests):
+ * keys int64[C], last int64[C], M fp32[C][dim].  Any argument may be NULL. */
+MPZCH_API int mpzch_state_views(mpzch_table* t, int64_t** keys, int64_t** last, float** M);
+
+/* Host-side last step (the step order check).  After restoring a saved state
+ * through mpzch_state_views, set it to the saved table's last step. */
+MPZCH_API int mpzch_get_last_step(mpzch_table* t, int64_t* step);
+MPZCH_API int mpzch_set_last_step(mpzch_table* t, int64_t step);
+
+/* Reads and clears the sticky device status word (MPZCH_STATUS_* bits).
+ * Synchronises `stream`. */
+MPZCH_API int mpzch_get_status(mpzch_table* t, int32_t* status, void* stream);
+
+/* Per-phase timing with CUDA events recorded around each kernel launch on the
+ * launching stream.  Phases (index): 0 lookup, 1 gather, 2 dedup, 3 insert,
+ * 4 writeback, 5 select, 6 export.  mpzch_trace_read synchronises the events
+ * recorded since the last read and returns, per phase, the summed device
+ * milliseconds and the number of kernel launches. */
+#define MPZCH_NPHASES 7
+MPZCH_API int mpzch_trace_enable(mpzch_table* t, int32_t on);
+MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t nphases);
+
+/* Options.  MPZCH_OPT_WIDE_ROUNDS: number of grid-wide insert conflict rounds
+ * before the single-block finisher takes the remaining keys (default 3, 0..16). */
+#define MPZCH_OPT_WIDE_ROUNDS 1
+MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
+
+/* Test hook: the next `count` device allocations made by this library fail as
+ * if the device were out of memory (no CUDA call is made for them). */
+MPZCH_API int mpzch_debug_fail_allocs(int32_t count);
+
+/* Number of kernel launches this library issued in the calling process. */
+MPZCH_API int64_t mpzch_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MPZCH_H */

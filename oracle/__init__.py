@@ -59,12 +59,13 @@ def lib():
         L.orc_serve_gather.argtypes = [p, i64, i32, p, p, i32, p, i64, p, p, p]
         L.orc_state.argtypes = [p, p, p, p]
         L.orc_get_row.argtypes = [p, i32, p]
+        L.orc_get_rows.argtypes = [p, p, i64, p]
         L.orc_set_row.argtypes = [p, i32, p]
         L.orc_set_state.argtypes = [p, p, p, i64]
         for f in ("orc_create", "orc_track_rows", "orc_lookup", "orc_gather_fused", "orc_dedup",
                   "orc_writeback", "orc_select_written_since", "orc_quantize_row",
                   "orc_export_int8", "orc_serve_gather", "orc_state", "orc_get_row",
-                  "orc_set_row", "orc_set_state"):
+                  "orc_set_row", "orc_set_state", "orc_get_rows"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -213,7 +214,11 @@ class OracleTable:
         return out
 
     def rows(self, rs):
-        return np.stack([self.row(r) for r in rs]) if len(rs) else np.empty((0, self.dim), np.float32)
+        rs = _c(rs, np.int32)
+        out = np.empty((rs.size, self.dim), np.float32)
+        rc = lib().orc_get_rows(self.h, _ptr(rs), rs.size, _ptr(out))
+        assert rc == ORC_OK, rc
+        return out
 
     def set_row(self, r, x):
         x = _c(x, np.float32)
@@ -228,7 +233,7 @@ class OracleTable:
 
     def values(self):
         """Dense copy of every value row (track_all tables only)."""
-        return np.stack([self.row(r) for r in range(self.capacity)])
+        return self.rows(np.arange(self.capacity, dtype=np.int32))
 
 
 def oracle_lib_path() -> str:

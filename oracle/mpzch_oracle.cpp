@@ -358,6 +358,15 @@ extern "C" int orc_get_row(const orc_table* t, int32_t row, float* out) {
   return ORC_OK;
 }
 
+extern "C" int orc_get_rows(const orc_table* t, const int32_t* rows, int64_t n, float* out) {
+  if (!t || (n > 0 && (!rows || !out))) return ORC_EINVAL;
+  for (int64_t i = 0; i < n; ++i) {
+    int rc = orc_get_row(t, rows[i], out + i * t->D);
+    if (rc) return rc;
+  }
+  return ORC_OK;
+}
+
 extern "C" int orc_set_row(orc_table* t, int32_t row, const float* in) {
   if (!t || !in || row < 0 || row >= t->C) return ORC_EINVAL;
   float* m = row_ptr(t, row);

@@ -66,6 +66,8 @@ int orc_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probes,
 /* State access for comparisons (host pointers owned by the table). */
 int orc_state(orc_table* t, int64_t** keys, int64_t** last, int64_t* last_step);
 int orc_get_row(const orc_table* t, int32_t row, float* out);
+/* Copies rows[0..n) of M into out[n][D] (every listed row must be kept). */
+int orc_get_rows(const orc_table* t, const int32_t* rows, int64_t n, float* out);
 int orc_set_row(orc_table* t, int32_t row, const float* in);
 int orc_set_state(orc_table* t, const int64_t* keys, const int64_t* last, int64_t last_step);
 

@@ -1,0 +1,132 @@
+"""Drives one workload through the CUDA library and the CPU oracle side by side
+and compares every output bit for bit (GPU tests only)."""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle
+from hashed_sparse_table_b200 import inputs
+
+STATS_KEYS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped")
+
+
+def bits(a: np.ndarray) -> np.ndarray:
+    """Bit pattern view: equality on it is byte equality (+0 vs -0, NaN payloads)."""
+    a = np.ascontiguousarray(a)
+    return a.view({4: np.uint32, 8: np.uint64, 1: np.uint8, 2: np.uint16}[a.dtype.itemsize])
+
+
+def assert_bitwise(gpu: np.ndarray, ref: np.ndarray, what: str):
+    assert gpu.shape == ref.shape, (what, gpu.shape, ref.shape)
+    g, r = bits(gpu), bits(ref)
+    if not np.array_equal(g, r):
+        bad = np.argwhere(g != r)
+        i = tuple(bad[0])
+        raise AssertionError(f"{what}: {len(bad)} mismatches, first at {i}: gpu={gpu[i]!r} "
+                             f"oracle={ref[i]!r}")
+
+
+def stats_dict(t: torch.Tensor) -> dict:
+    v = t.cpu().tolist()
+    return dict(zip(STATS_KEYS + ("n_rounds",), v))
+
+
+@dataclasses.dataclass
+class RunResult:
+    tbl: object
+    orc: object
+    steps: int
+    stats: list
+
+
+def make_pair(w: inputs.Workload, track_all: bool = True, track_rows: Optional[np.ndarray] = None):
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(w.capacity, w.dim, w.probes)
+    orc = oracle.OracleTable(w.capacity, w.dim, w.probes, track_all=track_all)
+    if track_rows is not None:
+        orc.track_rows(track_rows)
+    return tbl, orc
+
+
+def compare_state(tbl, orc, what: str, value_rows: Optional[np.ndarray] = None, values=True):
+    keys, last, M = tbl.state()
+    ok, ol, _ = orc.state()
+    assert_bitwise(keys.cpu().numpy(), ok, f"{what}: keys")
+    assert_bitwise(last.cpu().numpy(), ol, f"{what}: last")
+    if not values:
+        return
+    if value_rows is None:
+        assert_bitwise(M.cpu().numpy(), orc.values(), f"{what}: M")
+    else:
+        idx = torch.from_numpy(value_rows.astype(np.int64)).to(M.device)
+        assert_bitwise(M.index_select(0, idx).cpu().numpy(), orc.rows(value_rows), f"{what}: M rows")
+
+
+def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None, start: int = 0,
+             state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
+             ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None) -> RunResult:
+    """Runs steps [start, start+steps) of workload w on both sides.
+
+    Per step: lookup of the labeled ids, fused gather (with the always-on concat
+    when the workload has one), Writeback of the whole batch.  Compares rows,
+    hit, gathered features (first `gather_rows` rows, -1 = all), Writeback
+    counters, and the table state every `state_every` / `values_every` steps."""
+    from hashed_sparse_table_b200 import binding
+    if tbl is None:
+        tbl, orc = make_pair(w)
+    if wide_rounds is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, wide_rounds)
+    T = w.steps if steps is None else steps
+    dev = tbl.device
+    ao = inputs.author_table(w)
+    ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None
+    stats_d = torch.zeros(7, dtype=torch.int64, device=dev)
+    all_stats = []
+    for t in range(start, start + T):
+        ids = ids_fn(t) if ids_fn else inputs.step_ids(w, t)
+        e = e_fn(t, ids.size) if e_fn else inputs.step_e(w, t, rows=ids.size)
+        lab = min(w.labeled, ids.size)
+        ids_d = torch.from_numpy(ids).to(dev)
+        e_d = torch.from_numpy(e).to(dev)
+        aor = inputs.author_rows(w, ids[:lab])
+        aor_d = torch.from_numpy(aor).to(dev) if aor is not None else None
+        rows_d, hit_d = tbl.lookup(ids_d[:lab])
+        out_d = tbl.gather_fused(rows_d, hit_d, ao_d, aor_d)
+        tbl.writeback(ids_d, e_d, t, stats_d)
+        # oracle
+        rc, orows, ohit = orc.lookup(ids[:lab])
+        assert rc == 0
+        n_g = lab if gather_rows < 0 else min(gather_rows, lab)
+        oout = orc.gather_fused(orows[:n_g], ohit[:n_g], ao, None if aor is None else aor[:n_g])
+        rc, ost = orc.writeback(ids, e, t)
+        assert rc == 0
+        assert_bitwise(rows_d.cpu().numpy(), orows, f"step {t}: rows")
+        assert_bitwise(hit_d.cpu().numpy(), ohit, f"step {t}: hit")
+        assert_bitwise(out_d[:n_g].cpu().numpy(), oout, f"step {t}: gathered features")
+        gst = stats_dict(stats_d)
+        for k in STATS_KEYS:
+            assert gst[k] == ost[k], (t, k, gst, ost)
+        assert (gst["n_rounds"] >= 1) == (ost["n_inserted"] > 0), (t, gst)
+        all_stats.append(gst)
+        last_step = t == start + T - 1
+        if last_step or (state_every and (t - start) % state_every == 0):
+            with_values = last_step or (values_every and (t - start) % values_every == 0)
+            compare_state(tbl, orc, f"step {t}", value_rows, values=with_values)
+    assert tbl.status() == 0
+    return RunResult(tbl, orc, T, all_stats)
+
+
+def snapshot_from_export(capacity: int, dim: int, rows: np.ndarray, q: np.ndarray, scale: np.ndarray,
+                         keys: np.ndarray):
+    """Serving snapshot image: exported rows at their own row index, -1 elsewhere."""
+    snap_keys = np.full(capacity, -1, np.int64)
+    snap_q = np.zeros((capacity, dim), np.int8)
+    snap_s = np.zeros(capacity, np.float32)
+    snap_keys[rows] = keys
+    snap_q[rows] = q
+    snap_s[rows] = scale
+    return snap_keys, snap_q, snap_s

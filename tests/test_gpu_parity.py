@@ -1,0 +1,267 @@
+"""CUDA path vs CPU oracle, bit for bit, at sizes the oracle finishes in seconds.
+
+Every case spans several 1024-id tiles and several thread blocks with a
+ragged tail, and compares the lookup rows / hit mask, the fused gather
+(cached branch + always-on concat), the Writeback counters and the whole table
+state (keys, last-write steps, values) after every step.  Edge cases: empty
+batches, bad ids and rows, non-power-of-two capacity, P = 1, P = C, P > 32,
+windows wrapping past the last row, heavy eviction with dropped writes, the
+insert rounds forced fully into the grid-wide path or fully into the
+single-block finisher, checkpoint/resume, and repeatability.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from hashed_sparse_table_b200 import inputs
+from gpu_harness import assert_bitwise, make_pair, run_pair, snapshot_from_export, compare_state
+
+pytestmark = pytest.mark.gpu
+
+W = inputs.Workload
+SCALED = {
+    # a 1M-row-style stream at 1/64 scale: Zipf 1.1 + 15% fresh keys
+    "c2_small": W("c2_small", 2, capacity=1 << 14, dim=512, probes=8, steps=20, labeled=3000,
+                  pool=0, zipf_alpha=1.1, zipf_keys=300_000, fresh_frac=0.15),
+    # multi-table: labeled + pool, author concat by mixed key (ragged sizes)
+    "c3_small": W("c3_small", 3, capacity=1 << 13, dim=512, probes=8, steps=20, labeled=700,
+                  pool=2900, zipf_alpha=0.9, zipf_keys=40_000, ao_rows=1 << 13, ao_dim=128,
+                  ao_kind="mix"),
+    # capacity stress: more distinct ids per step than rows, heavy eviction and drops
+    "c4_stress": W("c4_stress", 4, capacity=1 << 12, dim=64, probes=8, steps=12, labeled=6000,
+                   pool=0, zipf_alpha=1.2, zipf_keys=100_000, fresh_frac=0.2),
+    "nonpow2": W("nonpow2", 6, capacity=3001, dim=32, probes=5, steps=10, labeled=2500, pool=0,
+                 zipf_alpha=1.0001, zipf_keys=20_000, fresh_frac=0.1, ao_rows=700, ao_dim=4,
+                 ao_kind="mod"),
+    "p1_direct": W("p1_direct", 7, capacity=2048, dim=16, probes=1, steps=10, labeled=1500,
+                   pool=0, zipf_alpha=1.05, zipf_keys=10_000),
+    "p_eq_c": W("p_eq_c", 8, capacity=64, dim=8, probes=64, steps=20, labeled=100, pool=0,
+                zipf_alpha=1.1, zipf_keys=500),
+    "p40": W("p40", 9, capacity=997, dim=8, probes=40, steps=10, labeled=700, pool=0,
+             zipf_alpha=0.95, zipf_keys=5_000),
+    "tiny_table": W("tiny_table", 10, capacity=8, dim=4, probes=3, steps=30, labeled=40, pool=0,
+                    zipf_alpha=1.1, zipf_keys=60),
+}
+
+
+def test_tiny_workload_bit_exact_every_step():
+    run_pair(inputs.CFG1_TINY)
+
+
+@pytest.mark.parametrize("name", list(SCALED))
+def test_scaled_workloads_bit_exact_every_step(name):
+    run_pair(SCALED[name])
+
+
+@pytest.mark.parametrize("wide", [0, 1, 16])
+def test_insert_rounds_split_does_not_change_results(wide):
+    r = run_pair(SCALED["c4_stress"], wide_rounds=wide)
+    assert max(s["n_rounds"] for s in r.stats) >= 2  # conflicts really happened
+    assert sum(s["n_dropped"] for s in r.stats) > 0
+
+
+def test_repeatable_bytes():
+    w = SCALED["c3_small"].scaled(steps=6)
+    a = run_pair(w)
+    b = run_pair(w)
+    for x, y in zip(a.tbl.state(), b.tbl.state()):
+        assert torch.equal(x, y)
+
+
+def test_checkpoint_resume_is_bit_identical():
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c2_small"].scaled(steps=12)
+    full = run_pair(w, state_every=0)
+    part = run_pair(w, steps=6, state_every=0)
+    keys, last, M = (x.clone() for x in part.tbl.state())
+    saved_step = binding.mpzch_get_last_step(part.tbl.h)
+    part.tbl.close()
+    tbl2, orc2 = make_pair(w)
+    k2, l2, m2 = tbl2.state()
+    k2.copy_(keys)
+    l2.copy_(last)
+    m2.copy_(M)
+    binding.mpzch_set_last_step(tbl2.h, saved_step)
+    ok, ol, ols = part.orc.state()
+    orc2.set_state(ok, ol, ols)
+    for r in range(w.capacity):
+        orc2.set_row(r, part.orc.row(r))
+    torch.cuda.synchronize()
+    resumed = run_pair(w, steps=6, start=6, tbl=tbl2, orc=orc2, state_every=0)
+    for x, y in zip(full.tbl.state(), resumed.tbl.state()):
+        assert torch.equal(x, y)
+
+
+# ------------------------------------------------------------------ dedup
+@pytest.mark.parametrize("n", [0, 1, 5, 1023, 1024, 1025, 4097, 70_001])
+def test_dedup_matches_oracle(n):
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(1024, 4, 2)
+    rng = np.random.default_rng(n)
+    ids = inputs.zipf_keys(rng, 1.1, 50_000, n)
+    uniq, pos, cnt = tbl.dedup(torch.from_numpy(ids).cuda())
+    ou, op = oracle.dedup(ids)
+    c = int(cnt.item())
+    assert c == ou.size
+    assert_bitwise(uniq[:c].cpu().numpy(), ou, "uniq")
+    assert_bitwise(pos[:c].cpu().numpy().astype(np.int64), op, "pos")
+    # scratch hash is left clean: a second call gives the same answer
+    uniq2, pos2, cnt2 = tbl.dedup(torch.from_numpy(ids).cuda())
+    assert int(cnt2.item()) == c and torch.equal(uniq2[:c], uniq[:c])
+
+
+def test_dedup_all_same_and_all_distinct():
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(1024, 4, 2)
+    for ids in (np.full(5000, 7, np.int64), np.arange(5000, dtype=np.int64)[::-1].copy()):
+        uniq, pos, cnt = tbl.dedup(torch.from_numpy(ids).cuda())
+        ou, op = oracle.dedup(ids)
+        c = int(cnt.item())
+        assert_bitwise(uniq[:c].cpu().numpy(), ou, "uniq")
+        assert_bitwise(pos[:c].cpu().numpy().astype(np.int64), op, "pos")
+
+
+# ------------------------------------------------------------------ export + serving
+def test_select_export_and_serve_match_oracle():
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c3_small"]
+    r = run_pair(w, state_every=5)
+    tbl, orc = r.tbl, r.orc
+    since = w.steps - 10
+    rows_d, cnt_d = tbl.select_written_since(since)
+    orows = orc.select_written_since(since)
+    n = int(cnt_d.item())
+    assert n == orows.size
+    assert_bitwise(rows_d[:n].cpu().numpy(), orows, "select rows")
+    # export consumes the device count directly (no host round trip)
+    q, s, k = tbl.export_int8(rows_d, n=w.capacity, dev_n=cnt_d)
+    oq, os_, ok = orc.export_int8(orows)
+    assert_bitwise(q[:n].cpu().numpy(), oq, "int8 q")
+    assert_bitwise(s[:n].cpu().numpy(), os_, "scale")
+    assert_bitwise(k[:n].cpu().numpy(), ok, "keys")
+    sk, sq, ss = snapshot_from_export(w.capacity, w.dim, orows, oq, os_, ok)
+    cand = inputs.zipf_keys(np.random.default_rng(1), 0.9, w.zipf_keys, 5000)
+    cand[::97] = 10**12 + np.arange(cand[::97].size)  # never-seen ids
+    rc, orow, ohit, oout = oracle.serve_gather(sk, w.capacity, w.probes, sq, ss, w.dim, cand)
+    assert rc == 0
+    dev = tbl.device
+    out = torch.empty((cand.size, w.dim), dtype=torch.float32, device=dev)
+    grow = torch.empty(cand.size, dtype=torch.int32, device=dev)
+    ghit = torch.empty(cand.size, dtype=torch.uint8, device=dev)
+    binding.mpzch_serve_gather(torch.from_numpy(sk).to(dev), w.probes, torch.from_numpy(sq).to(dev),
+                               torch.from_numpy(ss).to(dev), torch.from_numpy(cand).to(dev),
+                               grow, ghit, out)
+    assert_bitwise(grow.cpu().numpy(), orow, "serve rows")
+    assert_bitwise(ghit.cpu().numpy(), ohit, "serve hit")
+    assert_bitwise(out.cpu().numpy(), oout, "serve features")
+    assert 0 < ohit.mean() < 1
+
+
+def test_export_edge_rows():
+    """All-zero rows (scale 0), rows with a single large element, negative absmax."""
+    from hashed_sparse_table_b200 import binding
+    C, D = 64, 16
+    tbl = binding.MpzchTable(C, D, 4)
+    orc = oracle.OracleTable(C, D, 4)
+    _, _, M = tbl.state()
+    rng = np.random.default_rng(3)
+    vals = rng.standard_normal((C, D)).astype(np.float32)
+    vals[0] = 0
+    vals[1] = 0
+    vals[1, 5] = -3e-38
+    vals[2] = np.float32(127.0) * np.arange(-8, 8, dtype=np.float32)
+    vals[3] = np.float32(1e30)
+    vals[4, :] = np.float32(-0.0)
+    M.copy_(torch.from_numpy(vals))
+    for r in range(C):
+        orc.set_row(r, vals[r])
+    rows = np.arange(C, dtype=np.int32)
+    q, s, k = tbl.export_int8(torch.from_numpy(rows).cuda())
+    oq, os_, ok = orc.export_int8(rows)
+    assert_bitwise(q.cpu().numpy(), oq, "q")
+    assert_bitwise(s.cpu().numpy(), os_, "scale")
+
+
+# ------------------------------------------------------------------ error paths and empties
+def test_empty_calls_and_step_order():
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(256, 8, 4)
+    dev = tbl.device
+    empty_i = torch.empty(0, dtype=torch.int64, device=dev)
+    rows, hit = tbl.lookup(empty_i)
+    assert rows.numel() == 0
+    st = torch.full((7,), 99, dtype=torch.int64, device=dev)
+    tbl.writeback(empty_i, torch.empty((0, 8), device=dev), 0, st)
+    assert st.sum().item() == 0
+    with pytest.raises(binding.MpzchError) as ei:
+        tbl.writeback(empty_i, torch.empty((0, 8), device=dev), 0, st)
+    assert ei.value.code == binding.MPZCH_EINVAL
+    ids = torch.tensor([5, 6], dtype=torch.int64, device=dev)
+    tbl.writeback(ids, torch.ones((2, 8), device=dev), 3, st)
+    with pytest.raises(binding.MpzchError):
+        tbl.writeback(ids, torch.ones((2, 8), device=dev), 2, st)
+    # misaligned e
+    big = torch.ones(2 * 8 + 1, device=dev)
+    with pytest.raises(binding.MpzchError):
+        binding.mpzch_writeback(tbl.h, ids, big[1:].view(2, 8), 9, st)
+    assert tbl.status() == 0
+
+
+def test_bad_ids_set_status_and_are_skipped():
+    w = inputs.Workload("bad", 11, capacity=512, dim=8, probes=4, steps=3, labeled=300, pool=0,
+                        zipf_alpha=1.1, zipf_keys=2000)
+
+    def ids_fn(t):
+        ids = inputs.step_ids(w, t)
+        ids[::37] = -7
+        return ids
+    tbl, orc = make_pair(w)
+    dev = tbl.device
+    for t in range(3):
+        ids = ids_fn(t)
+        e = inputs.step_e(w, t)
+        ids_d = torch.from_numpy(ids).to(dev)
+        rows, hit = tbl.lookup(ids_d)
+        st = torch.zeros(7, dtype=torch.int64, device=dev)
+        tbl.writeback(ids_d, torch.from_numpy(e).to(dev), t, st)
+        rc, orows, ohit = orc.lookup(ids)
+        rc2, ost = orc.writeback(ids, e, t)
+        assert rc == oracle.ORC_EBADKEY and rc2 == oracle.ORC_EBADKEY
+        assert_bitwise(rows.cpu().numpy(), orows, "rows")
+        assert st[0].item() == ost["n_ids"] and st[1].item() == ost["n_unique"]
+        assert tbl.status() & 1
+    compare_state(tbl, orc, "after bad ids")
+    assert tbl.status() == 0  # cleared by the read
+
+
+def test_gather_bad_rows_set_status_and_give_zeros():
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(128, 8, 4)
+    dev = tbl.device
+    rows = torch.tensor([0, 500, -3, 7], dtype=torch.int32, device=dev)
+    hit = torch.tensor([1, 1, 1, 0], dtype=torch.uint8, device=dev)
+    ao = torch.arange(16 * 4, dtype=torch.float32, device=dev).view(16, 4)
+    aor = torch.tensor([1, 2, 99, 3], dtype=torch.int32, device=dev)
+    out = tbl.gather_fused(rows, hit, ao, aor)
+    st = tbl.status()
+    assert st & binding.MPZCH_STATUS_BADROW and st & binding.MPZCH_STATUS_BADAO
+    o = out.cpu().numpy()
+    assert (o[1:3, :8] == 0).all() and (o[2, 8:] == 0).all()
+    assert (o[0, 8:] == np.arange(4, 8)).all()
+    with pytest.raises(binding.MpzchError):  # ao_dim not a multiple of 4
+        tbl.gather_fused(rows, hit, torch.zeros((4, 6), device=dev), aor)
+
+
+def test_launch_counter_and_trace():
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c2_small"].scaled(steps=3)
+    tbl, orc = make_pair(w)
+    binding.mpzch_trace_enable(tbl.h, True)
+    before = binding.mpzch_launch_count()
+    run_pair(w, tbl=tbl, orc=orc, state_every=0)
+    tr = binding.mpzch_trace_read(tbl.h)
+    assert binding.mpzch_launch_count() > before
+    for ph in ("lookup", "gather", "dedup", "insert", "writeback"):
+        ms, launches = tr[ph]
+        assert launches > 0 and ms > 0, (ph, tr[ph])
