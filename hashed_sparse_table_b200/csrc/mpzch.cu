@@ -8,6 +8,7 @@
 #include <atomic>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -259,7 +260,96 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch of mpzch_dedup_static: a fixed static device array, so that call
+// never allocates.  Layout (256-byte aligned sections), for at most
+// MPZCH_DEDUP_STATIC_MAX_IDS ids:
+//   hash keys   8 B x kStaticHash   (all ones = empty)
+//   hash pos    4 B x kStaticHash   (all ones = none)
+//   slot_of     4 B x max ids
+//   tile counts 4 B x (max ids / kTile + 1)
+//   StepCtr     (cleared by k_dedup_insert)
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int64_t kStaticMaxIds = MPZCH_DEDUP_STATIC_MAX_IDS;
+constexpr uint64_t kStaticHash = 2 * (uint64_t)kStaticMaxIds;  // a power of two
+static_assert((kStaticHash & (kStaticHash - 1)) == 0, "static hash size must be a power of two");
+constexpr size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+constexpr size_t kOffHkey = 0;
+constexpr size_t kOffHpos = align256(kOffHkey + 8 * kStaticHash);
+constexpr size_t kOffSlot = align256(kOffHpos + 4 * kStaticHash);
+constexpr size_t kOffBcnt = align256(kOffSlot + 4 * (size_t)kStaticMaxIds);
+constexpr size_t kOffCtr = align256(kOffBcnt + 4 * (size_t)(kStaticMaxIds / kTile + 1));
+constexpr size_t kStaticBytes = align256(kOffCtr + sizeof(StepCtr));
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_dedup_scratch[kStaticBytes];
+
+namespace {
+std::mutex g_static_mu;
+constexpr int kMaxDevices = 64;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_dedup_scratch on the current device, looked up once per
+// device.  (In host code the array's name is only a host-side stand-in.)
+int static_scratch(unsigned char** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MPZCH_ECUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dedup_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return MPZCH_ECUDA;
+    }
+    g_static_addr[dev] = p;
+  }
+  *out = static_cast<unsigned char*>(g_static_addr[dev]);
+  return MPZCH_OK;
+}
+}  // namespace
+
 extern "C" {
+
+int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
+                       int64_t* dev_count, int32_t* dev_status, void* stream) {
+  if (n < 0 || !dev_count) return MPZCH_EINVAL;
+  if (n > kStaticMaxIds) return MPZCH_ERANGE;
+  if (n > 0 && (!ids || !uniq || !pos)) return MPZCH_EINVAL;
+  unsigned char* base = nullptr;
+  int rc = static_scratch(&base);
+  if (rc) return rc;
+  cudaStream_t st = S(stream);
+  if (n == 0)
+    return cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess ? MPZCH_OK
+                                                                              : MPZCH_ECUDA;
+  unsigned long long* hkey = reinterpret_cast<unsigned long long*>(base + kOffHkey);
+  uint32_t* hpos = reinterpret_cast<uint32_t*>(base + kOffHpos);
+  int32_t* slot_of = reinterpret_cast<int32_t*>(base + kOffSlot);
+  int32_t* bcount = reinterpret_cast<int32_t*>(base + kOffBcnt);
+  StepCtr* ctr = reinterpret_cast<StepCtr*>(base + kOffCtr);
+  // Hash of 2^k >= 2n slots; clear only that part (the rest is not read).
+  uint64_t H = pow2_at_least((uint64_t)n * 2);
+  if (H < 1024) H = 1024;
+  if (cudaMemsetAsync(hkey, 0xFF, H * sizeof(unsigned long long), st) != cudaSuccess ||
+      cudaMemsetAsync(hpos, 0xFF, H * sizeof(uint32_t), st) != cudaSuccess)
+    return MPZCH_ECUDA;
+  const long long* id = reinterpret_cast<const long long*>(ids);
+  const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
+  k_dedup_insert<<<grid_for(n, kBlock), kBlock, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr,
+                                                         nullptr, dev_status);
+  if (after_launch()) return MPZCH_ECUDA;
+  k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
+  if (after_launch()) return MPZCH_ECUDA;
+  k_dedup_compact<<<tiles, kBlock, 0, st>>>(
+      id, n, slot_of, hkey, hpos, bcount, reinterpret_cast<long long*>(uniq), pos,
+      reinterpret_cast<long long*>(dev_count), nullptr, nullptr, Geo{}, 0, nullptr, nullptr,
+      nullptr, ctr, nullptr);
+  return after_launch();
+}
 
 int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mpzch_table** out) {
   if (!out) return MPZCH_EINVAL;

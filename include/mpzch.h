@@ -58,6 +58,7 @@ extern "C" {
 #define MPZCH_ENOMEM (-2)  /* device allocation failed */
 #define MPZCH_ECUDA (-3)   /* a CUDA runtime call or launch failed */
 #define MPZCH_ECAPTURE (-5) /* would allocate while the stream is being captured */
+#define MPZCH_ERANGE (-6)  /* batch larger than a fixed maximum (mpzch_dedup_static) */
 
 /* Sticky device status bits (mpzch_get_status). */
 #define MPZCH_STATUS_BADKEY 1   /* a negative item id was given */
@@ -126,6 +127,35 @@ MPZCH_API int mpzch_gather_fused(mpzch_table* t, const int32_t* rows, const uint
  * Negative ids are skipped (MPZCH_STATUS_BADKEY).  Uses the table's scratch. */
 MPZCH_API int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
                 int64_t* dev_count, void* stream);
+
+/* Dedup that allocates no device memory.  The pages have no counterpart to
+ * this call; it is a variant of mpzch_dedup for callers that cannot call
+ * cudaMalloc -- for example a plug-in running inside an inference server or
+ * another framework that owns all device memory through its own pool (a raw
+ * cudaMalloc there can fail once the pool has reserved the device, and it
+ * bypasses the host's memory accounting), or a latency-critical path where a
+ * cudaMalloc/cudaFree would synchronise the device.  Such a caller cannot
+ * create a table handle either, so this call needs none.
+ *
+ * Output and argument meaning are those of mpzch_dedup: ids device int64[n];
+ * uniq device int64[n] and pos device int32[n] receive the distinct ids and
+ * the index of their first occurrence, in first-occurrence order; dev_count
+ * (device int64) receives their number.  dev_status: nullable device int32,
+ * OR-ed with MPZCH_STATUS_BADKEY when a negative id is skipped.
+ *
+ * Scratch: one fixed static device array of this library, about 7 MiB, which
+ * every GPU that loads the library holds until the process exits.  n must be
+ * at most MPZCH_DEDUP_STATIC_MAX_IDS; larger n returns MPZCH_ERANGE and
+ * launches nothing.  The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress) with that device current; make that first
+ * call before any stream capture.  Every call uses the same array and each
+ * call clears the part of it that must start empty, so the contents left by
+ * the previous call do not matter -- but calls that can overlap on the GPU
+ * (different streams, or several host threads) race with each other and give
+ * wrong results: order them on one stream. */
+#define MPZCH_DEDUP_STATIC_MAX_IDS 262144
+MPZCH_API int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
+                                 int64_t* dev_count, int32_t* dev_status, void* stream);
 
 /* One training step of the table (Memory Layer section 2, MPZCH and Writeback
  * paragraphs).  ids: device int64[n]; e: device fp32 [n][dim], the item-tower
