@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e-pool", type=int, default=inputs.E_POOL,
+                    help="distinct item-tower target batches cycled through (memory bound for "
+                         "profiling runs)")
     return ap.parse_args()
 
 
@@ -213,7 +216,8 @@ def run_ours(args):
     host = [host_step(t, rank) for t in range(total)]
     ids_d = [torch.from_numpy(h[0]).to(dev) for h in host]
     aor_d = [torch.from_numpy(h[1]).to(dev) for h in host]
-    e_host = [torch.from_numpy(inputs.step_e(W, t)) for t in range(inputs.E_POOL)]
+    E = max(1, min(args.e_pool, inputs.E_POOL))
+    e_host = [torch.from_numpy(inputs.step_e(W, t)) for t in range(E)]
     e_d = [x.to(dev) for x in e_host]
     ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
     lab = W.labeled
@@ -228,7 +232,7 @@ def run_ours(args):
     def step(t):
         binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])
         binding.mpzch_gather_fused(tbl.h, rows, hits[t], out, ao_d, aor_d[t])
-        binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % inputs.E_POOL], t, stats[t])
+        binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % E], t, stats[t])
 
     for t in range(Pf):
         step(t)
@@ -286,7 +290,7 @@ def run_ours(args):
     # end to end: host inputs (pinned) -> device -> step -> counters back to host
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host)
+        e2e = run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E)
 
     result = None
     if rank == 0:
@@ -313,6 +317,8 @@ def run_ours(args):
             "gather_writeback_frac_of_8tbs": gw_gbs / 8000.0,
             "phase_ms_per_step": {k: v[0] / K for k, v in trace.items() if v[1]},
             "unique_rows_per_step": n_unique / K,
+            "inserted_per_step": float(st[:, 3].sum()) / K,
+            "insert_rounds_per_step": float(st[:, 6].sum()) / K,
             "hit_rate_labeled": n_hit_lab / (K * lab),
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -326,7 +332,7 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host):
+def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
     """Same steps (continuing the stream) with host inputs copied in every step."""
     import torch.distributed as dist
     lab = W.labeled
@@ -354,7 +360,7 @@ def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host):
         t = n0 + j
         ids_d.copy_(ids_h[j], non_blocking=True)
         aor_d.copy_(aor_h[j], non_blocking=True)
-        e_d.copy_(e_h[t % inputs.E_POOL], non_blocking=True)
+        e_d.copy_(e_h[t % E], non_blocking=True)
         binding.mpzch_lookup(tbl.h, ids_d[:lab], rows, hit)
         binding.mpzch_gather_fused(tbl.h, rows, hit, out, ao_d, aor_d)
         binding.mpzch_writeback(tbl.h, ids_d, e_d, t, st_d)

@@ -106,7 +106,8 @@ struct mpzch_table {
   long long* ukey = nullptr;
   int32_t* upos = nullptr;
   int32_t* urow = nullptr;
-  int32_t* lists[3] = {nullptr, nullptr, nullptr};
+  long long* lkey[3] = {nullptr, nullptr, nullptr};  // insert round lists: keys
+  int32_t* lidx[3] = {nullptr, nullptr, nullptr};    // and their distinct-id index
   // small device words
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
@@ -137,7 +138,8 @@ void free_batch_scratch(mpzch_table* t) {
   dev_free(t->ukey);
   dev_free(t->upos);
   dev_free(t->urow);
-  for (auto& l : t->lists) dev_free(l), l = nullptr;
+  for (auto& l : t->lkey) dev_free(l), l = nullptr;
+  for (auto& l : t->lidx) dev_free(l), l = nullptr;
   t->hkey = nullptr;
   t->hpos = nullptr;
   t->slot_of = t->bcount = t->upos = t->urow = nullptr;
@@ -184,7 +186,8 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
   if (!rc) rc = dev_alloc((void**)&t->upos, cap * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->urow, cap * sizeof(int32_t));
-  for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lists[i], cap * sizeof(int32_t));
+  for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lkey[i], cap * sizeof(long long));
+  for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lidx[i], cap * sizeof(int32_t));
   if (rc) {
     free_batch_scratch(t);
     return rc;
@@ -240,10 +243,9 @@ struct PhaseScope {
   }
 };
 
-// The three dedup phases; with `wb` the compaction also re-probes the table,
-// refreshes resident rows and opens insert round 0.
+// The three dedup phases.
 int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, int32_t* pos,
-              long long* dev_count, bool wb, int64_t step, WbStats* stats, cudaStream_t st) {
+              long long* dev_count, WbStats* stats, cudaStream_t st) {
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<grid_for(n, kBlock), kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask,
@@ -251,10 +253,8 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
-  k_dedup_compact<<<tiles, kBlock, 0, st>>>(
-      id, n, t->slot_of, t->hkey, t->hpos, t->bcount, uniq, pos, dev_count,
-      wb ? t->keys : nullptr, t->last, t->geo, (long long)step, t->urow, t->lists[0],
-      t->claims[0], t->ctr, stats);
+  k_dedup_compact<<<tiles, kBlock, 0, st>>>(id, n, t->slot_of, t->hkey, t->hpos, t->bcount, uniq,
+                                            pos, dev_count, stats);
   return after_launch();
 }
 
@@ -344,10 +344,9 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
-  k_dedup_compact<<<tiles, kBlock, 0, st>>>(
-      id, n, slot_of, hkey, hpos, bcount, reinterpret_cast<long long*>(uniq), pos,
-      reinterpret_cast<long long*>(dev_count), nullptr, nullptr, Geo{}, 0, nullptr, nullptr,
-      nullptr, ctr, nullptr);
+  k_dedup_compact<<<tiles, kBlock, 0, st>>>(id, n, slot_of, hkey, hpos, bcount,
+                                            reinterpret_cast<long long*>(uniq), pos,
+                                            reinterpret_cast<long long*>(dev_count), nullptr);
   return after_launch();
 }
 
@@ -461,7 +460,7 @@ int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, in
   if (rc) return rc;
   PhaseScope ps(t, PH_DEDUP, st);
   return run_dedup(t, ids, n, reinterpret_cast<long long*>(uniq), pos,
-                   reinterpret_cast<long long*>(dev_count), false, 0, nullptr, st);
+                   reinterpret_cast<long long*>(dev_count), nullptr, st);
 }
 
 int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
@@ -482,8 +481,12 @@ int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t 
   if (rc) return rc;
   {
     PhaseScope ps(t, PH_DEDUP, st);
-    rc = run_dedup(t, ids, n, t->ukey, t->upos, nullptr, true, step, stats, st);
+    rc = run_dedup(t, ids, n, t->ukey, t->upos, nullptr, stats, st);
     if (rc) return rc;
+    k_reprobe<<<grid_for(n, kBlock), kBlock, 0, st>>>(t->ukey, &stats->n_unique, t->keys, t->last,
+                                                      t->geo, (long long)step, t->urow, t->lkey[0],
+                                                      t->lidx[0], t->claims[0], t->ctr, stats);
+    if (after_launch()) return MPZCH_ECUDA;
   }
   {
     PhaseScope ps(t, PH_INSERT, st);
@@ -491,15 +494,19 @@ int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t 
     const int R = t->wide_rounds;
     for (int r = 0; r < R; ++r) {
       k_insert_round<<<grid, kBlock, 0, st>>>(
-          r, t->ukey, t->keys, t->last, t->geo, (long long)step, t->urow, t->lists[(r + 2) % 3],
-          t->lists[r % 3], t->lists[(r + 1) % 3], t->claims[(r + 2) % 3], t->claims[r % 3],
-          t->claims[(r + 1) % 3], t->ctr, stats);
+          r, t->keys, t->last, t->geo, (long long)step, t->urow, t->lkey[(r + 2) % 3],
+          t->lkey[r % 3], t->lidx[r % 3], t->lkey[(r + 1) % 3], t->lidx[(r + 1) % 3],
+          t->claims[(r + 2) % 3], t->claims[r % 3], t->claims[(r + 1) % 3], t->ctr, stats);
       if (after_launch()) return MPZCH_ECUDA;
     }
-    k_insert_finish<<<1, 1024, 0, st>>>(R, t->ukey, t->keys, t->last, t->geo, (long long)step,
-                                        t->urow, t->lists[0], t->lists[1], t->lists[2],
-                                        t->claims[0], t->claims[1], t->claims[2], t->ctr, stats,
-                                        t->status);
+    Lists lists;
+    for (int i = 0; i < 3; ++i) {
+      lists.key[i] = t->lkey[i];
+      lists.idx[i] = t->lidx[i];
+    }
+    k_insert_finish<<<1, 1024, 0, st>>>(R, t->keys, t->last, t->geo, (long long)step, t->urow,
+                                        lists, t->claims[0], t->claims[1], t->claims[2], t->ctr,
+                                        stats, t->status);
     if (after_launch()) return MPZCH_ECUDA;
   }
   {

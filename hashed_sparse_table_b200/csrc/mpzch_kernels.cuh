@@ -6,10 +6,13 @@
 // requests at D = 512).  Every loop has a static bound; no kernel waits on a
 // flag written by another block, and no kernel traps.
 #pragma once
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace mpzch {
+
+namespace cg = cooperative_groups;
 
 constexpr unsigned long long kEmptyKey = 0xFFFFFFFFFFFFFFFFull;  // key -1
 constexpr unsigned long long kNoClaim = 0xFFFFFFFFFFFFFFFFull;   // larger than any key
@@ -76,13 +79,19 @@ __device__ __forceinline__ void set_status(int32_t* st, int bits) {
 }
 
 // Row of `k` by one thread scanning the whole window (first match in probe
-// order; the identity map holds at most one).  -1 if absent.
+// order; the identity map holds at most one).  -1 if absent.  Loads of 8
+// slots are issued together.
 __device__ __forceinline__ int64_t find_row_thread(const long long* __restrict__ keys, int64_t k,
                                                    int64_t h, const Geo& g) {
   int64_t found = -1;
-  for (int32_t j = 0; j < g.P; ++j) {
-    const int64_t s = wslot(h, j, g);
-    if (found < 0 && ld_cg(keys + s) == k) found = s;
+  for (int32_t j0 = 0; j0 < g.P; j0 += 8) {
+    long long v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      v[q] = (j0 + q < g.P) ? ld_cg(keys + wslot(h, j0 + q, g)) : -2;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (found < 0 && v[q] == k) found = wslot(h, j0 + q, g);
   }
   return found;
 }
@@ -296,20 +305,14 @@ __global__ void __launch_bounds__(kBlock) k_dedup_count(const int32_t* __restric
   if (threadIdx.x == 0) bcount[blockIdx.x] = (int32_t)t;
 }
 
-// Dedup, phase 3: ordered compaction of first occurrences into (uniq, pos), and
-// reset of the scratch hash slots for the next call.  With `keys` non-null
-// (Writeback) each distinct id is also re-probed in the table: a resident id
-// refreshes last[row] = step; a missing id joins insert round 0 and claims its
-// window in claims0.
+// Dedup, phase 3: ordered compaction of first occurrences into (uniq, pos),
+// and reset of the scratch hash slots for the next call.  The last block
+// writes the number of distinct ids.
 __global__ void __launch_bounds__(kBlock) k_dedup_compact(
     const long long* __restrict__ ids, int64_t n, const int32_t* __restrict__ slot_of,
     unsigned long long* __restrict__ hkey, uint32_t* __restrict__ hpos,
     const int32_t* __restrict__ bcount, long long* __restrict__ ukey, int32_t* __restrict__ upos,
-    long long* dev_count,
-    // Writeback extras (keys == nullptr for plain dedup)
-    const long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
-    int32_t* __restrict__ urow, int32_t* __restrict__ list0, unsigned long long* __restrict__ claims0,
-    StepCtr* ctr, WbStats* stats) {
+    long long* dev_count, WbStats* stats) {
   __shared__ long long sm[33];
   __shared__ int smi[33];
   const long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
@@ -329,45 +332,81 @@ __global__ void __launch_bounds__(kBlock) k_dedup_compact(
   }
   int total = 0;
   int rank = block_excl_scan(c, smi, total);
-  int hits = 0;
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     if (!(flags & (1 << u))) continue;
     const int64_t i = base + u;
     const int64_t uidx = offset + rank++;
-    const long long k = ids[i];
     const int32_t s = slot_of[i];
-    ukey[uidx] = k;
+    ukey[uidx] = ids[i];
     upos[uidx] = (int32_t)i;
     hkey[s] = kEmptyKey;  // only this thread owns slot s now
     hpos[s] = kNoPos;
-    if (keys) {
-      const int64_t h = home_slot(k, g);
-      const int64_t r = find_row_thread(keys, k, h, g);
-      if (r >= 0) {
-        urow[uidx] = (int32_t)r;
-        last[r] = step;
-        ++hits;
-      } else {
-        urow[uidx] = -1;
-        const int m = atomicAdd(&ctr->nlist[0], 1);
-        list0[m] = (int32_t)uidx;
-        for (int32_t j = 0; j < g.P; ++j) atomicMin(claims0 + wslot(h, j, g), (unsigned long long)k);
-      }
-    }
   }
   if (stats) {
-    const long long bh = block_sum_ll(hits, sm);
     const long long bv = block_sum_ll(nvalid, sm);
-    if (threadIdx.x == 0) {
-      if (bh) atomic_add_ll(&stats->n_hit_unique, bh);
-      if (bv) atomic_add_ll(&stats->n_ids, bv);
-    }
+    if (threadIdx.x == 0 && bv) atomic_add_ll(&stats->n_ids, bv);
   }
   if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
     const long long U = offset + total;
     if (dev_count) *dev_count = U;
     if (stats) stats->n_unique = U;
+  }
+}
+
+// Slot index of list entry m among the lanes of this warp that append together;
+// one atomic per warp instead of one per lane.
+__device__ __forceinline__ int warp_append(int32_t* counter) {
+  auto grp = cg::coalesced_threads();
+  int base = 0;
+  if (grp.thread_rank() == 0) base = atomicAdd(counter, (int)grp.size());
+  return grp.shfl(base, 0) + (int)grp.thread_rank();
+}
+
+__device__ __forceinline__ void claim_window(unsigned long long* claims, long long k, const Geo& g) {
+  const int64_t h = home_slot(k, g);
+  for (int32_t j = 0; j < g.P; ++j) atomicMin(claims + wslot(h, j, g), (unsigned long long)k);
+}
+
+__device__ __forceinline__ void clear_window(unsigned long long* claims, long long k, const Geo& g) {
+  const int64_t h = home_slot(k, g);
+  for (int32_t j = 0; j < g.P; ++j) claims[wslot(h, j, g)] = kNoClaim;
+}
+
+// Writeback, step 2: every distinct id is probed in the table (all window loads
+// issued together).  A resident id refreshes last[row] = step; a missing id
+// enters insert round 0 (list 0) and claims its window in claims0.
+__global__ void __launch_bounds__(kBlock) k_reprobe(
+    const long long* __restrict__ ukey, const long long* U_ptr, const long long* __restrict__ keys,
+    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
+    long long* __restrict__ lkey0, int32_t* __restrict__ lidx0, unsigned long long* claims0,
+    StepCtr* ctr, WbStats* stats) {
+  __shared__ long long sm[33];
+  const long long U = *U_ptr;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t first = (int64_t)blockIdx.x * blockDim.x;
+  long long hits = 0;
+  for (int64_t base = first; base < U; base += stride) {
+    const int64_t u = base + threadIdx.x;
+    if (u >= U) continue;
+    const long long k = ukey[u];
+    const int64_t h = home_slot(k, g);
+    const int64_t r = find_row_thread(keys, k, h, g);
+    if (r >= 0) {
+      urow[u] = (int32_t)r;
+      last[r] = step;
+      ++hits;
+    } else {
+      urow[u] = -1;
+      const int m = warp_append(&ctr->nlist[0]);
+      lkey0[m] = k;
+      lidx0[m] = (int32_t)u;
+      claim_window(claims0, k, g);
+    }
+  }
+  if (first < U) {
+    const long long bh = block_sum_ll(hits, sm);
+    if (threadIdx.x == 0 && bh && stats) atomic_add_ll(&stats->n_hit_unique, bh);
   }
 }
 
@@ -388,51 +427,58 @@ __global__ void __launch_bounds__(kBlock) k_dedup_compact(
 //
 // Round r checks claims[r % 3], makes round-(r+1) claims in claims[(r+1) % 3]
 // and clears round-(r-1) claims in claims[(r-1) % 3]: the three uses never
-// touch the same array inside one launch.
+// touch the same array inside one launch.  Lists hold (key, distinct-id index)
+// pairs and rotate the same way.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool try_commit(int64_t uidx, const long long* __restrict__ ukey,
+__device__ __forceinline__ bool try_commit(long long k, int32_t uidx,
                                            const unsigned long long* claims,
                                            long long* __restrict__ keys,
                                            long long* __restrict__ last, const Geo& g,
                                            long long step, int32_t* __restrict__ urow,
                                            long long& evicted) {
-  const long long k = ukey[uidx];
   const int64_t h = home_slot(k, g);
-  for (int32_t j = 0; j < g.P; ++j)
-    if (ld_cg(claims + wslot(h, j, g)) != (unsigned long long)k) return false;
   int64_t best = -1;
   long long best_last = 0;
-  for (int32_t j = 0; j < g.P; ++j) {
-    const int64_t s = wslot(h, j, g);
-    const long long l = ld_cg(last + s);
-    if (best < 0 || l < best_last || (l == best_last && s < best)) {
-      best = s;
-      best_last = l;
+  for (int32_t j0 = 0; j0 < g.P; j0 += 8) {
+    // claims and last-write steps of 8 window slots, all requests in flight together
+    unsigned long long c[8];
+    long long l[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const bool in = j0 + q < g.P;
+      const int64_t s = wslot(h, in ? j0 + q : 0, g);
+      c[q] = in ? ld_cg(claims + s) : (unsigned long long)k;
+      l[q] = in ? ld_cg(last + s) : 0;
+    }
+    bool mine = true;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) mine &= c[q] == (unsigned long long)k;
+    if (!mine) return false;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (j0 + q >= g.P) continue;
+      const int64_t s = wslot(h, j0 + q, g);
+      if (best < 0 || l[q] < best_last || (l[q] == best_last && s < best)) {
+        best = s;
+        best_last = l[q];
+      }
     }
   }
-  if (ld_cg(keys + best) != -1) ++evicted;
+  // A row is empty exactly when its last-write step is -1 (key and step are
+  // always set together), so a victim with a step is a live key.
+  if (best_last != -1) ++evicted;
   keys[best] = k;
   last[best] = step;
   urow[uidx] = (int32_t)best;
   return true;
 }
 
-__device__ __forceinline__ void claim_window(unsigned long long* claims, long long k, const Geo& g) {
-  const int64_t h = home_slot(k, g);
-  for (int32_t j = 0; j < g.P; ++j) atomicMin(claims + wslot(h, j, g), (unsigned long long)k);
-}
-
-__device__ __forceinline__ void clear_window(unsigned long long* claims, long long k, const Geo& g) {
-  const int64_t h = home_slot(k, g);
-  for (int32_t j = 0; j < g.P; ++j) claims[wslot(h, j, g)] = kNoClaim;
-}
-
 __global__ void __launch_bounds__(kBlock) k_insert_round(
-    int r, const long long* __restrict__ ukey, long long* __restrict__ keys,
-    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
-    int32_t* list_prev, int32_t* list_cur, int32_t* list_next, unsigned long long* claims_prev,
-    unsigned long long* claims_cur, unsigned long long* claims_next, StepCtr* ctr,
-    WbStats* stats) {
+    int r, long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
+    int32_t* __restrict__ urow, const long long* lkey_prev, const long long* lkey_cur,
+    const int32_t* lidx_cur, long long* lkey_next, int32_t* lidx_next,
+    unsigned long long* claims_prev, unsigned long long* claims_cur,
+    unsigned long long* claims_next, StepCtr* ctr, WbStats* stats) {
   __shared__ long long sm[33];
   const int32_t nprev = r > 0 ? ctr->nlist[r - 1] : 0;
   const int32_t ncur = ctr->nlist[r];
@@ -440,16 +486,17 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(
   long long evicted = 0;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t first = (int64_t)blockIdx.x * blockDim.x;
-  // Whole blocks iterate together (block_sum below needs every thread).
   for (int64_t base = first; base < nmax; base += stride) {
     const int64_t i = base + threadIdx.x;
-    if (i < nprev) clear_window(claims_prev, ukey[list_prev[i]], g);
+    if (i < nprev) clear_window(claims_prev, lkey_prev[i], g);
     if (i < ncur) {
-      const int32_t u = list_cur[i];
-      if (!try_commit(u, ukey, claims_cur, keys, last, g, step, urow, evicted)) {
-        const int m = atomicAdd(&ctr->nlist[r + 1], 1);
-        list_next[m] = u;
-        claim_window(claims_next, ukey[u], g);
+      const long long k = lkey_cur[i];
+      const int32_t u = lidx_cur[i];
+      if (!try_commit(k, u, claims_cur, keys, last, g, step, urow, evicted)) {
+        const int m = warp_append(&ctr->nlist[r + 1]);
+        lkey_next[m] = k;
+        lidx_next[m] = u;
+        claim_window(claims_next, k, g);
       }
     }
   }
@@ -460,17 +507,20 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(
   if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0 && stats) atomic_add_ll(&stats->n_rounds, 1LL);
 }
 
+struct Lists {
+  long long* key[3];
+  int32_t* idx[3];
+};
+
 // Remaining rounds in one block (block barriers only).  Lists and claims
-// rotate exactly as in k_insert_round; the list buffers come from the caller.
+// rotate exactly as in k_insert_round.
 __global__ void __launch_bounds__(1024) k_insert_finish(
-    int r0, const long long* __restrict__ ukey, long long* __restrict__ keys,
-    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
-    int32_t* lists0, int32_t* lists1, int32_t* lists2, unsigned long long* claims0,
+    int r0, long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
+    int32_t* __restrict__ urow, Lists lists, unsigned long long* claims0,
     unsigned long long* claims1, unsigned long long* claims2, StepCtr* ctr, WbStats* stats,
     int32_t* status) {
   __shared__ int32_t s_cnt[2];  // next-list counters, alternating by iteration parity
   __shared__ long long sm[33];
-  int32_t* lists[3] = {lists0, lists1, lists2};
   unsigned long long* claims[3] = {claims0, claims1, claims2};
   int32_t nprev = r0 > 0 ? ctr->nlist[r0 - 1] : 0;
   int32_t ncur = ctr->nlist[r0];
@@ -484,17 +534,21 @@ __global__ void __launch_bounds__(1024) k_insert_finish(
     if (threadIdx.x == 0) *s_next = 0;
     __syncthreads();
     const int32_t nmax = nprev > ncur ? nprev : ncur;
-    int32_t* lp = lists[(r + 2) % 3];
-    int32_t* lc = lists[r % 3];
-    int32_t* ln = lists[(r + 1) % 3];
+    const long long* kp = lists.key[(r + 2) % 3];
+    const long long* kc = lists.key[r % 3];
+    const int32_t* ic = lists.idx[r % 3];
+    long long* kn = lists.key[(r + 1) % 3];
+    int32_t* in_ = lists.idx[(r + 1) % 3];
     for (int32_t i = threadIdx.x; i < nmax; i += blockDim.x) {
-      if (i < nprev) clear_window(claims[(r + 2) % 3], ukey[lp[i]], g);
+      if (i < nprev) clear_window(claims[(r + 2) % 3], __ldcg(kp + i), g);
       if (i < ncur) {
-        const int32_t u = lc[i];
-        if (!try_commit(u, ukey, claims[r % 3], keys, last, g, step, urow, evicted)) {
+        const long long k = __ldcg(kc + i);
+        const int32_t u = __ldcg(ic + i);
+        if (!try_commit(k, u, claims[r % 3], keys, last, g, step, urow, evicted)) {
           const int m = atomicAdd(s_next, 1);
-          ln[m] = u;
-          claim_window(claims[(r + 1) % 3], ukey[u], g);
+          kn[m] = k;
+          in_[m] = u;
+          claim_window(claims[(r + 1) % 3], k, g);
         }
       }
     }
