@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--wide-rounds", type=int, default=None,
+                    help="grid-wide insert conflict rounds before the single-block finisher")
     ap.add_argument("--e-pool", type=int, default=inputs.E_POOL,
                     help="distinct item-tower target batches cycled through (memory bound for "
                          "profiling runs)")
@@ -228,6 +230,8 @@ def run_ours(args):
 
     tbl = binding.MpzchTable(W.capacity, W.dim, W.probes)
     binding.mpzch_reserve(tbl.h, W.batch)
+    if args.wide_rounds is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, args.wide_rounds)
 
     def step(t):
         binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])

@@ -115,7 +115,7 @@ struct mpzch_table {
   int32_t* sel_bcount = nullptr;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
-  int wide_rounds = 3;
+  int wide_rounds = 4;  // grid-wide insert rounds before the single-block finisher
   // tracing
   bool trace = false;
   struct Rec {
@@ -248,8 +248,8 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
               long long* dev_count, WbStats* stats, cudaStream_t st) {
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
-  k_dedup_insert<<<grid_for(n, kBlock), kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask,
-                                                         t->slot_of, t->ctr, stats, t->status);
+  k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
+                                           stats, t->status);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -339,8 +339,8 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
     return MPZCH_ECUDA;
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
-  k_dedup_insert<<<grid_for(n, kBlock), kBlock, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr,
-                                                         nullptr, dev_status);
+  k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
+                                           dev_status);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -479,41 +479,52 @@ int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t 
   }
   int rc = ensure_batch(t, n, st);
   if (rc) return rc;
+  WbParams p;
+  p.ids = reinterpret_cast<const long long*>(ids);
+  p.n = n;
+  p.e = reinterpret_cast<const float4*>(e);
+  p.D4 = t->D / 4;
+  p.hkey = t->hkey;
+  p.hpos = t->hpos;
+  p.hmask = t->hmask;
+  p.slot_of = t->slot_of;
+  p.ukey = t->ukey;
+  p.upos = t->upos;
+  p.urow = t->urow;
+  p.keys = t->keys;
+  p.last = t->last;
+  p.M = reinterpret_cast<float4*>(t->M);
+  p.g = t->geo;
+  p.step = (long long)step;
+  for (int i = 0; i < 3; ++i) {
+    p.lkey[i] = t->lkey[i];
+    p.lidx[i] = t->lidx[i];
+    p.claims[i] = t->claims[i];
+  }
+  p.ctr = t->ctr;
+  p.stats = stats;
+  p.status = t->status;
   {
     PhaseScope ps(t, PH_DEDUP, st);
-    rc = run_dedup(t, ids, n, t->ukey, t->upos, nullptr, stats, st);
-    if (rc) return rc;
-    k_reprobe<<<grid_for(n, kBlock), kBlock, 0, st>>>(t->ukey, &stats->n_unique, t->keys, t->last,
-                                                      t->geo, (long long)step, t->urow, t->lkey[0],
-                                                      t->lidx[0], t->claims[0], t->ctr, stats);
+    k_dedup_insert<<<(unsigned)((n + kTile - 1) / kTile), kBlock, 0, st>>>(
+        p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, stats, t->status);
+    if (after_launch()) return MPZCH_ECUDA;
+    k_first_reprobe<<<grid_for(n, kBlock), kBlock, 0, st>>>(p);
     if (after_launch()) return MPZCH_ECUDA;
   }
   {
     PhaseScope ps(t, PH_INSERT, st);
     const unsigned grid = grid_for(n, kBlock, 4);
-    const int R = t->wide_rounds;
-    for (int r = 0; r < R; ++r) {
-      k_insert_round<<<grid, kBlock, 0, st>>>(
-          r, t->keys, t->last, t->geo, (long long)step, t->urow, t->lkey[(r + 2) % 3],
-          t->lkey[r % 3], t->lidx[r % 3], t->lkey[(r + 1) % 3], t->lidx[(r + 1) % 3],
-          t->claims[(r + 2) % 3], t->claims[r % 3], t->claims[(r + 1) % 3], t->ctr, stats);
+    for (int r = 0; r < t->wide_rounds; ++r) {
+      k_insert_round<<<grid, kBlock, 0, st>>>(p, r);
       if (after_launch()) return MPZCH_ECUDA;
     }
-    Lists lists;
-    for (int i = 0; i < 3; ++i) {
-      lists.key[i] = t->lkey[i];
-      lists.idx[i] = t->lidx[i];
-    }
-    k_insert_finish<<<1, 1024, 0, st>>>(R, t->keys, t->last, t->geo, (long long)step, t->urow,
-                                        lists, t->claims[0], t->claims[1], t->claims[2], t->ctr,
-                                        stats, t->status);
+    k_insert_finish<<<1, 1024, 0, st>>>(p, t->wide_rounds);
     if (after_launch()) return MPZCH_ECUDA;
   }
   {
     PhaseScope ps(t, PH_WRITEBACK, st);
-    k_writeback<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
-        t->ukey, t->upos, t->urow, &stats->n_unique, t->keys, reinterpret_cast<float4*>(t->M),
-        reinterpret_cast<const float4*>(e), t->D / 4, stats);
+    k_writeback<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(p);
     if (after_launch()) return MPZCH_ECUDA;
   }
   t->last_step = step;
@@ -633,7 +644,7 @@ int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t npha
 int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
   if (!t) return MPZCH_EINVAL;
   if (option == MPZCH_OPT_WIDE_ROUNDS) {
-    if (value < 0 || value > kMaxRounds) return MPZCH_EINVAL;
+    if (value < 0 || value > 64) return MPZCH_EINVAL;
     t->wide_rounds = (int)value;
     return MPZCH_OK;
   }

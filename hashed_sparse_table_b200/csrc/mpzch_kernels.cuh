@@ -20,7 +20,6 @@ constexpr uint32_t kNoPos = 0xFFFFFFFFu;
 constexpr int kBlock = 256;
 constexpr int kTile = 1024;  // ids per block in the ordered compactions (4 per thread)
 constexpr int kSelTile = 4096;  // rows per block in select (16 per thread)
-constexpr int kMaxRounds = 16;
 
 // Status bits (mirror of the MPZCH_STATUS_* values of the public header).
 constexpr int kStBadKey = 1, kStBadRow = 2, kStBadAo = 4, kStInternal = 8;
@@ -32,11 +31,11 @@ struct Geo {
   int32_t P;
 };
 
-// Device counters of one Writeback.
+// Device counters of one Writeback (cleared at the start of each call).
 struct StepCtr {
-  int32_t nlist[kMaxRounds + 2];  // unresolved missing keys entering each insert round
-  uint32_t done_blocks;           // completion ticket of the last kernel's blocks
-  int32_t pad;
+  int32_t cnt[4];    // insert-round list sizes; round r appends to cnt[(r + 1) % 4]
+  int32_t n_unique;  // distinct ids of the batch
+  int32_t pad[3];
 };
 
 // Per-Writeback counters; same layout as mpzch_wb_stats.
@@ -186,56 +185,6 @@ __global__ void __launch_bounds__(kBlock) k_gather_fused(
   }
 }
 
-// ---------------------------------------------------------------------------
-// Dedup, phase 1: insert every id into an open-addressing scratch hash (key,
-// smallest position).  Lanes of a warp holding the same id elect the lowest
-// lane first, so a hot id costs one atomic per warp instead of one per copy.
-// Block 0 also clears the step counters used by the later phases.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kBlock) k_dedup_insert(
-    const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
-    uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status) {
-  if (blockIdx.x == 0 && threadIdx.x < sizeof(StepCtr) / 4)
-    reinterpret_cast<int32_t*>(ctr)[threadIdx.x] = 0;
-  if (stats && blockIdx.x == 0 && threadIdx.x < 7) reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // Whole warps iterate together so that __match_any_sync sees all lanes.
-  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); base < n;
-       base += stride) {
-    const int64_t i = base + (threadIdx.x & 31);
-    const bool valid = i < n;
-    const long long k = valid ? ids[i] : -1;
-    const unsigned active = __ballot_sync(0xFFFFFFFFu, valid);
-    const unsigned same = __match_any_sync(0xFFFFFFFFu, (unsigned long long)k) & active;
-    if (!valid) continue;
-    if (k < 0) {
-      slot_of[i] = -1;
-      set_status(status, kStBadKey);
-      continue;
-    }
-    const int leader = __ffs(same) - 1;
-    int64_t s = (int64_t)(splitmix64((uint64_t)k ^ 0xD6E8FEB86659FD93ull) & hmask);
-    if ((int)(threadIdx.x & 31) == leader) {
-      bool placed = false;
-      for (uint64_t probe = 0; probe <= hmask && !placed; ++probe) {
-        unsigned long long cur = __ldcg(hkey + s);
-        if (cur == kEmptyKey) cur = atomicCAS(hkey + s, kEmptyKey, (unsigned long long)k);
-        if (cur == kEmptyKey || cur == (unsigned long long)k) {
-          if (__ldcg(hpos + s) > (uint32_t)i) atomicMin(hpos + s, (uint32_t)i);
-          placed = true;
-        } else {
-          s = (s + 1) & (int64_t)hmask;
-        }
-      }
-      if (!placed) set_status(status, kStInternal);  // scratch hash sized >= 2n: never expected
-    }
-    // Every copy learns the slot from its leader.
-    s = __shfl_sync(same, s, leader);
-    slot_of[i] = (int32_t)s;
-  }
-}
-
 // Block-wide exclusive scan of one int per thread; returns the block total.
 __device__ __forceinline__ int block_excl_scan(int v, int* smem /* >= 33 ints */, int& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -276,6 +225,117 @@ __device__ __forceinline__ long long block_sum_ll(long long v, long long* smem /
   t = smem[0];
   __syncthreads();
   return t;
+}
+
+// ---------------------------------------------------------------------------
+// Dedup, phase 1: every id goes into an open-addressing scratch hash holding
+// (key, smallest position).  Each block first dedups its tile of kTile
+// positions in shared memory, so a hot id costs one global CAS per tile
+// instead of one per copy; then each distinct id of the tile is inserted once
+// with its smallest tile position, and every position learns its global slot.
+// Block 0 also clears the step counters used by the later phases.
+// ---------------------------------------------------------------------------
+constexpr int kTileHash = 2 * kTile;  // shared-memory slots per tile (load <= 1/2)
+
+__global__ void __launch_bounds__(kBlock) k_dedup_insert(
+    const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
+    uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
+    WbStats* stats, int32_t* status) {
+  __shared__ unsigned long long s_key[kTileHash];
+  __shared__ uint32_t s_pos[kTileHash];
+  __shared__ int32_t s_gslot[kTileHash];
+  __shared__ int16_t s_list[kTile];  // occupied shared slots (at most one per position)
+  __shared__ int s_scan[33];
+  if (blockIdx.x == 0 && threadIdx.x < sizeof(StepCtr) / 4)
+    reinterpret_cast<int32_t*>(ctr)[threadIdx.x] = 0;
+  if (stats && blockIdx.x == 0 && threadIdx.x < 7)
+    reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
+  for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
+    s_key[j] = kEmptyKey;
+    s_pos[j] = kNoPos;
+  }
+  __syncthreads();
+  constexpr int kPer = kTile / kBlock;
+  const int64_t tile = (int64_t)blockIdx.x * kTile;
+  int lslot[kPer];
+  // 1. tile-local dedup (positions strided by the block size: coalesced loads)
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int64_t i = tile + q * kBlock + threadIdx.x;
+    lslot[q] = -1;
+    if (i >= n) continue;
+    const long long k = ids[i];
+    if (k < 0) {
+      slot_of[i] = -1;
+      set_status(status, kStBadKey);
+      continue;
+    }
+    int j = (int)(splitmix64((uint64_t)k ^ 0x5851F42D4C957F2Dull) & (kTileHash - 1));
+    for (int probe = 0; probe < kTileHash; ++probe) {
+      const unsigned long long cur = atomicCAS(&s_key[j], kEmptyKey, (unsigned long long)k);
+      if (cur == kEmptyKey || cur == (unsigned long long)k) {
+        atomicMin(&s_pos[j], (uint32_t)i);
+        lslot[q] = j;
+        break;
+      }
+      j = (j + 1) & (kTileHash - 1);
+    }
+  }
+  __syncthreads();
+  // 2. one global insert per distinct id of the tile: compact the occupied
+  //    shared slots, then every thread issues the first probe of its (at most
+  //    kPer) ids together; a collision falls back to linear probing.
+  {
+    int occ = 0;
+    constexpr int kSlotsPer = kTileHash / kBlock;
+#pragma unroll
+    for (int q = 0; q < kSlotsPer; ++q) occ += s_key[threadIdx.x * kSlotsPer + q] != kEmptyKey;
+    int total = 0;
+    int at = block_excl_scan(occ, s_scan, total);
+#pragma unroll
+    for (int q = 0; q < kSlotsPer; ++q) {
+      const int j = threadIdx.x * kSlotsPer + q;
+      if (s_key[j] != kEmptyKey) s_list[at++] = j;
+    }
+    __syncthreads();
+    unsigned long long kk[kPer], cur[kPer];
+    int64_t ss[kPer];
+    int jj[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int e = threadIdx.x + q * kBlock;
+      jj[q] = e < total ? s_list[e] : -1;
+      kk[q] = jj[q] >= 0 ? s_key[jj[q]] : 0;
+      ss[q] = (int64_t)(splitmix64(kk[q] ^ 0xD6E8FEB86659FD93ull) & hmask);
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) cur[q] = jj[q] >= 0 ? __ldcg(hkey + ss[q]) : 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (jj[q] >= 0 && cur[q] == kEmptyKey) cur[q] = atomicCAS(hkey + ss[q], kEmptyKey, kk[q]);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      if (jj[q] < 0) continue;
+      int64_t sl = ss[q];
+      bool placed = cur[q] == kEmptyKey || cur[q] == kk[q];
+      for (uint64_t probe = 1; probe <= hmask && !placed; ++probe) {
+        sl = (sl + 1) & (int64_t)hmask;
+        unsigned long long c = __ldcg(hkey + sl);
+        if (c == kEmptyKey) c = atomicCAS(hkey + sl, kEmptyKey, kk[q]);
+        placed = c == kEmptyKey || c == kk[q];
+      }
+      if (!placed) set_status(status, kStInternal);  // scratch hash sized >= 2n: never expected
+      atomicMin(hpos + sl, s_pos[jj[q]]);
+      s_gslot[jj[q]] = (int32_t)sl;
+    }
+  }
+  __syncthreads();
+  // 3. every position learns the global slot of its id
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int64_t i = tile + q * kBlock + threadIdx.x;
+    if (i < n && lslot[q] >= 0) slot_of[i] = s_gslot[lslot[q]];
+  }
 }
 
 // Sum of cnt[0 .. upto) by the whole block.
@@ -373,43 +433,6 @@ __device__ __forceinline__ void clear_window(unsigned long long* claims, long lo
   for (int32_t j = 0; j < g.P; ++j) claims[wslot(h, j, g)] = kNoClaim;
 }
 
-// Writeback, step 2: every distinct id is probed in the table (all window loads
-// issued together).  A resident id refreshes last[row] = step; a missing id
-// enters insert round 0 (list 0) and claims its window in claims0.
-__global__ void __launch_bounds__(kBlock) k_reprobe(
-    const long long* __restrict__ ukey, const long long* U_ptr, const long long* __restrict__ keys,
-    long long* __restrict__ last, Geo g, long long step, int32_t* __restrict__ urow,
-    long long* __restrict__ lkey0, int32_t* __restrict__ lidx0, unsigned long long* claims0,
-    StepCtr* ctr, WbStats* stats) {
-  __shared__ long long sm[33];
-  const long long U = *U_ptr;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t first = (int64_t)blockIdx.x * blockDim.x;
-  long long hits = 0;
-  for (int64_t base = first; base < U; base += stride) {
-    const int64_t u = base + threadIdx.x;
-    if (u >= U) continue;
-    const long long k = ukey[u];
-    const int64_t h = home_slot(k, g);
-    const int64_t r = find_row_thread(keys, k, h, g);
-    if (r >= 0) {
-      urow[u] = (int32_t)r;
-      last[r] = step;
-      ++hits;
-    } else {
-      urow[u] = -1;
-      const int m = warp_append(&ctr->nlist[0]);
-      lkey0[m] = k;
-      lidx0[m] = (int32_t)u;
-      claim_window(claims0, k, g);
-    }
-  }
-  if (first < U) {
-    const long long bh = block_sum_ll(hits, sm);
-    if (threadIdx.x == 0 && bh && stats) atomic_add_ll(&stats->n_hit_unique, bh);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Insert of missing keys in conflict rounds.
 //
@@ -426,9 +449,9 @@ __global__ void __launch_bounds__(kBlock) k_reprobe(
 // independently.  The smallest unplaced key always commits, so rounds end.
 //
 // Round r checks claims[r % 3], makes round-(r+1) claims in claims[(r+1) % 3]
-// and clears round-(r-1) claims in claims[(r-1) % 3]: the three uses never
-// touch the same array inside one launch.  Lists hold (key, distinct-id index)
-// pairs and rotate the same way.
+// and clears round-(r-1) claims in claims[(r-1) % 3], so one round never uses
+// an array for two purposes.  The (key, distinct-id index) lists rotate the
+// same way.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool try_commit(long long k, int32_t uidx,
                                            const unsigned long long* claims,
@@ -473,58 +496,165 @@ __device__ __forceinline__ bool try_commit(long long k, int32_t uidx,
   return true;
 }
 
-__global__ void __launch_bounds__(kBlock) k_insert_round(
-    int r, long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
-    int32_t* __restrict__ urow, const long long* lkey_prev, const long long* lkey_cur,
-    const int32_t* lidx_cur, long long* lkey_next, int32_t* lidx_next,
-    unsigned long long* claims_prev, unsigned long long* claims_cur,
-    unsigned long long* claims_next, StepCtr* ctr, WbStats* stats) {
+// Arguments of the Writeback kernels.
+struct WbParams {
+  const long long* ids;
+  int64_t n;
+  const float4* e;
+  int D4;
+  unsigned long long* hkey;
+  uint32_t* hpos;
+  uint64_t hmask;
+  int32_t* slot_of;
+  long long* ukey;
+  int32_t* upos;
+  int32_t* urow;
+  long long* keys;
+  long long* last;
+  float4* M;
+  Geo g;
+  long long step;
+  long long* lkey[3];
+  int32_t* lidx[3];
+  unsigned long long* claims[3];
+  StepCtr* ctr;
+  WbStats* stats;
+  int32_t* status;
+};
+
+// Two per-thread counts packed as 16-bit halves (each <= the block size).
+__device__ __forceinline__ int pack2(int a, int b) { return a | (b << 16); }
+
+// Block-aggregated append: every thread with want != 0 gets a distinct slot of
+// the list whose length counter is `counter`; one global atomic per block.
+// All threads of the block must call it.
+__device__ __forceinline__ void block_append2(int wa, int wb, int32_t* ca, int32_t* cb, int& ia,
+                                              int& ib, int* smi) {
+  int total = 0;
+  const int before = block_excl_scan(pack2(wa, wb), smi, total);
+  __shared__ int s_base[2];
+  if (threadIdx.x == 0) {
+    const int ta = total & 0xFFFF, tb = total >> 16;
+    s_base[0] = ta ? atomicAdd(ca, ta) : 0;
+    s_base[1] = tb ? atomicAdd(cb, tb) : 0;
+  }
+  __syncthreads();
+  ia = s_base[0] + (before & 0xFFFF);
+  ib = s_base[1] + (before >> 16);
+  __syncthreads();
+}
+
+// Writeback, dedup phase 2 + re-probe, one pass over the batch positions: a
+// position whose id's scratch-hash entry holds that position is the id's
+// first occurrence.  Its thread appends the distinct id (key, first position)
+// to the distinct-id list (in block order; the Writeback result does not
+// depend on that order), resets the hash slot for the next call, and probes
+// the table: a resident id refreshes last[row] = step; a missing id enters
+// insert round 0 (list 0) and claims its window in claims[0].
+__global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
   __shared__ long long sm[33];
-  const int32_t nprev = r > 0 ? ctr->nlist[r - 1] : 0;
-  const int32_t ncur = ctr->nlist[r];
-  const int32_t nmax = nprev > ncur ? nprev : ncur;
-  long long evicted = 0;
+  __shared__ int smi[33];
+  const Geo g = p.g;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  const int64_t first = (int64_t)blockIdx.x * blockDim.x;
-  for (int64_t base = first; base < nmax; base += stride) {
+  long long hits = 0, nvalid = 0;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < p.n; base += stride) {
     const int64_t i = base + threadIdx.x;
-    if (i < nprev) clear_window(claims_prev, lkey_prev[i], g);
-    if (i < ncur) {
-      const long long k = lkey_cur[i];
-      const int32_t u = lidx_cur[i];
-      if (!try_commit(k, u, claims_cur, keys, last, g, step, urow, evicted)) {
-        const int m = warp_append(&ctr->nlist[r + 1]);
-        lkey_next[m] = k;
-        lidx_next[m] = u;
-        claim_window(claims_next, k, g);
+    bool first = false;
+    long long k = 0;
+    int64_t h = 0, r = -1;
+    if (i < p.n) {
+      const int32_t s = p.slot_of[i];
+      if (s >= 0) {
+        ++nvalid;
+        if (__ldcg(p.hpos + s) == (uint32_t)i) {
+          first = true;
+          k = p.ids[i];
+          p.hkey[s] = kEmptyKey;  // only this thread owns slot s now
+          p.hpos[s] = kNoPos;
+          h = home_slot(k, g);
+          r = find_row_thread(p.keys, k, h, g);
+        }
+      }
+    }
+    int u = 0, m = 0;
+    block_append2(first, first && r < 0, &p.ctr->n_unique, &p.ctr->cnt[0], u, m, smi);
+    if (first) {
+      p.ukey[u] = k;
+      p.upos[u] = (int32_t)i;
+      p.urow[u] = (int32_t)r;
+      if (r >= 0) {
+        p.last[r] = p.step;
+        ++hits;
+      } else {
+        p.lkey[0][m] = k;
+        p.lidx[0][m] = u;
+        claim_window(p.claims[0], k, g);
       }
     }
   }
-  if (first < nmax) {
-    const long long ev = block_sum_ll(evicted, sm);
-    if (threadIdx.x == 0 && ev && stats) atomic_add_ll(&stats->n_evicted, ev);
+  const long long bh = block_sum_ll(hits, sm);
+  const long long bv = block_sum_ll(nvalid, sm);
+  if (threadIdx.x == 0) {
+    if (bh) atomic_add_ll(&p.stats->n_hit_unique, bh);
+    if (bv) atomic_add_ll(&p.stats->n_ids, bv);
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0 && stats) atomic_add_ll(&stats->n_rounds, 1LL);
 }
 
-struct Lists {
-  long long* key[3];
-  int32_t* idx[3];
-};
+// Grid-wide insert round r (see the insert comment above): clears the claims
+// of round r-1, tries to commit every key of round r, and moves the others to
+// round r+1 (block-aggregated append, claims in claims[(r+1) % 3]).
+__global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
+  __shared__ long long sm[33];
+  __shared__ int smi[33];
+  const Geo g = p.g;
+  const int32_t nprev = r > 0 ? p.ctr->cnt[(r + 3) & 3] : 0;
+  const int32_t ncur = p.ctr->cnt[r & 3];
+  const int32_t nmax = nprev > ncur ? nprev : ncur;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    // counter that round r+1 appends to; its last reader was round r-1
+    p.ctr->cnt[(r + 2) & 3] = 0;
+    if (r == 0) p.stats->n_inserted = ncur;
+  }
+  const int64_t first_i = (int64_t)blockIdx.x * blockDim.x;
+  if (first_i >= nmax) return;  // whole block idle (block-uniform)
+  const int rp = (r + 2) % 3, rc = r % 3, rn = (r + 1) % 3;
+  long long evicted = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = first_i; base < nmax; base += stride) {
+    const int64_t i = base + threadIdx.x;
+    if (i < nprev) clear_window(p.claims[rp], p.lkey[rp][i], g);
+    bool defer = false;
+    long long k = 0;
+    int32_t u = 0;
+    if (i < ncur) {
+      k = p.lkey[rc][i];
+      u = p.lidx[rc][i];
+      defer = !try_commit(k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted);
+    }
+    int m = 0, unused = 0;
+    block_append2(defer, 0, &p.ctr->cnt[(r + 1) & 3], &p.ctr->cnt[(r + 1) & 3], m, unused, smi);
+    if (defer) {
+      p.lkey[rn][m] = k;
+      p.lidx[rn][m] = u;
+      claim_window(p.claims[rn], k, g);
+    }
+  }
+  const long long ev = block_sum_ll(evicted, sm);
+  if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
+}
 
-// Remaining rounds in one block (block barriers only).  Lists and claims
-// rotate exactly as in k_insert_round.
-__global__ void __launch_bounds__(1024) k_insert_finish(
-    int r0, long long* __restrict__ keys, long long* __restrict__ last, Geo g, long long step,
-    int32_t* __restrict__ urow, Lists lists, unsigned long long* claims0,
-    unsigned long long* claims1, unsigned long long* claims2, StepCtr* ctr, WbStats* stats,
-    int32_t* status) {
+// The rounds left after the grid-wide ones, in one block (block barriers only);
+// lists, claims and counters rotate exactly as in k_insert_round.  Also writes
+// the final counters of the row map.
+__global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
   __shared__ int32_t s_cnt[2];  // next-list counters, alternating by iteration parity
   __shared__ long long sm[33];
-  unsigned long long* claims[3] = {claims0, claims1, claims2};
-  int32_t nprev = r0 > 0 ? ctr->nlist[r0 - 1] : 0;
-  int32_t ncur = ctr->nlist[r0];
+  const Geo g = p.g;
+  int32_t nprev = r0 > 0 ? p.ctr->cnt[(r0 + 3) & 3] : 0;
+  int32_t ncur = p.ctr->cnt[r0 & 3];
   const int32_t bound = ncur + 2;  // each round commits at least one key
+  if (r0 == 0 && threadIdx.x == 0) p.stats->n_inserted = ncur;
   long long evicted = 0, rounds = 0;
   int r = r0;
   for (int32_t it = 0; it <= bound; ++it) {
@@ -534,21 +664,17 @@ __global__ void __launch_bounds__(1024) k_insert_finish(
     if (threadIdx.x == 0) *s_next = 0;
     __syncthreads();
     const int32_t nmax = nprev > ncur ? nprev : ncur;
-    const long long* kp = lists.key[(r + 2) % 3];
-    const long long* kc = lists.key[r % 3];
-    const int32_t* ic = lists.idx[r % 3];
-    long long* kn = lists.key[(r + 1) % 3];
-    int32_t* in_ = lists.idx[(r + 1) % 3];
+    const int rp = (r + 2) % 3, rc = r % 3, rn = (r + 1) % 3;
     for (int32_t i = threadIdx.x; i < nmax; i += blockDim.x) {
-      if (i < nprev) clear_window(claims[(r + 2) % 3], __ldcg(kp + i), g);
+      if (i < nprev) clear_window(p.claims[rp], __ldcg(p.lkey[rp] + i), g);
       if (i < ncur) {
-        const long long k = __ldcg(kc + i);
-        const int32_t u = __ldcg(ic + i);
-        if (!try_commit(k, u, claims[r % 3], keys, last, g, step, urow, evicted)) {
+        const long long k = __ldcg(p.lkey[rc] + i);
+        const int32_t u = __ldcg(p.lidx[rc] + i);
+        if (!try_commit(k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted)) {
           const int m = atomicAdd(s_next, 1);
-          kn[m] = k;
-          in_[m] = u;
-          claim_window(claims[(r + 1) % 3], k, g);
+          p.lkey[rn][m] = k;
+          p.lidx[rn][m] = u;
+          claim_window(p.claims[rn], k, g);
         }
       }
     }
@@ -559,47 +685,41 @@ __global__ void __launch_bounds__(1024) k_insert_finish(
     ncur = *s_next;
     ++r;
     if (nprev == 0 && ncur == 0) break;
-    if (it == bound && threadIdx.x == 0) set_status(status, kStInternal);
+    if (it == bound && threadIdx.x == 0) set_status(p.status, kStInternal);
   }
   const long long ev = block_sum_ll(evicted, sm);
-  if (threadIdx.x == 0 && stats) {
-    if (ev) atomic_add_ll(&stats->n_evicted, ev);
-    if (rounds) atomic_add_ll(&stats->n_rounds, rounds);
-    stats->n_inserted = ctr->nlist[0];
+  if (threadIdx.x == 0) {
+    if (ev) atomic_add_ll(&p.stats->n_evicted, ev);
+    if (rounds) atomic_add_ll(&p.stats->n_rounds, rounds);
   }
 }
 
 // ---------------------------------------------------------------------------
-// Writeback: M[r] <- fl(e_hat - fl(e_hat - e)) for every distinct id still owning
-// its row; one warp per row, 16-byte vectors, loads of a chunk before stores.
+// Writeback row update: M[r] <- fl(e_hat - fl(e_hat - e)) for every distinct id
+// still owning its row; one warp per row, 16-byte vectors, loads of a chunk
+// issued before its stores.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kBlock) k_writeback(
-    const long long* __restrict__ ukey, const int32_t* __restrict__ upos,
-    const int32_t* __restrict__ urow, const long long* U_ptr, const long long* __restrict__ keys,
-    float4* __restrict__ M, const float4* __restrict__ e, int D4, WbStats* stats) {
+__global__ void __launch_bounds__(kBlock) k_writeback(WbParams p) {
   __shared__ long long sm[33];
   const int lane = threadIdx.x & 31;
-  const long long U = *U_ptr;
+  const long long U = p.ctr->n_unique;
+  if (blockIdx.x == 0 && threadIdx.x == 0) p.stats->n_unique = U;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   long long dropped = 0;
   for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
-    const int32_t r = urow[u];
-    if (r < 0) {  // every distinct id gets a row; never expected
+    const int32_t r = __ldcg(p.urow + u);
+    if (r < 0 || __ldcg(p.keys + r) != __ldcg(p.ukey + u)) {  // evicted again in this step
       dropped += lane == 0;
       continue;
     }
-    if (__ldcg(keys + r) != ukey[u]) {
-      dropped += lane == 0;
-      continue;
-    }
-    float4* m = M + (int64_t)r * D4;
-    const float4* ev = e + (int64_t)upos[u] * D4;
-    for (int base = 0; base < D4; base += 4 * 32) {
+    float4* m = p.M + (int64_t)r * p.D4;
+    const float4* ev = p.e + (int64_t)__ldcg(p.upos + u) * p.D4;
+    for (int base = 0; base < p.D4; base += 4 * 32) {
       float4 a[4], b[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
-        if (c < D4) {
+        if (c < p.D4) {
           a[q] = __ldcg(m + c);
           b[q] = __ldcs(ev + c);
         }
@@ -607,7 +727,7 @@ __global__ void __launch_bounds__(kBlock) k_writeback(
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
-        if (c < D4) {
+        if (c < p.D4) {
           float4 o;
           o.x = __fsub_rn(a[q].x, __fsub_rn(a[q].x, b[q].x));
           o.y = __fsub_rn(a[q].y, __fsub_rn(a[q].y, b[q].y));
@@ -618,10 +738,8 @@ __global__ void __launch_bounds__(kBlock) k_writeback(
       }
     }
   }
-  if (stats) {
-    const long long d = block_sum_ll(dropped, sm);
-    if (threadIdx.x == 0 && d) atomic_add_ll(&stats->n_dropped, d);
-  }
+  const long long d = block_sum_ll(dropped, sm);
+  if (threadIdx.x == 0 && d) atomic_add_ll(&p.stats->n_dropped, d);
 }
 
 // ---------------------------------------------------------------------------

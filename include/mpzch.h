@@ -218,17 +218,20 @@ MPZCH_API int mpzch_set_last_step(mpzch_table* t, int64_t step);
  * Synchronises `stream`. */
 MPZCH_API int mpzch_get_status(mpzch_table* t, int32_t* status, void* stream);
 
-/* Per-phase timing with CUDA events recorded around each kernel launch on the
- * launching stream.  Phases (index): 0 lookup, 1 gather, 2 dedup, 3 insert,
- * 4 writeback, 5 select, 6 export.  mpzch_trace_read synchronises the events
- * recorded since the last read and returns, per phase, the summed device
- * milliseconds and the number of kernel launches. */
+/* Per-phase timing with CUDA events recorded around each phase's launches on
+ * the launching stream.  Phases (index): 0 lookup, 1 gather, 2 dedup (inside
+ * mpzch_writeback: dedup, re-probe and refresh; also mpzch_dedup), 3 insert
+ * (conflict rounds), 4 writeback (the row update kernel alone), 5 select,
+ * 6 export.  mpzch_trace_read synchronises the events recorded since the last
+ * read and returns, per phase, the summed device milliseconds and the number
+ * of kernel launches. */
 #define MPZCH_NPHASES 7
 MPZCH_API int mpzch_trace_enable(mpzch_table* t, int32_t on);
 MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t nphases);
 
 /* Options.  MPZCH_OPT_WIDE_ROUNDS: number of grid-wide insert conflict rounds
- * before the single-block finisher takes the remaining keys (default 3, 0..16). */
+ * launched before a single-block kernel runs the remaining rounds (default 4,
+ * range 0..64).  Results do not depend on it. */
 #define MPZCH_OPT_WIDE_ROUNDS 1
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 
