@@ -139,6 +139,21 @@ def gpu_id_for(local_rank: int) -> str:
     return str(local_rank)
 
 
+# ------------------------------------------------------------------ ranks
+def reduce_over_ranks(units: float, ms: float, device):
+    """Whole-job aggregate: units summed over ranks, time = max over ranks.
+    Without an initialised process group this is the identity."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(units), float(ms)
+    u = torch.tensor([float(units)], dtype=torch.float64, device=device)
+    m = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    dist.all_reduce(m, op=dist.ReduceOp.MAX)
+    return float(u.item()), float(m.item())
+
+
 # ------------------------------------------------------------------ host-side inputs
 def host_step(t: int, rank: int):
     tt = t + rank * REPLICA_STRIDE
@@ -271,15 +286,7 @@ def run_ours(args):
     n_unique = int(st[:, 1].sum())
     n_written = int((st[:, 1] - st[:, 5]).sum())
     n_hit_lab = int(hits[Pf + Wm:].sum().item())
-    t_units = torch.tensor([float(n_unique), ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        u = t_units[:1].clone()
-        m = t_units[1:].clone()
-        dist.all_reduce(u, op=dist.ReduceOp.SUM)
-        dist.all_reduce(m, op=dist.ReduceOp.MAX)
-        tot_units, max_ms = float(u.item()), float(m.item())
-    else:
-        tot_units, max_ms = float(n_unique), ms
+    tot_units, max_ms = reduce_over_ranks(n_unique, ms, dev)
 
     # roofline of the dominant kernel (the Writeback row update)
     D, A = W.dim, W.ao_dim
@@ -372,13 +379,7 @@ def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
     ev1.record()
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
-    units = float(st_h[:, 1].sum().item())
-    if world > 1:
-        u = torch.tensor([units], dtype=torch.float64, device=dev)
-        m = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(u, op=dist.ReduceOp.SUM)
-        dist.all_reduce(m, op=dist.ReduceOp.MAX)
-        units, ms = float(u.item()), float(m.item())
+    units, ms = reduce_over_ranks(float(st_h[:, 1].sum().item()), ms, dev)
     h2d = W.batch * 8 + lab * 4 + W.batch * W.dim * 4
     return {"value": units / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": 7 * 8, "ms_per_step": ms / K}
