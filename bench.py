@@ -5,7 +5,10 @@ per step a labeled batch of 32,768 ids and an unlabeled candidate-pool batch of
 131,072 ids, both Zipf(0.9) over 5M keys, merged labeled-first).  One step =
 MPZCH lookup of the labeled ids -> fused gather (cached row or zeros, plus the
 128-d author embedding from a 1M-row always-on table) -> Writeback of the
-merged batch (dedup, refresh, ascending-key insert/evict, exact row write).
+merged batch (dedup, refresh, ascending-key insert/evict, exact row write),
+issued as one mpzch_train_step call per step with an inputs-ready event, so a
+step's row map overlaps the previous step's row update (--no-pipeline: without
+the event; --separate-calls: three calls).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -51,6 +54,12 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--side-priority", type=int, default=None, choices=[0, 1],
+                    help="priority of the table's side stream (1 = highest)")
+    ap.add_argument("--no-pipeline", action="store_true",
+                    help="do not pass an inputs-ready event (no overlap across steps)")
+    ap.add_argument("--separate-calls", action="store_true",
+                    help="lookup, gather and Writeback as three calls instead of mpzch_train_step")
     ap.add_argument("--wide-rounds", type=int, default=None,
                     help="grid-wide insert conflict rounds before the single-block finisher")
     ap.add_argument("--e-pool", type=int, default=inputs.E_POOL,
@@ -243,15 +252,27 @@ def run_ours(args):
     out = torch.empty((lab, W.dim + W.ao_dim), dtype=torch.float32, device=dev)
     stats = torch.zeros((total, 7), dtype=torch.int64, device=dev)
 
+    # per-step outputs the next (pipelined) step may not overwrite early: the
+    # hit masks and counters are kept per step, the row buffers alternate
+    rows_t = [torch.empty(lab, dtype=torch.int32, device=dev) for _ in range(2)]
+    ready = torch.cuda.Event()
+    ready.record(stream)  # every step's inputs are resident from here on
     tbl = binding.MpzchTable(W.capacity, W.dim, W.probes)
     binding.mpzch_reserve(tbl.h, W.batch)
+    if args.side_priority is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SIDE_PRIORITY, args.side_priority)
     if args.wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, args.wide_rounds)
 
     def step(t):
-        binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])
-        binding.mpzch_gather_fused(tbl.h, rows, hits[t], out, ao_d, aor_d[t])
-        binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % E], t, stats[t])
+        if args.separate_calls:
+            binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])
+            binding.mpzch_gather_fused(tbl.h, rows, hits[t], out, ao_d, aor_d[t])
+            binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % E], t, stats[t])
+        else:
+            binding.mpzch_train_step(tbl.h, ids_d[t], lab, e_d[t % E], t, rows_t[t % 2], hits[t],
+                                     out, ao_d, aor_d[t], stats[t],
+                                     inputs_ready=None if args.no_pipeline else ready)
 
     for t in range(Pf):
         step(t)
@@ -372,9 +393,10 @@ def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
         ids_d.copy_(ids_h[j], non_blocking=True)
         aor_d.copy_(aor_h[j], non_blocking=True)
         e_d.copy_(e_h[t % E], non_blocking=True)
-        binding.mpzch_lookup(tbl.h, ids_d[:lab], rows, hit)
-        binding.mpzch_gather_fused(tbl.h, rows, hit, out, ao_d, aor_d)
-        binding.mpzch_writeback(tbl.h, ids_d, e_d, t, st_d)
+        ev_in = torch.cuda.Event()
+        ev_in.record()
+        binding.mpzch_train_step(tbl.h, ids_d, lab, e_d, t, rows, hit, out, ao_d, aor_d, st_d,
+                                 inputs_ready=ev_in)
         st_h[j].copy_(st_d, non_blocking=True)
     ev1.record()
     torch.cuda.synchronize()

@@ -29,6 +29,7 @@ MPZCH_STATUS_BADAO = 4
 MPZCH_STATUS_INTERNAL = 8
 MPZCH_NPHASES = 7
 MPZCH_OPT_WIDE_ROUNDS = 1
+MPZCH_OPT_SIDE_PRIORITY = 2
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")
@@ -47,6 +48,8 @@ _SIGS = {
     "mpzch_gather_fused": [_p, _p, _p, _i64, _p, _i64, _i32, _p, _p, _p],
     "mpzch_dedup": [_p, _p, _i64, _p, _p, _p, _p],
     "mpzch_writeback": [_p, _p, _p, _i64, _i64, _p, _p],
+    "mpzch_train_step": [_p, _p, _i64, _i64, _p, _i64, _p, _i64, _i32, _p, _p, _p, _p, _p, _p,
+                         _p],
     "mpzch_select_written_since": [_p, _i64, _p, _p, _p],
     "mpzch_export_int8": [_p, _p, _i64, _p, _p, _p, _p, _p],
     "mpzch_serve_gather": [_p, _i64, _i32, _p, _p, _i32, _p, _i64, _p, _p, _p, _p, _p],
@@ -160,6 +163,31 @@ def mpzch_writeback(h, ids, e, step: int, stats=None, stream=None) -> None:
     assert e.dim() == 2 and e.shape[0] >= n
     _check("mpzch_writeback", _lib.mpzch_writeback(h, _ptr(ids), _ptr(e), n, step, _ptr(stats),
                                                    _stream(stream)))
+
+
+def mpzch_train_step(h, ids, n_labeled: int, e, step: int, rows, hit, out, ao_table=None,
+                     ao_rows=None, stats=None, inputs_ready=None, stream=None) -> None:
+    """inputs_ready: None or a torch.cuda.Event recorded after this step's inputs."""
+    _need(ids, torch.int64, "ids")
+    _need(e, torch.float32, "e")
+    n = ids.numel()
+    assert 0 <= n_labeled <= n and e.dim() == 2 and e.shape[0] >= n
+    if n_labeled:
+        _need(rows, torch.int32, "rows")
+        _need(hit, torch.uint8, "hit")
+        _need(out, torch.float32, "out")
+    ao_n, ao_dim = 0, 0
+    if ao_table is not None:
+        _need(ao_table, torch.float32, "ao_table")
+        _need(ao_rows, torch.int32, "ao_rows")
+        ao_n, ao_dim = ao_table.shape
+    if stats is not None:
+        _need(stats, torch.int64, "stats")
+        assert stats.numel() >= 7
+    _check("mpzch_train_step", _lib.mpzch_train_step(
+        h, _ptr(ids), n, n_labeled, _ptr(e), step, _ptr(ao_table), ao_n, ao_dim, _ptr(ao_rows),
+        _ptr(rows), _ptr(hit), _ptr(out), _ptr(stats),
+        None if inputs_ready is None else C.c_void_p(inputs_ready.cuda_event), _stream(stream)))
 
 
 def mpzch_select_written_since(h, since: int, rows_out, count, stream=None) -> None:
@@ -311,6 +339,17 @@ class MpzchTable:
 
     def writeback(self, ids, e, step, stats=None, stream=None):
         mpzch_writeback(self.h, ids, e, step, stats, stream)
+
+    def train_step(self, ids, n_labeled, e, step, ao_table=None, ao_rows=None, stats=None,
+                   inputs_ready=None, stream=None):
+        dev = ids.device
+        w = self.dim + (0 if ao_table is None else ao_table.shape[1])
+        rows = torch.empty(n_labeled, dtype=torch.int32, device=dev)
+        hit = torch.empty(n_labeled, dtype=torch.uint8, device=dev)
+        out = torch.empty((n_labeled, w), dtype=torch.float32, device=dev)
+        mpzch_train_step(self.h, ids, n_labeled, e, step, rows, hit, out, ao_table, ao_rows, stats,
+                         inputs_ready, stream)
+        return rows, hit, out
 
     def select_written_since(self, since, stream=None):
         rows = torch.empty(self.capacity, dtype=torch.int32, device=self.device)

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <cstdlib>
+#include <utility>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -66,6 +67,62 @@ int after_launch() {
   return cudaGetLastError() == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
 }
 
+// Launches a kernel; with `pdl` it may start while the previous kernel of the
+// stream drains (programmatic dependent launch: every kernel waits for its
+// predecessors with griddepcontrol.wait before touching memory).
+template <typename... KArgs, typename... Args>
+int launch(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t st, bool pdl,
+           Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MPZCH_ECUDA;
+  }
+  return MPZCH_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_smem(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                cudaStream_t st, bool pdl, Args&&... args) {
+  static bool attr_set = false;  // one kernel per instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return MPZCH_ECUDA;
+    }
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return MPZCH_ECUDA;
+  }
+  return MPZCH_OK;
+}
+
 uint64_t pow2_at_least(uint64_t x) {
   uint64_t p = 1;
   while (p < x) p <<= 1;
@@ -108,6 +165,11 @@ struct mpzch_table {
   int32_t* urow = nullptr;
   long long* lkey[3] = {nullptr, nullptr, nullptr};  // insert round lists: keys
   int32_t* lidx[3] = {nullptr, nullptr, nullptr};    // and their distinct-id index
+  // write lists (row, position of e), two buffers used by alternate Writebacks
+  int32_t* wrow[2] = {nullptr, nullptr};
+  int32_t* wpos[2] = {nullptr, nullptr};
+  int32_t* wcnt = nullptr;  // device int32[2]
+  int wset = 0;             // buffer of the next Writeback
   // small device words
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
@@ -115,7 +177,14 @@ struct mpzch_table {
   int32_t* sel_bcount = nullptr;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
-  int wide_rounds = 4;  // grid-wide insert rounds before the single-block finisher
+  int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
+  int side_high_priority = 0;  // priority of the side stream (set before its first use)
+  // mpzch_train_step: the row map runs on a second (high-priority) stream
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_fork = nullptr, ev_lookup = nullptr, ev_map = nullptr;
+  cudaEvent_t ev_update[2] = {nullptr, nullptr};  // row update that read write list b
+  cudaEvent_t ev_user = nullptr;    // end of the last other call on a caller stream
+  cudaEvent_t ev_gather = nullptr;  // end of the last train step's gather
   // tracing
   bool trace = false;
   struct Rec {
@@ -140,6 +209,8 @@ void free_batch_scratch(mpzch_table* t) {
   dev_free(t->urow);
   for (auto& l : t->lkey) dev_free(l), l = nullptr;
   for (auto& l : t->lidx) dev_free(l), l = nullptr;
+  for (auto& l : t->wrow) dev_free(l), l = nullptr;
+  for (auto& l : t->wpos) dev_free(l), l = nullptr;
   t->hkey = nullptr;
   t->hpos = nullptr;
   t->slot_of = t->bcount = t->upos = t->urow = nullptr;
@@ -155,6 +226,7 @@ void free_all(mpzch_table* t) {
   dev_free(t->M);
   for (auto& c : t->claims) dev_free(c), c = nullptr;
   dev_free(t->ctr);
+  dev_free(t->wcnt);
   dev_free(t->stats);
   dev_free(t->status);
   dev_free(t->sel_bcount);
@@ -164,6 +236,33 @@ void free_all(mpzch_table* t) {
     cudaEventDestroy(r.b);
   }
   for (auto e : t->pool) cudaEventDestroy(e);
+  if (t->ev_fork) cudaEventDestroy(t->ev_fork);
+  if (t->ev_lookup) cudaEventDestroy(t->ev_lookup);
+  if (t->ev_map) cudaEventDestroy(t->ev_map);
+  for (auto& e : t->ev_update)
+    if (e) cudaEventDestroy(e);
+  if (t->ev_user) cudaEventDestroy(t->ev_user);
+  if (t->ev_gather) cudaEventDestroy(t->ev_gather);
+  if (t->side) cudaStreamDestroy(t->side);
+}
+
+int ensure_side_stream(mpzch_table* t) {
+  if (t->side) return MPZCH_OK;
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&t->side, cudaStreamNonBlocking,
+                                   t->side_high_priority ? greatest : least) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_lookup, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_map, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_update[0], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_update[1], cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_user, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&t->ev_gather, cudaEventDisableTiming) != cudaSuccess) {
+    cudaGetLastError();
+    return MPZCH_ECUDA;
+  }
+  return MPZCH_OK;
 }
 
 // Grow the per-batch scratch to hold batches of n ids.
@@ -188,6 +287,8 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   if (!rc) rc = dev_alloc((void**)&t->urow, cap * sizeof(int32_t));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lkey[i], cap * sizeof(long long));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lidx[i], cap * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->wrow[i], cap * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->wpos[i], cap * sizeof(int32_t));
   if (rc) {
     free_batch_scratch(t);
     return rc;
@@ -249,13 +350,155 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
-                                           stats, t->status);
+                                           stats, t->status, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_compact<<<tiles, kBlock, 0, st>>>(id, n, t->slot_of, t->hkey, t->hpos, t->bcount, uniq,
                                             pos, dev_count, stats);
   return after_launch();
+}
+
+}  // namespace
+
+namespace {
+
+int enqueue_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit,
+                   cudaStream_t st, bool pdl) {
+  PhaseScope ps(t, PH_LOOKUP, st);
+  int G = (int)pow2_at_least((uint64_t)t->P);
+  if (G > 32) G = 32;
+  return launch(k_lookup, grid_for(n * G, kBlock), kBlock, st, pdl,
+                reinterpret_cast<const long long*>(ids), n, (const long long*)t->keys, t->geo, G,
+                rows, hit, t->status);
+}
+
+int check_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
+                 const float* ao_table, int64_t ao_nrows, int32_t ao_dim, const int32_t* ao_rows,
+                 const float* out) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  const bool has_ao = ao_table != nullptr;
+  if (has_ao && (ao_dim <= 0 || ao_dim % 4 != 0 || ao_nrows <= 0 || !ao_rows)) return MPZCH_EINVAL;
+  if (!has_ao && (ao_dim != 0 || ao_rows)) return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!rows || !hit || !out || !on_device(t)) return MPZCH_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) ||
+      (has_ao && (reinterpret_cast<uintptr_t>(ao_table) & 15)))
+    return MPZCH_EINVAL;
+  return MPZCH_OK;
+}
+
+int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
+                   const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
+                   const int32_t* ao_rows, float* out, cudaStream_t st, bool pdl) {
+  PhaseScope ps(t, PH_GATHER, st);
+  const bool has_ao = ao_table != nullptr;
+  return launch(k_gather_fused, grid_for(n * 32, kBlock), kBlock, st, pdl, rows, hit, n,
+                reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
+                reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
+                ao_rows, reinterpret_cast<float4*>(out), t->status);
+}
+
+int check_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step) {
+  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
+  if (step <= t->last_step) return MPZCH_EINVAL;
+  if (n > 0 && (!ids || !e)) return MPZCH_EINVAL;
+  if (!on_device(t)) return MPZCH_EINVAL;
+  if (reinterpret_cast<uintptr_t>(e) & 15) return MPZCH_EINVAL;
+  return MPZCH_OK;
+}
+
+WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
+                     WbStats* stats) {
+  WbParams p;
+  p.ids = reinterpret_cast<const long long*>(ids);
+  p.n = n;
+  p.e = reinterpret_cast<const float4*>(e);
+  p.D4 = t->D / 4;
+  p.hkey = t->hkey;
+  p.hpos = t->hpos;
+  p.hmask = t->hmask;
+  p.slot_of = t->slot_of;
+  p.ukey = t->ukey;
+  p.upos = t->upos;
+  p.urow = t->urow;
+  p.keys = t->keys;
+  p.last = t->last;
+  p.M = reinterpret_cast<float4*>(t->M);
+  p.g = t->geo;
+  p.step = (long long)step;
+  for (int i = 0; i < 3; ++i) {
+    p.lkey[i] = t->lkey[i];
+    p.lidx[i] = t->lidx[i];
+    p.claims[i] = t->claims[i];
+  }
+  p.ctr = t->ctr;
+  p.stats = stats;
+  p.status = t->status;
+  p.wide_rounds = t->wide_rounds;
+  p.wrow = t->wrow[t->wset];
+  p.wpos = t->wpos[t->wset];
+  p.wcount = t->wcnt + t->wset;
+  return p;
+}
+
+// Row map of one Writeback on stream `st`: dedup + re-probe + refresh, then
+// (optionally) the lookup of the first n_lookup ids -- which must read the keys
+// before any insert of this step -- then the insert rounds and the write list.
+// ev_lookup (optional) is recorded after the lookup.
+int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, int32_t* rows,
+                    uint8_t* hit, int64_t n_lookup, cudaEvent_t ev_lookup, void* unused) {
+  (void)unused;
+  const int64_t n = p.n;
+  int rc;
+  {
+    PhaseScope ps(t, PH_DEDUP, st);
+    rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kBlock, st, false, p.ids, n,
+                t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status, p.wcount);
+    if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
+    if (rc) return rc;
+  }
+  if (n_lookup > 0) {
+    rc = enqueue_lookup(t, reinterpret_cast<const int64_t*>(p.ids), n_lookup, rows, hit, st, true);
+    if (rc) return rc;
+  }
+  if (ev_lookup && cudaEventRecord(ev_lookup, st) != cudaSuccess) return MPZCH_ECUDA;
+  {
+    PhaseScope ps(t, PH_INSERT, st);
+    const unsigned grid = grid_for(n, kBlock, 4);
+    for (int r = 0; r < t->wide_rounds && !rc; ++r)
+      rc = launch(k_insert_round, grid, kBlock, st, !ev_lookup || r > 0, p, r);
+    if (!rc)
+      rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, t->wide_rounds);
+    if (!rc) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
+  }
+  return rc;
+}
+
+int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool pdl) {
+  {
+    PhaseScope ps(t, PH_WRITEBACK, st);
+    const int rc = launch(k_writeback, grid_for(p.n * 32, kBlock), kBlock, st, pdl,
+                          (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount,
+                          p.M, p.e, p.D4);
+    if (rc) return rc;
+  }
+  if (t->side && cudaEventRecord(t->ev_update[t->wset], st) != cudaSuccess) return MPZCH_ECUDA;
+  t->wset ^= 1;
+  return MPZCH_OK;
+}
+
+// Calls other than mpzch_train_step run on the caller's stream: they first
+// wait for the side stream's work, and the next train step's side-stream work
+// waits for them (ev_user).
+int join_side(mpzch_table* t, cudaStream_t st) {
+  if (!t->side) return MPZCH_OK;
+  return cudaStreamWaitEvent(st, t->ev_map, 0) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
+}
+
+int mark_user(mpzch_table* t, cudaStream_t st, int rc) {
+  if (rc || !t->side) return rc;
+  return cudaEventRecord(t->ev_user, st) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
 }
 
 }  // namespace
@@ -340,7 +583,7 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
-                                           dev_status);
+                                           dev_status, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -370,6 +613,7 @@ int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mp
   for (int i = 0; i < 3 && !rc; ++i)
     rc = dev_alloc((void**)&t->claims[i], capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
+  if (!rc) rc = dev_alloc((void**)&t->wcnt, 2 * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
   if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
   if (!rc)
@@ -421,32 +665,21 @@ int mpzch_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, u
   if (n == 0) return MPZCH_OK;
   if (!ids || !rows || !hit || !on_device(t)) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  PhaseScope ps(t, PH_LOOKUP, st);
-  int G = (int)pow2_at_least((uint64_t)t->P);
-  if (G > 32) G = 32;
-  k_lookup<<<grid_for(n * G, kBlock), kBlock, 0, st>>>(
-      reinterpret_cast<const long long*>(ids), n, t->keys, t->geo, G, rows, hit, t->status);
-  return after_launch();
+  int rc = join_side(t, st);
+  if (!rc) rc = enqueue_lookup(t, ids, n, rows, hit, st, false);
+  return mark_user(t, st, rc);
 }
 
 int mpzch_gather_fused(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
                        const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
                        const int32_t* ao_rows, float* out, void* stream) {
-  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
-  const bool has_ao = ao_table != nullptr;
-  if (has_ao && (ao_dim <= 0 || ao_dim % 4 != 0 || ao_nrows <= 0 || !ao_rows)) return MPZCH_EINVAL;
-  if (!has_ao && (ao_dim != 0 || ao_rows)) return MPZCH_EINVAL;
-  if (n == 0) return MPZCH_OK;
-  if (!rows || !hit || !out || !on_device(t)) return MPZCH_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(out) & 15) || (has_ao && (reinterpret_cast<uintptr_t>(ao_table) & 15)))
-    return MPZCH_EINVAL;
+  int rc = check_gather(t, rows, hit, n, ao_table, ao_nrows, ao_dim, ao_rows, out);
+  if (rc || n == 0) return rc;
   cudaStream_t st = S(stream);
-  PhaseScope ps(t, PH_GATHER, st);
-  k_gather_fused<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
-      rows, hit, n, reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
-      reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0, ao_rows,
-      reinterpret_cast<float4*>(out), t->status);
-  return after_launch();
+  rc = join_side(t, st);
+  if (!rc)
+    rc = enqueue_gather(t, rows, hit, n, ao_table, ao_nrows, ao_dim, ao_rows, out, st, false);
+  return mark_user(t, st, rc);
 }
 
 int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, int32_t* pos,
@@ -455,78 +688,100 @@ int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, in
   if (n > 0 && (!ids || !uniq || !pos)) return MPZCH_EINVAL;
   if (!on_device(t)) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  if (n == 0) return cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
-  int rc = ensure_batch(t, n, st);
+  if (n == 0)
+    return cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess ? MPZCH_OK
+                                                                              : MPZCH_ECUDA;
+  int rc = join_side(t, st);
+  if (!rc) rc = ensure_batch(t, n, st);
   if (rc) return rc;
-  PhaseScope ps(t, PH_DEDUP, st);
-  return run_dedup(t, ids, n, reinterpret_cast<long long*>(uniq), pos,
+  {
+    PhaseScope ps(t, PH_DEDUP, st);
+    rc = run_dedup(t, ids, n, reinterpret_cast<long long*>(uniq), pos,
                    reinterpret_cast<long long*>(dev_count), nullptr, st);
+  }
+  return mark_user(t, st, rc);
 }
 
 int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
                     mpzch_wb_stats* dev_stats, void* stream) {
-  if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
-  if (step <= t->last_step) return MPZCH_EINVAL;
-  if (n > 0 && (!ids || !e)) return MPZCH_EINVAL;
-  if (!on_device(t)) return MPZCH_EINVAL;
-  if (reinterpret_cast<uintptr_t>(e) & 15) return MPZCH_EINVAL;
+  int rc = check_writeback(t, ids, e, n, step);
+  if (rc) return rc;
   cudaStream_t st = S(stream);
   WbStats* stats = dev_stats ? reinterpret_cast<WbStats*>(dev_stats) : t->stats;
+  rc = join_side(t, st);
+  if (rc) return rc;
   if (n == 0) {
     if (cudaMemsetAsync(stats, 0, sizeof(WbStats), st) != cudaSuccess) return MPZCH_ECUDA;
     t->last_step = step;
-    return MPZCH_OK;
+    return mark_user(t, st, MPZCH_OK);
   }
-  int rc = ensure_batch(t, n, st);
+  rc = ensure_batch(t, n, st);
   if (rc) return rc;
-  WbParams p;
-  p.ids = reinterpret_cast<const long long*>(ids);
-  p.n = n;
-  p.e = reinterpret_cast<const float4*>(e);
-  p.D4 = t->D / 4;
-  p.hkey = t->hkey;
-  p.hpos = t->hpos;
-  p.hmask = t->hmask;
-  p.slot_of = t->slot_of;
-  p.ukey = t->ukey;
-  p.upos = t->upos;
-  p.urow = t->urow;
-  p.keys = t->keys;
-  p.last = t->last;
-  p.M = reinterpret_cast<float4*>(t->M);
-  p.g = t->geo;
-  p.step = (long long)step;
-  for (int i = 0; i < 3; ++i) {
-    p.lkey[i] = t->lkey[i];
-    p.lidx[i] = t->lidx[i];
-    p.claims[i] = t->claims[i];
+  const WbParams p = make_params(t, ids, e, n, step, stats);
+  rc = enqueue_row_map(t, p, st, nullptr, nullptr, 0, nullptr, nullptr);
+  if (!rc) rc = enqueue_row_update(t, p, st, true);
+  if (rc) return rc;
+  t->last_step = step;
+  return mark_user(t, st, MPZCH_OK);
+}
+
+int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_labeled,
+                     const float* e, int64_t step, const float* ao_table, int64_t ao_nrows,
+                     int32_t ao_dim, const int32_t* ao_rows, int32_t* rows, uint8_t* hit,
+                     float* out, mpzch_wb_stats* dev_stats, void* inputs_ready, void* stream) {
+  if (!t || n_labeled < 0 || n_labeled > n) return MPZCH_EINVAL;
+  int rc = check_writeback(t, ids, e, n, step);
+  if (rc) return rc;
+  if (n_labeled > 0) {
+    if (!rows || !hit) return MPZCH_EINVAL;
+    rc = check_gather(t, rows, hit, n_labeled, ao_table, ao_nrows, ao_dim, ao_rows, out);
+    if (rc) return rc;
   }
-  p.ctr = t->ctr;
-  p.stats = stats;
-  p.status = t->status;
-  {
-    PhaseScope ps(t, PH_DEDUP, st);
-    k_dedup_insert<<<(unsigned)((n + kTile - 1) / kTile), kBlock, 0, st>>>(
-        p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, stats, t->status);
-    if (after_launch()) return MPZCH_ECUDA;
-    k_first_reprobe<<<grid_for(n, kBlock), kBlock, 0, st>>>(p);
-    if (after_launch()) return MPZCH_ECUDA;
+  cudaStream_t st = S(stream);
+  WbStats* stats = dev_stats ? reinterpret_cast<WbStats*>(dev_stats) : t->stats;
+  rc = ensure_batch(t, n > 0 ? n : 1, st);
+  if (!rc) rc = ensure_side_stream(t);
+  if (rc) return rc;
+  if (n == 0) {
+    if (cudaStreamWaitEvent(st, t->ev_map, 0) != cudaSuccess ||
+        cudaMemsetAsync(stats, 0, sizeof(WbStats), st) != cudaSuccess)
+      return MPZCH_ECUDA;
+    t->last_step = step;
+    return mark_user(t, st, MPZCH_OK);
   }
-  {
-    PhaseScope ps(t, PH_INSERT, st);
-    const unsigned grid = grid_for(n, kBlock, 4);
-    for (int r = 0; r < t->wide_rounds; ++r) {
-      k_insert_round<<<grid, kBlock, 0, st>>>(p, r);
-      if (after_launch()) return MPZCH_ECUDA;
-    }
-    k_insert_finish<<<1, 1024, 0, st>>>(p, t->wide_rounds);
-    if (after_launch()) return MPZCH_ECUDA;
+  const WbParams p = make_params(t, ids, e, n, step, stats);
+  // Side stream: dedup + refresh, lookup, inserts, write list.  It starts after
+  // the caller's stream (no inputs_ready), or -- pipelined -- after the inputs,
+  // the last other call, the row update that last read this write-list buffer
+  // and the previous gather (which read rows/hit), but not after the rest of
+  // the caller's stream, so it overlaps the previous step's row update.
+  if (inputs_ready) {
+    if (cudaStreamWaitEvent(t->side, reinterpret_cast<cudaEvent_t>(inputs_ready), 0) !=
+            cudaSuccess ||
+        cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->side, t->ev_gather, 0) != cudaSuccess)
+      return MPZCH_ECUDA;
+  } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
+             cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess) {
+    return MPZCH_ECUDA;
   }
-  {
-    PhaseScope ps(t, PH_WRITEBACK, st);
-    k_writeback<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(p);
-    if (after_launch()) return MPZCH_ECUDA;
+  rc = enqueue_row_map(t, p, t->side, rows, hit, n_labeled, t->ev_lookup, nullptr);
+  if (rc) return rc;
+  if (cudaEventRecord(t->ev_map, t->side) != cudaSuccess) return MPZCH_ECUDA;
+  // Caller's stream: gather once the lookup is done, then the row update once
+  // the row map is done (and after the gather has read the values).
+  if (n_labeled > 0) {
+    if (cudaStreamWaitEvent(st, t->ev_lookup, 0) != cudaSuccess) return MPZCH_ECUDA;
+    rc = enqueue_gather(t, rows, hit, n_labeled, ao_table, ao_nrows, ao_dim, ao_rows, out, st,
+                        false);
+    if (rc) return rc;
   }
+  if (cudaEventRecord(t->ev_gather, st) != cudaSuccess ||
+      cudaStreamWaitEvent(st, t->ev_map, 0) != cudaSuccess)
+    return MPZCH_ECUDA;
+  rc = enqueue_row_update(t, p, st, false);
+  if (rc) return rc;
   t->last_step = step;
   return MPZCH_OK;
 }
@@ -535,15 +790,22 @@ int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows
                                int64_t* dev_count, void* stream) {
   if (!t || !rows_out || !dev_count || !on_device(t)) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  PhaseScope ps(t, PH_SELECT, st);
-  const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
-  k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
-                                           t->sel_bcount);
-  if (after_launch()) return MPZCH_ECUDA;
-  k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
-                                             t->sel_bcount, rows_out,
-                                             reinterpret_cast<long long*>(dev_count));
-  return after_launch();
+  int rc = join_side(t, st);
+  if (rc) return rc;
+  {
+    PhaseScope ps(t, PH_SELECT, st);
+    const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
+    k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
+                                             t->sel_bcount);
+    rc = after_launch();
+    if (!rc) {
+      k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
+                                                 t->sel_bcount, rows_out,
+                                                 reinterpret_cast<long long*>(dev_count));
+      rc = after_launch();
+    }
+  }
+  return mark_user(t, st, rc);
 }
 
 int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n,
@@ -553,12 +815,17 @@ int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int6
   if (!rows || !q || !scale || !keys_out || !on_device(t)) return MPZCH_EINVAL;
   if (reinterpret_cast<uintptr_t>(q) & 3) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  PhaseScope ps(t, PH_EXPORT, st);
-  k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
-      rows, n, reinterpret_cast<const long long*>(dev_n), reinterpret_cast<const float4*>(t->M),
-      t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale,
-      reinterpret_cast<long long*>(keys_out), t->status);
-  return after_launch();
+  int rc = join_side(t, st);
+  if (rc) return rc;
+  {
+    PhaseScope ps(t, PH_EXPORT, st);
+    k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+        rows, n, reinterpret_cast<const long long*>(dev_n), reinterpret_cast<const float4*>(t->M),
+        t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale,
+        reinterpret_cast<long long*>(keys_out), t->status);
+    rc = after_launch();
+  }
+  return mark_user(t, st, rc);
 }
 
 int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probes,
@@ -604,7 +871,8 @@ int mpzch_set_last_step(mpzch_table* t, int64_t step) {
 int mpzch_get_status(mpzch_table* t, int32_t* status, void* stream) {
   if (!t || !status || !on_device(t)) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  if (cudaMemcpyAsync(t->h_status, t->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
+  if (join_side(t, st) != MPZCH_OK ||
+      cudaMemcpyAsync(t->h_status, t->status, sizeof(int32_t), cudaMemcpyDeviceToHost, st) !=
           cudaSuccess ||
       cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) != cudaSuccess ||
       cudaStreamSynchronize(st) != cudaSuccess)
@@ -643,6 +911,11 @@ int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t npha
 
 int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
   if (!t) return MPZCH_EINVAL;
+  if (option == MPZCH_OPT_SIDE_PRIORITY) {
+    if ((value != 0 && value != 1) || t->side) return MPZCH_EINVAL;
+    t->side_high_priority = (int)value;
+    return MPZCH_OK;
+  }
   if (option == MPZCH_OPT_WIDE_ROUNDS) {
     if (value < 0 || value > 64) return MPZCH_EINVAL;
     t->wide_rounds = (int)value;

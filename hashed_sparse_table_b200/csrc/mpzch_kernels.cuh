@@ -77,6 +77,16 @@ __device__ __forceinline__ void set_status(int32_t* st, int bits) {
   if (st) atomicOr(st, bits);
 }
 
+// Programmatic dependent launch: let the next kernel of the stream start its
+// launch now, then wait until every earlier grid of the stream has completed
+// and its memory is visible.  Both are no-ops for a kernel launched without
+// the programmatic-serialisation attribute.  Every kernel calls this first,
+// so nothing is read before the producer has finished.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // Row of `k` by one thread scanning the whole window (first match in probe
 // order; the identity map holds at most one).  -1 if absent.  Loads of 8
 // slots are issued together.
@@ -103,6 +113,7 @@ __global__ void __launch_bounds__(kBlock) k_lookup(const long long* __restrict__
                                                    const long long* __restrict__ keys, Geo g,
                                                    int G, int32_t* __restrict__ rows,
                                                    uint8_t* __restrict__ hit, int32_t* status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int sub = lane & (G - 1);
   const unsigned gmask = (G == 32) ? 0xFFFFFFFFu : (((1u << G) - 1u) << (lane & ~(G - 1)));
@@ -141,6 +152,7 @@ __global__ void __launch_bounds__(kBlock) k_gather_fused(
     const float4* __restrict__ M, int64_t C, int D4, const float4* __restrict__ ao,
     int64_t ao_n, int A4, const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
     int32_t* status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int W4 = D4 + A4;
@@ -240,7 +252,8 @@ constexpr int kTileHash = 2 * kTile;  // shared-memory slots per tile (load <= 1
 __global__ void __launch_bounds__(kBlock) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status) {
+    WbStats* stats, int32_t* status, int32_t* wcount) {
+  pdl_enter();
   __shared__ unsigned long long s_key[kTileHash];
   __shared__ uint32_t s_pos[kTileHash];
   __shared__ int32_t s_gslot[kTileHash];
@@ -250,6 +263,7 @@ __global__ void __launch_bounds__(kBlock) k_dedup_insert(
     reinterpret_cast<int32_t*>(ctr)[threadIdx.x] = 0;
   if (stats && blockIdx.x == 0 && threadIdx.x < 7)
     reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
+  if (wcount && blockIdx.x == 0 && threadIdx.x == 0) *wcount = 0;
   for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
     s_key[j] = kEmptyKey;
     s_pos[j] = kNoPos;
@@ -350,6 +364,7 @@ __device__ __forceinline__ long long block_prefix_of_counts(const int32_t* cnt, 
 __global__ void __launch_bounds__(kBlock) k_dedup_count(const int32_t* __restrict__ slot_of,
                                                         const uint32_t* __restrict__ hpos,
                                                         int64_t n, int32_t* __restrict__ bcount) {
+  pdl_enter();
   __shared__ long long sm[33];
   const int64_t base = (int64_t)blockIdx.x * kTile + threadIdx.x * 4;
   int c = 0;
@@ -373,6 +388,7 @@ __global__ void __launch_bounds__(kBlock) k_dedup_compact(
     unsigned long long* __restrict__ hkey, uint32_t* __restrict__ hpos,
     const int32_t* __restrict__ bcount, long long* __restrict__ ukey, int32_t* __restrict__ upos,
     long long* dev_count, WbStats* stats) {
+  pdl_enter();
   __shared__ long long sm[33];
   __shared__ int smi[33];
   const long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
@@ -520,6 +536,12 @@ struct WbParams {
   StepCtr* ctr;
   WbStats* stats;
   int32_t* status;
+  int wide_rounds;  // grid-wide insert rounds of this Writeback
+  // write list of this Writeback: (row, position of e) of every distinct id
+  // that still owns its row; one of two buffers, alternating by call
+  int32_t* wrow;
+  int32_t* wpos;
+  int32_t* wcount;
 };
 
 // Two per-thread counts packed as 16-bit halves (each <= the block size).
@@ -552,6 +574,7 @@ __device__ __forceinline__ void block_append2(int wa, int wb, int32_t* ca, int32
 // the table: a resident id refreshes last[row] = step; a missing id enters
 // insert round 0 (list 0) and claims its window in claims[0].
 __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
+  pdl_enter();
   __shared__ long long sm[33];
   __shared__ int smi[33];
   const Geo g = p.g;
@@ -604,6 +627,7 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
 // of round r-1, tries to commit every key of round r, and moves the others to
 // round r+1 (block-aggregated append, claims in claims[(r+1) % 3]).
 __global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
+  pdl_enter();
   __shared__ long long sm[33];
   __shared__ int smi[33];
   const Geo g = p.g;
@@ -636,7 +660,8 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
     if (defer) {
       p.lkey[rn][m] = k;
       p.lidx[rn][m] = u;
-      claim_window(p.claims[rn], k, g);
+      // the single-block finisher claims for itself if it needs claims
+      if (r + 1 < p.wide_rounds) claim_window(p.claims[rn], k, g);
     }
   }
   const long long ev = block_sum_ll(evicted, sm);
@@ -644,18 +669,14 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
   if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
 }
 
-// The rounds left after the grid-wide ones, in one block (block barriers only);
-// lists, claims and counters rotate exactly as in k_insert_round.  Also writes
-// the final counters of the row map.
-__global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
+// Remaining rounds in one block by the claim rule (block barriers only); lists,
+// claims and counters rotate exactly as in k_insert_round.  Used when too many
+// keys are left for the cluster path.
+__device__ void finish_by_rounds(const WbParams& p, int r0, int32_t nprev, int32_t ncur,
+                                 long long& evicted, long long& rounds) {
   __shared__ int32_t s_cnt[2];  // next-list counters, alternating by iteration parity
-  __shared__ long long sm[33];
   const Geo g = p.g;
-  int32_t nprev = r0 > 0 ? p.ctr->cnt[(r0 + 3) & 3] : 0;
-  int32_t ncur = p.ctr->cnt[r0 & 3];
   const int32_t bound = ncur + 2;  // each round commits at least one key
-  if (r0 == 0 && threadIdx.x == 0) p.stats->n_inserted = ncur;
-  long long evicted = 0, rounds = 0;
   int r = r0;
   for (int32_t it = 0; it <= bound; ++it) {
     // s_cnt[it & 1] was last read right after the barrier that ended iteration
@@ -687,6 +708,185 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
     if (nprev == 0 && ncur == 0) break;
     if (it == bound && threadIdx.x == 0) set_status(p.status, kStInternal);
   }
+}
+
+// Places one missing key by the sequential rule (victim = smallest (last, row)
+// in its window).  The caller guarantees that no other thread touches the
+// window meanwhile.
+__device__ __forceinline__ void place_key(const WbParams& p, long long k, int32_t u,
+                                          long long& evicted) {
+  const Geo& g = p.g;
+  const int64_t h = home_slot(k, g);
+  int64_t best = -1;
+  long long best_last = 0;
+  for (int32_t j0 = 0; j0 < g.P; j0 += 8) {
+    long long l[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      l[q] = j0 + q < g.P ? ld_cg(p.last + wslot(h, j0 + q, g)) : 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (j0 + q >= g.P) continue;
+      const int64_t s = wslot(h, j0 + q, g);
+      if (best < 0 || l[q] < best_last || (l[q] == best_last && s < best)) {
+        best = s;
+        best_last = l[q];
+      }
+    }
+  }
+  if (best_last != -1) ++evicted;
+  p.keys[best] = k;
+  p.last[best] = p.step;
+  p.urow[u] = (int32_t)best;
+}
+
+// Keys left after the grid-wide rounds, in one block.
+//
+// Cluster path (at most kClusterMax keys): every key still unplaced only
+// conflicts with unplaced keys whose windows overlap its own (keys placed in
+// earlier rounds are smaller than every unplaced key overlapping them, so
+// their effect already precedes in the sequential order).  The unplaced keys
+// are sorted by home slot (bucket counting sort + insertion sort per bucket in
+// shared memory); maximal runs whose consecutive home slots are less than P
+// apart (cyclically) are clusters with pairwise disjoint window sets; one
+// thread places a cluster's keys in ascending key order.  Claims left behind
+// by the last grid-wide round are cleared by k_write_list (spread over the
+// whole grid).  Larger leftovers fall back to claim rounds.
+constexpr int kClusterMax = 4096;
+constexpr int kClusterBuckets = 4096;
+constexpr size_t kClusterSmem = (size_t)kClusterMax * (4 + 8 + 4) + (kClusterBuckets + 1) * 4;
+
+__global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
+  pdl_enter();
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ long long sm[33];
+  __shared__ int smi[33];
+  const Geo g = p.g;
+  const int32_t nprev = r0 > 0 ? p.ctr->cnt[(r0 + 3) & 3] : 0;
+  const int32_t ncur = p.ctr->cnt[r0 & 3];
+  if (r0 == 0 && threadIdx.x == 0) p.stats->n_inserted = ncur;
+  long long evicted = 0, rounds = 0;
+  if (ncur > kClusterMax) {
+    // claim rounds need this round's claims, which the last grid-wide round skipped
+    for (int32_t i = threadIdx.x; i < ncur; i += blockDim.x)
+      claim_window(p.claims[r0 % 3], __ldcg(p.lkey[r0 % 3] + i), g);
+    __threadfence();
+    __syncthreads();
+    finish_by_rounds(p, r0, nprev, ncur, evicted, rounds);
+  } else {
+    long long* s_k = reinterpret_cast<long long*>(dsm);
+    uint32_t* s_h = reinterpret_cast<uint32_t*>(dsm + 8 * kClusterMax);
+    int32_t* s_u = reinterpret_cast<int32_t*>(dsm + 12 * kClusterMax);
+    int32_t* s_off = reinterpret_cast<int32_t*>(dsm + 16 * kClusterMax);
+    const int rc = r0 % 3;
+    for (int b = threadIdx.x; b <= kClusterBuckets; b += blockDim.x) s_off[b] = 0;
+    __syncthreads();
+    // bucket of each key (buckets partition the slot range in order)
+    constexpr int kPer = kClusterMax / 1024;
+    long long kk[kPer];
+    int32_t uu[kPer], bb[kPer], rk[kPer];
+    uint32_t hh[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int32_t i = threadIdx.x + q * 1024;
+      bb[q] = -1;
+      if (i < ncur) {
+        kk[q] = __ldcg(p.lkey[rc] + i);
+        uu[q] = __ldcg(p.lidx[rc] + i);
+        hh[q] = (uint32_t)home_slot(kk[q], g);
+        bb[q] = (int32_t)(((uint64_t)hh[q] * kClusterBuckets) / (uint64_t)g.C);
+        rk[q] = atomicAdd(&s_off[bb[q]], 1);
+      }
+    }
+    __syncthreads();
+    {  // exclusive scan of the bucket counts (4 buckets per thread)
+      constexpr int kBper = kClusterBuckets / 1024;
+      int c[kBper], sum = 0;
+#pragma unroll
+      for (int q = 0; q < kBper; ++q) {
+        c[q] = s_off[threadIdx.x * kBper + q];
+        sum += c[q];
+      }
+      int total = 0;
+      int run = block_excl_scan(sum, smi, total);
+#pragma unroll
+      for (int q = 0; q < kBper; ++q) {
+        s_off[threadIdx.x * kBper + q] = run;
+        run += c[q];
+      }
+      if (threadIdx.x == 0) s_off[kClusterBuckets] = total;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      if (bb[q] < 0) continue;
+      const int32_t at = s_off[bb[q]] + rk[q];
+      s_k[at] = kk[q];
+      s_h[at] = hh[q];
+      s_u[at] = uu[q];
+    }
+    __syncthreads();
+    // insertion sort of each bucket by home slot
+    for (int b = threadIdx.x; b < kClusterBuckets; b += blockDim.x) {
+      const int32_t lo = s_off[b], hi = s_off[b + 1];
+      for (int32_t i = lo + 1; i < hi; ++i) {
+        const uint32_t h = s_h[i];
+        const long long k = s_k[i];
+        const int32_t u = s_u[i];
+        int32_t j = i - 1;
+        while (j >= lo && s_h[j] > h) {
+          s_h[j + 1] = s_h[j];
+          s_k[j + 1] = s_k[j];
+          s_u[j + 1] = s_u[j];
+          --j;
+        }
+        s_h[j + 1] = h;
+        s_k[j + 1] = k;
+        s_u[j + 1] = u;
+      }
+    }
+    __syncthreads();
+    // clusters: a run ends where the next home slot is P or more further on
+    const int32_t N = ncur;
+    const bool wrap = N > 1 && ((int64_t)s_h[0] + g.C - (int64_t)s_h[N - 1]) < g.P;
+    int any_inner_head = 0;
+    for (int32_t i = 1 + threadIdx.x; i < N; i += blockDim.x)
+      any_inner_head |= ((int64_t)s_h[i] - (int64_t)s_h[i - 1]) >= g.P;
+    any_inner_head = __syncthreads_or(any_inner_head);
+    for (int32_t i = threadIdx.x; i < N; i += blockDim.x) {
+      bool head;
+      if (i == 0)
+        head = !wrap || !any_inner_head;
+      else
+        head = ((int64_t)s_h[i] - (int64_t)s_h[i - 1]) >= g.P;
+      if (!head) continue;
+      // members: i, i+1, ... up to (not including) the next head, cyclically
+      int32_t m = 1;
+      while (m < N) {
+        const int32_t j = (i + m) % N;
+        const bool jhead =
+            j == 0 ? (!wrap || !any_inner_head) : ((int64_t)s_h[j] - (int64_t)s_h[j - 1]) >= g.P;
+        if (jhead) break;
+        ++m;
+      }
+      // place the members in ascending key order (placed members marked -1)
+      for (int32_t done = 0; done < m; ++done) {
+        int32_t arg = -1;
+        long long kmin = 0;
+        for (int32_t t = 0; t < m; ++t) {
+          const int32_t j = (i + t) % N;
+          const long long k = s_k[j];
+          if (k >= 0 && (arg < 0 || k < kmin)) {
+            arg = j;
+            kmin = k;
+          }
+        }
+        place_key(p, kmin, s_u[arg], evicted);
+        s_k[arg] = -1;
+      }
+    }
+    rounds = N > 0;
+  }
   const long long ev = block_sum_ll(evicted, sm);
   if (threadIdx.x == 0) {
     if (ev) atomic_add_ll(&p.stats->n_evicted, ev);
@@ -695,31 +895,70 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
 }
 
 // ---------------------------------------------------------------------------
-// Writeback row update: M[r] <- fl(e_hat - fl(e_hat - e)) for every distinct id
-// still owning its row; one warp per row, 16-byte vectors, loads of a chunk
-// issued before its stores.
+// End of the row map: the write list holds (row, position of e) for every
+// distinct id that still owns its row after all inserts (a distinct id evicted
+// again later in the same step gets no write, n_dropped).  Also clears the
+// claims checked by the last grid-wide round (list 0's when there was none),
+// still set at this point, and writes the remaining counters.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kBlock) k_writeback(WbParams p) {
+__global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
+  pdl_enter();
   __shared__ long long sm[33];
-  const int lane = threadIdx.x & 31;
-  const long long U = p.ctr->n_unique;
+  __shared__ int smi[33];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  {
+    // clearing a window that is already clear is harmless
+    const int L = p.wide_rounds > 0 ? p.wide_rounds - 1 : 0;
+    const int32_t nl = p.ctr->cnt[L & 3];
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nl; i += stride)
+      clear_window(p.claims[L % 3], p.lkey[L % 3][i], p.g);
+  }
+  const int32_t U = p.ctr->n_unique;
   if (blockIdx.x == 0 && threadIdx.x == 0) p.stats->n_unique = U;
-  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   long long dropped = 0;
-  for (int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; u < U; u += warps) {
-    const int32_t r = __ldcg(p.urow + u);
-    if (r < 0 || __ldcg(p.keys + r) != __ldcg(p.ukey + u)) {  // evicted again in this step
-      dropped += lane == 0;
-      continue;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < U; base += stride) {
+    const int64_t u = base + threadIdx.x;
+    bool owned = false;
+    int32_t r = -1;
+    if (u < U) {
+      r = p.urow[u];
+      owned = r >= 0 && p.keys[r] == p.ukey[u];
+      dropped += !owned;
     }
-    float4* m = p.M + (int64_t)r * p.D4;
-    const float4* ev = p.e + (int64_t)__ldcg(p.upos + u) * p.D4;
-    for (int base = 0; base < p.D4; base += 4 * 32) {
+    int m = 0, unused = 0;
+    block_append2(owned, 0, p.wcount, p.wcount, m, unused, smi);
+    if (owned) {
+      p.wrow[m] = r;
+      p.wpos[m] = p.upos[u];
+    }
+  }
+  const long long d = block_sum_ll(dropped, sm);
+  if (threadIdx.x == 0 && d) atomic_add_ll(&p.stats->n_dropped, d);
+}
+
+// ---------------------------------------------------------------------------
+// Writeback row update: M[r] <- fl(e_hat - fl(e_hat - e)) for every entry of the
+// write list; one warp per row, 16-byte vectors, loads of a chunk issued
+// before its stores.  Reads only the write list, M and e.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict__ wrow,
+                                                      const int32_t* __restrict__ wpos,
+                                                      const int32_t* wcount,
+                                                      float4* __restrict__ M,
+                                                      const float4* __restrict__ e, int D4) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int32_t W = *wcount;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < W; w += warps) {
+    float4* m = M + (int64_t)wrow[w] * D4;
+    const float4* ev = e + (int64_t)wpos[w] * D4;
+    for (int base = 0; base < D4; base += 4 * 32) {
       float4 a[4], b[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
-        if (c < p.D4) {
+        if (c < D4) {
           a[q] = __ldcg(m + c);
           b[q] = __ldcs(ev + c);
         }
@@ -727,7 +966,7 @@ __global__ void __launch_bounds__(kBlock) k_writeback(WbParams p) {
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
-        if (c < p.D4) {
+        if (c < D4) {
           float4 o;
           o.x = __fsub_rn(a[q].x, __fsub_rn(a[q].x, b[q].x));
           o.y = __fsub_rn(a[q].y, __fsub_rn(a[q].y, b[q].y));
@@ -738,8 +977,6 @@ __global__ void __launch_bounds__(kBlock) k_writeback(WbParams p) {
       }
     }
   }
-  const long long d = block_sum_ll(dropped, sm);
-  if (threadIdx.x == 0 && d) atomic_add_ll(&p.stats->n_dropped, d);
 }
 
 // ---------------------------------------------------------------------------
@@ -749,6 +986,7 @@ __global__ void __launch_bounds__(kBlock) k_select_count(const long long* __rest
                                                          const long long* __restrict__ last,
                                                          int64_t C, long long since,
                                                          int32_t* __restrict__ bcount) {
+  pdl_enter();
   __shared__ long long sm[33];
   const int64_t base = (int64_t)blockIdx.x * kSelTile + threadIdx.x;
   int c = 0;
@@ -767,6 +1005,7 @@ __global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __re
                                                            const int32_t* __restrict__ bcount,
                                                            int32_t* __restrict__ rows_out,
                                                            long long* dev_count) {
+  pdl_enter();
   __shared__ long long sm[33];
   __shared__ int smi[33];
   long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
@@ -791,6 +1030,7 @@ __global__ void __launch_bounds__(kBlock) k_export_int8(
     const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C, int D4,
     char4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
     int32_t* status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   int64_t nn = n;
   if (dev_n) {
@@ -849,6 +1089,7 @@ __global__ void __launch_bounds__(kBlock) k_serve_gather(
     const float* __restrict__ scale, int D4, const long long* __restrict__ ids, int64_t n,
     int32_t* __restrict__ rows, uint8_t* __restrict__ hit, float4* __restrict__ out,
     int32_t* status) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += warps) {

@@ -173,6 +173,37 @@ MPZCH_API int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, i
 MPZCH_API int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
                     mpzch_wb_stats* dev_stats, void* stream);
 
+/* One multi-table training step in one call (Memory Layer section 2,
+ * Multi-Table paragraph: a labeled batch and an unlabeled candidate-pool batch
+ * are merged, the item tower runs once, one Writeback covers both, and the
+ * loss reads only the labeled part).  ids: device int64[n], the merged batch
+ * with its n_labeled labeled ids first (0 <= n_labeled <= n); e: device fp32
+ * [n][dim].  The call gives, bit for bit, the outputs of
+ *   mpzch_lookup(ids, n_labeled, rows, hit);
+ *   mpzch_gather_fused(rows, hit, n_labeled, ao_table, ao_nrows, ao_dim, ao_rows, out);
+ *   mpzch_writeback(ids, e, n, step, dev_stats);
+ * rows/hit/out/ao_* as in those calls (may be NULL when n_labeled == 0).
+ *
+ * Inside, the row map (dedup, refresh, the lookup, inserts) runs on a second
+ * stream of the table (MPZCH_OPT_SIDE_PRIORITY); the gather and the row update run on
+ * `stream`, the gather once the lookup is done and the row update once the
+ * row map is done.  Later work on `stream` is ordered after all of it (rows,
+ * hit, out, stats and the table are complete there).
+ *
+ * inputs_ready: NULL, or a cudaEvent_t (as void*) recorded after ids, e and
+ * ao_rows of this step were written.  With NULL the step starts after all
+ * earlier work on `stream`.  With an event the step's row map starts as soon
+ * as that event, the previous step's gather and the previous calls on the
+ * table allow -- so it overlaps the previous step's row update (pipelined
+ * steps, identical results).  Then the caller must also order every read of
+ * the previous step's rows, hit and stats buffers, if they are reused for
+ * this step, before inputs_ready. */
+MPZCH_API int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_labeled,
+                               const float* e, int64_t step, const float* ao_table,
+                               int64_t ao_nrows, int32_t ao_dim, const int32_t* ao_rows,
+                               int32_t* rows, uint8_t* hit, float* out,
+                               mpzch_wb_stats* dev_stats, void* inputs_ready, void* stream);
+
 /* Rows written recently (Memory Layer section 2, RES paragraph: fresh rows are
  * streamed to the predictors): rows_out (device int32[C]) receives, in
  * ascending order, every row r with keys[r] != -1 and last[r] >= since_step;
@@ -230,9 +261,13 @@ MPZCH_API int mpzch_trace_enable(mpzch_table* t, int32_t on);
 MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t nphases);
 
 /* Options.  MPZCH_OPT_WIDE_ROUNDS: number of grid-wide insert conflict rounds
- * launched before a single-block kernel runs the remaining rounds (default 4,
+ * launched before a single-block kernel places the remaining keys (default 3,
  * range 0..64).  Results do not depend on it. */
 #define MPZCH_OPT_WIDE_ROUNDS 1
+/* MPZCH_OPT_SIDE_PRIORITY: 1 = the side stream of mpzch_train_step gets the
+ * device's highest stream priority, 0 (default) = the lowest; only before the
+ * first mpzch_train_step of the table (MPZCH_EINVAL afterwards). */
+#define MPZCH_OPT_SIDE_PRIORITY 2
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 
 /* Test hook: the next `count` device allocations made by this library fail as

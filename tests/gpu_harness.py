@@ -68,7 +68,8 @@ def compare_state(tbl, orc, what: str, value_rows: Optional[np.ndarray] = None, 
 
 def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None, start: int = 0,
              state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
-             ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None) -> RunResult:
+             ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None,
+             fused_step: bool = False) -> RunResult:
     """Runs steps [start, start+steps) of workload w on both sides.
 
     Per step: lookup of the labeled ids, fused gather (with the always-on concat
@@ -94,9 +95,12 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
         e_d = torch.from_numpy(e).to(dev)
         aor = inputs.author_rows(w, ids[:lab])
         aor_d = torch.from_numpy(aor).to(dev) if aor is not None else None
-        rows_d, hit_d = tbl.lookup(ids_d[:lab])
-        out_d = tbl.gather_fused(rows_d, hit_d, ao_d, aor_d)
-        tbl.writeback(ids_d, e_d, t, stats_d)
+        if fused_step:
+            rows_d, hit_d, out_d = tbl.train_step(ids_d, lab, e_d, t, ao_d, aor_d, stats_d)
+        else:
+            rows_d, hit_d = tbl.lookup(ids_d[:lab])
+            out_d = tbl.gather_fused(rows_d, hit_d, ao_d, aor_d)
+            tbl.writeback(ids_d, e_d, t, stats_d)
         # oracle
         rc, orows, ohit = orc.lookup(ids[:lab])
         assert rc == 0
@@ -130,3 +134,53 @@ def snapshot_from_export(capacity: int, dim: int, rows: np.ndarray, q: np.ndarra
     snap_q[rows] = q
     snap_s[rows] = scale
     return snap_keys, snap_q, snap_s
+
+
+def run_pipelined(w: inputs.Workload, steps: Optional[int] = None):
+    """All steps' inputs uploaded first, then every step issued back to back as
+    a pipelined mpzch_train_step (inputs_ready = one event after the uploads),
+    each step with its own output buffers; then every output and the final
+    table are compared with the oracle run step by step."""
+    from hashed_sparse_table_b200 import binding
+    T = w.steps if steps is None else steps
+    tbl, orc = make_pair(w)
+    dev = tbl.device
+    ao = inputs.author_table(w)
+    ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None
+    host = []
+    for t in range(T):
+        ids = inputs.step_ids(w, t)
+        e = inputs.step_e(w, t, rows=ids.size)
+        host.append((ids, e, inputs.author_rows(w, ids[:w.labeled])))
+    dev_in = [(torch.from_numpy(i).to(dev), torch.from_numpy(e).to(dev),
+               None if a is None else torch.from_numpy(a).to(dev)) for i, e, a in host]
+    ready = torch.cuda.Event()
+    ready.record()
+    lab = w.labeled
+    width = w.dim + (0 if ao is None else ao.shape[1])
+    outs = []
+    for t in range(T):
+        ids_d, e_d, aor_d = dev_in[t]
+        rows = torch.empty(lab, dtype=torch.int32, device=dev)
+        hit = torch.empty(lab, dtype=torch.uint8, device=dev)
+        out = torch.empty((lab, width), dtype=torch.float32, device=dev)
+        st = torch.zeros(7, dtype=torch.int64, device=dev)
+        binding.mpzch_train_step(tbl.h, ids_d, lab, e_d, t, rows, hit, out, ao_d, aor_d, st,
+                                 inputs_ready=ready)
+        outs.append((rows, hit, out, st))
+    torch.cuda.synchronize()
+    for t in range(T):
+        ids, e, aor = host[t]
+        rows, hit, out, st = outs[t]
+        rc, orows, ohit = orc.lookup(ids[:lab])
+        oout = orc.gather_fused(orows, ohit, ao, aor)
+        rc, ost = orc.writeback(ids, e, t)
+        assert_bitwise(rows.cpu().numpy(), orows, f"pipelined step {t}: rows")
+        assert_bitwise(hit.cpu().numpy(), ohit, f"pipelined step {t}: hit")
+        assert_bitwise(out.cpu().numpy(), oout, f"pipelined step {t}: features")
+        gst = stats_dict(st)
+        for k in STATS_KEYS:
+            assert gst[k] == ost[k], (t, k, gst, ost)
+    compare_state(tbl, orc, "after pipelined steps")
+    assert tbl.status() == 0
+    return tbl, orc
