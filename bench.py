@@ -42,6 +42,11 @@ W = inputs.CFG3_MULTI
 METRIC = "unique rows/s through lookup+gather+writeback"
 UNIT = "unique rows/s"
 PREFILL = 20  # untimed steps that bring the table to its steady state
+# DRAM bytes (read + write) of one k_writeback launch of this workload, from
+# one ncu capture of the current kernel (profiles/k_writeback_multitable_c1m_d512.md)
+WB_TRAFFIC_BYTES = 544.69e6
+WB_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
+                     "(23rd step of the multi-table workload)")
 REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
 
 
@@ -312,7 +317,8 @@ def run_ours(args):
     # roofline of the dominant kernel (the Writeback row update)
     D, A = W.dim, W.ao_dim
     wb_ms, wb_launches = trace["writeback"]
-    wb_bytes = n_written * 12 * D + n_unique * 24  # e + M read, M write; 24 B of index data per id
+    # e row + M row read, M row written, 8 B of write-list entry per written row
+    wb_bytes = n_written * (12 * D + 8)
     g_ms, _ = trace["gather"]
     g_bytes = n_hit_lab * 4 * D + K * lab * (4 * A + 4 * (D + A) + 9)
     peak, peak_kind = load_peaks()
@@ -341,7 +347,8 @@ def run_ours(args):
             "gpu_launches": launches,
             "roofline": {"bound": "hbm", "kernel": "k_writeback", "achieved": wb_gbs,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": wb_gbs / peak, "traffic": None,
+                         "frac": wb_gbs / peak, "traffic": WB_TRAFFIC_BYTES,
+                         "traffic_source": WB_TRAFFIC_SOURCE,
                          "bytes_per_launch": wb_bytes / max(1, wb_launches),
                          "avg_launch_us": wb_ms * 1e3 / max(1, wb_launches)},
             "gather_writeback_gbs": gw_gbs,

@@ -349,7 +349,7 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
               long long* dev_count, WbStats* stats, cudaStream_t st) {
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
-  k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
+  k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
                                            stats, t->status, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
@@ -453,7 +453,7 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, int32_t*
   int rc;
   {
     PhaseScope ps(t, PH_DEDUP, st);
-    rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kBlock, st, false, p.ids, n,
+    rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false, p.ids, n,
                 t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status, p.wcount);
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
@@ -582,7 +582,7 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
     return MPZCH_ECUDA;
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
-  k_dedup_insert<<<tiles, kBlock, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
+  k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
                                            dev_status, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);

@@ -248,8 +248,9 @@ __device__ __forceinline__ long long block_sum_ll(long long v, long long* smem /
 // Block 0 also clears the step counters used by the later phases.
 // ---------------------------------------------------------------------------
 constexpr int kTileHash = 2 * kTile;  // shared-memory slots per tile (load <= 1/2)
+constexpr int kDedupThreads = kTile;  // one tile position per thread
 
-__global__ void __launch_bounds__(kBlock) k_dedup_insert(
+__global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
     WbStats* stats, int32_t* status, int32_t* wcount) {
@@ -269,87 +270,58 @@ __global__ void __launch_bounds__(kBlock) k_dedup_insert(
     s_pos[j] = kNoPos;
   }
   __syncthreads();
-  constexpr int kPer = kTile / kBlock;
-  const int64_t tile = (int64_t)blockIdx.x * kTile;
-  int lslot[kPer];
-  // 1. tile-local dedup (positions strided by the block size: coalesced loads)
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int64_t i = tile + q * kBlock + threadIdx.x;
-    lslot[q] = -1;
-    if (i >= n) continue;
+  // 1. tile-local dedup
+  const int64_t i = (int64_t)blockIdx.x * kTile + threadIdx.x;
+  int lslot = -1;
+  if (i < n) {
     const long long k = ids[i];
     if (k < 0) {
       slot_of[i] = -1;
       set_status(status, kStBadKey);
-      continue;
-    }
-    int j = (int)(splitmix64((uint64_t)k ^ 0x5851F42D4C957F2Dull) & (kTileHash - 1));
-    for (int probe = 0; probe < kTileHash; ++probe) {
-      const unsigned long long cur = atomicCAS(&s_key[j], kEmptyKey, (unsigned long long)k);
-      if (cur == kEmptyKey || cur == (unsigned long long)k) {
-        atomicMin(&s_pos[j], (uint32_t)i);
-        lslot[q] = j;
-        break;
+    } else {
+      int j = (int)(splitmix64((uint64_t)k ^ 0x5851F42D4C957F2Dull) & (kTileHash - 1));
+      for (int probe = 0; probe < kTileHash; ++probe) {
+        const unsigned long long cur = atomicCAS(&s_key[j], kEmptyKey, (unsigned long long)k);
+        if (cur == kEmptyKey || cur == (unsigned long long)k) {
+          atomicMin(&s_pos[j], (uint32_t)i);
+          lslot = j;
+          break;
+        }
+        j = (j + 1) & (kTileHash - 1);
       }
-      j = (j + 1) & (kTileHash - 1);
     }
   }
   __syncthreads();
-  // 2. one global insert per distinct id of the tile: compact the occupied
-  //    shared slots, then every thread issues the first probe of its (at most
-  //    kPer) ids together; a collision falls back to linear probing.
+  // 2. one global insert per distinct id of the tile (compacted: at most one
+  //    per thread); a collision falls back to linear probing.
   {
-    int occ = 0;
-    constexpr int kSlotsPer = kTileHash / kBlock;
-#pragma unroll
-    for (int q = 0; q < kSlotsPer; ++q) occ += s_key[threadIdx.x * kSlotsPer + q] != kEmptyKey;
+    const int occ = (s_key[2 * threadIdx.x] != kEmptyKey) + (s_key[2 * threadIdx.x + 1] != kEmptyKey);
     int total = 0;
     int at = block_excl_scan(occ, s_scan, total);
-#pragma unroll
-    for (int q = 0; q < kSlotsPer; ++q) {
-      const int j = threadIdx.x * kSlotsPer + q;
-      if (s_key[j] != kEmptyKey) s_list[at++] = j;
-    }
+    if (s_key[2 * threadIdx.x] != kEmptyKey) s_list[at++] = (int16_t)(2 * threadIdx.x);
+    if (s_key[2 * threadIdx.x + 1] != kEmptyKey) s_list[at++] = (int16_t)(2 * threadIdx.x + 1);
     __syncthreads();
-    unsigned long long kk[kPer], cur[kPer];
-    int64_t ss[kPer];
-    int jj[kPer];
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      const int e = threadIdx.x + q * kBlock;
-      jj[q] = e < total ? s_list[e] : -1;
-      kk[q] = jj[q] >= 0 ? s_key[jj[q]] : 0;
-      ss[q] = (int64_t)(splitmix64(kk[q] ^ 0xD6E8FEB86659FD93ull) & hmask);
-    }
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) cur[q] = jj[q] >= 0 ? __ldcg(hkey + ss[q]) : 0;
-#pragma unroll
-    for (int q = 0; q < kPer; ++q)
-      if (jj[q] >= 0 && cur[q] == kEmptyKey) cur[q] = atomicCAS(hkey + ss[q], kEmptyKey, kk[q]);
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      if (jj[q] < 0) continue;
-      int64_t sl = ss[q];
-      bool placed = cur[q] == kEmptyKey || cur[q] == kk[q];
+    if ((int)threadIdx.x < total) {
+      const int jj = s_list[threadIdx.x];
+      const unsigned long long kk = s_key[jj];
+      int64_t sl = (int64_t)(splitmix64(kk ^ 0xD6E8FEB86659FD93ull) & hmask);
+      unsigned long long cur = __ldcg(hkey + sl);
+      if (cur == kEmptyKey) cur = atomicCAS(hkey + sl, kEmptyKey, kk);
+      bool placed = cur == kEmptyKey || cur == kk;
       for (uint64_t probe = 1; probe <= hmask && !placed; ++probe) {
         sl = (sl + 1) & (int64_t)hmask;
         unsigned long long c = __ldcg(hkey + sl);
-        if (c == kEmptyKey) c = atomicCAS(hkey + sl, kEmptyKey, kk[q]);
-        placed = c == kEmptyKey || c == kk[q];
+        if (c == kEmptyKey) c = atomicCAS(hkey + sl, kEmptyKey, kk);
+        placed = c == kEmptyKey || c == kk;
       }
       if (!placed) set_status(status, kStInternal);  // scratch hash sized >= 2n: never expected
-      atomicMin(hpos + sl, s_pos[jj[q]]);
-      s_gslot[jj[q]] = (int32_t)sl;
+      atomicMin(hpos + sl, s_pos[jj]);
+      s_gslot[jj] = (int32_t)sl;
     }
   }
   __syncthreads();
   // 3. every position learns the global slot of its id
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int64_t i = tile + q * kBlock + threadIdx.x;
-    if (i < n && lslot[q] >= 0) slot_of[i] = s_gslot[lslot[q]];
-  }
+  if (i < n && lslot >= 0) slot_of[i] = s_gslot[lslot];
 }
 
 // Sum of cnt[0 .. upto) by the whole block.
