@@ -37,7 +37,9 @@ class WbStats(C.Structure):
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # MPZCH_ORACLE_LIB lets the mutation tests load a deliberately broken
+        # copy of the oracle; normally the library is built from this folder.
+        path = os.environ.get("MPZCH_ORACLE_LIB") or _build.build()
         L = C.CDLL(path)
         p = C.c_void_p
         i64, i32 = C.c_int64, C.c_int32

@@ -1,0 +1,74 @@
+"""The oracle's pins catch planted mistakes (no GPU needed).
+
+Each case copies the oracle source to a temporary folder, plants one plausible
+mistake there by a textual edit (a dropped term, a wrong comparison, order,
+constant or rounding), builds that copy, and runs the pin suite
+(tests/test_oracle_pins.py) against it in a subprocess.  The suite must fail
+for every mutant.  The oracle in oracle/ itself is never modified.
+"""
+import os
+import shutil
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "mpzch_oracle.cpp")
+HDR = os.path.join(ROOT, "oracle", "mpzch_oracle.h")
+
+# (name, text in the oracle, replacement)
+MUTANTS = [
+    ("hash: final xor-shift dropped", "return z ^ (z >> 31);", "return z;"),
+    ("lookup: window one slot short",
+     "  for (int32_t j = 0; j < t->P; ++j) {\n    int64_t s = window_slot(t, key, j);\n    if (t->keys[s] == key && found < 0) found = s;",
+     "  for (int32_t j = 0; j + 1 < t->P; ++j) {\n    int64_t s = window_slot(t, key, j);\n    if (t->keys[s] == key && found < 0) found = s;"),
+    ("lookup: stops at the first empty slot",
+     "if (t->keys[s] == key && found < 0) found = s;",
+     "if (t->keys[s] == -1) break;\n    if (t->keys[s] == key && found < 0) found = s;"),
+    ("victim: ties broken by probe order, not row index",
+     "(t->last[s] == t->last[best] && s < best)", "false"),
+    ("victim: most recently used instead of least",
+     "t->last[s] < t->last[best] ||", "t->last[s] > t->last[best] ||"),
+    ("resident ids not refreshed", "      t->last[r] = step;\n", "\n"),
+    ("missing ids inserted in descending key order",
+     "return uniq[a] < uniq[b];", "return uniq[a] > uniq[b];"),
+    ("evictions not counted", "if (t->keys[best] != -1) ++n_evicted;", ""),
+    ("Writeback stores e instead of e_hat - (e_hat - e)",
+     "m[d] = e_hat - g;", "m[d] = ek[d];"),
+    ("Writeback sign flipped", "float g = e_hat - ek[d];", "float g = ek[d] - e_hat;"),
+    ("dedup keeps the last occurrence",
+     "    if (first.emplace(ids[i], i).second) {\n      uniq[u] = ids[i];\n      pos[u] = i;\n      ++u;\n    }",
+     "    auto it = first.find(ids[i]);\n    if (it == first.end()) {\n      first.emplace(ids[i], u);\n      uniq[u] = ids[i];\n      pos[u] = i;\n      ++u;\n    } else {\n      pos[it->second] = i;\n    }"),
+    ("miss feature is -0.0", "o[d] = 0.0f;", "o[d] = -0.0f;"),
+    ("select uses > instead of >=", "t->last[r] >= since", "t->last[r] > since"),
+    ("int8 scale divides by 128", "const float s = a / 127.0f;", "const float s = a / 128.0f;"),
+    ("int8 rounds by truncation", "float v = std::nearbyint(x[d] / s);",
+     "float v = std::trunc(x[d] / s);"),
+    ("serving divides by the scale",
+     "(float)snap_q[r * (int64_t)dim + d] * snap_scale[r]",
+     "(float)snap_q[r * (int64_t)dim + d] / snap_scale[r]"),
+]
+
+
+def build_mutant(tmp, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique: {old!r}"
+    with open(os.path.join(tmp, "mpzch_oracle.cpp"), "w") as f:
+        f.write(src.replace(old, new))
+    shutil.copy(HDR, os.path.join(tmp, "mpzch_oracle.h"))
+    lib = os.path.join(tmp, "libmutant.so")
+    subprocess.run(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+                    "-shared", os.path.join(tmp, "mpzch_oracle.cpp"), "-o", lib], check=True)
+    return lib
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(tmp_path, name, old, new):
+    lib = build_mutant(str(tmp_path), old, new)
+    env = dict(os.environ, MPZCH_ORACLE_LIB=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join("tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode != 0, f"planted mistake survived every pin: {name}\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout, r.stdout[-2000:]
