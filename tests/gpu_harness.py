@@ -154,20 +154,21 @@ def run_pipelined(w: inputs.Workload, steps: Optional[int] = None):
         host.append((ids, e, inputs.author_rows(w, ids[:w.labeled])))
     dev_in = [(torch.from_numpy(i).to(dev), torch.from_numpy(e).to(dev),
                None if a is None else torch.from_numpy(a).to(dev)) for i, e, a in host]
-    ready = torch.cuda.Event()
-    ready.record()
     lab = w.labeled
     width = w.dim + (0 if ao is None else ao.shape[1])
-    outs = []
+    # every buffer a pipelined step writes exists before the inputs-ready event
+    # (the counters are cleared by the library itself)
+    outs = [(torch.empty(lab, dtype=torch.int32, device=dev),
+             torch.empty(lab, dtype=torch.uint8, device=dev),
+             torch.empty((lab, width), dtype=torch.float32, device=dev),
+             torch.empty(7, dtype=torch.int64, device=dev)) for _ in range(T)]
+    ready = torch.cuda.Event()
+    ready.record()
     for t in range(T):
         ids_d, e_d, aor_d = dev_in[t]
-        rows = torch.empty(lab, dtype=torch.int32, device=dev)
-        hit = torch.empty(lab, dtype=torch.uint8, device=dev)
-        out = torch.empty((lab, width), dtype=torch.float32, device=dev)
-        st = torch.zeros(7, dtype=torch.int64, device=dev)
+        rows, hit, out, st = outs[t]
         binding.mpzch_train_step(tbl.h, ids_d, lab, e_d, t, rows, hit, out, ao_d, aor_d, st,
                                  inputs_ready=ready)
-        outs.append((rows, hit, out, st))
     torch.cuda.synchronize()
     for t in range(T):
         ids, e, aor = host[t]

@@ -1,6 +1,8 @@
 """CUDA path vs CPU oracle at the full workload sizes, through the same calls
-and launch configuration the benchmark times (mpzch_reserve for the batch, then
-lookup -> fused gather -> Writeback per step on the current stream).
+and launch configuration the benchmark times: mpzch_reserve for the batch, then
+one pipelined mpzch_train_step per step (lookup -> fused gather -> Writeback,
+with an inputs-ready event so a step's row map overlaps the previous step's
+row update), the item-tower target pool resident on the device.
 
 * 1M rows x 512, 8 probes, 100 steps of 65,536 ids (Zipf 1.1 over 20M + 15%
   fresh): every lookup row / hit and Writeback counter, the identity map and
@@ -40,7 +42,11 @@ class Pool:
         return self.host[t % inputs.E_POOL], self.dev[t % inputs.E_POOL]
 
 
-def run_full(w, check_state_every, full_gather_every, value_rows=None, gather_sample=2048):
+def run_full(w, check_state_every, full_gather_every, value_rows=None, gather_sample=2048,
+             chunk=10):
+    """Steps are issued as the benchmark issues them: pipelined mpzch_train_step
+    calls with an inputs-ready event, `chunk` steps at a time with their own
+    output buffers; then each step is checked against the oracle in order."""
     from hashed_sparse_table_b200 import binding
     dev = torch.device("cuda", torch.cuda.current_device())
     tbl = binding.MpzchTable(w.capacity, w.dim, w.probes)
@@ -53,39 +59,56 @@ def run_full(w, check_state_every, full_gather_every, value_rows=None, gather_sa
     pool = Pool(w, dev)
     ao = inputs.author_table(w)
     ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None
-    stats_d = torch.zeros(7, dtype=torch.int64, device=dev)
     lab = w.labeled
+    width = w.dim + (0 if ao is None else ao.shape[1])
     rng = np.random.default_rng(99)
-    for t in range(w.steps):
-        ids = inputs.step_ids(w, t)
-        e_h, e_d = pool(t)
-        aor = inputs.author_rows(w, ids[:lab])
-        ids_d = torch.from_numpy(ids).to(dev)
-        aor_d = torch.from_numpy(aor).to(dev) if aor is not None else None
-        rows_d, hit_d = tbl.lookup(ids_d[:lab])
-        out_d = tbl.gather_fused(rows_d, hit_d, ao_d, aor_d)
-        tbl.writeback(ids_d, e_d, t, stats_d)
-        rc, orows, ohit = orc.lookup(ids[:lab])
-        assert rc == 0
-        assert_bitwise(rows_d.cpu().numpy(), orows, f"step {t}: rows")
-        assert_bitwise(hit_d.cpu().numpy(), ohit, f"step {t}: hit")
-        # gathered features: all rows every few steps, a sample otherwise; with a
-        # value-row sample only positions whose row is kept (or misses) are checked
-        if t % full_gather_every == 0 or t == w.steps - 1:
-            pos = np.arange(lab)
-        else:
-            pos = np.sort(rng.choice(lab, size=min(gather_sample, lab), replace=False))
-        if value_rows is not None:
-            pos = pos[(ohit[pos] == 0) | tracked[np.maximum(orows[pos], 0)]]
-        oout = orc.gather_fused(orows[pos], ohit[pos], ao, None if aor is None else aor[pos])
-        got = out_d[torch.from_numpy(pos).to(dev)].cpu().numpy()
-        assert_bitwise(got, oout, f"step {t}: gathered features")
-        rc, ost = orc.writeback(ids, e_h, t)
-        assert rc == 0
-        gst = stats_dict(stats_d)
-        for k in STATS_KEYS:
-            assert gst[k] == ost[k], (t, k, gst, ost)
-        if t % check_state_every == 0 or t == w.steps - 1:
+    assert check_state_every % chunk == 0
+    for c0 in range(0, w.steps, chunk):
+        steps = list(range(c0, min(c0 + chunk, w.steps)))
+        host = {t: inputs.step_ids(w, t) for t in steps}
+        aor = {t: inputs.author_rows(w, host[t][:lab]) for t in steps}
+        dev_ids = {t: torch.from_numpy(host[t]).to(dev) for t in steps}
+        dev_aor = {t: None if aor[t] is None else torch.from_numpy(aor[t]).to(dev) for t in steps}
+        # every buffer a pipelined step writes exists before the inputs-ready event
+        # (the counters are cleared by the library itself)
+        outs = {t: (torch.empty(lab, dtype=torch.int32, device=dev),
+                    torch.empty(lab, dtype=torch.uint8, device=dev),
+                    torch.empty((lab, width), dtype=torch.float32, device=dev),
+                    torch.empty(7, dtype=torch.int64, device=dev)) for t in steps}
+        ready = torch.cuda.Event()
+        ready.record()
+        for t in steps:
+            rows, hit, out, st = outs[t]
+            binding.mpzch_train_step(tbl.h, dev_ids[t], lab, pool(t)[1], t, rows, hit, out, ao_d,
+                                     dev_aor[t], st, inputs_ready=ready)
+        torch.cuda.synchronize()
+        for t in steps:
+            ids = host[t]
+            rows_d, hit_d, out_d, st_d = outs[t]
+            rc, orows, ohit = orc.lookup(ids[:lab])
+            assert rc == 0
+            assert_bitwise(rows_d.cpu().numpy(), orows, f"step {t}: rows")
+            assert_bitwise(hit_d.cpu().numpy(), ohit, f"step {t}: hit")
+            # gathered features: all rows every few steps, a sample otherwise; with a
+            # value-row sample only positions whose row is kept (or misses) are checked
+            if t % full_gather_every == 0 or t == w.steps - 1:
+                pos = np.arange(lab)
+            else:
+                pos = np.sort(rng.choice(lab, size=min(gather_sample, lab), replace=False))
+            if value_rows is not None:
+                pos = pos[(ohit[pos] == 0) | tracked[np.maximum(orows[pos], 0)]]
+            a = aor[t]
+            oout = orc.gather_fused(orows[pos], ohit[pos], ao, None if a is None else a[pos])
+            got = out_d[torch.from_numpy(pos).to(dev)].cpu().numpy()
+            assert_bitwise(got, oout, f"step {t}: gathered features")
+            rc, ost = orc.writeback(ids, pool(t)[0], t)
+            assert rc == 0
+            gst = stats_dict(st_d)
+            for k in STATS_KEYS:
+                assert gst[k] == ost[k], (t, k, gst, ost)
+        del outs
+        t = steps[-1]
+        if (t + 1) % check_state_every == 0 or t == w.steps - 1:
             keys, last, _ = tbl.state()
             ok, ol, _ = orc.state()
             assert_bitwise(keys.cpu().numpy(), ok, f"step {t}: keys")
@@ -150,5 +173,5 @@ def test_full_16m_rows_capacity_stress():
     w = inputs.CFG4_16M
     sample = np.sort(np.random.default_rng(4).choice(w.capacity, size=8192, replace=False))
     tbl, orc = run_full(w, check_state_every=20, full_gather_every=25,
-                        value_rows=sample.astype(np.int32))
+                        value_rows=sample.astype(np.int32), chunk=10)
     tbl.close()
