@@ -55,6 +55,7 @@ def lib():
         L.orc_gather_fused.argtypes = [p, p, p, i64, p, i64, i32, p, p]
         L.orc_dedup.argtypes = [p, i64, p, p, p]
         L.orc_writeback.argtypes = [p, p, p, i64, i64, p]
+        L.orc_set_learning_rate.argtypes = [p, C.c_float]
         L.orc_select_written_since.argtypes = [p, i64, p, p]
         L.orc_quantize_row.argtypes = [p, i32, p, p]
         L.orc_export_int8.argtypes = [p, p, i64, p, p, p]
@@ -67,7 +68,7 @@ def lib():
         for f in ("orc_create", "orc_track_rows", "orc_lookup", "orc_gather_fused", "orc_dedup",
                   "orc_writeback", "orc_select_written_since", "orc_quantize_row",
                   "orc_export_int8", "orc_serve_gather", "orc_state", "orc_get_row",
-                  "orc_set_row", "orc_set_state", "orc_get_rows"):
+                  "orc_set_row", "orc_set_state", "orc_get_rows", "orc_set_learning_rate"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -180,6 +181,10 @@ class OracleTable:
         st = WbStats()
         rc = lib().orc_writeback(self.h, _ptr(ids), _ptr(e), ids.size, step, C.byref(st))
         return rc, st.as_dict()
+
+    def set_learning_rate(self, eta):
+        rc = lib().orc_set_learning_rate(self.h, float(eta))
+        assert rc == ORC_OK, rc
 
     def select_written_since(self, since):
         out = np.empty(self.capacity, np.int32)

@@ -19,6 +19,9 @@
 //  * Memory Layer section 2, Writeback paragraph: gradient g = e_hat - e,
 //    exact SGD with learning rate 1, M[i] <- e_hat - (e_hat - e); duplicate
 //    ids of one batch are deduplicated first so each row gets one exact write.
+//    The same paragraph compares it with minimising ||M[i] - sg(e_i)||^2,
+//    whose SGD step with rate a is the same update with learning rate 2a;
+//    orc_set_learning_rate covers that general step.
 //  * Memory Layer section 2, always-on paragraph: on a miss the cached branch
 //    is zeroed and the always-on (author id) embedding remains.
 //  * Memory Layer section 2, RES paragraph and section 5: streamed rows are
@@ -43,6 +46,7 @@ struct orc_table {
   std::vector<float> M;       // value rows (track_all)
   std::unordered_map<int32_t, std::vector<float>> tracked;  // value rows (!track_all)
   int64_t last_step;
+  float eta;  // learning rate of the SGD step (1: Writeback)
 };
 
 extern "C" uint64_t orc_splitmix64(uint64_t x) {
@@ -98,6 +102,7 @@ extern "C" int orc_create(int64_t capacity, int32_t dim, int32_t probes, int32_t
     t->last.assign((size_t)capacity, -1);
     if (t->track_all) t->M.assign((size_t)capacity * dim, 0.0f);
     t->last_step = -1;
+    t->eta = 1.0f;
   } catch (...) {
     delete t;
     return ORC_ENOMEM;
@@ -231,10 +236,12 @@ extern "C" int orc_writeback(orc_table* t, const int64_t* ids, const float* e, i
     row_of[u] = best;
   }
 
-  // 4. Writeback: every key still owning its row gets
-  //    M[r] <- e_hat - (e_hat - e), e_hat = the row's content before this step.
-  //    A row is owned by at most one key, so each row is read and written once
-  //    and reading it here still gives its pre-step content.
+  // 4. Writeback: every key still owning its row gets the SGD step with
+  //    gradient g = e_hat - e and learning rate eta,
+  //    M[r] <- e_hat - eta * g   (eta = 1: M[r] <- e_hat - (e_hat - e)),
+  //    e_hat = the row's content before this step.  A row is owned by at most
+  //    one key, so each row is read and written once and reading it here still
+  //    gives its pre-step content.
   int64_t n_dropped = 0;
   for (int64_t u = 0; u < U; ++u) {
     int64_t r = row_of[u];
@@ -248,7 +255,8 @@ extern "C" int orc_writeback(orc_table* t, const int64_t* ids, const float* e, i
     for (int32_t d = 0; d < t->D; ++d) {
       float e_hat = m[d];
       float g = e_hat - ek[d];  // Writeback gradient
-      m[d] = e_hat - g;         // SGD step, learning rate 1
+      float step_d = t->eta * g;  // rounded before the subtraction (no FMA)
+      m[d] = e_hat - step_d;      // SGD step
     }
   }
   t->last_step = step;
@@ -264,6 +272,12 @@ extern "C" int orc_writeback(orc_table* t, const int64_t* ids, const float* e, i
     stats->n_dropped = n_dropped;
   }
   return rc;
+}
+
+extern "C" int orc_set_learning_rate(orc_table* t, float eta) {
+  if (!t || !std::isfinite(eta)) return ORC_EINVAL;
+  t->eta = eta;
+  return ORC_OK;
 }
 
 // Rows (ascending) whose key is live and whose last write is at or after `since`.

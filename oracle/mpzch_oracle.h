@@ -55,6 +55,9 @@ int orc_gather_fused(const orc_table* t, const int32_t* rows, const uint8_t* hit
 int orc_dedup(const int64_t* ids, int64_t n, int64_t* uniq, int64_t* pos, int64_t* n_unique);
 int orc_writeback(orc_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step,
                   orc_wb_stats* stats);
+/* Learning rate eta of the Writeback step M <- e_hat - eta * (e_hat - e)
+ * (default 1: the exact assignment). */
+int orc_set_learning_rate(orc_table* t, float eta);
 int orc_select_written_since(const orc_table* t, int64_t since, int32_t* rows_out, int64_t* count);
 int orc_quantize_row(const float* x, int32_t dim, int8_t* q, float* scale);
 int orc_export_int8(const orc_table* t, const int32_t* rows, int64_t n, int8_t* q, float* scale,

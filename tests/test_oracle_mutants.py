@@ -35,7 +35,8 @@ MUTANTS = [
      "return uniq[a] < uniq[b];", "return uniq[a] > uniq[b];"),
     ("evictions not counted", "if (t->keys[best] != -1) ++n_evicted;", ""),
     ("Writeback stores e instead of e_hat - (e_hat - e)",
-     "m[d] = e_hat - g;", "m[d] = ek[d];"),
+     "m[d] = e_hat - step_d;", "m[d] = ek[d];"),
+    ("learning rate ignored", "float step_d = t->eta * g;", "float step_d = g;"),
     ("Writeback sign flipped", "float g = e_hat - ek[d];", "float g = ek[d] - e_hat;"),
     ("dedup keeps the last occurrence",
      "    if (first.emplace(ids[i], i).second) {\n      uniq[u] = ids[i];\n      pos[u] = i;\n      ++u;\n    }",

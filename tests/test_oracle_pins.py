@@ -209,6 +209,62 @@ def test_writeback_hand_worked_binary32_cases():
         assert got.view(np.uint32).tolist() == [np.float32(want).view(np.uint32)] * 4, case["why"]
 
 
+def _val_eta(s):
+    s = s.strip()
+    if "/" in s:
+        a, b = s.split("/")
+        return float(np.float32(float(a) / float(b)))
+    return _val(s)
+
+
+def test_writeback_learning_rate_hand_worked_cases():
+    g = load("writeback_eta_cases.json")
+    for case in g["cases"]:
+        e_hat, e, eta = (np.float32(_val_eta(case[k])) for k in ("e_hat", "e", "eta"))
+        want = np.float32(float(case["expect"]))
+        T = OracleTable(8, 4, 8)
+        k = np.array([11])
+        T.writeback(k, np.zeros((1, 4), np.float32), 0)
+        r = int(T.lookup(k)[1][0])
+        T.set_row(r, np.full(4, e_hat, np.float32))
+        T.set_learning_rate(eta)
+        T.writeback(k, np.full((1, 4), e, np.float32), 1)
+        got = T.row(r)
+        assert got.view(np.uint32).tolist() == [want.view(np.uint32)] * 4, case["why"]
+
+
+def test_writeback_learning_rate_zero_keeps_every_value():
+    rng = np.random.default_rng(21)
+    T = OracleTable(128, 8, 4)
+    for t in range(3):
+        ids = rng.integers(0, 300, size=60).astype(np.int64)
+        T.writeback(ids, rng.standard_normal((60, 8)).astype(np.float32), t)
+    before = T.values()
+    T.set_learning_rate(0.0)
+    ids = rng.integers(0, 300, size=60).astype(np.int64)
+    T.writeback(ids, rng.standard_normal((60, 8)).astype(np.float32), 3)
+    np.testing.assert_array_equal(T.values(), before)
+
+
+@pytest.mark.parametrize("eta", [0.5, 0.1, 0.9])
+def test_writeback_learning_rate_is_an_ema_toward_the_target(eta):
+    """Repeated steps toward a fixed target from a zero row follow the closed
+    form M_k = e (1 - (1 - eta)^k) up to k binary32 roundings."""
+    rng = np.random.default_rng(22)
+    e = rng.standard_normal((1, 16)).astype(np.float32)
+    T = OracleTable(16, 16, 4)
+    T.set_learning_rate(eta)
+    key = np.array([5])
+    T.writeback(key, np.zeros((1, 16), np.float32), 0)  # insert; row stays 0
+    r = int(T.lookup(key)[1][0])
+    for k in range(1, 40):
+        T.writeback(key, e, k)
+        eta32 = float(np.float32(eta))
+        exact = e[0].astype(np.float64) * (1.0 - (1.0 - eta32) ** k)
+        bound = k * 4 * 2.0 ** -24 * np.abs(e[0]).astype(np.float64) + 1e-30
+        assert (np.abs(T.row(r).astype(np.float64) - exact) <= bound).all(), k
+
+
 def test_writeback_from_empty_table_is_exact_and_first_occurrence():
     rng = np.random.default_rng(7)
     T = OracleTable(1024, 16, 8)
