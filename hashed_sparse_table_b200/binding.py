@@ -61,6 +61,7 @@ _SIGS = {
     "mpzch_trace_read": [_p, C.POINTER(C.c_double), C.POINTER(_i64), _i32],
     "mpzch_set_option": [_p, _i32, _i64],
     "mpzch_debug_fail_allocs": [_i32],
+    "mpzch_set_learning_rate": [_p, C.c_float],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -261,6 +262,10 @@ def mpzch_trace_read(h):
 
 def mpzch_set_option(h, option: int, value: int) -> None:
     _check("mpzch_set_option", _lib.mpzch_set_option(h, option, value))
+
+
+def mpzch_set_learning_rate(h, eta: float) -> None:
+    _check("mpzch_set_learning_rate", _lib.mpzch_set_learning_rate(h, float(eta)))
 
 
 def mpzch_debug_fail_allocs(count: int) -> None:

@@ -179,6 +179,7 @@ struct mpzch_table {
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
   int side_high_priority = 0;  // priority of the side stream (set before its first use)
+  float eta = 1.0f;            // learning rate of the Writeback step
   // mpzch_train_step: the row map runs on a second (high-priority) stream
   cudaStream_t side = nullptr;
   cudaEvent_t ev_fork = nullptr, ev_lookup = nullptr, ev_map = nullptr;
@@ -480,7 +481,7 @@ int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool 
     PhaseScope ps(t, PH_WRITEBACK, st);
     const int rc = launch(k_writeback, grid_for(p.n * 32, kBlock), kBlock, st, pdl,
                           (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount,
-                          p.M, p.e, p.D4);
+                          p.M, p.e, p.D4, t->eta);
     if (rc) return rc;
   }
   if (t->side && cudaEventRecord(t->ev_update[t->wset], st) != cudaSuccess) return MPZCH_ECUDA;
@@ -922,6 +923,12 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     return MPZCH_OK;
   }
   return MPZCH_EINVAL;
+}
+
+int mpzch_set_learning_rate(mpzch_table* t, float eta) {
+  if (!t || !(eta == eta) || eta > 3.0e38f || eta < -3.0e38f) return MPZCH_EINVAL;
+  t->eta = eta;
+  return MPZCH_OK;
 }
 
 int mpzch_debug_fail_allocs(int32_t count) {

@@ -909,15 +909,16 @@ __global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// Writeback row update: M[r] <- fl(e_hat - fl(e_hat - e)) for every entry of the
-// write list; one warp per row, 16-byte vectors, loads of a chunk issued
+// Writeback row update: M[r] <- fl(e_hat - fl(eta * fl(e_hat - e))) (eta = 1:
+// the exact Writeback) for every entry of the write list; one warp per row, 16-byte vectors, loads of a chunk issued
 // before its stores.  Reads only the write list, M and e.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict__ wrow,
                                                       const int32_t* __restrict__ wpos,
                                                       const int32_t* wcount,
                                                       float4* __restrict__ M,
-                                                      const float4* __restrict__ e, int D4) {
+                                                      const float4* __restrict__ e, int D4,
+                                                      float eta) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int32_t W = *wcount;
@@ -939,11 +940,14 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
         if (c < D4) {
+          // SGD step with gradient g = e_hat - e: M <- e_hat - fl(eta * g); every
+          // operation rounded separately (eta = 1: e_hat - (e_hat - e) exactly,
+          // since fl(1 * g) = g)
           float4 o;
-          o.x = __fsub_rn(a[q].x, __fsub_rn(a[q].x, b[q].x));
-          o.y = __fsub_rn(a[q].y, __fsub_rn(a[q].y, b[q].y));
-          o.z = __fsub_rn(a[q].z, __fsub_rn(a[q].z, b[q].z));
-          o.w = __fsub_rn(a[q].w, __fsub_rn(a[q].w, b[q].w));
+          o.x = __fsub_rn(a[q].x, __fmul_rn(eta, __fsub_rn(a[q].x, b[q].x)));
+          o.y = __fsub_rn(a[q].y, __fmul_rn(eta, __fsub_rn(a[q].y, b[q].y)));
+          o.z = __fsub_rn(a[q].z, __fmul_rn(eta, __fsub_rn(a[q].z, b[q].z)));
+          o.w = __fsub_rn(a[q].w, __fmul_rn(eta, __fsub_rn(a[q].w, b[q].w)));
           m[c] = o;
         }
       }

@@ -270,6 +270,16 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
 #define MPZCH_OPT_SIDE_PRIORITY 2
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 
+/* Learning rate of the Writeback step for the following calls (Memory Layer
+ * section 2, Writeback paragraph: the exact step is SGD at rate 1 on
+ * g = e_hat - e; the alternative it is compared with, minimising
+ * ||M[i] - sg(e_i)||^2, is the same SGD step at rate 2a for loss rate a; an
+ * EMA cache c <- alpha c + (1 - alpha) v is the step at 1 - alpha).  Every
+ * written row becomes M[r] <- fl(e_hat - fl(eta * fl(e_hat - e))); eta = 1
+ * (the default) is the exact Writeback M[r] <- e_hat - (e_hat - e).  eta must
+ * be finite (MPZCH_EINVAL otherwise).  Host-side only; affects later calls. */
+MPZCH_API int mpzch_set_learning_rate(mpzch_table* t, float eta);
+
 /* Test hook: the next `count` device allocations made by this library fail as
  * if the device were out of memory (no CUDA call is made for them). */
 MPZCH_API int mpzch_debug_fail_allocs(int32_t count);

@@ -69,7 +69,7 @@ def compare_state(tbl, orc, what: str, value_rows: Optional[np.ndarray] = None, 
 def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None, start: int = 0,
              state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
              ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None,
-             fused_step: bool = False) -> RunResult:
+             fused_step: bool = False, eta: Optional[float] = None) -> RunResult:
     """Runs steps [start, start+steps) of workload w on both sides.
 
     Per step: lookup of the labeled ids, fused gather (with the always-on concat
@@ -81,6 +81,9 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
         tbl, orc = make_pair(w)
     if wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, wide_rounds)
+    if eta is not None:
+        binding.mpzch_set_learning_rate(tbl.h, eta)
+        orc.set_learning_rate(eta)
     T = w.steps if steps is None else steps
     dev = tbl.device
     ao = inputs.author_table(w)

@@ -97,6 +97,20 @@ def test_insert_rounds_split_does_not_change_results(wide):
     assert sum(s["n_dropped"] for s in r.stats) > 0
 
 
+@pytest.mark.parametrize("eta", [0.5, 0.1, 2.0 / 3.0, 0.0, 1.75])
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress"])
+def test_learning_rate_writeback_bit_exact(name, eta):
+    run_pair(SCALED[name], eta=eta, fused_step=True)
+
+
+def test_learning_rate_rejects_non_finite():
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(64, 4, 2)
+    for bad in (float("nan"), float("inf"), -float("inf")):
+        with pytest.raises(binding.MpzchError):
+            binding.mpzch_set_learning_rate(tbl.h, bad)
+
+
 def test_repeatable_bytes():
     w = SCALED["c3_small"].scaled(steps=6)
     a = run_pair(w)
