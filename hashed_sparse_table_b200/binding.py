@@ -23,6 +23,9 @@ MPZCH_EINVAL = -1
 MPZCH_ENOMEM = -2
 MPZCH_ECUDA = -3
 MPZCH_ECAPTURE = -5
+MPZCH_ERANGE = -6
+MPZCH_EBUSY = -7
+MPZCH_ETIMEDOUT = -8
 MPZCH_STATUS_BADKEY = 1
 MPZCH_STATUS_BADROW = 2
 MPZCH_STATUS_BADAO = 4
@@ -62,6 +65,13 @@ _SIGS = {
     "mpzch_set_option": [_p, _i32, _i64],
     "mpzch_debug_fail_allocs": [_i32],
     "mpzch_set_learning_rate": [_p, C.c_float],
+    "mpzch_res_create": [_p, _i64, _i32, _i32, C.POINTER(_p)],
+    "mpzch_res_stream": [_p, _i64, _i64, _p],
+    "mpzch_res_flush": [_p, _i32],
+    "mpzch_res_read": [_p, _p, _p, _p, _p, C.POINTER(_i64), C.POINTER(_i64)],
+    "mpzch_res_latency": [_p, C.POINTER(C.c_double), C.POINTER(C.c_double),
+                          C.POINTER(C.c_double), C.POINTER(_i64), C.POINTER(_i64)],
+    "mpzch_res_destroy": [_p],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -274,6 +284,60 @@ def mpzch_debug_fail_allocs(count: int) -> None:
 
 def mpzch_launch_count() -> int:
     return int(_lib.mpzch_launch_count())
+
+
+class MpzchRes:
+    """Streaming exporter of fresh rows to a host int8 snapshot (RES)."""
+
+    def __init__(self, table: "MpzchTable", max_rows: int = 0, slots: int = 2,
+                 period_ms: int = 15000):
+        self.capacity, self.dim = table.capacity, table.dim
+        h = C.c_void_p()
+        _check("mpzch_res_create", _lib.mpzch_res_create(table.h, max_rows, slots, period_ms,
+                                                         C.byref(h)))
+        self.h = h
+
+    def stream(self, since_step: int, upto_step: int, stream=None) -> int:
+        """Returns MPZCH_OK or MPZCH_EBUSY (every staging slot still in use)."""
+        rc = _lib.mpzch_res_stream(self.h, since_step, upto_step, _stream(stream))
+        if rc not in (MPZCH_OK, MPZCH_EBUSY):
+            raise MpzchError("mpzch_res_stream", rc)
+        return rc
+
+    def flush(self, timeout_ms: int = 60000) -> None:
+        _check("mpzch_res_flush", _lib.mpzch_res_flush(self.h, timeout_ms))
+
+    def read(self):
+        import numpy as np
+        keys = np.empty(self.capacity, np.int64)
+        q = np.empty((self.capacity, self.dim), np.int8)
+        scale = np.empty(self.capacity, np.float32)
+        last = np.empty(self.capacity, np.int64)
+        ver, upto = C.c_int64(), C.c_int64()
+        _check("mpzch_res_read", _lib.mpzch_res_read(
+            self.h, keys.ctypes.data_as(C.c_void_p), q.ctypes.data_as(C.c_void_p),
+            scale.ctypes.data_as(C.c_void_p), last.ctypes.data_as(C.c_void_p), C.byref(ver),
+            C.byref(upto)))
+        return keys, q, scale, last, ver.value, upto.value
+
+    def latency(self):
+        p50, p99, mx = C.c_double(), C.c_double(), C.c_double()
+        n, ovf = C.c_int64(), C.c_int64()
+        _check("mpzch_res_latency", _lib.mpzch_res_latency(
+            self.h, C.byref(p50), C.byref(p99), C.byref(mx), C.byref(n), C.byref(ovf)))
+        return {"p50_ms": p50.value, "p99_ms": p99.value, "max_ms": mx.value,
+                "samples": n.value, "overflow_rows": ovf.value}
+
+    def close(self):
+        if getattr(self, "h", None):
+            _check("mpzch_res_destroy", _lib.mpzch_res_destroy(self.h))
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ------------------------------------------------------------------ handle helper

@@ -1,6 +1,7 @@
 // libmpzch: C ABI, table handle and launch orchestration for the Memory Layer
 // table kernels (see include/mpzch.h for the contract of every entry point).
 #include "mpzch.h"
+#include "mpzch_internal.h"
 #include "mpzch_kernels.cuh"
 
 #include <cuda_runtime.h>
@@ -823,7 +824,7 @@ int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int6
     k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
         rows, n, reinterpret_cast<const long long*>(dev_n), reinterpret_cast<const float4*>(t->M),
         t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale,
-        reinterpret_cast<long long*>(keys_out), t->status);
+        reinterpret_cast<long long*>(keys_out), t->status, nullptr, nullptr);
     rc = after_launch();
   }
   return mark_user(t, st, rc);
@@ -940,3 +941,45 @@ int mpzch_debug_fail_allocs(int32_t count) {
 int64_t mpzch_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Internal entry points used by the streaming exporter (mpzch_res.cu).
+// ---------------------------------------------------------------------------
+namespace mpzch_internal {
+
+int64_t table_capacity(const mpzch_table* t) { return t->C; }
+int32_t table_dim(const mpzch_table* t) { return t->D; }
+int table_device(const mpzch_table* t) { return t->device; }
+
+int export_since(mpzch_table* t, int64_t since, int32_t* rows, int64_t* dev_count, int64_t max_rows,
+                 int8_t* q, float* scale, int64_t* keys, int64_t* last, cudaStream_t st) {
+  if (!t || !rows || !dev_count || !q || !scale || !keys || !last || max_rows < 1) return MPZCH_EINVAL;
+  if (!on_device(t)) return MPZCH_EINVAL;
+  int rc = join_side(t, st);
+  if (rc) return rc;
+  {
+    PhaseScope ps(t, PH_SELECT, st);
+    const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
+    k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since,
+                                             t->sel_bcount);
+    rc = after_launch();
+    if (!rc) {
+      k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since,
+                                                 t->sel_bcount, rows,
+                                                 reinterpret_cast<long long*>(dev_count));
+      rc = after_launch();
+    }
+  }
+  if (!rc) {
+    PhaseScope ps(t, PH_EXPORT, st);
+    k_export_int8<<<grid_for(max_rows * 32, kBlock), kBlock, 0, st>>>(
+        rows, max_rows, reinterpret_cast<const long long*>(dev_count),
+        reinterpret_cast<const float4*>(t->M), t->keys, t->C, t->D / 4,
+        reinterpret_cast<char4*>(q), scale, reinterpret_cast<long long*>(keys), t->status,
+        t->last, reinterpret_cast<long long*>(last));
+    rc = after_launch();
+  }
+  return mark_user(t, st, rc);
+}
+
+}  // namespace mpzch_internal

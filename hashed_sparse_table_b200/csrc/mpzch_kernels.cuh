@@ -999,13 +999,14 @@ __global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __re
 
 // ---------------------------------------------------------------------------
 // int8 export: one warp per row.  a = max|x| (exact), scale = a/127 and x/scale
-// as IEEE divisions, round-half-even, clamp to +-127.
+// as IEEE divisions, round-half-even, clamp to +-127.  With last_out, the row's
+// last-write step is exported too (metadata of the streamed snapshot).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBlock) k_export_int8(
     const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
     const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C, int D4,
     char4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
-    int32_t* status) {
+    int32_t* status, const long long* __restrict__ last, long long* __restrict__ last_out) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   int64_t nn = n;
@@ -1022,6 +1023,7 @@ __global__ void __launch_bounds__(kBlock) k_export_int8(
         set_status(status, kStBadRow);
         scale[i] = 0.f;
         keys_out[i] = -1;
+        if (last_out) last_out[i] = -1;
       }
       for (int c = lane; c < D4; c += 32) qo[c] = make_char4(0, 0, 0, 0);
       continue;
@@ -1050,6 +1052,7 @@ __global__ void __launch_bounds__(kBlock) k_export_int8(
     if (lane == 0) {
       scale[i] = s;
       keys_out[i] = keys[r];
+      if (last_out) last_out[i] = last[r];
     }
   }
 }

@@ -59,6 +59,8 @@ extern "C" {
 #define MPZCH_ECUDA (-3)   /* a CUDA runtime call or launch failed */
 #define MPZCH_ECAPTURE (-5) /* would allocate while the stream is being captured */
 #define MPZCH_ERANGE (-6)  /* batch larger than a fixed maximum (mpzch_dedup_static) */
+#define MPZCH_EBUSY (-7)   /* every staging slot of a streaming exporter is in use */
+#define MPZCH_ETIMEDOUT (-8) /* a wait with a time limit ran out */
 
 /* Sticky device status bits (mpzch_get_status). */
 #define MPZCH_STATUS_BADKEY 1   /* a negative item id was given */
@@ -235,6 +237,52 @@ MPZCH_API int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int
                        const int8_t* snap_q, const float* snap_scale, int32_t dim,
                        const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit, float* out,
                        int32_t* dev_status, void* stream);
+
+/* ---- Streaming export of fresh rows to a host serving snapshot (RES) ----
+ * Memory Layer section 2, RES paragraph: new vectors are copied to the host
+ * asynchronously while they are in HBM; in the background they are deduped by
+ * id, quantised and merged, and vectors + identity map + metadata are pushed
+ * atomically every 15 s without blocking training.  Section 5: serving reads
+ * int8 rows.  The host snapshot is a table image: keys[C] (-1 = empty), int8
+ * q[C][dim], scale[C], last-write step last[C], at the table's row indices. */
+typedef struct mpzch_res mpzch_res;
+
+/* Exporter for table t (current device = the table's): `slots` device staging
+ * slots of max_rows rows (max_rows <= 0: the capacity), a background host
+ * thread, and a publish period in milliseconds.  Destroy it before the table. */
+MPZCH_API int mpzch_res_create(mpzch_table* t, int64_t max_rows, int32_t slots, int32_t period_ms,
+                               mpzch_res** out);
+
+/* On `stream` (ordered like any table call): selects every row with a live key
+ * written at or after since_step and exports it (int8 q, scale, key,
+ * last-write step) into a free staging slot; the background thread copies it
+ * to the host and merges it into the snapshot by row index (a row written
+ * several times since the previous call is exported once, with its latest
+ * value; a row reassigned to a new key carries the new key).  upto_step labels
+ * the data (normally the last step written before the call).  Never waits on
+ * the host: returns MPZCH_EBUSY if every slot is still being copied (a later
+ * call with an earlier since_step covers the rows).  Rows beyond max_rows in
+ * one call are not exported and are counted (mpzch_res_latency). */
+MPZCH_API int mpzch_res_stream(mpzch_res* r, int64_t since_step, int64_t upto_step, void* stream);
+
+/* Waits (at most timeout_ms) until every streamed slot is merged and a
+ * snapshot containing them is published.  MPZCH_ETIMEDOUT otherwise. */
+MPZCH_API int mpzch_res_flush(mpzch_res* r, int32_t timeout_ms);
+
+/* Copies the latest published snapshot (host buffers of C entries each; any may
+ * be NULL), its version (number of publishes) and the largest upto_step it
+ * contains.  The copy is taken under the publish lock: one whole version. */
+MPZCH_API int mpzch_res_read(mpzch_res* r, int64_t* keys, int8_t* q, float* scale, int64_t* last,
+                             int64_t* version, int64_t* upto_step);
+
+/* Propagation latency from mpzch_res_stream to the publish that contains its
+ * rows: median, 99th percentile and maximum in ms over `samples` streamed
+ * batches, and the number of rows dropped for exceeding max_rows. */
+MPZCH_API int mpzch_res_latency(mpzch_res* r, double* p50_ms, double* p99_ms, double* max_ms,
+                                int64_t* samples, int64_t* overflow_rows);
+
+/* Stops the background thread after it has merged what is pending, frees all. */
+MPZCH_API int mpzch_res_destroy(mpzch_res* r);
 
 /* Device pointers to the table's state (for checkpoint/resume and tests):
  * keys int64[C], last int64[C], M fp32[C][dim].  Any argument may be NULL. */

@@ -111,6 +111,20 @@ def test_serve_gather_rejects_null_buffers_and_accepts_empty(lib):
                                   None) == 0
 
 
+def test_res_create_rejects_bad_arguments(lib):
+    p = _setup(lib)
+    lib.mpzch_res_create.argtypes = [p, C.c_int64, C.c_int32, C.c_int32, C.POINTER(p)]
+    h = p()
+    assert lib.mpzch_res_create(None, 0, 2, 100, C.byref(h)) == -1
+    assert lib.mpzch_res_create(None, 0, 2, 100, None) == -1
+    lib.mpzch_res_stream.argtypes = [p, C.c_int64, C.c_int64, p]
+    assert lib.mpzch_res_stream(None, 0, 0, None) == -1
+    lib.mpzch_res_flush.argtypes = [p, C.c_int32]
+    assert lib.mpzch_res_flush(None, 10) == -1
+    lib.mpzch_res_destroy.argtypes = [p]
+    assert lib.mpzch_res_destroy(None) == 0
+
+
 def test_python_binding_loads(lib):
     from hashed_sparse_table_b200 import binding
     assert binding.mpzch_launch_count() >= 0
