@@ -59,6 +59,13 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--res-every", type=int, default=0,
+                    help="after the timed region, train for --res-seconds more while streaming "
+                         "the rows written every N steps to a host int8 snapshot (RES); "
+                         "reports its propagation latency under a 'res' key (0 = off)")
+    ap.add_argument("--res-period-ms", type=int, default=1000,
+                    help="RES publish period (the pages' deployment pushes every 15 s)")
+    ap.add_argument("--res-seconds", type=float, default=5.0)
     ap.add_argument("--side-priority", type=int, default=None, choices=[0, 1],
                     help="priority of the table's side stream (1 = highest)")
     ap.add_argument("--no-pipeline", action="store_true",
@@ -269,14 +276,16 @@ def run_ours(args):
     if args.wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, args.wide_rounds)
 
-    def step(t):
+    def step(t, i=None):
+        # step t of the stream reads the resident inputs of slot i (default t)
+        i = t if i is None else i
         if args.separate_calls:
-            binding.mpzch_lookup(tbl.h, ids_d[t][:lab], rows, hits[t])
-            binding.mpzch_gather_fused(tbl.h, rows, hits[t], out, ao_d, aor_d[t])
-            binding.mpzch_writeback(tbl.h, ids_d[t], e_d[t % E], t, stats[t])
+            binding.mpzch_lookup(tbl.h, ids_d[i][:lab], rows, hits[i])
+            binding.mpzch_gather_fused(tbl.h, rows, hits[i], out, ao_d, aor_d[i])
+            binding.mpzch_writeback(tbl.h, ids_d[i], e_d[t % E], t, stats[i])
         else:
-            binding.mpzch_train_step(tbl.h, ids_d[t], lab, e_d[t % E], t, rows_t[t % 2], hits[t],
-                                     out, ao_d, aor_d[t], stats[t],
+            binding.mpzch_train_step(tbl.h, ids_d[i], lab, e_d[t % E], t, rows_t[t % 2], hits[i],
+                                     out, ao_d, aor_d[i], stats[i],
                                      inputs_ready=None if args.no_pipeline else ready)
 
     for t in range(Pf):
@@ -325,6 +334,11 @@ def run_ours(args):
     wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
     gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
 
+    res_info = None
+    if args.res_every > 0:
+        res_info = run_res(tbl, binding, torch, args, step_fn=step, first_step=total,
+                           n_inputs=total)
+
     # end to end: host inputs (pinned) -> device -> step -> counters back to host
     e2e = None
     if not args.no_e2e:
@@ -363,6 +377,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
         }
+        if res_info is not None:
+            result["res"] = res_info
     tbl.close()
     if world > 1:
         dist.barrier()
@@ -371,12 +387,51 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
+def run_res(tbl, binding, torch, args, step_fn, first_step, n_inputs):
+    """Training continues (cycling through the resident id batches with new step
+    numbers) while every --res-every steps the rows written since the last
+    export are streamed to the host snapshot; reports the propagation latency
+    from each export call to the publish that contains it."""
+    res = binding.MpzchRes(tbl, slots=2, period_ms=args.res_period_ms)
+    t = first_step
+    streamed_upto = first_step - 1
+    busy = 0
+    streams = 0
+    t_end = time.perf_counter() + args.res_seconds
+    steps = 0
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    while time.perf_counter() < t_end:
+        step_fn(t, t % n_inputs)
+        steps += 1
+        if steps % args.res_every == 0:
+            rc = res.stream(streamed_upto + 1, t)
+            if rc == binding.MPZCH_OK:
+                streamed_upto = t
+                streams += 1
+            else:
+                busy += 1
+        t += 1
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    res.flush(120_000)
+    lat = res.latency()
+    _, _, _, _, version, upto = res.read()
+    res.close()
+    return {"every_steps": args.res_every, "period_ms": args.res_period_ms,
+            "train_steps": steps, "train_steps_per_s": steps / wall, "streams": streams,
+            "busy_skips": busy, "publishes": version, "snapshot_upto_step": upto,
+            "latency_ms": {"p50": lat["p50_ms"], "p99": lat["p99_ms"], "max": lat["max_ms"],
+                           "samples": lat["samples"]},
+            "overflow_rows": lat["overflow_rows"]}
+
+
 def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
     """Same steps (continuing the stream) with host inputs copied in every step."""
     import torch.distributed as dist
     lab = W.labeled
-    n0 = total
-    host = [host_step(t, rank) for t in range(n0, n0 + K)]
+    n0 = max(total, binding.mpzch_get_last_step(tbl.h) + 1)  # continue the step sequence
+    host = [host_step(t, rank) for t in range(total, total + K)]
     ids_h = [torch.from_numpy(h[0]).pin_memory() for h in host]
     aor_h = [torch.from_numpy(h[1]).pin_memory() for h in host]
     e_h = [x.pin_memory() for x in e_host]

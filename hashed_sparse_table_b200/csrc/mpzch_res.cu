@@ -17,10 +17,11 @@
 //    earlier `since` covers the skipped rows.
 //  * one background host thread per exporter: waits for a slot's event,
 //    copies exactly that many rows to pinned host buffers on its own copy
-//    stream, merges them into the working snapshot by row index (a row
-//    reassigned to a new key simply carries the new key), frees the slot,
-//    and every period publishes: the working snapshot is copied into the
-//    published one under a lock and the version increases.  Readers copy the
+//    stream, merges them into the working snapshot by row index with a few
+//    host threads (a row reassigned to a new key simply carries the new key),
+//    frees the slot, and every period publishes what has been merged: the
+//    working snapshot is copied into the published one under a lock and the
+//    version increases.  Readers copy the
 //    published snapshot under the same lock, so they always see one whole
 //    version.
 #include <cuda_runtime.h>
@@ -91,6 +92,7 @@ struct mpzch_res {
   std::deque<int> pending;
   bool stop = false;
   int64_t flush_requests = 0, flushes_done = 0;
+  int merge_threads = 1;
   std::thread th;
 };
 
@@ -168,12 +170,28 @@ int merge_slot(mpzch_res* r, Slot& s) {
         cudaStreamSynchronize(cs))
       return MPZCH_ECUDA;
   }
-  for (int64_t i = 0; i < n; ++i) {
-    const int64_t row = s.h_rows[i];
-    r->w_keys[row] = s.h_keys[i];
-    r->w_last[row] = s.h_last[i];
-    r->w_scale[row] = s.h_scale[i];
-    std::memcpy(&r->w_q[row * D], &s.h_q[i * D], D);
+  // Merge by row index; the rows of one export are distinct, so host threads
+  // can take disjoint ranges of it.
+  auto merge_range = [&](int64_t i0, int64_t i1) {
+    for (int64_t i = i0; i < i1; ++i) {
+      const int64_t row = s.h_rows[i];
+      r->w_keys[row] = s.h_keys[i];
+      r->w_last[row] = s.h_last[i];
+      r->w_scale[row] = s.h_scale[i];
+      std::memcpy(&r->w_q[row * D], &s.h_q[i * D], D);
+    }
+  };
+  const int64_t per = 65536;
+  const int nt = (int)std::min<int64_t>(r->merge_threads, (n + per - 1) / per);
+  if (nt <= 1) {
+    merge_range(0, n);
+  } else {
+    std::vector<std::thread> pool;
+    pool.reserve(nt);
+    const int64_t chunk = (n + nt - 1) / nt;
+    for (int k = 0; k < nt; ++k)
+      pool.emplace_back(merge_range, std::min(n, k * chunk), std::min(n, (k + 1) * chunk));
+    for (auto& th : pool) th.join();
   }
   return MPZCH_OK;
 }
@@ -183,10 +201,17 @@ void worker(mpzch_res* r) {
   double next_publish = now_ms() + r->period_ms;
   std::unique_lock<std::mutex> lk(r->mu);
   while (true) {
+    // Publish on the period whatever is still queued (what has been merged so
+    // far); a flush publishes once everything queued before it is merged.
+    if (now_ms() >= next_publish) {
+      publish_locked(r);
+      next_publish = now_ms() + r->period_ms;
+      r->cv.notify_all();
+    }
     const bool flush_wanted = r->flush_requests > r->flushes_done;
     if (r->pending.empty()) {
       if (r->stop) break;
-      if (flush_wanted || now_ms() >= next_publish) {
+      if (flush_wanted) {
         publish_locked(r);
         r->flushes_done = r->flush_requests;
         next_publish = now_ms() + r->period_ms;
@@ -274,6 +299,7 @@ int mpzch_res_create(mpzch_table* t, int64_t max_rows, int32_t slots, int32_t pe
     delete r;
     return rc;
   }
+  r->merge_threads = (int)std::max(1u, std::min(8u, std::thread::hardware_concurrency() / 2));
   r->th = std::thread(worker, r);
   *out = r;
   return MPZCH_OK;
