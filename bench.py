@@ -44,7 +44,7 @@ UNIT = "unique rows/s"
 PREFILL = 20  # untimed steps that bring the table to its steady state
 # DRAM bytes (read + write) of one k_writeback launch of this workload, from
 # one ncu capture of the current kernel (profiles/k_writeback_multitable_c1m_d512.md)
-WB_TRAFFIC_BYTES = None  # kernel changed since the last capture; re-captured below when set
+WB_TRAFFIC_BYTES = 545.38e6
 WB_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                      "(23rd step of the multi-table workload)")
 REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--prefill", type=int, default=PREFILL)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-serving", action="store_true",
+                    help="skip the export + serving measurement after the timed region")
     ap.add_argument("--res-every", type=int, default=0,
                     help="after the timed region, train for --res-seconds more while streaming "
                          "the rows written every N steps to a host int8 snapshot (RES); "
@@ -334,6 +336,8 @@ def run_ours(args):
     wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
     gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
 
+    serving = None if args.no_serving else run_export_and_serve(tbl, binding, torch, dev, peak)
+
     res_info = None
     if args.res_every > 0:
         res_info = run_res(tbl, binding, torch, args, step_fn=step, first_step=total,
@@ -377,6 +381,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
         }
+        if serving is not None:
+            result.update(serving)
         if res_info is not None:
             result["res"] = res_info
     tbl.close()
@@ -385,6 +391,83 @@ def run_ours(args):
         dist.destroy_process_group()
     if result is not None:
         print(json.dumps(result), flush=True)
+
+
+def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):
+    """Export and serving on the trained table: rows written in the last 50
+    steps -> int8 export (select + quantise), the serving snapshot image, and the
+    serving gather of 4,096 requests x 1,024 candidates (Zipf 0.9 over 5M) in
+    512-request chunks.  CUDA events on the current stream; L2 is not flushed
+    between repetitions (each pass moves several GB)."""
+    D, P, C = W.dim, W.probes, W.capacity
+    last_step = binding.mpzch_get_last_step(tbl.h)
+    since = last_step - inputs.CFG5_SERVE_SINCE + 1
+    rows_d = torch.empty(C, dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int64, device=dev)
+    q = torch.empty((C, D), dtype=torch.int8, device=dev)
+    scale = torch.empty(C, dtype=torch.float32, device=dev)
+    keys = torch.empty(C, dtype=torch.int64, device=dev)
+    binding.mpzch_trace_read(tbl.h)
+    binding.mpzch_trace_enable(tbl.h, True)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(reps):
+        binding.mpzch_select_written_since(tbl.h, since, rows_d, cnt)
+        binding.mpzch_export_int8(tbl.h, rows_d, q, scale, keys, n=C, dev_n=cnt)
+    ev1.record()
+    torch.cuda.synchronize()
+    tr = binding.mpzch_trace_read(tbl.h)
+    binding.mpzch_trace_enable(tbl.h, False)
+    n = int(cnt.item())
+    export_ms = ev0.elapsed_time(ev1) / reps
+    sel_ms, _ = tr["select"]
+    exp_ms, _ = tr["export"]
+    exp_bytes = n * (4 * D + D + 4 + 8 + 4 + 8)  # row read, int8 + scale + key written, row id, key read
+    sel_bytes = C * 16 + n * 4                   # keys + last scanned, selected rows written
+    # serving snapshot image (the push target): exported rows at their row index
+    snap_keys = torch.full((C,), -1, dtype=torch.int64, device=dev)
+    snap_q = torch.zeros((C, D), dtype=torch.int8, device=dev)
+    snap_s = torch.zeros(C, dtype=torch.float32, device=dev)
+    idx = rows_d[:n].long()
+    snap_keys[idx] = keys[:n]
+    snap_q[idx] = q[:n]
+    snap_s[idx] = scale[:n]
+    cand = torch.from_numpy(inputs.serve_candidates()).to(dev)
+    chunk = 512 * inputs.CFG5_CANDIDATES
+    out = torch.empty((chunk, D), dtype=torch.float32, device=dev)
+    grow = torch.empty(chunk, dtype=torch.int32, device=dev)
+    ghit = torch.empty(cand.numel(), dtype=torch.uint8, device=dev)
+    for _ in range(2):  # warm-up
+        binding.mpzch_serve_gather(snap_keys, P, snap_q, snap_s, cand[:chunk], grow,
+                                   ghit[:chunk], out)
+    torch.cuda.synchronize()
+    ev0.record()
+    for c0 in range(0, cand.numel(), chunk):
+        binding.mpzch_serve_gather(snap_keys, P, snap_q, snap_s, cand[c0:c0 + chunk], grow,
+                                   ghit[c0:c0 + chunk], out)
+    ev1.record()
+    torch.cuda.synchronize()
+    serve_ms = ev0.elapsed_time(ev1)
+    n_ids = cand.numel()
+    hits = int(ghit.sum().item())
+    serve_bytes = n_ids * (8 + 8 * P + 5 + 4 * D) + hits * (D + 4)
+    serve_gbs = serve_bytes / (serve_ms * 1e-3) / 1e9
+    exp_gbs = exp_bytes / (exp_ms / reps * 1e-3) / 1e9 if exp_ms > 0 else 0.0
+    return {
+        "export": {"rows": n, "since_step": since, "ms": export_ms,
+                   "rows_per_s": n / (export_ms * 1e-3),
+                   "roofline": {"bound": "hbm", "kernel": "k_export_int8", "achieved": exp_gbs,
+                                "peak": peak, "unit": "GB/s", "frac": exp_gbs / peak,
+                                "bytes_per_launch": exp_bytes,
+                                "avg_launch_us": exp_ms / reps * 1e3},
+                   "select_gbs": sel_bytes / (sel_ms / reps * 1e-3) / 1e9 if sel_ms > 0 else 0.0},
+        "serve": {"ids": n_ids, "chunk_ids": chunk, "hit_rate": hits / n_ids, "ms": serve_ms,
+                  "ids_per_s": n_ids / (serve_ms * 1e-3),
+                  "roofline": {"bound": "hbm", "kernel": "k_serve_gather", "achieved": serve_gbs,
+                               "peak": peak, "unit": "GB/s", "frac": serve_gbs / peak,
+                               "bytes_per_launch": serve_bytes / (n_ids // chunk)}},
+    }
 
 
 def run_res(tbl, binding, torch, args, step_fn, first_step, n_inputs):

@@ -1002,6 +1002,102 @@ __global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __re
 // as IEEE divisions, round-half-even, clamp to +-127.  With last_out, the row's
 // last-write step is exported too (metadata of the streamed snapshot).
 // ---------------------------------------------------------------------------
+// q = rne(fl(x / s)), clamped to +-127.  Fast path: p = fl(x * fl(1/s)) differs
+// from the exact quotient t = x/s by at most |t| 2^-23 + |t| 2^-24, and fl(t)
+// from t by at most |t| 2^-24, so |p - fl(x/s)| < |t| 2^-22 <= 127.00001 * 2^-22
+// < 3.1e-5.  When p is more than 1e-4 away from every half-integer, fl(x/s)
+// rounds to the same integer as p; otherwise the IEEE division is taken.  (A
+// reciprocal that is not finite, for a subnormal s, sends every element to
+// the division.)
+__device__ __forceinline__ signed char quant1(float xv, float s, float rcp, bool fast) {
+  int t;
+  const float p = __fmul_rn(xv, rcp);
+  const float dist = fabsf(fabsf(p - truncf(p)) - 0.5f);
+  if (fast && dist > 1e-4f)
+    t = __float2int_rn(p);
+  else
+    t = __float2int_rn(__fdiv_rn(xv, s));
+  t = t > 127 ? 127 : (t < -127 ? -127 : t);
+  return (signed char)t;
+}
+
+__device__ __forceinline__ uint32_t quant4(float4 v, float s, float rcp, bool fast) {
+  const uint32_t b0 = (uint8_t)quant1(v.x, s, rcp, fast), b1 = (uint8_t)quant1(v.y, s, rcp, fast);
+  const uint32_t b2 = (uint8_t)quant1(v.z, s, rcp, fast), b3 = (uint8_t)quant1(v.w, s, rcp, fast);
+  return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+}
+
+// Export of one row by one warp, the row held in registers: lane l owns the
+// 16-byte vectors 4l..4l+3 of each 2 KiB chunk (64 contiguous input bytes) and
+// writes their 16 int8 values with one 16-byte store.  kChunks chunks of 128
+// vectors cover dim = 512 * kChunks.
+template <int kChunks>
+__device__ __forceinline__ void export_row_regs(const float4* __restrict__ x, uint4* qo, float* sc,
+                                                long long* ko, long long* lo, long long key,
+                                                long long lastv, int lane) {
+  float4 v[kChunks][4];
+#pragma unroll
+  for (int ch = 0; ch < kChunks; ++ch)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[ch][j] = __ldcs(x + ch * 128 + 4 * lane + j);
+  float a = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < kChunks; ++ch)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      a = fmaxf(a, fmaxf(fmaxf(fabsf(v[ch][j].x), fabsf(v[ch][j].y)),
+                         fmaxf(fabsf(v[ch][j].z), fabsf(v[ch][j].w))));
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+  const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
+  const float rcp = a == 0.f ? 0.f : __frcp_rn(s);
+  const bool fast = a != 0.f && isfinite(rcp);
+#pragma unroll
+  for (int ch = 0; ch < kChunks; ++ch) {
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (a != 0.f) {
+      o.x = quant4(v[ch][0], s, rcp, fast);
+      o.y = quant4(v[ch][1], s, rcp, fast);
+      o.z = quant4(v[ch][2], s, rcp, fast);
+      o.w = quant4(v[ch][3], s, rcp, fast);
+    }
+    __stcs(qo + ch * 32 + lane, o);
+  }
+  if (lane == 0) {
+    *sc = s;
+    *ko = key;
+    if (lo) *lo = lastv;
+  }
+}
+
+// Any dim (multiple of 4): two passes over the row (max, then quantise) with
+// 4-byte stores.
+__device__ __forceinline__ void export_row_generic(const float4* __restrict__ x, char4* qo, int D4,
+                                                   float* sc, long long* ko, long long* lo,
+                                                   long long key, long long lastv, int lane) {
+  float a = 0.f;
+  for (int c = lane; c < D4; c += 32) {
+    const float4 v = x[c];
+    a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+  const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
+  const float rcp = a == 0.f ? 0.f : __frcp_rn(s);
+  const bool fast = a != 0.f && isfinite(rcp);
+  for (int c = lane; c < D4; c += 32) {
+    const float4 v = x[c];
+    char4 o = make_char4(0, 0, 0, 0);
+    if (a != 0.f)
+      o = make_char4(quant1(v.x, s, rcp, fast), quant1(v.y, s, rcp, fast),
+                     quant1(v.z, s, rcp, fast), quant1(v.w, s, rcp, fast));
+    qo[c] = o;
+  }
+  if (lane == 0) {
+    *sc = s;
+    *ko = key;
+    if (lo) *lo = lastv;
+  }
+}
+
 __global__ void __launch_bounds__(kBlock) k_export_int8(
     const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
     const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C, int D4,
@@ -1014,46 +1110,34 @@ __global__ void __launch_bounds__(kBlock) k_export_int8(
     const long long d = *dev_n;
     nn = d < nn ? d : nn;
   }
+  // 16-byte output rows need dim % 16 == 0 and an aligned q
+  const bool vec16 = (D4 % 128 == 0) && ((reinterpret_cast<uintptr_t>(q) & 15) == 0);
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nn; i += warps) {
     const int32_t r = rows[i];
     char4* qo = q + i * (int64_t)D4;
+    long long* lo = last_out ? last_out + i : nullptr;
     if (r < 0 || (int64_t)r >= C) {
       if (lane == 0) {
         set_status(status, kStBadRow);
         scale[i] = 0.f;
         keys_out[i] = -1;
-        if (last_out) last_out[i] = -1;
+        if (lo) *lo = -1;
       }
       for (int c = lane; c < D4; c += 32) qo[c] = make_char4(0, 0, 0, 0);
       continue;
     }
     const float4* x = M + (int64_t)r * D4;
-    float a = 0.f;
-    for (int c = lane; c < D4; c += 32) {
-      const float4 v = x[c];
-      a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
-    for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-    const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
-    for (int c = lane; c < D4; c += 32) {
-      const float4 v = x[c];
-      char4 o = make_char4(0, 0, 0, 0);
-      if (a != 0.f) {
-        auto qz = [s](float xv) -> signed char {
-          int t = __float2int_rn(__fdiv_rn(xv, s));
-          t = t > 127 ? 127 : (t < -127 ? -127 : t);
-          return (signed char)t;
-        };
-        o = make_char4(qz(v.x), qz(v.y), qz(v.z), qz(v.w));
-      }
-      qo[c] = o;
-    }
-    if (lane == 0) {
-      scale[i] = s;
-      keys_out[i] = keys[r];
-      if (last_out) last_out[i] = last[r];
-    }
+    const long long key = keys[r];
+    const long long lastv = last_out ? last[r] : 0;
+    if (vec16 && D4 == 128)
+      export_row_regs<1>(x, reinterpret_cast<uint4*>(qo), scale + i, keys_out + i, lo, key, lastv,
+                         lane);
+    else if (vec16 && D4 == 256)
+      export_row_regs<2>(x, reinterpret_cast<uint4*>(qo), scale + i, keys_out + i, lo, key, lastv,
+                         lane);
+    else
+      export_row_generic(x, qo, D4, scale + i, keys_out + i, lo, key, lastv, lane);
   }
 }
 

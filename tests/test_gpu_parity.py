@@ -233,6 +233,39 @@ def test_export_edge_rows():
     assert_bitwise(s.cpu().numpy(), os_, "scale")
 
 
+def test_export_near_half_integer_quotients():
+    """Rows built so that x/scale lands on or within a few ulps of k + 1/2 (the
+    rounding boundary), plus subnormal-scale rows: every int8 byte must match
+    the oracle's IEEE division and round-half-even."""
+    from hashed_sparse_table_b200 import binding
+    C, D = 512, 64
+    tbl = binding.MpzchTable(C, D, 4)
+    orc = oracle.OracleTable(C, D, 4)
+    rng = np.random.default_rng(11)
+    vals = np.empty((C, D), np.float32)
+    for r in range(C):
+        a = np.float32(10.0 ** rng.uniform(-30, 30)) if r % 8 else np.float32(127.0)
+        if r % 61 == 0:
+            a = np.float32(3e-42)  # subnormal absmax: subnormal scale
+        sc = np.float32(a / np.float32(127.0))
+        k = rng.integers(-127, 127, size=D).astype(np.float32)
+        x = ((k + np.float32(0.5)) * sc).astype(np.float32)
+        nudge = rng.integers(-3, 4, size=D)
+        x = np.array([np.nextafter(v, np.float32(np.inf) if n > 0 else np.float32(-np.inf))
+                      if n else v for v, n in zip(x, nudge)], np.float32)
+        x[0] = a  # the absmax element
+        vals[r] = x
+    _, _, M = tbl.state()
+    M.copy_(torch.from_numpy(vals))
+    for r in range(C):
+        orc.set_row(r, vals[r])
+    rows = np.arange(C, dtype=np.int32)
+    q, s, k = tbl.export_int8(torch.from_numpy(rows).cuda())
+    oq, os_, ok = orc.export_int8(rows)
+    assert_bitwise(s.cpu().numpy(), os_, "scale")
+    assert_bitwise(q.cpu().numpy(), oq, "q near half-integers")
+
+
 # ------------------------------------------------------------------ error paths and empties
 def test_empty_calls_and_step_order():
     from hashed_sparse_table_b200 import binding
