@@ -179,10 +179,11 @@ struct mpzch_table {
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
-  int side_high_priority = 0;  // priority of the side stream (set before its first use)
+  int side_high_priority = 1;  // priority of the side stream (set before its first use)
   float eta = 1.0f;            // learning rate of the Writeback step
   // mpzch_train_step: the row map runs on a second (high-priority) stream
   cudaStream_t side = nullptr;
+  cudaStream_t look = nullptr;  // the train step's lookup: highest stream priority
   cudaEvent_t ev_fork = nullptr, ev_lookup = nullptr, ev_map = nullptr;
   cudaEvent_t ev_update[2] = {nullptr, nullptr};  // row update that read write list b
   cudaEvent_t ev_user = nullptr;    // end of the last other call on a caller stream
@@ -246,6 +247,7 @@ void free_all(mpzch_table* t) {
   if (t->ev_user) cudaEventDestroy(t->ev_user);
   if (t->ev_gather) cudaEventDestroy(t->ev_gather);
   if (t->side) cudaStreamDestroy(t->side);
+  if (t->look) cudaStreamDestroy(t->look);
 }
 
 int ensure_side_stream(mpzch_table* t) {
@@ -254,6 +256,7 @@ int ensure_side_stream(mpzch_table* t) {
   if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
       cudaStreamCreateWithPriority(&t->side, cudaStreamNonBlocking,
                                    t->side_high_priority ? greatest : least) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&t->look, cudaStreamNonBlocking, greatest) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_lookup, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_map, cudaEventDisableTiming) != cudaSuccess ||
@@ -445,31 +448,26 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
 }
 
 // Row map of one Writeback on stream `st`: dedup + re-probe + refresh, then
-// (optionally) the lookup of the first n_lookup ids -- which must read the keys
-// before any insert of this step -- then the insert rounds and the write list.
-// ev_lookup (optional) is recorded after the lookup.
-int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, int32_t* rows,
-                    uint8_t* hit, int64_t n_lookup, cudaEvent_t ev_lookup, void* unused) {
-  (void)unused;
+// the insert rounds and the write list.  With `keys_free` the inserts (the
+// first writes to the key array in the step) wait for that event: a lookup of
+// this step on another stream must read the keys first.
+int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEvent_t keys_free) {
   const int64_t n = p.n;
   int rc;
   {
     PhaseScope ps(t, PH_DEDUP, st);
-    rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false, p.ids, n,
-                t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status, p.wcount);
+    rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false,
+                p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status,
+                p.wcount);
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
   }
-  if (n_lookup > 0) {
-    rc = enqueue_lookup(t, reinterpret_cast<const int64_t*>(p.ids), n_lookup, rows, hit, st, true);
-    if (rc) return rc;
-  }
-  if (ev_lookup && cudaEventRecord(ev_lookup, st) != cudaSuccess) return MPZCH_ECUDA;
+  if (keys_free && cudaStreamWaitEvent(st, keys_free, 0) != cudaSuccess) return MPZCH_ECUDA;
   {
     PhaseScope ps(t, PH_INSERT, st);
     const unsigned grid = grid_for(n, kBlock, 4);
     for (int r = 0; r < t->wide_rounds && !rc; ++r)
-      rc = launch(k_insert_round, grid, kBlock, st, !ev_lookup || r > 0, p, r);
+      rc = launch(k_insert_round, grid, kBlock, st, !keys_free || r > 0, p, r);
     if (!rc)
       rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, t->wide_rounds);
     if (!rc) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
@@ -720,7 +718,7 @@ int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t 
   rc = ensure_batch(t, n, st);
   if (rc) return rc;
   const WbParams p = make_params(t, ids, e, n, step, stats);
-  rc = enqueue_row_map(t, p, st, nullptr, nullptr, 0, nullptr, nullptr);
+  rc = enqueue_row_map(t, p, st, nullptr);
   if (!rc) rc = enqueue_row_update(t, p, st, true);
   if (rc) return rc;
   t->last_step = step;
@@ -752,23 +750,38 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
     return mark_user(t, st, MPZCH_OK);
   }
   const WbParams p = make_params(t, ids, e, n, step, stats);
-  // Side stream: dedup + refresh, lookup, inserts, write list.  It starts after
-  // the caller's stream (no inputs_ready), or -- pipelined -- after the inputs,
-  // the last other call, the row update that last read this write-list buffer
-  // and the previous gather (which read rows/hit), but not after the rest of
-  // the caller's stream, so it overlaps the previous step's row update.
+  // Three streams.  Lookup stream (highest priority): the lookup, once the
+  // keys hold the previous step's inserts.  Side stream (low priority):
+  // dedup + refresh, then -- after the lookup has read the keys -- inserts and
+  // the write list.  Caller's stream: gather, then the row update.  Without
+  // inputs_ready both helper streams start after everything earlier on the
+  // caller's stream.  With it (pipelined) they wait only for what they need:
+  // the inputs, the last other call on the table, the previous gather (which
+  // read rows/hit), the previous row map (lookup: final keys) and the row
+  // update that last read this write-list buffer (side stream) -- so they
+  // overlap the previous step's row update.
   if (inputs_ready) {
-    if (cudaStreamWaitEvent(t->side, reinterpret_cast<cudaEvent_t>(inputs_ready), 0) !=
-            cudaSuccess ||
+    cudaEvent_t in = reinterpret_cast<cudaEvent_t>(inputs_ready);
+    if (cudaStreamWaitEvent(t->look, in, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->look, t->ev_user, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->look, t->ev_gather, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->look, t->ev_map, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(t->side, in, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_gather, 0) != cudaSuccess)
       return MPZCH_ECUDA;
   } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
+             cudaStreamWaitEvent(t->look, t->ev_fork, 0) != cudaSuccess ||
              cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess) {
     return MPZCH_ECUDA;
   }
-  rc = enqueue_row_map(t, p, t->side, rows, hit, n_labeled, t->ev_lookup, nullptr);
+  if (n_labeled > 0) {
+    rc = enqueue_lookup(t, ids, n_labeled, rows, hit, t->look, false);
+    if (rc) return rc;
+  }
+  if (cudaEventRecord(t->ev_lookup, t->look) != cudaSuccess) return MPZCH_ECUDA;
+  rc = enqueue_row_map(t, p, t->side, t->ev_lookup);
   if (rc) return rc;
   if (cudaEventRecord(t->ev_map, t->side) != cudaSuccess) return MPZCH_ECUDA;
   // Caller's stream: gather once the lookup is done, then the row update once

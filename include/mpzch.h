@@ -186,10 +186,11 @@ MPZCH_API int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e
  *   mpzch_writeback(ids, e, n, step, dev_stats);
  * rows/hit/out/ao_* as in those calls (may be NULL when n_labeled == 0).
  *
- * Inside, the row map (dedup, refresh, the lookup, inserts) runs on a second
- * stream of the table (MPZCH_OPT_SIDE_PRIORITY); the gather and the row update run on
- * `stream`, the gather once the lookup is done and the row update once the
- * row map is done.  Later work on `stream` is ordered after all of it (rows,
+ * Inside, the lookup runs on a highest-priority stream of the table and the
+ * rest of the row map (dedup, refresh, inserts) on a second stream
+ * (MPZCH_OPT_SIDE_PRIORITY); the gather and the row update run on `stream`,
+ * the gather once the lookup is done and the row update once the row map is
+ * done.  Later work on `stream` is ordered after all of it (rows,
  * hit, out, stats and the table are complete there).
  *
  * inputs_ready: NULL, or a cudaEvent_t (as void*) recorded after ids, e and
@@ -312,8 +313,8 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * launched before a single-block kernel places the remaining keys (default 3,
  * range 0..64).  Results do not depend on it. */
 #define MPZCH_OPT_WIDE_ROUNDS 1
-/* MPZCH_OPT_SIDE_PRIORITY: 1 = the side stream of mpzch_train_step gets the
- * device's highest stream priority, 0 (default) = the lowest; only before the
+/* MPZCH_OPT_SIDE_PRIORITY: 1 (default) = the side stream of mpzch_train_step
+ * gets the device's highest stream priority, 0 = the lowest; only before the
  * first mpzch_train_step of the table (MPZCH_EINVAL afterwards). */
 #define MPZCH_OPT_SIDE_PRIORITY 2
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
