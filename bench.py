@@ -68,6 +68,8 @@ def parse():
     ap.add_argument("--res-period-ms", type=int, default=1000,
                     help="RES publish period (the pages' deployment pushes every 15 s)")
     ap.add_argument("--res-seconds", type=float, default=5.0)
+    ap.add_argument("--row-grid", type=int, default=None,
+                    help="row kernels: 0 = one row per warp, k = k blocks per SM grid-stride")
     ap.add_argument("--side-priority", type=int, default=None, choices=[0, 1],
                     help="priority of the table's side stream (1 = highest)")
     ap.add_argument("--no-pipeline", action="store_true",
@@ -273,6 +275,8 @@ def run_ours(args):
     ready.record(stream)  # every step's inputs are resident from here on
     tbl = binding.MpzchTable(W.capacity, W.dim, W.probes)
     binding.mpzch_reserve(tbl.h, W.batch)
+    if args.row_grid is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_ROW_GRID, args.row_grid)
     if args.side_priority is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SIDE_PRIORITY, args.side_priority)
     if args.wide_rounds is not None:

@@ -33,6 +33,7 @@ MPZCH_STATUS_INTERNAL = 8
 MPZCH_NPHASES = 7
 MPZCH_OPT_WIDE_ROUNDS = 1
 MPZCH_OPT_SIDE_PRIORITY = 2
+MPZCH_OPT_ROW_GRID = 3
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")

@@ -124,6 +124,18 @@ int launch_smem(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t sm
   return MPZCH_OK;
 }
 
+// Grid of a one-warp-per-row kernel over n rows: per_sm > 0 caps it at per_sm
+// resident blocks per SM (grid-stride, long-lived blocks); per_sm == 0 gives
+// one row per warp (short-lived blocks, so blocks of other streams find free
+// slots while it runs).
+unsigned row_grid(int64_t n, int per_sm) {
+  if (per_sm > 0) return grid_for(n * 32, kBlock, per_sm);
+  int64_t g = (n * 32 + kBlock - 1) / kBlock;
+  if (g < 1) g = 1;
+  if (g > 0x7FFFFFFF) g = 0x7FFFFFFF;
+  return (unsigned)g;
+}
+
 uint64_t pow2_at_least(uint64_t x) {
   uint64_t p = 1;
   while (p < x) p <<= 1;
@@ -181,6 +193,7 @@ struct mpzch_table {
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
   int side_high_priority = 1;  // priority of the side stream (set before its first use)
   float eta = 1.0f;            // learning rate of the Writeback step
+  int row_blocks_per_sm = 8;   // row kernels: 0 = one row per warp, else grid-stride cap
   // mpzch_train_step: the row map runs on a second (high-priority) stream
   cudaStream_t side = nullptr;
   cudaStream_t look = nullptr;  // the train step's lookup: highest stream priority
@@ -398,7 +411,7 @@ int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int6
                    const int32_t* ao_rows, float* out, cudaStream_t st, bool pdl) {
   PhaseScope ps(t, PH_GATHER, st);
   const bool has_ao = ao_table != nullptr;
-  return launch(k_gather_fused, grid_for(n * 32, kBlock), kBlock, st, pdl, rows, hit, n,
+  return launch(k_gather_fused, row_grid(n, t->row_blocks_per_sm), kBlock, st, pdl, rows, hit, n,
                 reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
                 reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
                 ao_rows, reinterpret_cast<float4*>(out), t->status);
@@ -478,7 +491,7 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
 int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool pdl) {
   {
     PhaseScope ps(t, PH_WRITEBACK, st);
-    const int rc = launch(k_writeback, grid_for(p.n * 32, kBlock), kBlock, st, pdl,
+    const int rc = launch(k_writeback, row_grid(p.n, t->row_blocks_per_sm), kBlock, st, pdl,
                           (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount,
                           p.M, p.e, p.D4, t->eta);
     if (rc) return rc;
@@ -929,6 +942,11 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
   if (option == MPZCH_OPT_SIDE_PRIORITY) {
     if ((value != 0 && value != 1) || t->side) return MPZCH_EINVAL;
     t->side_high_priority = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_ROW_GRID) {
+    if (value < 0 || value > 32) return MPZCH_EINVAL;
+    t->row_blocks_per_sm = (int)value;
     return MPZCH_OK;
   }
   if (option == MPZCH_OPT_WIDE_ROUNDS) {

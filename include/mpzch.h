@@ -317,6 +317,10 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * gets the device's highest stream priority, 0 = the lowest; only before the
  * first mpzch_train_step of the table (MPZCH_EINVAL afterwards). */
 #define MPZCH_OPT_SIDE_PRIORITY 2
+/* MPZCH_OPT_ROW_GRID: grid of the row kernels (fused gather, row update):
+ * 0 = one row per warp, short-lived blocks; k > 0 = at most k blocks of 256
+ * threads per SM, each striding over many rows (default 8). */
+#define MPZCH_OPT_ROW_GRID 3
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 
 /* Learning rate of the Writeback step for the following calls (Memory Layer
