@@ -68,6 +68,10 @@ def parse():
     ap.add_argument("--res-period-ms", type=int, default=1000,
                     help="RES publish period (the pages' deployment pushes every 15 s)")
     ap.add_argument("--res-seconds", type=float, default=5.0)
+    ap.add_argument("--host-values", action="store_true",
+                    help="table values in pinned host memory (host-memory tier): the row "
+                         "kernels move them over the host link; reports the link's copy "
+                         "bandwidth as 'host_link'")
     ap.add_argument("--row-grid", type=int, default=None,
                     help="row kernels: 0 = one row per warp, k = k blocks per SM grid-stride")
     ap.add_argument("--side-priority", type=int, default=None, choices=[0, 1],
@@ -273,7 +277,8 @@ def run_ours(args):
     rows_t = [torch.empty(lab, dtype=torch.int32, device=dev) for _ in range(2)]
     ready = torch.cuda.Event()
     ready.record(stream)  # every step's inputs are resident from here on
-    tbl = binding.MpzchTable(W.capacity, W.dim, W.probes)
+    tbl = binding.MpzchTable(W.capacity, W.dim, W.probes,
+                             flags=binding.MPZCH_VALUES_IN_HOST_MEMORY if args.host_values else 0)
     binding.mpzch_reserve(tbl.h, W.batch)
     if args.row_grid is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_ROW_GRID, args.row_grid)
@@ -387,6 +392,15 @@ def run_ours(args):
         }
         if serving is not None:
             result.update(serving)
+        if args.host_values:
+            link = host_link_bandwidth(torch, dev)
+            # the row update moves each written row over the link twice (read + write)
+            link_bytes = n_written * 2 * 4 * D
+            link_gbs = link_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
+            link["row_update_link_gbs"] = link_gbs
+            link["row_update_frac_of_bidirectional"] = link_gbs / link["bidirectional_gbs"]
+            result["host_link"] = link
+            result["config"]["values"] = "pinned host memory, mapped (host-memory tier)"
         if res_info is not None:
             result["res"] = res_info
     tbl.close()
@@ -395,6 +409,35 @@ def run_ours(args):
         dist.destroy_process_group()
     if result is not None:
         print(json.dumps(result), flush=True)
+
+
+def host_link_bandwidth(torch, dev, nbytes: int = 1 << 30):
+    """Pinned host <-> device copy bandwidth (GB/s): H2D, D2H, and both at once."""
+    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h2 = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d2 = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def timed(fn, reps=3):
+        best = 1e30
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            best = min(best, time.perf_counter() - t0)
+        return best
+    h2d = nbytes / timed(lambda: d.copy_(h, non_blocking=True)) / 1e9
+    d2h = nbytes / timed(lambda: h.copy_(d, non_blocking=True)) / 1e9
+
+    def both():
+        with torch.cuda.stream(s1):
+            d2.copy_(h2, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h.copy_(d, non_blocking=True)
+    bidir = 2 * nbytes / timed(both) / 1e9
+    return {"h2d_gbs": h2d, "d2h_gbs": d2h, "bidirectional_gbs": bidir}
 
 
 def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):

@@ -32,6 +32,7 @@ MPZCH_STATUS_BADAO = 4
 MPZCH_STATUS_INTERNAL = 8
 MPZCH_NPHASES = 7
 MPZCH_OPT_WIDE_ROUNDS = 1
+MPZCH_VALUES_IN_HOST_MEMORY = 1
 MPZCH_OPT_SIDE_PRIORITY = 2
 MPZCH_OPT_ROW_GRID = 3
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
@@ -46,6 +47,7 @@ _lib = C.CDLL(LIB_PATH)
 _p, _i64, _i32 = C.c_void_p, C.c_int64, C.c_int32
 _SIGS = {
     "mpzch_create": [_i64, _i32, _i32, _p, C.POINTER(_p)],
+    "mpzch_create_ex": [_i64, _i32, _i32, C.c_uint32, _p, C.POINTER(_p)],
     "mpzch_destroy": [_p],
     "mpzch_reserve": [_p, _i64, _p],
     "mpzch_lookup": [_p, _p, _i64, _p, _p, _p],
@@ -121,6 +123,13 @@ def lib() -> C.CDLL:
 def mpzch_create(capacity: int, dim: int, probes: int, stream=None) -> C.c_void_p:
     h = C.c_void_p()
     _check("mpzch_create", _lib.mpzch_create(capacity, dim, probes, _stream(stream), C.byref(h)))
+    return h
+
+
+def mpzch_create_ex(capacity: int, dim: int, probes: int, flags: int, stream=None) -> C.c_void_p:
+    h = C.c_void_p()
+    _check("mpzch_create_ex", _lib.mpzch_create_ex(capacity, dim, probes, flags, _stream(stream),
+                                                   C.byref(h)))
     return h
 
 
@@ -362,10 +371,10 @@ def _view(addr: int, shape, dtype, device) -> torch.Tensor:
 class MpzchTable:
     """Owns one table handle; methods forward to the entry points above."""
 
-    def __init__(self, capacity: int, dim: int, probes: int, stream=None):
+    def __init__(self, capacity: int, dim: int, probes: int, stream=None, flags: int = 0):
         self.capacity, self.dim, self.probes = capacity, dim, probes
         self.device = torch.device("cuda", torch.cuda.current_device())
-        self.h = mpzch_create(capacity, dim, probes, stream)
+        self.h = mpzch_create_ex(capacity, dim, probes, flags, stream)
 
     def close(self):
         if getattr(self, "h", None):

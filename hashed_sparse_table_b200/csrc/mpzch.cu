@@ -40,6 +40,30 @@ void dev_free(void* p) {
   if (p) cudaFree(p);
 }
 
+// Pinned host memory mapped into the device address space, zero-filled: the
+// kernels reach it over the host link with the same pointer arithmetic.
+int host_mapped_alloc(void** dev_ptr, void** host_ptr, size_t bytes) {
+  *dev_ptr = *host_ptr = nullptr;
+  if (g_fail_allocs.load() > 0) {
+    g_fail_allocs.fetch_sub(1);
+    return MPZCH_ENOMEM;
+  }
+  if (cudaHostAlloc(host_ptr, bytes, cudaHostAllocMapped | cudaHostAllocPortable) != cudaSuccess) {
+    cudaGetLastError();
+    *host_ptr = nullptr;
+    return MPZCH_ENOMEM;
+  }
+  std::memset(*host_ptr, 0, bytes);
+  if (cudaHostGetDevicePointer(dev_ptr, *host_ptr, 0) != cudaSuccess) {
+    cudaGetLastError();
+    cudaFreeHost(*host_ptr);
+    *host_ptr = nullptr;
+    *dev_ptr = nullptr;
+    return MPZCH_ECUDA;
+  }
+  return MPZCH_OK;
+}
+
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int sm_count() {
@@ -163,7 +187,9 @@ struct mpzch_table {
   // table state (row-indexed arrays)
   long long* keys = nullptr;
   long long* last = nullptr;
-  float* M = nullptr;
+  float* M = nullptr;          // device-accessible address of the values
+  void* M_host = nullptr;      // host allocation when the values live in host memory
+  bool values_on_host = false;
   // insert scratch: three claim arrays of C slots
   unsigned long long* claims[3] = {nullptr, nullptr, nullptr};
   // per-batch scratch, sized for `cap` ids
@@ -239,7 +265,10 @@ void free_all(mpzch_table* t) {
   free_batch_scratch(t);
   dev_free(t->keys);
   dev_free(t->last);
-  dev_free(t->M);
+  if (t->M_host)
+    cudaFreeHost(t->M_host);
+  else
+    dev_free(t->M);
   for (auto& c : t->claims) dev_free(c), c = nullptr;
   dev_free(t->ctr);
   dev_free(t->wcnt);
@@ -607,10 +636,15 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
 }
 
 int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mpzch_table** out) {
+  return mpzch_create_ex(capacity, dim, probes, 0u, stream, out);
+}
+
+int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flags, void* stream,
+                    mpzch_table** out) {
   if (!out) return MPZCH_EINVAL;
   *out = nullptr;
   if (capacity < 1 || capacity > 0x7FFFFFFFLL || dim <= 0 || dim % 4 != 0 || probes < 1 ||
-      (int64_t)probes > capacity)
+      (int64_t)probes > capacity || (flags & ~(uint32_t)MPZCH_VALUES_IN_HOST_MEMORY))
     return MPZCH_EINVAL;
   mpzch_table* t = new (std::nothrow) mpzch_table;
   if (!t) return MPZCH_ENOMEM;
@@ -618,11 +652,18 @@ int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mp
   t->D = dim;
   t->P = probes;
   t->geo = make_geo(capacity, probes);
+  t->values_on_host = (flags & MPZCH_VALUES_IN_HOST_MEMORY) != 0;
   cudaStream_t st = S(stream);
   int rc = MPZCH_OK;
   if (!rc) rc = dev_alloc((void**)&t->keys, capacity * sizeof(long long));
   if (!rc) rc = dev_alloc((void**)&t->last, capacity * sizeof(long long));
-  if (!rc) rc = dev_alloc((void**)&t->M, (size_t)capacity * dim * sizeof(float));
+  if (!rc) {
+    const size_t bytes = (size_t)capacity * dim * sizeof(float);
+    if (t->values_on_host)
+      rc = host_mapped_alloc((void**)&t->M, &t->M_host, bytes);
+    else
+      rc = dev_alloc((void**)&t->M, bytes);
+  }
   for (int i = 0; i < 3 && !rc; ++i)
     rc = dev_alloc((void**)&t->claims[i], capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
@@ -639,7 +680,9 @@ int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mp
   if (!rc) {
     bool ok = cudaMemsetAsync(t->keys, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
               cudaMemsetAsync(t->last, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
-              cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) == cudaSuccess &&
+              (t->values_on_host ||
+               cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) ==
+                   cudaSuccess) &&
               cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
               cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;

@@ -91,6 +91,16 @@ typedef struct {
  * `out`, MPZCH_ENOMEM if an allocation fails (nothing is leaked). */
 MPZCH_API int mpzch_create(int64_t capacity, int32_t dim, int32_t probes, void* stream, mpzch_table** out);
 
+/* As mpzch_create, with flags.  MPZCH_VALUES_IN_HOST_MEMORY: the value rows
+ * M[C][dim] live in pinned host memory mapped into the device's address space
+ * (zero-filled), the identity map, metadata and scratch stay in device memory;
+ * every kernel reaches the values over the host link, so tables larger than
+ * HBM fit (Memory Layer section 2: the 512-d vector table is sharded across
+ * GPU and CPU), at host-link bandwidth.  Other flag bits: MPZCH_EINVAL. */
+#define MPZCH_VALUES_IN_HOST_MEMORY 1u
+MPZCH_API int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flags,
+                              void* stream, mpzch_table** out);
+
 /* Free all device memory of the table (synchronises the device). NULL is a no-op. */
 MPZCH_API int mpzch_destroy(mpzch_table* t);
 

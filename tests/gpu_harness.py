@@ -43,9 +43,10 @@ class RunResult:
     stats: list
 
 
-def make_pair(w: inputs.Workload, track_all: bool = True, track_rows: Optional[np.ndarray] = None):
+def make_pair(w: inputs.Workload, track_all: bool = True, track_rows: Optional[np.ndarray] = None,
+              flags: int = 0):
     from hashed_sparse_table_b200 import binding
-    tbl = binding.MpzchTable(w.capacity, w.dim, w.probes)
+    tbl = binding.MpzchTable(w.capacity, w.dim, w.probes, flags=flags)
     orc = oracle.OracleTable(w.capacity, w.dim, w.probes, track_all=track_all)
     if track_rows is not None:
         orc.track_rows(track_rows)
@@ -69,7 +70,8 @@ def compare_state(tbl, orc, what: str, value_rows: Optional[np.ndarray] = None, 
 def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None, start: int = 0,
              state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
              ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None,
-             fused_step: bool = False, eta: Optional[float] = None) -> RunResult:
+             fused_step: bool = False, eta: Optional[float] = None,
+             flags: int = 0) -> RunResult:
     """Runs steps [start, start+steps) of workload w on both sides.
 
     Per step: lookup of the labeled ids, fused gather (with the always-on concat
@@ -78,7 +80,7 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
     counters, and the table state every `state_every` / `values_every` steps."""
     from hashed_sparse_table_b200 import binding
     if tbl is None:
-        tbl, orc = make_pair(w)
+        tbl, orc = make_pair(w, flags=flags)
     if wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, wide_rounds)
     if eta is not None:
@@ -139,14 +141,14 @@ def snapshot_from_export(capacity: int, dim: int, rows: np.ndarray, q: np.ndarra
     return snap_keys, snap_q, snap_s
 
 
-def run_pipelined(w: inputs.Workload, steps: Optional[int] = None):
+def run_pipelined(w: inputs.Workload, steps: Optional[int] = None, flags: int = 0):
     """All steps' inputs uploaded first, then every step issued back to back as
     a pipelined mpzch_train_step (inputs_ready = one event after the uploads),
     each step with its own output buffers; then every output and the final
     table are compared with the oracle run step by step."""
     from hashed_sparse_table_b200 import binding
     T = w.steps if steps is None else steps
-    tbl, orc = make_pair(w)
+    tbl, orc = make_pair(w, flags=flags)
     dev = tbl.device
     ao = inputs.author_table(w)
     ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None

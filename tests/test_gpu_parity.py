@@ -111,6 +111,33 @@ def test_learning_rate_rejects_non_finite():
             binding.mpzch_set_learning_rate(tbl.h, bad)
 
 
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress", "nonpow2"])
+@pytest.mark.parametrize("fused", [False, True])
+def test_values_in_host_memory_bit_exact(name, fused):
+    from hashed_sparse_table_b200 import binding
+    run_pair(SCALED[name], fused_step=fused, flags=binding.MPZCH_VALUES_IN_HOST_MEMORY)
+
+
+def test_values_in_host_memory_pipelined_and_export():
+    from hashed_sparse_table_b200 import binding
+    from gpu_harness import run_pipelined
+    w = SCALED["c3_small"]
+    tbl, orc = run_pipelined(w, flags=binding.MPZCH_VALUES_IN_HOST_MEMORY)
+    rows_d, cnt_d = tbl.select_written_since(w.steps - 10)
+    n = int(cnt_d.item())
+    orows = orc.select_written_since(w.steps - 10)
+    q, s, k = tbl.export_int8(rows_d, n=w.capacity, dev_n=cnt_d)
+    oq, os_, ok = orc.export_int8(orows)
+    assert_bitwise(q[:n].cpu().numpy(), oq, "int8 export from host values")
+    assert_bitwise(s[:n].cpu().numpy(), os_, "scales from host values")
+
+
+def test_create_ex_rejects_unknown_flags():
+    from hashed_sparse_table_b200 import binding
+    with pytest.raises(binding.MpzchError):
+        binding.mpzch_create_ex(64, 4, 2, 0x80)
+
+
 def test_repeatable_bytes():
     w = SCALED["c3_small"].scaled(steps=6)
     a = run_pair(w)
