@@ -47,6 +47,9 @@ def lib():
         L.orc_splitmix64.argtypes = [C.c_uint64]
         L.orc_home_slot.restype = i64
         L.orc_home_slot.argtypes = [i64, i64]
+        L.orc_owner.restype = i32
+        L.orc_owner.argtypes = [i64, i32]
+        L.orc_owners.argtypes = [p, i64, i32, p]
         L.orc_create.argtypes = [i64, i32, i32, i32, C.POINTER(p)]
         L.orc_destroy.argtypes = [p]
         L.orc_destroy.restype = None
@@ -68,7 +71,8 @@ def lib():
         for f in ("orc_create", "orc_track_rows", "orc_lookup", "orc_gather_fused", "orc_dedup",
                   "orc_writeback", "orc_select_written_since", "orc_quantize_row",
                   "orc_export_int8", "orc_serve_gather", "orc_state", "orc_get_row",
-                  "orc_set_row", "orc_set_state", "orc_get_rows", "orc_set_learning_rate"):
+                  "orc_set_row", "orc_set_state", "orc_get_rows", "orc_set_learning_rate",
+                  "orc_owners"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -88,6 +92,18 @@ def splitmix64(x: int) -> int:
 
 def home_slot(key: int, capacity: int) -> int:
     return int(lib().orc_home_slot(key, capacity))
+
+
+def owner(key: int, n_owners: int) -> int:
+    return int(lib().orc_owner(key, n_owners))
+
+
+def owners(ids: np.ndarray, n_owners: int) -> np.ndarray:
+    ids = _c(ids, np.int64)
+    out = np.empty(ids.size, np.int32)
+    rc = lib().orc_owners(_ptr(ids), ids.size, n_owners, _ptr(out))
+    assert rc == ORC_OK, rc
+    return out
 
 
 def dedup(ids: np.ndarray):
@@ -245,3 +261,78 @@ class OracleTable:
 
 def oracle_lib_path() -> str:
     return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmpzch_oracle.so")
+
+
+class ShardedOracle:
+    """Hash-owner sharding of the table over G shards, one per rank.
+
+    Memory Layer section 2 shards the table across devices and keeps the
+    distributed lookup's all-to-all exchange; MTGR section 3.3 exchanges ids
+    all-to-all and dedups twice, before and after the exchange.  Key k lives
+    in shard owner(k) = (splitmix64(k) >> 32) mod G, an ordinary oracle table
+    of `shard_capacity` rows.  Global row of shard s, local row r: s*C_s + r.
+
+    One step, for the batches of ranks 0..G-1:
+      1. each rank's labeled ids are looked up (and gathered, with the
+         rank's always-on rows) at their owners, on the tables as they were
+         before the step;
+      2. each rank dedups its whole batch (first occurrence keeps its e row),
+         sends each distinct id with its e row to its owner; an owner receives
+         the ids of ranks 0..G-1 in rank order, each rank's in batch order, and
+         runs the Writeback on that batch, which dedups again.
+    """
+
+    def __init__(self, n_shards: int, shard_capacity: int, dim: int, probes: int):
+        self.G, self.Cs, self.dim, self.probes = n_shards, shard_capacity, dim, probes
+        self.shards = [OracleTable(shard_capacity, dim, probes) for _ in range(n_shards)]
+
+    def close(self):
+        for t in self.shards:
+            t.close()
+
+    def lookup_gather(self, ids, ao=None, ao_rows=None):
+        """Rows (global), hit and gathered features of one rank's labeled ids."""
+        ids = _c(ids, np.int64)
+        n = ids.size
+        own = owners(ids, self.G)
+        rows = np.full(n, -1, np.int32)
+        hit = np.zeros(n, np.uint8)
+        width = self.dim + (0 if ao is None else ao.shape[1])
+        out = np.zeros((n, width), np.float32)
+        rc_all = ORC_OK
+        for s in range(self.G):
+            at = np.nonzero(own == s)[0]
+            if at.size == 0:
+                continue
+            rc, r, h = self.shards[s].lookup(ids[at])
+            rc_all = rc_all or rc
+            out[at] = self.shards[s].gather_fused(r, h, ao, None if ao_rows is None else ao_rows[at])
+            rows[at] = np.where(h != 0, r + s * self.Cs, -1)
+            hit[at] = h
+        return rc_all, rows, hit, out
+
+    def routed_batches(self, rank_ids, rank_e):
+        """What each owner receives: (ids, e) per shard after the first dedup."""
+        recv_ids = [[] for _ in range(self.G)]
+        recv_e = [[] for _ in range(self.G)]
+        for ids, e in zip(rank_ids, rank_e):  # ranks in order
+            uniq, pos = dedup(ids)
+            own = owners(uniq, self.G)
+            for s in range(self.G):
+                sel = own == s
+                recv_ids[s].append(uniq[sel])
+                recv_e[s].append(_c(e, np.float32)[pos[sel]])
+        return ([np.concatenate(x) for x in recv_ids],
+                [np.concatenate(x).reshape(-1, self.dim) for x in recv_e])
+
+    def writeback(self, rank_ids, rank_e, step):
+        """Per-shard (rc, stats) of the step's Writeback."""
+        recv_ids, recv_e = self.routed_batches(rank_ids, rank_e)
+        return [self.shards[s].writeback(recv_ids[s], recv_e[s], step) for s in range(self.G)]
+
+    def state(self, s):
+        return self.shards[s].state()
+
+    def values(self, s):
+        return self.shards[s].values()
+

@@ -62,6 +62,21 @@ extern "C" int64_t orc_home_slot(int64_t key, int64_t capacity) {
   return (int64_t)(orc_splitmix64((uint64_t)key) % (uint64_t)capacity);
 }
 
+// Hash-owner sharding (Memory Layer section 2: the table is sharded across
+// devices and the distributed lookup keeps its all-to-all path; MTGR section
+// 3.3: ids are exchanged all-to-all between devices).  The owning shard takes
+// the upper 32 bits of the same SplitMix64 output, so the shard and the home
+// slot inside the shard (lower bits, mod C) come from different bits.
+extern "C" int32_t orc_owner(int64_t key, int32_t n_owners) {
+  return (int32_t)((orc_splitmix64((uint64_t)key) >> 32) % (uint64_t)n_owners);
+}
+
+extern "C" int orc_owners(const int64_t* ids, int64_t n, int32_t n_owners, int32_t* out) {
+  if (n_owners < 1 || (n > 0 && (!ids || !out))) return ORC_EINVAL;
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_owner(ids[i], n_owners);
+  return ORC_OK;
+}
+
 // The P-slot probe window of a key, in probe order.
 static int64_t window_slot(const orc_table* t, int64_t key, int32_t j) {
   return (orc_home_slot(key, t->C) + j) % t->C;

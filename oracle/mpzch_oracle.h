@@ -40,6 +40,11 @@ uint64_t orc_splitmix64(uint64_t x);
 /* Start slot h(k) = splitmix64(k) mod C. */
 int64_t orc_home_slot(int64_t key, int64_t capacity);
 
+/* Owning shard of a key among n_owners shards: (splitmix64(k) >> 32) mod n_owners. */
+int32_t orc_owner(int64_t key, int32_t n_owners);
+/* out[i] = orc_owner(ids[i], n_owners) for i < n. */
+int orc_owners(const int64_t* ids, int64_t n, int32_t n_owners, int32_t* out);
+
 /* track_all != 0: keep every value row (C*D floats of host memory).
  * track_all == 0: keep only rows later registered with orc_track_rows; the
  * identity map (keys, last-access) is always kept in full. */

@@ -6,6 +6,11 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+# The mutation tests point this at a folder holding a deliberately broken copy
+# of the oracle package, imported in place of the real one.
+MUTANT = os.environ.get("MPZCH_ORACLE_PKG_PARENT")
+if MUTANT:
+    sys.path.insert(0, MUTANT)
 HERE = os.path.dirname(os.path.abspath(__file__))
 if HERE not in sys.path:
     sys.path.insert(0, HERE)

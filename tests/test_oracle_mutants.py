@@ -46,10 +46,27 @@ MUTANTS = [
     ("int8 scale divides by 128", "const float s = a / 127.0f;", "const float s = a / 128.0f;"),
     ("int8 rounds by truncation", "float v = std::nearbyint(x[d] / s);",
      "float v = std::trunc(x[d] / s);"),
+    ("owner taken from the low hash bits",
+     "(int32_t)((orc_splitmix64((uint64_t)key) >> 32) % (uint64_t)n_owners)",
+     "(int32_t)(orc_splitmix64((uint64_t)key) % (uint64_t)n_owners)"),
     ("serving divides by the scale",
      "(float)snap_q[r * (int64_t)dim + d] * snap_scale[r]",
      "(float)snap_q[r * (int64_t)dim + d] / snap_scale[r]"),
 ]
+
+
+# Mistakes in the sharded oracle (Python, oracle/__init__.py): (name, text, replacement)
+PY_MUTANTS = [
+    ("owner receives ranks in reverse order",
+     "for ids, e in zip(rank_ids, rank_e):  # ranks in order",
+     "for ids, e in list(zip(rank_ids, rank_e))[::-1]:"),
+    ("first dedup sends the e row at the distinct id's index, not its batch position",
+     "recv_e[s].append(_c(e, np.float32)[pos[sel]])",
+     "recv_e[s].append(_c(e, np.float32)[np.nonzero(sel)[0]])"),
+    ("global row misses the shard offset", "rows[at] = np.where(h != 0, r + s * self.Cs, -1)",
+     "rows[at] = np.where(h != 0, r, -1)"),
+]
+PKG = os.path.join(ROOT, "oracle")
 
 
 def build_mutant(tmp, old, new):
@@ -71,5 +88,34 @@ def test_pins_catch_planted_mistake(tmp_path, name, old, new):
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join("tests", "test_oracle_pins.py")],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode != 0, f"planted mistake survived every pin: {name}\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout, r.stdout[-2000:]
+
+
+def run_pins_on_py_copy(tmp_path, old, new):
+    import oracle
+    lib = oracle.lib()._name  # the real C++ oracle, already built
+    dst = tmp_path / "oracle"
+    dst.mkdir()
+    src = open(os.path.join(PKG, "__init__.py")).read()
+    assert src.count(old) == 1, f"mutation site not unique: {old!r}"
+    (dst / "__init__.py").write_text(src.replace(old, new))
+    shutil.copy(os.path.join(PKG, "build.py"), dst / "build.py")
+    env = dict(os.environ, MPZCH_ORACLE_LIB=lib, MPZCH_ORACLE_PKG_PARENT=str(tmp_path))
+    return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           os.path.join("tests", "test_oracle_pins.py"), "-k",
+                           "owner or shard or exchange"],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+
+
+def test_unmutated_copy_of_the_sharded_oracle_passes(tmp_path):
+    """Control: the copy mechanism itself breaks nothing."""
+    r = run_pins_on_py_copy(tmp_path, "class ShardedOracle:", "class ShardedOracle:")
+    assert r.returncode == 0, r.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTANTS, ids=[m[0] for m in PY_MUTANTS])
+def test_pins_catch_planted_mistake_in_sharded_oracle(tmp_path, name, old, new):
+    r = run_pins_on_py_copy(tmp_path, old, new)
     assert r.returncode != 0, f"planted mistake survived every pin: {name}\n{r.stdout[-2000:]}"
     assert "failed" in r.stdout, r.stdout[-2000:]

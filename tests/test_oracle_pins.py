@@ -435,3 +435,149 @@ def test_zipf_sampler_matches_exact_pmf(alpha, n):
     chi2 = (((f - p * s.size) ** 2) / (p * s.size)).sum()
     # n-1 degrees of freedom: mean n-1, sd sqrt(2(n-1)); 6 sd is a generous gate
     assert chi2 < (n - 1) + 6 * np.sqrt(2 * (n - 1)), chi2
+
+
+# ---------------------------------------------------------------- hash-owner sharding
+def _signed(x):
+    return x - (1 << 64) if x >= 1 << 63 else x
+
+
+def test_owner_takes_the_upper_bits_of_published_outputs():
+    g = load("splitmix64_seed0.json")
+    gamma = int(g["gamma"], 16)
+    for i, want in enumerate(g["outputs_seed0"]):
+        state = (i * gamma) & ((1 << 64) - 1)
+        h = int(want, 16)
+        for G in (1, 2, 3, 8, 1000):
+            assert oracle.owner(_signed(state), G) == (h >> 32) % G
+    keys = np.random.default_rng(3).integers(0, 2**63 - 1, size=500, dtype=np.int64)
+    for G in (2, 5, 8):
+        want = np.array([(pyref.splitmix64(int(k)) >> 32) % G for k in keys])
+        assert np.array_equal(oracle.owners(keys, G), want)
+
+
+@pytest.mark.parametrize("G", [2, 3, 8])
+def test_owner_spreads_consecutive_keys_evenly(G):
+    own = oracle.owners(np.arange(240_000, dtype=np.int64), G)
+    f = np.bincount(own, minlength=G)
+    expect = own.size / G
+    chi2 = (((f - expect) ** 2) / expect).sum()
+    assert chi2 < (G - 1) + 6 * np.sqrt(2 * (G - 1)), (f, chi2)
+
+
+def _rank_batches(seed, G, steps, n, n_keys, dim, dup_frac=0.0):
+    """Zipf-like skewed batches per rank and step (heavy cross-rank overlap)."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for t in range(steps):
+        ranks = []
+        for r in range(G):
+            ids = (rng.pareto(1.1, size=n) * 7).astype(np.int64) % n_keys
+            e = rng.standard_normal((n, dim)).astype(np.float32)
+            ranks.append((ids, e))
+        out.append(ranks)
+    return out
+
+
+def test_sharded_single_shard_is_the_table():
+    C, D, P = 64, 8, 4
+    so = oracle.ShardedOracle(1, C, D, P)
+    one = OracleTable(C, D, P)
+    ao = np.random.default_rng(1).standard_normal((32, 4)).astype(np.float32)
+    saw_evict = 0
+    for t, ranks in enumerate(_rank_batches(5, 1, 12, 60, 400, D)):
+        ids, e = ranks[0]
+        lab = ids[:25]
+        aor = (lab % 32).astype(np.int32)
+        rc, rows, hit, out = so.lookup_gather(lab, ao, aor)
+        rc1, rows1, hit1 = one.lookup(lab)
+        assert rc == rc1 == 0
+        assert np.array_equal(rows, rows1) and np.array_equal(hit, hit1)
+        assert np.array_equal(out.view(np.uint32), one.gather_fused(rows1, hit1, ao, aor).view(np.uint32))
+        (rc, st), = so.writeback([ids], [e], t)
+        rc1, st1 = one.writeback(ids, e, t)
+        assert rc == rc1 == 0
+        for k in ("n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped"):
+            assert st[k] == st1[k], (t, k)
+        assert st["n_ids"] == st["n_unique"]  # the owner receives distinct ids only
+        saw_evict += st1["n_evicted"]
+        k0, l0, _ = so.state(0)
+        k1, l1, _ = one.state()
+        assert np.array_equal(k0, k1) and np.array_equal(l0, l1)
+        assert np.array_equal(so.values(0).view(np.uint32), one.values().view(np.uint32))
+    assert saw_evict > 0  # the case exercises eviction
+
+
+def test_sharded_without_eviction_matches_one_table_per_key():
+    """With room for every key, each key's row content and last step depend on
+    its own history only, so G shards fed the rank-order concatenation must hold
+    exactly what one table holds.  Cross-rank duplicates with different e rows
+    make the rank order and the first-occurrence rule visible."""
+    G, Cs, D, P = 4, 4096, 8, 8
+    so = oracle.ShardedOracle(G, Cs, D, P)
+    one = OracleTable(1 << 15, D, P)
+    ao = np.random.default_rng(2).standard_normal((64, 4)).astype(np.float32)
+    cross_dups = 0
+    for t, ranks in enumerate(_rank_batches(6, G, 10, 80, 600, D)):
+        concat = np.concatenate([ids for ids, _ in ranks])
+        for r, (ids, e) in enumerate(ranks):
+            lab = ids[:30]
+            aor = (lab % 64).astype(np.int32)
+            rc, rows, hit, out = so.lookup_gather(lab, ao, aor)
+            rc1, rows1, hit1 = one.lookup(lab)
+            assert np.array_equal(hit, hit1), (t, r)
+            assert np.array_equal(out.view(np.uint32),
+                                  one.gather_fused(rows1, hit1, ao, aor).view(np.uint32)), (t, r)
+            own = oracle.owners(lab, G)
+            assert np.all((rows < 0) | (rows // Cs == own))
+        sets = [set(ids.tolist()) for ids, _ in ranks]
+        cross_dups += sum(len(sets[a] & sets[b]) for a in range(G) for b in range(a + 1, G))
+        res = so.writeback([ids for ids, _ in ranks], [e for _, e in ranks], t)
+        rc1, st1 = one.writeback(concat, np.concatenate([e for _, e in ranks]), t)
+        assert all(rc == 0 for rc, _ in res) and rc1 == 0
+        assert st1["n_evicted"] == 0 and all(st["n_evicted"] == 0 for _, st in res)
+        assert sum(st["n_unique"] for _, st in res) == st1["n_unique"]
+        assert sum(st["n_inserted"] for _, st in res) == st1["n_inserted"]
+    assert cross_dups > 100
+    keys1, last1, _ = one.state()
+    live = np.nonzero(keys1 >= 0)[0]
+    vals1 = one.values()
+    placed = 0
+    for s in range(G):
+        ks, ls, _ = so.state(s)
+        vs = so.values(s)
+        live_s = np.nonzero(ks >= 0)[0]
+        assert np.all(oracle.owners(ks[live_s], G) == s)
+        where = {int(k): i for i, k in zip(live_s, ks[live_s])}
+        for r in live:
+            k = int(keys1[r])
+            if oracle.owner(k, G) != s:
+                continue
+            i = where[k]
+            assert ls[i] == last1[r]
+            assert np.array_equal(vs[i].view(np.uint32), vals1[r].view(np.uint32)), k
+            placed += 1
+    assert placed == live.size
+
+
+def test_dedup_before_the_exchange_changes_no_result():
+    """Sending every id (no first dedup) must leave the owners in the same
+    state: the owner's Writeback keeps the first occurrence in rank order."""
+    G, Cs, D, P = 3, 48, 8, 4
+    a = oracle.ShardedOracle(G, Cs, D, P)
+    b = [OracleTable(Cs, D, P) for _ in range(G)]
+    for t, ranks in enumerate(_rank_batches(7, G, 10, 70, 500, D)):
+        ids_all = np.concatenate([ids for ids, _ in ranks])
+        e_all = np.concatenate([e for _, e in ranks])
+        res = a.writeback([ids for ids, _ in ranks], [e for _, e in ranks], t)
+        own = oracle.owners(ids_all, G)
+        for s in range(G):
+            rc, st = b[s].writeback(ids_all[own == s], e_all[own == s], t)
+            assert rc == 0 and res[s][0] == 0
+            for k in ("n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped"):
+                assert st[k] == res[s][1][k], (t, s, k)
+    for s in range(G):
+        ka, la, _ = a.state(s)
+        kb, lb, _ = b[s].state()
+        assert np.array_equal(ka, kb) and np.array_equal(la, lb)
+        assert np.array_equal(a.values(s).view(np.uint32), b[s].values().view(np.uint32))
