@@ -82,6 +82,9 @@ def parse():
                     help="lookup, gather and Writeback as three calls instead of mpzch_train_step")
     ap.add_argument("--wide-rounds", type=int, default=None,
                     help="grid-wide insert conflict rounds before the single-block finisher")
+    ap.add_argument("--shard", action="store_true",
+                    help="hash-owner sharding: one shard per GPU, ids routed to their owner "
+                         "with NCCL all-to-all (a one-rank group at --gpus 1)")
     ap.add_argument("--e-pool", type=int, default=inputs.E_POOL,
                     help="distinct item-tower target batches cycled through (memory bound for "
                          "profiling runs)")
@@ -599,10 +602,129 @@ def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
             "d2h_bytes_per_step": 7 * 8, "ms_per_step": ms / K}
 
 
+def run_sharded(args):
+    """The sharded step (partition by owner, first dedup, NCCL all-to-all of ids
+    and e rows, owner lookup / gather / Writeback, answers back, combine) on
+    every rank; each rank holds one shard of W.capacity rows and draws its own
+    id stream from the same key universe, so ranks share keys."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    from hashed_sparse_table_b200 import binding, sharded
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world == 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        if "MASTER_PORT" not in os.environ:
+            with socket.socket() as so:
+                so.bind(("127.0.0.1", 0))
+                os.environ["MASTER_PORT"] = str(so.getsockname()[1])
+        dist.init_process_group("nccl", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    K, Wm, Pf = args.steps, args.warmup, args.prefill
+    total = Pf + Wm + K
+    host = [host_step(t, rank) for t in range(total)]
+    ids_d = [torch.from_numpy(h[0]).to(dev) for h in host]
+    aor_d = [torch.from_numpy(h[1]).to(dev) for h in host]
+    E = max(1, min(args.e_pool, inputs.E_POOL))
+    e_d = [torch.from_numpy(inputs.step_e(W, t)).to(dev) for t in range(E)]
+    ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
+    lab = W.labeled
+    rows = torch.empty(lab, dtype=torch.int32, device=dev)
+    hit = torch.empty(lab, dtype=torch.uint8, device=dev)
+    out = torch.empty((lab, W.dim + W.ao_dim), dtype=torch.float32, device=dev)
+    stats = torch.zeros((total, 7), dtype=torch.int64, device=dev)
+    shard = sharded.ShardedMpzch(W.capacity, W.dim, W.probes, sharded.DistExchange())
+    binding.mpzch_reserve(shard.table.h, W.batch * world)
+    sent = {"lookup": 0, "writeback": 0}
+
+    def step(t):
+        tr = {}
+        shard.train_step(ids_d[t], lab, e_d[t % E], t, ao_d, aor_d[t], rows, hit, out, stats[t],
+                         trace=tr)
+        return tr
+
+    for t in range(Pf + Wm):
+        step(t)
+    binding.mpzch_trace_read(shard.table.h)
+    binding.mpzch_trace_enable(shard.table.h, True)
+    clocks = ClockSampler(gpu_id_for(local)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.1)
+    dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    l0 = binding.mpzch_launch_count()
+    ev0.record(stream)
+    for t in range(Pf + Wm, total):
+        tr = step(t)
+        sent["lookup"] += tr["sent_lookup"]
+        sent["writeback"] += tr["sent_writeback"]
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    launches = binding.mpzch_launch_count() - l0
+    dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    trace = binding.mpzch_trace_read(shard.table.h)
+    clk = clocks.stop() if clocks else None
+    st = stats[Pf + Wm:].cpu().numpy()
+    n_unique = int(st[:, 1].sum())
+    n_written = int((st[:, 1] - st[:, 5]).sum())
+    tot_units, max_ms = reduce_over_ranks(n_unique, ms, dev)
+    D, A = W.dim, W.ao_dim
+    wb_ms, wb_launches = trace["writeback"]
+    wb_bytes = n_written * (12 * D + 8)
+    wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
+    peak, peak_kind = load_peaks()
+    # bytes this rank hands to the all-to-all per step: ids out, ids + e rows
+    # out, and the owners' answers (row + D values) back
+    x_bytes = (sent["lookup"] * (8 + 4 + 4 * D) + sent["writeback"] * (8 + 4 * D)) / K
+    table_ms = sum(v[0] for v in trace.values())
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": tot_units / (max_ms * 1e-3), "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": max_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded Zipf id streams, N(0,1) item-tower targets)",
+            "config": config_dict({
+                "prefill_steps": Pf, "shards": world,
+                "parallelism": f"hash-owner sharding: one {W.capacity}-row shard per GPU, ids, "
+                               "e rows and lookup answers exchanged all-to-all (NCCL)"}),
+            "gpu_launches": launches,
+            "roofline": {"bound": "hbm", "kernel": "k_writeback", "achieved": wb_gbs,
+                         "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": wb_gbs / peak, "traffic": None,
+                         "bytes_per_launch": wb_bytes / max(1, wb_launches),
+                         "avg_launch_us": wb_ms * 1e3 / max(1, wb_launches)},
+            "phase_ms_per_step": {k: v[0] / K for k, v in trace.items() if v[1]},
+            "partition_exchange_combine_ms_per_step": (ms - table_ms) / K,
+            "exchange_bytes_per_step_rank0": x_bytes,
+            "unique_rows_per_step": n_unique / K,
+            "clocks": clk, "cpu_baseline": None, "e2e": None,
+        }
+    shard.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    if result is not None:
+        print(json.dumps(result), flush=True)
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard:
+        run_sharded(args)
     else:
         run_ours(args)
 

@@ -75,6 +75,9 @@ _SIGS = {
     "mpzch_res_latency": [_p, C.POINTER(C.c_double), C.POINTER(C.c_double),
                           C.POINTER(C.c_double), C.POINTER(_i64), C.POINTER(_i64)],
     "mpzch_res_destroy": [_p],
+    "mpzch_owner_partition": [_p, _p, _i64, _p, _i32, _p, _i32, _p, _p, _p, _p, _p, _i64, _p],
+    "mpzch_owner_combine": [_p, _p, _i64, _i32, _i64, _p, _p, _i32, _p, _i64, _i32, _p, _p, _p,
+                            _p, _p, _p],
 }
 for _name, _args in _SIGS.items():
     _f = getattr(_lib, _name)
@@ -82,6 +85,9 @@ for _name, _args in _SIGS.items():
     _f.restype = C.c_int
 _lib.mpzch_launch_count.argtypes = []
 _lib.mpzch_launch_count.restype = _i64
+_lib.mpzch_owner_partition_workspace.argtypes = [_i64, _i32]
+_lib.mpzch_owner_partition_workspace.restype = _i64
+MPZCH_MAX_OWNERS = 256
 
 
 class MpzchError(RuntimeError):
@@ -366,6 +372,64 @@ def _view(addr: int, shape, dtype, device) -> torch.Tensor:
     t = torch.as_tensor(_Iface(), device=device)
     assert t.numel() == numel and t.element_size() == itemsize
     return t
+
+
+def mpzch_owner_partition_workspace(n: int, n_owners: int) -> int:
+    b = _lib.mpzch_owner_partition_workspace(n, n_owners)
+    if b < 0:
+        raise MpzchError("mpzch_owner_partition_workspace", MPZCH_EINVAL)
+    return b
+
+
+def mpzch_owner_partition(ids, n_owners: int, ids_out, pos_out, counts, workspace, src_pos=None,
+                          dev_n=None, e=None, e_out=None, stream=None) -> None:
+    _need(ids, torch.int64, "ids")
+    _need(ids_out, torch.int64, "ids_out")
+    _need(pos_out, torch.int32, "pos_out")
+    _need(counts, torch.int64, "counts")
+    _need(workspace, torch.uint8, "workspace")
+    if src_pos is not None:
+        _need(src_pos, torch.int32, "src_pos")
+    if dev_n is not None:
+        _need(dev_n, torch.int64, "dev_n")
+    dim = 0
+    if e is not None:
+        _need(e, torch.float32, "e")
+        _need(e_out, torch.float32, "e_out")
+        dim = e.shape[1]
+        assert e_out.dim() == 2 and e_out.shape[1] == dim
+    n = ids.numel()
+    assert ids_out.numel() >= n and pos_out.numel() >= n and counts.numel() >= n_owners
+    assert e_out is None or e_out.shape[0] >= n
+    _check("mpzch_owner_partition", _lib.mpzch_owner_partition(
+        _ptr(ids), _ptr(src_pos), n, _ptr(dev_n), n_owners, _ptr(e), dim, _ptr(ids_out),
+        _ptr(pos_out), _ptr(e_out), _ptr(counts), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+
+
+def mpzch_owner_combine(send_ids, pos, n_owners: int, shard_capacity: int, recv_rows, recv_feat,
+                        rows, hit, out, ao_table=None, ao_rows=None, status=None, stream=None,
+                        n=None) -> None:
+    n = send_ids.numel() if n is None else n
+    _need(send_ids, torch.int64, "send_ids")
+    _need(pos, torch.int32, "pos")
+    _need(recv_rows, torch.int32, "recv_rows")
+    _need(recv_feat, torch.float32, "recv_feat")
+    _need(rows, torch.int32, "rows")
+    _need(hit, torch.uint8, "hit")
+    _need(out, torch.float32, "out")
+    ao_n, ao_dim = 0, 0
+    if ao_table is not None:
+        _need(ao_table, torch.float32, "ao_table")
+        _need(ao_rows, torch.int32, "ao_rows")
+        ao_n, ao_dim = ao_table.shape
+    if status is not None:
+        _need(status, torch.int32, "status")
+    assert recv_rows.numel() >= n and recv_feat.dim() == 2 and recv_feat.shape[0] >= n
+    _check("mpzch_owner_combine", _lib.mpzch_owner_combine(
+        _ptr(send_ids), _ptr(pos), n, n_owners, shard_capacity, _ptr(recv_rows), _ptr(recv_feat),
+        recv_feat.shape[1], _ptr(ao_table), ao_n, ao_dim, _ptr(ao_rows), _ptr(rows), _ptr(hit),
+        _ptr(out), _ptr(status), _stream(stream)))
 
 
 class MpzchTable:

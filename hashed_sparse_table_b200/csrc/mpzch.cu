@@ -919,6 +919,67 @@ int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probe
   return after_launch();
 }
 
+int64_t mpzch_owner_partition_workspace(int64_t n, int32_t n_owners) {
+  if (n < 0 || n > 0x7FFFFFFFLL || n_owners < 1 || n_owners > kMaxOwners) return -1;
+  const int64_t nb = (n + kPartTile - 1) / kPartTile;
+  return ((nb * n_owners * (int64_t)sizeof(int32_t)) + 255) / 256 * 256;
+}
+
+int mpzch_owner_partition(const int64_t* ids, const int32_t* src_pos, int64_t n,
+                          const int64_t* dev_n, int32_t n_owners, const float* e, int32_t dim,
+                          int64_t* ids_out, int32_t* pos_out, float* e_out, int64_t* dev_counts,
+                          void* workspace, int64_t workspace_bytes, void* stream) {
+  const int64_t need = mpzch_owner_partition_workspace(n, n_owners);
+  if (need < 0 || !dev_counts) return MPZCH_EINVAL;
+  if (e && (dim <= 0 || dim % 4 != 0 || !e_out || (reinterpret_cast<uintptr_t>(e) & 15) ||
+            (reinterpret_cast<uintptr_t>(e_out) & 15)))
+    return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  const int nb = (int)((n + kPartTile - 1) / kPartTile);
+  if (n > 0 && (!ids || !ids_out || !pos_out || !workspace || workspace_bytes < need))
+    return MPZCH_EINVAL;
+  int32_t* blk = static_cast<int32_t*>(workspace);
+  const long long* dn = reinterpret_cast<const long long*>(dev_n);
+  long long* cnt = reinterpret_cast<long long*>(dev_counts);
+  if (nb == 0) {  // empty batch: every owner gets nothing
+    return cudaMemsetAsync(dev_counts, 0, sizeof(int64_t) * n_owners, st) == cudaSuccess
+               ? MPZCH_OK
+               : MPZCH_ECUDA;
+  }
+  const long long* k = reinterpret_cast<const long long*>(ids);
+  int rc = launch(k_owner_count, nb, kPartTile, st, false, k, n, dn, (int)n_owners, blk);
+  if (!rc) rc = launch(k_owner_offsets, 1, 1024, st, true, blk, nb, (int)n_owners, cnt);
+  if (!rc)
+    rc = launch(k_owner_scatter, nb, kPartTile, st, true, k, src_pos, n, dn, (int)n_owners,
+                static_cast<const int32_t*>(blk), reinterpret_cast<const float4*>(e),
+                e ? dim / 4 : 0, reinterpret_cast<long long*>(ids_out), pos_out,
+                reinterpret_cast<float4*>(e_out));
+  return rc;
+}
+
+int mpzch_owner_combine(const int64_t* send_ids, const int32_t* pos, int64_t n, int32_t n_owners,
+                        int64_t shard_capacity, const int32_t* recv_rows, const float* recv_feat,
+                        int32_t dim, const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
+                        const int32_t* ao_rows, int32_t* rows, uint8_t* hit, float* out,
+                        int32_t* dev_status, void* stream) {
+  if (n < 0 || n > 0x7FFFFFFFLL || n_owners < 1 || n_owners > kMaxOwners || shard_capacity < 1 ||
+      (int64_t)n_owners * shard_capacity > 0x7FFFFFFFLL || dim <= 0 || dim % 4 != 0)
+    return MPZCH_EINVAL;
+  if (ao_table && (ao_dim <= 0 || ao_dim % 4 != 0 || ao_nrows < 1 || !ao_rows)) return MPZCH_EINVAL;
+  if (!ao_table && (ao_dim != 0 || ao_nrows != 0 || ao_rows)) return MPZCH_EINVAL;
+  if (n == 0) return MPZCH_OK;
+  if (!send_ids || !pos || !recv_rows || !recv_feat || !rows || !hit || !out) return MPZCH_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(recv_feat) & 15) ||
+      (reinterpret_cast<uintptr_t>(ao_table) & 15))
+    return MPZCH_EINVAL;
+  cudaStream_t st = S(stream);
+  return launch(k_owner_combine, grid_for(n * 32, kBlock), kBlock, st, false,
+                reinterpret_cast<const long long*>(send_ids), pos, n, (int)n_owners,
+                shard_capacity, recv_rows, reinterpret_cast<const float4*>(recv_feat), dim / 4,
+                reinterpret_cast<const float4*>(ao_table), ao_nrows, ao_table ? ao_dim / 4 : 0,
+                ao_rows, rows, hit, reinterpret_cast<float4*>(out), dev_status);
+}
+
 int mpzch_state_views(mpzch_table* t, int64_t** keys, int64_t** last, float** M) {
   if (!t) return MPZCH_EINVAL;
   if (keys) *keys = reinterpret_cast<int64_t*>(t->keys);

@@ -1186,4 +1186,215 @@ __global__ void __launch_bounds__(kBlock) k_serve_gather(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Hash-owner sharding (Memory Layer section 2: the table is sharded across
+// devices and the distributed lookup keeps its all-to-all path; MTGR section
+// 3.3: ids are exchanged all-to-all, with a dedup before and after).  Key k
+// belongs to shard owner(k) = (splitmix64(k) >> 32) mod G.
+//
+// The partition is a stable counting sort by owner in three launches over
+// tiles of kPartTile ids (one id per thread):
+//   k_owner_count    per tile and owner, the number of ids (owner-major matrix);
+//   k_owner_offsets  one block: exclusive scan of that matrix in owner-major
+//                    order (= each tile's first output slot per owner) and the
+//                    per-owner totals;
+//   k_owner_scatter  each id's slot = its tile's offset for its owner + the ids
+//                    of that owner in earlier warps of the tile + earlier lanes
+//                    of its warp (__match_any_sync groups a warp by owner), then
+//                    each warp copies its ids' e rows to the packed send buffer.
+// Order within an owner is batch order, so the owner sees each rank's ids in
+// the order the rank had them.
+// ---------------------------------------------------------------------------
+constexpr int kPartTile = 1024;
+constexpr int kMaxOwners = 256;
+
+__device__ __forceinline__ int owner_of(long long k, int G) {
+  return (int)((splitmix64((uint64_t)k) >> 32) % (uint64_t)G);
+}
+
+__device__ __forceinline__ int64_t part_n(int64_t n, const long long* dev_n) {
+  if (!dev_n) return n;
+  const long long m = *dev_n;
+  return m < 0 ? 0 : (m < n ? m : n);
+}
+
+// Per-warp owner counts of this thread's tile in wcnt[warp * G + o]; returns the
+// thread's owner (G for an id past the end) and its rank among the earlier lanes
+// of its warp with the same owner.
+__device__ __forceinline__ int tile_owner_ranks(const long long* __restrict__ ids, int64_t i,
+                                                int64_t n_eff, int G, uint16_t* wcnt,
+                                                long long& key, int& rank) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int x = threadIdx.x; x < 32 * G; x += blockDim.x) wcnt[x] = 0;
+  key = -1;
+  int o = G;
+  if (i < n_eff) {
+    key = ids[i];
+    o = owner_of(key, G);
+  }
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, o);
+  rank = __popc(peers & ((1u << lane) - 1u));
+  __syncthreads();
+  if (o < G && rank == 0) wcnt[warp * G + o] = (uint16_t)__popc(peers);
+  __syncthreads();
+  return o;
+}
+
+__global__ void __launch_bounds__(kPartTile) k_owner_count(const long long* __restrict__ ids,
+                                                          int64_t n, const long long* dev_n,
+                                                          int G, int32_t* __restrict__ blk) {
+  pdl_enter();
+  __shared__ uint16_t wcnt[32 * kMaxOwners];
+  const int64_t n_eff = part_n(n, dev_n);
+  const int64_t i = (int64_t)blockIdx.x * kPartTile + threadIdx.x;
+  long long key;
+  int rank;
+  tile_owner_ranks(ids, i, n_eff, G, wcnt, key, rank);
+  for (int o = threadIdx.x; o < G; o += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < 32; ++w) c += wcnt[w * G + o];
+    blk[(int64_t)o * gridDim.x + blockIdx.x] = c;
+  }
+}
+
+// One block.  blk[o * nb + b] (counts) becomes the exclusive prefix in
+// owner-major order; counts[o] = the owner's total.
+__global__ void __launch_bounds__(1024) k_owner_offsets(int32_t* __restrict__ blk, int nb, int G,
+                                                        long long* __restrict__ counts) {
+  pdl_enter();
+  __shared__ int sm[33];
+  __shared__ int carry_s;
+  const int64_t L = (int64_t)nb * G;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < L; base += blockDim.x) {
+    const int64_t x = base + threadIdx.x;
+    const int v = x < L ? blk[x] : 0;
+    int total;
+    const int before = block_excl_scan(v, sm, total);
+    const int carry = carry_s;
+    if (x < L) blk[x] = carry + before;
+    __syncthreads();
+    if (threadIdx.x == 0) carry_s = carry + total;
+    __syncthreads();
+  }
+  const int all = carry_s;
+  for (int o = threadIdx.x; o < G; o += blockDim.x) {
+    const int lo = blk[(int64_t)o * nb];
+    const int hi = o + 1 < G ? blk[(int64_t)(o + 1) * nb] : all;
+    counts[o] = hi - lo;
+  }
+}
+
+__global__ void __launch_bounds__(kPartTile) k_owner_scatter(
+    const long long* __restrict__ ids, const int32_t* __restrict__ src_pos, int64_t n,
+    const long long* dev_n, int G, const int32_t* __restrict__ off, const float4* __restrict__ e,
+    int D4, long long* __restrict__ ids_out, int32_t* __restrict__ pos_out,
+    float4* __restrict__ e_out) {
+  pdl_enter();
+  __shared__ uint16_t wcnt[32 * kMaxOwners];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t n_eff = part_n(n, dev_n);
+  const int64_t i = (int64_t)blockIdx.x * kPartTile + threadIdx.x;
+  long long key;
+  int rank;
+  const int o = tile_owner_ranks(ids, i, n_eff, G, wcnt, key, rank);
+  // exclusive prefix over the warps of the tile, per owner, in place
+  for (int q = threadIdx.x; q < G; q += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wcnt[w * G + q];
+      wcnt[w * G + q] = (uint16_t)run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  int64_t dst = -1;
+  int32_t src = 0;
+  if (o < G) {
+    dst = (int64_t)off[(int64_t)o * gridDim.x + blockIdx.x] + wcnt[warp * G + o] + rank;
+    src = src_pos ? src_pos[i] : (int32_t)i;
+    ids_out[dst] = key;
+    pos_out[dst] = src;
+  }
+  if (!e) return;
+  // the warp's rows, one after another; lane l moves 16-byte vectors l + 32c
+  for (int l = 0; l < 32; ++l) {
+    const long long d = __shfl_sync(0xFFFFFFFFu, dst, l);
+    const int32_t sp = __shfl_sync(0xFFFFFFFFu, src, l);
+    if (d < 0) continue;
+    const float4* srow = e + (int64_t)sp * D4;
+    float4* drow = e_out + d * D4;
+    for (int base = 0; base < D4; base += 4 * 32) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        if (c < D4) v[u] = __ldcs(srow + c);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        if (c < D4) __stcs(drow + c, v[u]);
+      }
+    }
+  }
+}
+
+// Combine: the owners' answers come back in send order.  Id j of the send
+// buffer came from batch position pos[j]; the answer is its owner's local row
+// (-1 = miss) and D gathered values (+0 on a miss).  Writes, at pos[j], the
+// global row owner * Cs + row (or -1), hit, and the fused feature row: the
+// owner's D values, then the always-on row ao[ao_rows[pos[j]]].
+__global__ void __launch_bounds__(kBlock) k_owner_combine(
+    const long long* __restrict__ send_ids, const int32_t* __restrict__ pos, int64_t n, int G,
+    int64_t Cs, const int32_t* __restrict__ recv_rows, const float4* __restrict__ recv_feat,
+    int D4, const float4* __restrict__ ao, int64_t ao_n, int A4,
+    const int32_t* __restrict__ ao_rows, int32_t* __restrict__ rows, uint8_t* __restrict__ hit,
+    float4* __restrict__ out, int32_t* status) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int W4 = D4 + A4;
+  for (int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; j < n; j += warps) {
+    const int32_t p = pos[j];
+    const int32_t r = recv_rows[j];
+    int32_t a = 0;
+    bool has_a = A4 > 0;
+    if (has_a) {
+      a = ao_rows[p];
+      if (a < 0 || (int64_t)a >= ao_n) {
+        if (lane == 0) set_status(status, kStBadAo);
+        has_a = false;
+      }
+    }
+    if (lane == 0) {
+      const int o = owner_of(send_ids[j], G);
+      rows[p] = r >= 0 ? (int32_t)((int64_t)o * Cs + r) : -1;
+      hit[p] = r >= 0;
+    }
+    const float4* src = recv_feat + j * (int64_t)D4;
+    const float4* asrc = ao + (int64_t)a * A4;
+    float4* dst = out + (int64_t)p * W4;
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int base = 0; base < W4; base += 4 * 32) {
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        v[u] = z;
+        if (c < D4)
+          v[u] = __ldcs(src + c);
+        else if (c < W4 && has_a)
+          v[u] = __ldg(asrc + (c - D4));
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = base + u * 32 + lane;
+        if (c < W4) __stcs(dst + c, v[u]);
+      }
+    }
+  }
+}
+
 }  // namespace mpzch

@@ -249,6 +249,66 @@ MPZCH_API int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int
                        const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit, float* out,
                        int32_t* dev_status, void* stream);
 
+/* ---- Hash-owner sharding --------------------------------------------------
+ * Memory Layer section 2 shards the table across devices and keeps the
+ * distributed lookup's all-to-all path; MTGR (page "MTGR: Industrial-Scale
+ * Generative Recommendation Framework in Meituan") section 3.3 exchanges ids
+ * all-to-all between devices with a dedup before and after the exchange.
+ * With G shards (one table per rank), key k belongs to shard
+ *   owner(k) = (splitmix64(k) >> 32) mod G,
+ * the upper half of the hash whose lower bits pick the home slot inside the
+ * shard.  A rank partitions its ids (and e rows) by owner into one contiguous
+ * segment per owner, exchanges the segments all-to-all (NCCL; the owner
+ * receives ranks 0..G-1 in rank order), runs lookup/gather/Writeback on its
+ * own table, and sends lookup answers back in the order received; the combine
+ * step puts them at their batch positions.  Global row of shard s, local row
+ * r: s * shard_capacity + r.  At most MPZCH_MAX_OWNERS shards. */
+#define MPZCH_MAX_OWNERS 256
+
+/* Bytes of device workspace mpzch_owner_partition needs for n ids and
+ * n_owners owners (a multiple of 256), or -1 for bad sizes. */
+MPZCH_API int64_t mpzch_owner_partition_workspace(int64_t n, int32_t n_owners);
+
+/* Stable partition of ids by owner.  For i < n_eff (n_eff = n, or
+ * min(n, *dev_n) when dev_n is given -- e.g. the dev_count of mpzch_dedup):
+ * ids[i] goes to the segment of owner(ids[i]); segments are laid out in
+ * ascending owner order and keep batch order inside, in ids_out (device
+ * int64[n]).  pos_out[j] (device int32[n]) = src_pos ? src_pos[i] : i for the
+ * id placed at j.  With e (device fp32 [..][dim], dim % 4 == 0, 16-byte
+ * aligned) non-NULL, e_out row j (device fp32 [n][dim], 16-byte aligned) =
+ * e row pos_out[j]: the packed send buffer of the ids' e rows.  dev_counts:
+ * device int64[n_owners], the segment sizes (they sum to n_eff).  Slots past
+ * n_eff are not written.  workspace: device memory of at least
+ * mpzch_owner_partition_workspace(n, n_owners) bytes, owned by the caller,
+ * not used after the call's work completes on `stream`.  Allocates nothing.
+ * MPZCH_EINVAL for bad sizes, null pointers or misaligned rows. */
+MPZCH_API int mpzch_owner_partition(const int64_t* ids, const int32_t* src_pos, int64_t n,
+                                    const int64_t* dev_n, int32_t n_owners, const float* e,
+                                    int32_t dim, int64_t* ids_out, int32_t* pos_out, float* e_out,
+                                    int64_t* dev_counts, void* workspace,
+                                    int64_t workspace_bytes, void* stream);
+
+/* Combine the owners' lookup answers (they arrive in send order).  For j < n:
+ * send_ids/pos are the ids_out/pos_out of the partition of the looked-up ids
+ * (batch positions pos[j] < the caller's batch size), recv_rows (device
+ * int32[n]) the owner's local row or -1, recv_feat (device fp32 [n][dim],
+ * 16-byte aligned) the owner's gathered values (+0 on a miss).  Writes at
+ * p = pos[j]:
+ *   rows[p] = recv_rows[j] >= 0 ? owner(send_ids[j]) * shard_capacity + recv_rows[j] : -1,
+ *   hit[p]  = recv_rows[j] >= 0,
+ *   out[p][0:dim] = recv_feat[j],  out[p][dim:dim+ao_dim] = ao_table[ao_rows[p]]
+ * -- bit for bit what mpzch_gather_fused gives on one table.  ao_* as in
+ * mpzch_gather_fused (NULL/0 for no concat).  out: device fp32 [..][dim +
+ * ao_dim], 16-byte aligned.  An always-on row outside [0, ao_nrows) gives
+ * zeros and ORs MPZCH_STATUS_BADAO into dev_status (nullable device int32).
+ * n_owners * shard_capacity must be below 2^31.  Needs no table handle. */
+MPZCH_API int mpzch_owner_combine(const int64_t* send_ids, const int32_t* pos, int64_t n,
+                                  int32_t n_owners, int64_t shard_capacity,
+                                  const int32_t* recv_rows, const float* recv_feat, int32_t dim,
+                                  const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
+                                  const int32_t* ao_rows, int32_t* rows, uint8_t* hit, float* out,
+                                  int32_t* dev_status, void* stream);
+
 /* ---- Streaming export of fresh rows to a host serving snapshot (RES) ----
  * Memory Layer section 2, RES paragraph: new vectors are copied to the host
  * asynchronously while they are in HBM; in the background they are deduped by

@@ -130,3 +130,39 @@ def test_python_binding_loads(lib):
     assert binding.mpzch_launch_count() >= 0
     with pytest.raises(binding.MpzchError):
         binding.mpzch_debug_fail_allocs(-3)
+
+
+def test_owner_partition_and_combine_reject_bad_arguments_without_the_gpu(lib):
+    p, i64, i32 = C.c_void_p, C.c_int64, C.c_int32
+    lib.mpzch_owner_partition_workspace.argtypes = [i64, i32]
+    lib.mpzch_owner_partition_workspace.restype = i64
+    assert lib.mpzch_owner_partition_workspace(0, 1) == 0
+    assert lib.mpzch_owner_partition_workspace(1, 1) == 256
+    assert lib.mpzch_owner_partition_workspace(163840, 8) == 160 * 8 * 4  # 1024-id tiles
+    for n, g in ((-1, 4), (10, 0), (10, 257), (1 << 31, 4)):
+        assert lib.mpzch_owner_partition_workspace(n, g) == -1
+    lib.mpzch_owner_partition.argtypes = [p, p, i64, p, i32, p, i32, p, p, p, p, p, i64, p]
+    fake = C.c_void_p(0x1000)
+    # bad owner counts, missing counts, missing buffers, short workspace, odd dim
+    assert lib.mpzch_owner_partition(fake, None, 10, None, 0, None, 0, fake, fake, None, fake,
+                                     fake, 4096, None) == -1
+    assert lib.mpzch_owner_partition(fake, None, 10, None, 4, None, 0, fake, fake, None, None,
+                                     fake, 4096, None) == -1
+    assert lib.mpzch_owner_partition(fake, None, 10, None, 4, None, 0, None, fake, None, fake,
+                                     fake, 4096, None) == -1
+    assert lib.mpzch_owner_partition(fake, None, 10, None, 4, None, 0, fake, fake, None, fake,
+                                     fake, 16, None) == -1
+    assert lib.mpzch_owner_partition(fake, None, 10, None, 4, fake, 6, fake, fake, fake, fake,
+                                     fake, 4096, None) == -1
+    lib.mpzch_owner_combine.argtypes = [p, p, i64, i32, i64, p, p, i32, p, i64, i32, p, p, p, p,
+                                        p, p]
+    def comb(n=10, G=4, cs=1000, dim=16, ao=None, ao_n=0, ao_dim=0, aor=None, out=fake):
+        return lib.mpzch_owner_combine(fake, fake, n, G, cs, fake, fake, dim, ao, ao_n, ao_dim,
+                                       aor, fake, fake, out, None, None)
+    assert comb(G=0) == -1 and comb(G=257) == -1
+    assert comb(cs=1 << 30, G=4) == -1      # global rows would pass 2^31
+    assert comb(dim=6) == -1
+    assert comb(ao=fake, ao_n=5, ao_dim=8, aor=None) == -1
+    assert comb(ao=None, ao_dim=8) == -1
+    assert comb(out=None) == -1
+    assert comb(n=0) == 0                   # nothing to do, nothing launched
