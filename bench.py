@@ -80,6 +80,8 @@ def parse():
                     help="do not pass an inputs-ready event (no overlap across steps)")
     ap.add_argument("--separate-calls", action="store_true",
                     help="lookup, gather and Writeback as three calls instead of mpzch_train_step")
+    ap.add_argument("--insert", choices=["cluster", "rounds"], default=None,
+                    help="insert path: grid-wide cluster placement (default) or claim rounds")
     ap.add_argument("--wide-rounds", type=int, default=None,
                     help="grid-wide insert conflict rounds before the single-block finisher")
     ap.add_argument("--shard", action="store_true",
@@ -289,6 +291,9 @@ def run_ours(args):
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SIDE_PRIORITY, args.side_priority)
     if args.wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, args.wide_rounds)
+    if args.insert is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT,
+                                 1 if args.insert == "cluster" else 0)
 
     def step(t, i=None):
         # step t of the stream reads the resident inputs of slot i (default t)

@@ -35,6 +35,7 @@ MPZCH_OPT_WIDE_ROUNDS = 1
 MPZCH_VALUES_IN_HOST_MEMORY = 1
 MPZCH_OPT_SIDE_PRIORITY = 2
 MPZCH_OPT_ROW_GRID = 3
+MPZCH_OPT_CLUSTER_INSERT = 4
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")

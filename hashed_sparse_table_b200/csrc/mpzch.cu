@@ -190,8 +190,14 @@ struct mpzch_table {
   float* M = nullptr;          // device-accessible address of the values
   void* M_host = nullptr;      // host allocation when the values live in host memory
   bool values_on_host = false;
-  // insert scratch: three claim arrays of C slots
+  // insert scratch: three claim arrays of C slots (claim-round path)
   unsigned long long* claims[3] = {nullptr, nullptr, nullptr};
+  // cluster placement path: tagged per-slot list heads (C slots) and the tag
+  // of the last call (0 is never a call's tag; shead starts all zero)
+  unsigned long long* shead = nullptr;
+  uint32_t tag = 0;
+  bool tag_wrapped = false;
+  int cluster_insert = 1;
   // per-batch scratch, sized for `cap` ids
   int64_t cap = 0;
   uint64_t hmask = 0;
@@ -202,6 +208,7 @@ struct mpzch_table {
   long long* ukey = nullptr;
   int32_t* upos = nullptr;
   int32_t* urow = nullptr;
+  int32_t* snext = nullptr;  // next key of the same home slot (cluster path)
   long long* lkey[3] = {nullptr, nullptr, nullptr};  // insert round lists: keys
   int32_t* lidx[3] = {nullptr, nullptr, nullptr};    // and their distinct-id index
   // write lists (row, position of e), two buffers used by alternate Writebacks
@@ -249,6 +256,8 @@ void free_batch_scratch(mpzch_table* t) {
   dev_free(t->ukey);
   dev_free(t->upos);
   dev_free(t->urow);
+  dev_free(t->snext);
+  t->snext = nullptr;
   for (auto& l : t->lkey) dev_free(l), l = nullptr;
   for (auto& l : t->lidx) dev_free(l), l = nullptr;
   for (auto& l : t->wrow) dev_free(l), l = nullptr;
@@ -270,6 +279,7 @@ void free_all(mpzch_table* t) {
   else
     dev_free(t->M);
   for (auto& c : t->claims) dev_free(c), c = nullptr;
+  dev_free(t->shead);
   dev_free(t->ctr);
   dev_free(t->wcnt);
   dev_free(t->stats);
@@ -332,6 +342,7 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
   if (!rc) rc = dev_alloc((void**)&t->upos, cap * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->urow, cap * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->snext, cap * sizeof(int32_t));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lkey[i], cap * sizeof(long long));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lidx[i], cap * sizeof(int32_t));
   for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->wrow[i], cap * sizeof(int32_t));
@@ -483,6 +494,14 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.stats = stats;
   p.status = t->status;
   p.wide_rounds = t->wide_rounds;
+  p.cluster = t->cluster_insert;
+  if (++t->tag == 0) {  // 2^32 calls: old entries could alias the new tag
+    t->tag = 1;
+    t->tag_wrapped = true;
+  }
+  p.tag = t->tag;
+  p.shead = t->shead;
+  p.snext = t->snext;
   p.wrow = t->wrow[t->wset];
   p.wpos = t->wpos[t->wset];
   p.wcount = t->wcnt + t->wset;
@@ -496,6 +515,11 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
 int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEvent_t keys_free) {
   const int64_t n = p.n;
   int rc;
+  if (t->tag_wrapped) {
+    if (cudaMemsetAsync(t->shead, 0, t->C * sizeof(unsigned long long), st) != cudaSuccess)
+      return MPZCH_ECUDA;
+    t->tag_wrapped = false;
+  }
   {
     PhaseScope ps(t, PH_DEDUP, st);
     rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false,
@@ -505,6 +529,16 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     if (rc) return rc;
   }
   if (keys_free && cudaStreamWaitEvent(st, keys_free, 0) != cudaSuccess) return MPZCH_ECUDA;
+  if (p.cluster) {
+    // cluster placement; the single-block finisher only acts when the
+    // windows may cover the whole ring
+    PhaseScope ps(t, PH_INSERT, st);
+    rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !keys_free, p);
+    if (!rc) rc = launch(k_place_multi, grid_for(n * 32, kBlock, 4), kBlock, st, true, p);
+    if (!rc) rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, 0);
+    if (!rc) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
+    return rc;
+  }
   {
     PhaseScope ps(t, PH_INSERT, st);
     const unsigned grid = grid_for(n, kBlock, 4);
@@ -666,6 +700,7 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   }
   for (int i = 0; i < 3 && !rc; ++i)
     rc = dev_alloc((void**)&t->claims[i], capacity * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->shead, capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
   if (!rc) rc = dev_alloc((void**)&t->wcnt, 2 * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
@@ -684,6 +719,8 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
                cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) ==
                    cudaSuccess) &&
               cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
+              cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
+                  cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
               cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
     for (int i = 0; i < 3 && ok; ++i)
@@ -812,10 +849,12 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
   // the write list.  Caller's stream: gather, then the row update.  Without
   // inputs_ready both helper streams start after everything earlier on the
   // caller's stream.  With it (pipelined) they wait only for what they need:
-  // the inputs, the last other call on the table, the previous gather (which
-  // read rows/hit), the previous row map (lookup: final keys) and the row
-  // update that last read this write-list buffer (side stream) -- so they
-  // overlap the previous step's row update.
+  // the inputs and the last other call on the table; the lookup also for the
+  // previous gather (which read rows/hit) and the previous row map (final
+  // keys); the side stream for the row update that last read this write-list
+  // buffer (the row map touches nothing a gather reads: keys, steps, scratch
+  // and the write list, never the values) -- so they overlap the previous
+  // step's gather and row update.
   if (inputs_ready) {
     cudaEvent_t in = reinterpret_cast<cudaEvent_t>(inputs_ready);
     if (cudaStreamWaitEvent(t->look, in, 0) != cudaSuccess ||
@@ -824,8 +863,7 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
         cudaStreamWaitEvent(t->look, t->ev_map, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, in, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->side, t->ev_gather, 0) != cudaSuccess)
+        cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess)
       return MPZCH_ECUDA;
   } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
              cudaStreamWaitEvent(t->look, t->ev_fork, 0) != cudaSuccess ||
@@ -1056,6 +1094,11 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
   if (option == MPZCH_OPT_WIDE_ROUNDS) {
     if (value < 0 || value > 64) return MPZCH_EINVAL;
     t->wide_rounds = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_CLUSTER_INSERT) {
+    if (value != 0 && value != 1) return MPZCH_EINVAL;
+    t->cluster_insert = (int)value;
     return MPZCH_OK;
   }
   return MPZCH_EINVAL;

@@ -35,7 +35,9 @@ struct Geo {
 struct StepCtr {
   int32_t cnt[4];    // insert-round list sizes; round r appends to cnt[(r + 1) % 4]
   int32_t n_unique;  // distinct ids of the batch
-  int32_t pad[3];
+  int32_t n_multi;   // cluster path: heads of clusters with several keys (list lidx[1])
+  int32_t n_serial;  // cluster path: clusters left to the single-block kernel (list lidx[2])
+  int32_t pad;
 };
 
 // Per-Writeback counters; same layout as mpzch_wb_stats.
@@ -183,9 +185,9 @@ __global__ void __launch_bounds__(kBlock) k_gather_fused(
         const int c = base + u * 32 + lane;
         v[u] = z;
         if (c < D4) {
-          if (h) v[u] = __ldg(src + c);
+          if (h) v[u] = __ldcs(src + c);
         } else if (c < W4 && has_a) {
-          v[u] = __ldg(asrc + (c - D4));
+          v[u] = __ldcs(asrc + (c - D4));
         }
       }
 #pragma unroll
@@ -508,7 +510,16 @@ struct WbParams {
   StepCtr* ctr;
   WbStats* stats;
   int32_t* status;
-  int wide_rounds;  // grid-wide insert rounds of this Writeback
+  int wide_rounds;  // grid-wide insert rounds of this Writeback (claim-round path)
+  // cluster placement path: per-slot lists of this call's missing keys.
+  // shead[s] = (tag << 32) | list-0 index of the last key linked at home slot
+  // s, valid only when its upper half equals this call's tag (so entries of
+  // earlier calls read as empty and nothing is ever cleared); snext[m] = the
+  // next key of the same home slot, or -1.
+  int cluster;
+  uint32_t tag;
+  unsigned long long* shead;
+  int32_t* snext;
   // write list of this Writeback: (row, position of e) of every distinct id
   // that still owns its row; one of two buffers, alternating by call
   int32_t* wrow;
@@ -583,7 +594,13 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
       } else {
         p.lkey[0][m] = k;
         p.lidx[0][m] = u;
-        claim_window(p.claims[0], k, g);
+        if (p.cluster) {
+          const unsigned long long old =
+              atomicExch(p.shead + h, ((unsigned long long)p.tag << 32) | (uint32_t)m);
+          p.snext[m] = (uint32_t)(old >> 32) == p.tag ? (int32_t)(uint32_t)old : -1;
+        } else {
+          claim_window(p.claims[0], k, g);
+        }
       }
     }
   }
@@ -728,6 +745,8 @@ constexpr int kClusterMax = 4096;
 constexpr int kClusterBuckets = 4096;
 constexpr size_t kClusterSmem = (size_t)kClusterMax * (4 + 8 + 4) + (kClusterBuckets + 1) * 4;
 
+__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, long long& evicted);
+
 __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
   pdl_enter();
   extern __shared__ __align__(16) unsigned char dsm[];
@@ -736,6 +755,19 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
   const Geo g = p.g;
   const int32_t nprev = r0 > 0 ? p.ctr->cnt[(r0 + 3) & 3] : 0;
   const int32_t ncur = p.ctr->cnt[r0 & 3];
+  // cluster placement path: when the windows may cover the whole ring the
+  // grid-wide passes placed nothing and this block places every key; otherwise
+  // it only places the clusters the warp path left (listed in lidx[2])
+  if (p.cluster && (int64_t)ncur * g.P < g.C) {
+    const int32_t S = p.ctr->n_serial;
+    if (S == 0) return;  // block-uniform
+    long long ev_serial = 0;
+    for (int32_t i = threadIdx.x; i < S; i += blockDim.x)
+      place_cluster_serial(p, __ldcg(p.lidx[2] + i), ncur, ev_serial);
+    const long long evs = block_sum_ll(ev_serial, sm);
+    if (threadIdx.x == 0 && evs) atomic_add_ll(&p.stats->n_evicted, evs);
+    return;
+  }
   if (r0 == 0 && threadIdx.x == 0) p.stats->n_inserted = ncur;
   long long evicted = 0, rounds = 0;
   if (ncur > kClusterMax) {
@@ -867,6 +899,378 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
 }
 
 // ---------------------------------------------------------------------------
+// Cluster placement (default insert path), grid-wide and exact.
+//
+// Windows W(a) and W(b) overlap exactly when the home slots are less than P
+// apart on the ring.  Cut the ring's occupied home slots wherever two
+// consecutive ones are P or more apart: each run (cluster) touches a set of
+// slots no other cluster touches, so placing each cluster's keys in ascending
+// key order, clusters independently, gives the state of the sequential insert
+// of all missing keys in ascending order.  The re-probe linked every missing
+// key into the list of its home slot; here the key whose index heads its slot's
+// list is the slot's representative, a representative with no occupied slot
+// among the P-1 slots before its own heads its cluster, and that thread walks
+// forward (the next occupied slot within P-1 of the last one found), collects
+// the cluster's keys from the slot lists and places them one after another
+// (victim = smallest (last, row) of the window, reading its own earlier
+// writes).  The common case -- a lone key with no neighbour within P-1 slots
+// -- is decided from one batch of loads issued together.
+//
+// Such a cut exists when the windows do not cover the whole ring, which is
+// certain when N * P < C (N missing keys).  Otherwise this kernel places
+// nothing and k_insert_finish places every key.
+// ---------------------------------------------------------------------------
+constexpr int kClusterLocal = 32;  // cluster keys sorted locally; larger clusters take the slow walk
+constexpr int kSpanLocal = 96;     // slots of a cluster's windows copied locally
+
+__device__ __forceinline__ bool slot_used(unsigned long long v, uint32_t tag) {
+  return (uint32_t)(v >> 32) == tag;
+}
+
+__device__ __forceinline__ int64_t ring_add(int64_t h, int64_t d, int64_t C) {
+  int64_t s = h + d;  // |d| < C
+  if (s < 0) s += C;
+  if (s >= C) s -= C;
+  return s;
+}
+
+// Adds (key, distinct-id index) to the first n entries of ck/cu, kept in
+// ascending key order; false when kClusterLocal entries are already held.
+__device__ __forceinline__ bool sorted_add(long long* ck, int32_t* cu, int& n, long long kk,
+                                           int32_t uu) {
+  if (n == kClusterLocal) return false;
+  int j = n++;
+  for (; j > 0 && ck[j - 1] > kk; --j) {
+    ck[j] = ck[j - 1];
+    cu[j] = cu[j - 1];
+  }
+  ck[j] = kk;
+  cu[j] = uu;
+  return true;
+}
+
+// Smallest unplaced key of the cluster [h, h + L] (urow < 0 until placed), by
+// walking the slot lists; returns its list-0 index or -1.  Slow path for
+// clusters too large to sort in registers (never on the benchmark workloads).
+__device__ int32_t cluster_min_unplaced(const WbParams& p, int64_t h, int64_t L, int32_t N) {
+  const Geo& g = p.g;
+  int32_t arg = -1;
+  long long kmin = 0;
+  for (int64_t off = 0; off <= L; ++off) {
+    const unsigned long long v = ld_cg(p.shead + ring_add(h, off, g.C));
+    if (!slot_used(v, p.tag)) continue;
+    for (int32_t x = (int32_t)(uint32_t)v, hops = 0; x >= 0 && hops <= N;
+         x = __ldcg(p.snext + x), ++hops) {
+      const long long k = __ldcg(p.lkey[0] + x);
+      if (__ldcg(p.urow + __ldcg(p.lidx[0] + x)) < 0 && (arg < 0 || k < kmin)) {
+        arg = x;
+        kmin = k;
+      }
+    }
+  }
+  return arg;
+}
+
+// Serial placement of the cluster headed at slot h by one thread: walk 8 slot
+// heads per batch, collect and sort the keys, copy the span's steps and decide
+// every placement on the copy; clusters beyond the local limits place key by
+// key in global memory.  Used where the warp path does not apply.
+__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, long long& evicted) {
+  const Geo& g = p.g;
+  unsigned long long heads[kClusterLocal];
+  int nh = 0;
+  bool overflow = false;
+  heads[nh++] = ld_cg(p.shead + h);
+  int64_t L = 0;
+  for (int64_t off = 1; off <= L + g.P - 1 && off < g.C;) {
+    unsigned long long w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      w[q] = off + q < g.C ? ld_cg(p.shead + ring_add(h, off + q, g.C)) : 0;
+    int q = 0;
+    for (; q < 8; ++q) {
+      const int64_t o = off + q;
+      if (o > L + g.P - 1 || o >= g.C) break;
+      if (slot_used(w[q], p.tag)) {
+        L = o;
+        if (nh < kClusterLocal)
+          heads[nh++] = w[q];
+        else
+          overflow = true;
+      }
+    }
+    off += q;
+    if (q < 8) break;
+  }
+  long long ck[kClusterLocal];
+  int32_t cu[kClusterLocal];
+  int n = 0;
+  for (int i = 0; i < nh && !overflow; ++i)
+    for (int32_t x = (int32_t)(uint32_t)heads[i], hops = 0; x >= 0 && hops <= N && !overflow;
+         x = __ldcg(p.snext + x), ++hops)
+      overflow |= !sorted_add(ck, cu, n, __ldcg(p.lkey[0] + x), __ldcg(p.lidx[0] + x));
+  const int64_t span = L + g.P;
+  if (!overflow && span <= kSpanLocal) {
+    long long sl[kSpanLocal];
+    for (int64_t o0 = 0; o0 < span; o0 += 16) {
+      long long v[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        v[q] = o0 + q < span ? ld_cg(p.last + ring_add(h, o0 + q, g.C)) : 0;
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (o0 + q < span) sl[o0 + q] = v[q];
+    }
+    for (int j = 0; j < n; ++j) {
+      const long long kk = ck[j];
+      int64_t off = home_slot(kk, g) - h;
+      if (off < 0) off += g.C;
+      int64_t best = -1, best_o = 0;
+      long long best_last = 0;
+      for (int32_t q = 0; q < g.P; ++q) {
+        const int64_t o = off + q;
+        const int64_t s = ring_add(h, o, g.C);
+        if (best < 0 || sl[o] < best_last || (sl[o] == best_last && s < best)) {
+          best = s;
+          best_o = o;
+          best_last = sl[o];
+        }
+      }
+      if (best_last != -1) ++evicted;
+      sl[best_o] = p.step;
+      p.keys[best] = kk;
+      p.last[best] = p.step;
+      p.urow[cu[j]] = (int32_t)best;
+    }
+    return;
+  }
+  if (!overflow) {
+    for (int j = 0; j < n; ++j) place_key(p, ck[j], cu[j], evicted);
+    return;
+  }
+  for (int32_t it = 0; it <= N; ++it) {
+    const int32_t x = cluster_min_unplaced(p, h, L, N);
+    if (x < 0) return;
+    place_key(p, __ldcg(p.lkey[0] + x), __ldcg(p.lidx[0] + x), evicted);
+  }
+  set_status(p.status, kStInternal);  // more placements than keys: never expected
+}
+
+// Per-warp shared scratch of the warp path: the cluster's keys as collected
+// and in ascending order.
+constexpr int kWarpSpan = 64;  // slots (offsets 0..63 from the head) one warp loads at once
+constexpr int kWarpKeys = 64;
+struct WarpCluster {
+  long long k[kWarpKeys];
+  long long ks[kWarpKeys];
+  int32_t u[kWarpKeys];
+  int32_t us[kWarpKeys];
+  int n;
+};
+
+// The whole warp places the cluster headed at slot h: lane l holds offsets l
+// and l + 32 (slot head and last-write step, one batch of loads), the cluster
+// end comes from the occupancy ballot, lanes fetch the slot lists' keys, a
+// rank count orders them, and each placement is an argmin of (step, row) over
+// lanes q < P of the window, exchanged by shuffles; lane 0 stores.  Returns
+// false, having written nothing to the table, when the cluster is outside the
+// path's limits (P > 32, span > 64 slots, more than 64 keys, C < 128).
+__device__ bool place_cluster_warp(const WbParams& p, int64_t h, int32_t N, WarpCluster& sw,
+                                   long long& evicted) {
+  const Geo& g = p.g;
+  const int lane = threadIdx.x & 31;
+  if (g.P > 32 || g.C < 2 * kWarpSpan) return false;
+  const int64_t s0 = ring_add(h, lane, g.C), s1 = ring_add(h, lane + 32, g.C);
+  const unsigned long long v0 = ld_cg(p.shead + s0), v1 = ld_cg(p.shead + s1);
+  long long l0 = ld_cg(p.last + s0), l1 = ld_cg(p.last + s1);
+  const unsigned long long occ =
+      (unsigned long long)__ballot_sync(0xFFFFFFFFu, slot_used(v0, p.tag)) |
+      ((unsigned long long)__ballot_sync(0xFFFFFFFFu, slot_used(v1, p.tag)) << 32);
+  int L = 0;  // offset of the cluster's last occupied slot
+  while (L < 63) {
+    const unsigned long long later = occ & ~((2ull << L) - 1ull);
+    if (!later) break;
+    const int o = __ffsll((long long)later) - 1;
+    if (o > L + g.P - 1) break;
+    L = o;
+  }
+  if (L + g.P > kWarpSpan) return false;
+  __syncwarp();
+  if (lane == 0) sw.n = 0;
+  __syncwarp();
+  bool too_many = false;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int o = lane + 32 * half;
+    const unsigned long long v = half ? v1 : v0;
+    if (o > L || !slot_used(v, p.tag)) continue;
+    for (int32_t x = (int32_t)(uint32_t)v, hops = 0; x >= 0 && hops <= N;
+         x = __ldcg(p.snext + x), ++hops) {
+      const int at = atomicAdd(&sw.n, 1);
+      if (at < kWarpKeys) {
+        sw.k[at] = __ldcg(p.lkey[0] + x);
+        sw.u[at] = __ldcg(p.lidx[0] + x);
+      } else {
+        too_many = true;
+      }
+    }
+  }
+  __syncwarp();
+  if (__any_sync(0xFFFFFFFFu, too_many)) return false;
+  const int n = sw.n;
+  for (int j = lane; j < n; j += 32) {  // rank = number of smaller keys (keys are distinct)
+    const long long kj = sw.k[j];
+    int r = 0;
+    for (int i = 0; i < n; ++i) r += sw.k[i] < kj;
+    sw.ks[r] = kj;
+    sw.us[r] = sw.u[j];
+  }
+  __syncwarp();
+  for (int j = 0; j < n; ++j) {
+    const long long k = sw.ks[j];
+    int64_t off = home_slot(k, g) - h;
+    if (off < 0) off += g.C;
+    const int o = (int)off + lane;  // window offset of lane q = lane (< 64 for q < P)
+    const long long a = __shfl_sync(0xFFFFFFFFu, l0, o & 31);
+    const long long b = __shfl_sync(0xFFFFFFFFu, l1, o & 31);
+    long long cl = o < 32 ? a : b;
+    long long cs = ring_add(h, o, g.C);
+    int co = o;
+    if (lane >= g.P) {
+      cl = 0x7FFFFFFFFFFFFFFFll;
+      cs = 0x7FFFFFFFFFFFFFFFll;
+    }
+    for (int d = 16; d > 0; d >>= 1) {
+      const long long ol = __shfl_xor_sync(0xFFFFFFFFu, cl, d);
+      const long long os = __shfl_xor_sync(0xFFFFFFFFu, cs, d);
+      const int oo = __shfl_xor_sync(0xFFFFFFFFu, co, d);
+      if (ol < cl || (ol == cl && os < cs)) {
+        cl = ol;
+        cs = os;
+        co = oo;
+      }
+    }
+    if (co < 32) {
+      if (lane == co) l0 = p.step;
+    } else if (lane == co - 32) {
+      l1 = p.step;
+    }
+    if (lane == 0) {
+      if (cl != -1) ++evicted;
+      p.keys[cs] = k;
+      p.last[cs] = p.step;
+      p.urow[sw.us[j]] = (int32_t)cs;
+    }
+  }
+  return true;
+}
+
+// First look at missing key m by its own thread.  Places a lone key (no other
+// key with a start slot within P-1 on either side, none sharing its own) from
+// one batch of loads and returns 0; returns 0 for a key that is not its slot's
+// representative or not the head of its cluster; returns 1, with its start
+// slot in h_out, for the head of a cluster that needs more than that.
+__device__ int place_lone(const WbParams& p, int32_t m, long long& evicted, int64_t& h_out) {
+  const Geo& g = p.g;
+  const long long k = __ldcg(p.lkey[0] + m);
+  const int64_t h = home_slot(k, g);
+  h_out = h;
+  if (g.P > 8) {
+    const unsigned long long vh = ld_cg(p.shead + h);
+    if (!slot_used(vh, p.tag) || (int32_t)(uint32_t)vh != m) return 0;
+    for (int64_t off = 1; off < g.P; ++off)
+      if (slot_used(ld_cg(p.shead + ring_add(h, -off, g.C)), p.tag)) return 0;
+    return 1;
+  }
+  // one batch: slot heads h-P+1 .. h+P-1, the key's list link, its window's steps
+  unsigned long long v[15];
+  long long l[8];
+#pragma unroll
+  for (int j = 0; j < 15; ++j)
+    v[j] = j < 2 * g.P - 1 ? ld_cg(p.shead + ring_add(h, j - (g.P - 1), g.C)) : 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) l[q] = q < g.P ? ld_cg(p.last + wslot(h, q, g)) : 0;
+  const int32_t nx = __ldcg(p.snext + m);
+  unsigned long long vh = 0;
+  bool back = false, fwd = false;
+#pragma unroll
+  for (int j = 0; j < 15; ++j) {
+    if (j >= 2 * g.P - 1) continue;
+    const bool u = slot_used(v[j], p.tag);
+    if (j < g.P - 1)
+      back |= u;
+    else if (j == g.P - 1)
+      vh = v[j];
+    else
+      fwd |= u;
+  }
+  if (!slot_used(vh, p.tag) || (int32_t)(uint32_t)vh != m) return 0;  // not the representative
+  if (back) return 0;  // not the head of its cluster
+  if (fwd || nx >= 0) return 1;
+  int64_t best = -1;
+  long long best_last = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    if (q >= g.P) continue;
+    const int64_t s = wslot(h, q, g);
+    if (best < 0 || l[q] < best_last || (l[q] == best_last && s < best)) {
+      best = s;
+      best_last = l[q];
+    }
+  }
+  if (best_last != -1) ++evicted;
+  p.keys[best] = k;
+  p.last[best] = p.step;
+  p.urow[__ldcg(p.lidx[0] + m)] = (int32_t)best;
+  return 0;
+}
+
+// Pass 1 of the cluster path: one thread per missing key; lone keys are placed,
+// heads of larger clusters are listed (start slot) for pass 2.
+__global__ void __launch_bounds__(kBlock) k_place_clusters(WbParams p) {
+  pdl_enter();
+  __shared__ long long sm[33];
+  const int32_t N = p.ctr->cnt[0];
+  const bool ring_may_be_covered = (int64_t)N * p.g.P >= p.g.C;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.stats->n_inserted = N;
+    if (N > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
+  }
+  long long evicted = 0;
+  if (!ring_may_be_covered) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < N; m += stride) {
+      int64_t h = 0;
+      if (place_lone(p, (int32_t)m, evicted, h)) p.lidx[1][warp_append(&p.ctr->n_multi)] = (int32_t)h;
+    }
+  }
+  const long long ev = block_sum_ll(evicted, sm);
+  if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
+}
+
+// Pass 2: one warp per listed cluster head; clusters outside the warp path's
+// limits are listed for the single-block kernel.
+__global__ void __launch_bounds__(kBlock) k_place_multi(WbParams p) {
+  pdl_enter();
+  __shared__ long long sm[33];
+  __shared__ WarpCluster s_warp[kBlock / 32];
+  const int32_t N = p.ctr->cnt[0];
+  const int32_t H = p.ctr->n_multi;
+  const int lane = threadIdx.x & 31;
+  WarpCluster& sw = s_warp[threadIdx.x >> 5];
+  long long evicted = 0;
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < H; w += warps) {
+    const int64_t h = __ldcg(p.lidx[1] + w);
+    if (!place_cluster_warp(p, h, N, sw, evicted) && lane == 0)
+      p.lidx[2][atomicAdd(&p.ctr->n_serial, 1)] = (int32_t)h;
+    __syncwarp();
+  }
+  const long long ev = block_sum_ll(evicted, sm);
+  if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
+}
+
+// ---------------------------------------------------------------------------
 // End of the row map: the write list holds (row, position of e) for every
 // distinct id that still owns its row after all inserts (a distinct id evicted
 // again later in the same step gets no write, n_dropped).  Also clears the
@@ -878,7 +1282,7 @@ __global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
   __shared__ long long sm[33];
   __shared__ int smi[33];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  {
+  if (!p.cluster) {
     // clearing a window that is already clear is harmless
     const int L = p.wide_rounds > 0 ? p.wide_rounds - 1 : 0;
     const int32_t nl = p.ctr->cnt[L & 3];
@@ -911,7 +1315,10 @@ __global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
 // ---------------------------------------------------------------------------
 // Writeback row update: M[r] <- fl(e_hat - fl(eta * fl(e_hat - e))) (eta = 1:
 // the exact Writeback) for every entry of the write list; one warp per row, 16-byte vectors, loads of a chunk issued
-// before its stores.  Reads only the write list, M and e.
+// before its stores.  Reads only the write list, M and e.  Rows and targets
+// are touched once per step, so they go through L2 as streaming (evict-first)
+// accesses, which leaves the identity map, step and list arrays of the row
+// map -- a few tens of MB -- resident in L2 while this kernel runs.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict__ wrow,
                                                       const int32_t* __restrict__ wpos,
@@ -932,7 +1339,7 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
       for (int q = 0; q < 4; ++q) {
         const int c = base + q * 32 + lane;
         if (c < D4) {
-          a[q] = __ldcg(m + c);
+          a[q] = __ldcs(m + c);
           b[q] = __ldcs(ev + c);
         }
       }
@@ -948,7 +1355,7 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
           o.y = __fsub_rn(a[q].y, __fmul_rn(eta, __fsub_rn(a[q].y, b[q].y)));
           o.z = __fsub_rn(a[q].z, __fmul_rn(eta, __fsub_rn(a[q].z, b[q].z)));
           o.w = __fsub_rn(a[q].w, __fmul_rn(eta, __fsub_rn(a[q].w, b[q].w)));
-          m[c] = o;
+          __stcs(m + c, o);
         }
       }
     }

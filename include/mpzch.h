@@ -379,10 +379,18 @@ MPZCH_API int mpzch_get_status(mpzch_table* t, int32_t* status, void* stream);
 MPZCH_API int mpzch_trace_enable(mpzch_table* t, int32_t on);
 MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t nphases);
 
-/* Options.  MPZCH_OPT_WIDE_ROUNDS: number of grid-wide insert conflict rounds
- * launched before a single-block kernel places the remaining keys (default 3,
- * range 0..64).  Results do not depend on it. */
+/* Options.  Results never depend on them.
+ * MPZCH_OPT_CLUSTER_INSERT: how the missing ids of a Writeback are inserted.
+ * 1 (default) = cluster placement: ids whose windows chain together (home
+ * slots less than P apart) form a cluster, each cluster is placed by one
+ * thread in ascending key order, clusters in parallel (when the windows may
+ * cover the whole ring -- missing ids x P >= C -- one block places them all).
+ * 0 = claim rounds: MPZCH_OPT_WIDE_ROUNDS grid-wide rounds in which every
+ * unplaced id claims its window, then one block places the rest.
+ * MPZCH_OPT_WIDE_ROUNDS: the number of those rounds (default 3, range
+ * 0..64). */
 #define MPZCH_OPT_WIDE_ROUNDS 1
+#define MPZCH_OPT_CLUSTER_INSERT 4
 /* MPZCH_OPT_SIDE_PRIORITY: 1 (default) = the side stream of mpzch_train_step
  * gets the device's highest stream priority, 0 = the lowest; only before the
  * first mpzch_train_step of the table (MPZCH_EINVAL afterwards). */

@@ -71,7 +71,7 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
              state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
              ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None,
              fused_step: bool = False, eta: Optional[float] = None,
-             flags: int = 0) -> RunResult:
+             flags: int = 0, cluster: Optional[int] = None) -> RunResult:
     """Runs steps [start, start+steps) of workload w on both sides.
 
     Per step: lookup of the labeled ids, fused gather (with the always-on concat
@@ -83,6 +83,8 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
         tbl, orc = make_pair(w, flags=flags)
     if wide_rounds is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, wide_rounds)
+    if cluster is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT, cluster)
     if eta is not None:
         binding.mpzch_set_learning_rate(tbl.h, eta)
         orc.set_learning_rate(eta)

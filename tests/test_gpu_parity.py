@@ -5,9 +5,10 @@ ragged tail, and compares the lookup rows / hit mask, the fused gather
 (cached branch + always-on concat), the Writeback counters and the whole table
 state (keys, last-write steps, values) after every step.  Edge cases: empty
 batches, bad ids and rows, non-power-of-two capacity, P = 1, P = C, P > 32,
-windows wrapping past the last row, heavy eviction with dropped writes, the
-insert rounds run fully grid-wide, fully in the single-block finisher or
-split between them, checkpoint/resume, and repeatability.
+windows wrapping past the last row, heavy eviction with dropped writes, both
+insert paths (cluster placement, with its whole-ring fallback, long chains and
+shared start slots; claim rounds run fully grid-wide, fully in the single-block
+finisher or split between them), checkpoint/resume, and repeatability.
 """
 import numpy as np
 import pytest
@@ -91,10 +92,71 @@ def test_fused_train_step_with_no_labeled_ids():
 
 @pytest.mark.parametrize("wide", [0, 1, 4, 64])
 def test_insert_rounds_split_does_not_change_results(wide):
-    r = run_pair(SCALED["c4_stress"], wide_rounds=wide)
+    r = run_pair(SCALED["c4_stress"], wide_rounds=wide, cluster=0)
     if wide >= 1:  # conflicts really happened (the single-block finisher counts as one round)
         assert max(s["n_rounds"] for s in r.stats) >= 2
     assert sum(s["n_dropped"] for s in r.stats) > 0
+
+
+CLUSTERED = {
+    # missing ids x P stay below C, so the grid-wide cluster placement runs;
+    # enough misses per step that multi-key clusters are common
+    "clus_p8": W("clus_p8", 11, capacity=1 << 15, dim=32, probes=8, steps=12, labeled=3000,
+                 pool=0, zipf_alpha=0.9, zipf_keys=60_000, fresh_frac=0.3),
+    "clus_p16": W("clus_p16", 12, capacity=1 << 14, dim=16, probes=16, steps=16, labeled=1200,
+                  pool=0, zipf_alpha=0.9, zipf_keys=80_000, fresh_frac=0.5),
+    "clus_p3_nonpow2": W("clus_p3_nonpow2", 13, capacity=30011, dim=16, probes=3, steps=12,
+                         labeled=4000, pool=0, zipf_alpha=0.95, zipf_keys=60_000,
+                         fresh_frac=0.3),
+}
+
+
+@pytest.mark.parametrize("name", list(CLUSTERED))
+@pytest.mark.parametrize("cluster", [1, 0])
+def test_cluster_placement_and_claim_rounds_bit_exact(name, cluster):
+    w = CLUSTERED[name]
+    r = run_pair(w, cluster=cluster)
+    # the cluster placement really ran (not the whole-ring fallback) on most steps
+    grid_wide = [s for s in r.stats if 0 < s["n_inserted"] and s["n_inserted"] * w.probes < w.capacity]
+    assert len(grid_wide) >= w.steps // 2
+    assert sum(s["n_evicted"] for s in r.stats) > 0
+
+
+def _keys_with_home(C, slots, count_per_slot, start):
+    # test-side hash (the published SplitMix64, as in the input generator) to
+    # build keys whose start slots are chosen
+    cand = np.arange(start, start + (1 << 22), dtype=np.int64)
+    homes = (inputs.splitmix64_np(cand) % np.uint64(C)).astype(np.int64)
+    out = []
+    for s_, c in zip(slots, count_per_slot):
+        ks = cand[homes == s_][:c]
+        assert ks.size == c
+        out.append(ks)
+    return np.concatenate(out)
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_cluster_placement_long_chains_and_shared_slots(fused):
+    """Clusters beyond the 32 keys sorted in registers: a chain of 40 keys with
+    start slots 2 apart that wraps past the last row, and 36 keys sharing one
+    start slot (28 of them are evicted again in the same step)."""
+    C, P, D = 1 << 16, 8, 16
+    w = W("crafted", 14, capacity=C, dim=D, probes=P, steps=4, labeled=400, pool=0,
+          zipf_alpha=1.0, zipf_keys=1000)
+    rng = np.random.default_rng(5)
+    batches = []
+    for t in range(4):
+        chain = _keys_with_home(C, [(C - 30 + 2 * i + (t % 2)) % C for i in range(40)], [1] * 40,
+                                start=(t + 1) << 24)
+        shared = _keys_with_home(C, [C // 2 + 3 * t], [36], start=(t + 9) << 24)
+        other = rng.integers(1 << 40, 1 << 41, size=200, dtype=np.int64)
+        repeat = batches[-1][:50] if batches else np.empty(0, np.int64)
+        ids = np.concatenate([chain, shared, other, repeat])
+        batches.append(ids[rng.permutation(ids.size)])
+    r = run_pair(w, steps=4, ids_fn=lambda t: batches[t], fused_step=fused)
+    for s in r.stats:
+        assert s["n_inserted"] * P < C  # the grid-wide cluster path
+    assert sum(s["n_dropped"] for s in r.stats) >= 4 * 28
 
 
 @pytest.mark.parametrize("eta", [0.5, 0.1, 2.0 / 3.0, 0.0, 1.75])
