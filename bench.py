@@ -44,7 +44,7 @@ UNIT = "unique rows/s"
 PREFILL = 20  # untimed steps that bring the table to its steady state
 # DRAM bytes (read + write) of one k_writeback launch of this workload, from
 # one ncu capture of the current kernel (profiles/k_writeback_multitable_c1m_d512.md)
-WB_TRAFFIC_BYTES = 545.38e6
+WB_TRAFFIC_BYTES = 550.74e6
 WB_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                      "(23rd step of the multi-table workload)")
 REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
