@@ -92,6 +92,32 @@ int after_launch() {
   return cudaGetLastError() == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
 }
 
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device) and size: the attribute belongs to the
+// kernel function on one device, so kernels sharing a signature (template
+// instances) and devices are tracked separately.
+int allow_dynamic_smem(const void* kern, size_t bytes) {
+  struct Entry {
+    const void* kern;
+    int device;
+    size_t bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MPZCH_ECUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : done)
+    if (e.kern == kern && e.device == dev && e.bytes >= bytes) return MPZCH_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MPZCH_ECUDA;
+  }
+  done.push_back({kern, dev, bytes});
+  return MPZCH_OK;
+}
+
 // Launches a kernel; with `pdl` it may start while the previous kernel of the
 // stream drains (programmatic dependent launch: every kernel waits for its
 // predecessors with griddepcontrol.wait before touching memory).
@@ -120,15 +146,8 @@ int launch(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t s
 template <typename... KArgs, typename... Args>
 int launch_smem(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
                 cudaStream_t st, bool pdl, Args&&... args) {
-  static bool attr_set = false;  // one kernel per instantiation
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
-      cudaGetLastError();
-      return MPZCH_ECUDA;
-    }
-    attr_set = true;
-  }
+  int rc = allow_dynamic_smem(reinterpret_cast<const void*>(kern), smem);
+  if (rc) return rc;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
@@ -917,6 +936,33 @@ int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows
   return mark_user(t, st, rc);
 }
 
+namespace {
+// Row export: the staged kernel (shared-memory double buffering) for dim 512
+// or 1024 with a 16-byte aligned q, the register kernel for every other shape.
+int launch_export(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n, int8_t* q,
+                  float* scale, int64_t* keys_out, int64_t* last_out, cudaStream_t st) {
+  const long long* dn = reinterpret_cast<const long long*>(dev_n);
+  const float4* M = reinterpret_cast<const float4*>(t->M);
+  long long* ko = reinterpret_cast<long long*>(keys_out);
+  long long* lo = reinterpret_cast<long long*>(last_out);
+  const bool q16 = (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+  uint4* q4 = reinterpret_cast<uint4*>(q);
+  const unsigned grid = grid_for(n * 32, kBlock, 4);
+  if (q16 && t->D == 512)
+    return launch_smem(k_export_int8_staged<1>, grid, kBlock, export_stage_smem(1), st, false,
+                       rows, n, dn, M, t->keys, t->C, q4, scale, ko, t->status,
+                       static_cast<const long long*>(t->last), lo);
+  if (q16 && t->D == 1024)
+    return launch_smem(k_export_int8_staged<2>, grid, kBlock, export_stage_smem(2), st, false,
+                       rows, n, dn, M, t->keys, t->C, q4, scale, ko, t->status,
+                       static_cast<const long long*>(t->last), lo);
+  k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+      rows, n, dn, M, t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale, ko, t->status,
+      t->last, lo);
+  return after_launch();
+}
+}  // namespace
+
 int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n,
                       int8_t* q, float* scale, int64_t* keys_out, void* stream) {
   if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
@@ -928,11 +974,7 @@ int mpzch_export_int8(mpzch_table* t, const int32_t* rows, int64_t n, const int6
   if (rc) return rc;
   {
     PhaseScope ps(t, PH_EXPORT, st);
-    k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
-        rows, n, reinterpret_cast<const long long*>(dev_n), reinterpret_cast<const float4*>(t->M),
-        t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale,
-        reinterpret_cast<long long*>(keys_out), t->status, nullptr, nullptr);
-    rc = after_launch();
+    rc = launch_export(t, rows, n, dev_n, q, scale, keys_out, nullptr, st);
   }
   return mark_user(t, st, rc);
 }
@@ -1150,12 +1192,7 @@ int export_since(mpzch_table* t, int64_t since, int32_t* rows, int64_t* dev_coun
   }
   if (!rc) {
     PhaseScope ps(t, PH_EXPORT, st);
-    k_export_int8<<<grid_for(max_rows * 32, kBlock), kBlock, 0, st>>>(
-        rows, max_rows, reinterpret_cast<const long long*>(dev_count),
-        reinterpret_cast<const float4*>(t->M), t->keys, t->C, t->D / 4,
-        reinterpret_cast<char4*>(q), scale, reinterpret_cast<long long*>(keys), t->status,
-        t->last, reinterpret_cast<long long*>(last));
-    rc = after_launch();
+    rc = launch_export(t, rows, max_rows, dev_count, q, scale, keys, last, st);
   }
   return mark_user(t, st, rc);
 }

@@ -1416,64 +1416,99 @@ __global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __re
 // rounds to the same integer as p; otherwise the IEEE division is taken.  (A
 // reciprocal that is not finite, for a subnormal s, sends every element to
 // the division.)
-__device__ __forceinline__ signed char quant1(float xv, float s, float rcp, bool fast) {
-  int t;
-  const float p = __fmul_rn(xv, rcp);
-  const float dist = fabsf(fabsf(p - truncf(p)) - 0.5f);
-  if (fast && dist > 1e-4f)
-    t = __float2int_rn(p);
-  else
-    t = __float2int_rn(__fdiv_rn(xv, s));
-  t = t > 127 ? 127 : (t < -127 ? -127 : t);
-  return (signed char)t;
+// Round-half-to-even of |v| < 2^22 without a conversion instruction: adding
+// 1.5 * 2^23 leaves v's nearest integer (ties to even, IEEE rounding of the
+// add) in the low mantissa bits, and subtracting it again gives that integer as
+// a float.  Only full-rate FP32 / integer operations.
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+constexpr int kRoundMagicBits = 0x4B400000;
+
+__device__ __forceinline__ int rne_small(float v) {
+  return __float_as_int(__fadd_rn(v, kRoundMagic)) - kRoundMagicBits;
 }
 
-__device__ __forceinline__ uint32_t quant4(float4 v, float s, float rcp, bool fast) {
-  const uint32_t b0 = (uint8_t)quant1(v.x, s, rcp, fast), b1 = (uint8_t)quant1(v.y, s, rcp, fast);
-  const uint32_t b2 = (uint8_t)quant1(v.z, s, rcp, fast), b3 = (uint8_t)quant1(v.w, s, rcp, fast);
-  return b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+// int8 code of x / s for the values of one lane.  The product p = x * fl(1/s)
+// is within 3.1e-5 of x / s, so rne(p) = rne(x / s) whenever p lies at least
+// 1e-4 from a half-integer; a lane with any value closer than that (or with no
+// usable reciprocal) recomputes all of its values from the IEEE quotient.
+// |x| <= a = 127 s, so every code lies in [-127, 127] (clamped all the same).
+template <int kN>
+__device__ __forceinline__ void quant_lane(const float (&x)[kN], float s, float rcp, bool fast,
+                                           int (&t)[kN]) {
+  bool amb = !fast;
+#pragma unroll
+  for (int e = 0; e < kN; ++e) {
+    const float p = __fmul_rn(x[e], rcp);
+    const float y = __fadd_rn(p, kRoundMagic);
+    const float r = __fsub_rn(y, kRoundMagic);
+    amb |= fabsf(__fsub_rn(p, r)) > 0.4999f;
+    t[e] = __float_as_int(y) - kRoundMagicBits;
+  }
+  if (amb) {
+#pragma unroll
+    for (int e = 0; e < kN; ++e) t[e] = rne_small(__fdiv_rn(x[e], s));
+  }
+#pragma unroll
+  for (int e = 0; e < kN; ++e) t[e] = max(-127, min(127, t[e]));
 }
 
-// Export of one row by one warp, the row held in registers: lane l owns the
-// 16-byte vectors 4l..4l+3 of each 2 KiB chunk (64 contiguous input bytes) and
-// writes their 16 int8 values with one 16-byte store.  kChunks chunks of 128
-// vectors cover dim = 512 * kChunks.
+__device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Quantise and store one row held by a warp: lane l holds the 16-byte
+// vectors 4l..4l+3 of each 2 KiB chunk (64 contiguous input bytes) as v and
+// writes their 16 int8 values with one 16-byte store per chunk.
 template <int kChunks>
-__device__ __forceinline__ void export_row_regs(const float4* __restrict__ x, uint4* qo, float* sc,
-                                                long long* ko, long long* lo, long long key,
-                                                long long lastv, int lane) {
-  float4 v[kChunks][4];
-#pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) v[ch][j] = __ldcs(x + ch * 128 + 4 * lane + j);
+__device__ __forceinline__ void export_values(const float (&v)[kChunks * 16], uint4* qo, float* sc,
+                                              long long* ko, long long* lo, long long key,
+                                              long long lastv, int lane) {
   float a = 0.f;
 #pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch)
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      a = fmaxf(a, fmaxf(fmaxf(fabsf(v[ch][j].x), fabsf(v[ch][j].y)),
-                         fmaxf(fabsf(v[ch][j].z), fabsf(v[ch][j].w))));
+  for (int e = 0; e < kChunks * 16; ++e) a = fmaxf(a, fabsf(v[e]));
   for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
   const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
   const float rcp = a == 0.f ? 0.f : __frcp_rn(s);
   const bool fast = a != 0.f && isfinite(rcp);
 #pragma unroll
   for (int ch = 0; ch < kChunks; ++ch) {
-    uint4 o = make_uint4(0u, 0u, 0u, 0u);
-    if (a != 0.f) {
-      o.x = quant4(v[ch][0], s, rcp, fast);
-      o.y = quant4(v[ch][1], s, rcp, fast);
-      o.z = quant4(v[ch][2], s, rcp, fast);
-      o.w = quant4(v[ch][3], s, rcp, fast);
+    float vc[16];
+    int c[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      vc[e] = v[ch * 16 + e];
+      c[e] = 0;
     }
-    __stcs(qo + ch * 32 + lane, o);
+    if (a != 0.f) quant_lane<16>(vc, s, rcp, fast, c);
+    __stcs(qo + ch * 32 + lane, make_uint4(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
+                                           pack4(c[8], c[9], c[10], c[11]),
+                                           pack4(c[12], c[13], c[14], c[15])));
   }
   if (lane == 0) {
     *sc = s;
     *ko = key;
     if (lo) *lo = lastv;
   }
+}
+
+// Export of one row by one warp, the row loaded into registers.  kChunks
+// chunks of 128 vectors cover dim = 512 * kChunks.
+template <int kChunks>
+__device__ __forceinline__ void export_row_regs(const float4* __restrict__ x, uint4* qo, float* sc,
+                                                long long* ko, long long* lo, long long key,
+                                                long long lastv, int lane) {
+  float v[kChunks * 16];
+#pragma unroll
+  for (int ch = 0; ch < kChunks; ++ch)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 f = __ldcs(x + ch * 128 + 4 * lane + j);
+      v[ch * 16 + 4 * j] = f.x;
+      v[ch * 16 + 4 * j + 1] = f.y;
+      v[ch * 16 + 4 * j + 2] = f.z;
+      v[ch * 16 + 4 * j + 3] = f.w;
+    }
+  export_values<kChunks>(v, qo, sc, ko, lo, key, lastv, lane);
 }
 
 // Any dim (multiple of 4): two passes over the row (max, then quantise) with
@@ -1491,12 +1526,11 @@ __device__ __forceinline__ void export_row_generic(const float4* __restrict__ x,
   const float rcp = a == 0.f ? 0.f : __frcp_rn(s);
   const bool fast = a != 0.f && isfinite(rcp);
   for (int c = lane; c < D4; c += 32) {
-    const float4 v = x[c];
-    char4 o = make_char4(0, 0, 0, 0);
-    if (a != 0.f)
-      o = make_char4(quant1(v.x, s, rcp, fast), quant1(v.y, s, rcp, fast),
-                     quant1(v.z, s, rcp, fast), quant1(v.w, s, rcp, fast));
-    qo[c] = o;
+    const float4 f = x[c];
+    const float v[4] = {f.x, f.y, f.z, f.w};
+    int t[4] = {0, 0, 0, 0};
+    if (a != 0.f) quant_lane<4>(v, s, rcp, fast, t);
+    qo[c] = make_char4((signed char)t[0], (signed char)t[1], (signed char)t[2], (signed char)t[3]);
   }
   if (lane == 0) {
     *sc = s;
@@ -1505,7 +1539,7 @@ __device__ __forceinline__ void export_row_generic(const float4* __restrict__ x,
   }
 }
 
-__global__ void __launch_bounds__(kBlock) k_export_int8(
+__global__ void __launch_bounds__(kBlock, 4) k_export_int8(
     const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
     const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C, int D4,
     char4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
@@ -1546,6 +1580,99 @@ __global__ void __launch_bounds__(kBlock) k_export_int8(
     else
       export_row_generic(x, qo, D4, scale + i, keys_out + i, lo, key, lastv, lane);
   }
+}
+
+// Asynchronous 16-byte global -> shared copy (L2 only) and its groups.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Export with the rows staged through shared memory (dim = 512 * kChunks,
+// 16-byte aligned q): each warp owns two row buffers and copies the next row
+// (cp.async) while it quantises the current one, so a row's load latency
+// overlaps the previous row's reduction, rounding and stores.  Lane l stages
+// exactly the vectors it later reads (4l..4l+3 of each chunk), so it waits only
+// for its own copies and no warp barrier is needed.  Same results as
+// k_export_int8.
+template <int kChunks>
+__global__ void __launch_bounds__(kBlock, 4) k_export_int8_staged(
+    const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
+    const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C,
+    uint4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
+    int32_t* status, const long long* __restrict__ last, long long* __restrict__ last_out) {
+  pdl_enter();
+  extern __shared__ __align__(16) float4 s_stage[];
+  constexpr int kVec = kChunks * 128;  // 16-byte vectors per row
+  const int lane = threadIdx.x & 31;
+  float4* buf = s_stage + (size_t)(threadIdx.x >> 5) * 2 * kVec;
+  int64_t nn = n;
+  if (dev_n) {
+    const long long d = *dev_n;
+    nn = d < nn ? d : nn;
+  }
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t first = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  auto issue = [&](int64_t i, int stage) {
+    if (i < nn) {
+      const int32_t r = rows[i];
+      if (r >= 0 && (int64_t)r < C) {
+        const float4* src = M + (int64_t)r * kVec + 4 * lane;
+        float4* dst = buf + stage * kVec + 4 * lane;
+#pragma unroll
+        for (int ch = 0; ch < kChunks; ++ch)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) cp_async16(dst + ch * 128 + j, src + ch * 128 + j);
+      }
+    }
+    cp_async_commit();  // one group per issue, empty or not, so the counts stay in step
+  };
+  issue(first, 0);
+  int stage = 0;
+  for (int64_t i = first; i < nn; i += warps, stage ^= 1) {
+    issue(i + warps, stage ^ 1);
+    cp_async_wait<1>();  // this lane's copies of row i have landed
+    const int32_t r = rows[i];
+    uint4* qo = q + i * (int64_t)(kChunks * 32);
+    long long* lo = last_out ? last_out + i : nullptr;
+    if (r < 0 || (int64_t)r >= C) {
+      if (lane == 0) {
+        set_status(status, kStBadRow);
+        scale[i] = 0.f;
+        keys_out[i] = -1;
+        if (lo) *lo = -1;
+      }
+#pragma unroll
+      for (int ch = 0; ch < kChunks; ++ch) qo[ch * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
+      continue;
+    }
+    const float4* mine = buf + stage * kVec + 4 * lane;
+    float v[kChunks * 16];
+#pragma unroll
+    for (int ch = 0; ch < kChunks; ++ch)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 f = mine[ch * 128 + j];
+        v[ch * 16 + 4 * j] = f.x;
+        v[ch * 16 + 4 * j + 1] = f.y;
+        v[ch * 16 + 4 * j + 2] = f.z;
+        v[ch * 16 + 4 * j + 3] = f.w;
+      }
+    export_values<kChunks>(v, qo, scale + i, keys_out + i, lo, keys[r], last_out ? last[r] : 0,
+                           lane);
+  }
+  cp_async_wait<0>();
+}
+
+constexpr size_t export_stage_smem(int kChunks) {
+  return (size_t)(kBlock / 32) * 2 * kChunks * 128 * sizeof(float4);
 }
 
 // ---------------------------------------------------------------------------

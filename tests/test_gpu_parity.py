@@ -297,10 +297,12 @@ def test_select_export_and_serve_match_oracle():
     assert 0 < ohit.mean() < 1
 
 
-def test_export_edge_rows():
-    """All-zero rows (scale 0), rows with a single large element, negative absmax."""
+@pytest.mark.parametrize("D", [16, 512, 1024])
+def test_export_edge_rows(D):
+    """All-zero rows (scale 0), rows with a single large element, negative absmax
+    (dims 512 and 1024 take the staged export kernel, others the register one)."""
     from hashed_sparse_table_b200 import binding
-    C, D = 64, 16
+    C = 64
     tbl = binding.MpzchTable(C, D, 4)
     orc = oracle.OracleTable(C, D, 4)
     _, _, M = tbl.state()
@@ -309,7 +311,7 @@ def test_export_edge_rows():
     vals[0] = 0
     vals[1] = 0
     vals[1, 5] = -3e-38
-    vals[2] = np.float32(127.0) * np.arange(-8, 8, dtype=np.float32)
+    vals[2] = np.float32(127.0) * (np.arange(D, dtype=np.float32) - np.float32(D // 2))
     vals[3] = np.float32(1e30)
     vals[4, :] = np.float32(-0.0)
     M.copy_(torch.from_numpy(vals))
@@ -320,14 +322,25 @@ def test_export_edge_rows():
     oq, os_, ok = orc.export_int8(rows)
     assert_bitwise(q.cpu().numpy(), oq, "q")
     assert_bitwise(s.cpu().numpy(), os_, "scale")
+    # rows outside [0, C): zero codes, scale 0, key -1 and the bad-row status
+    bad = np.array([3, -1, C, 5, 2**31 - 1], np.int32)
+    q, s, k = tbl.export_int8(torch.from_numpy(bad).cuda())
+    assert tbl.status() == binding.MPZCH_STATUS_BADROW
+    ok_at = np.array([0, 3])
+    oq, os_, _ = orc.export_int8(bad[ok_at])
+    assert_bitwise(q.cpu().numpy()[ok_at], oq, "q of valid rows")
+    assert_bitwise(s.cpu().numpy()[ok_at], os_, "scale of valid rows")
+    for i in (1, 2, 4):
+        assert not q[i].any() and s[i].item() == 0.0 and k[i].item() == -1
 
 
-def test_export_near_half_integer_quotients():
+@pytest.mark.parametrize("D", [64, 512, 1024])
+def test_export_near_half_integer_quotients(D):
     """Rows built so that x/scale lands on or within a few ulps of k + 1/2 (the
     rounding boundary), plus subnormal-scale rows: every int8 byte must match
     the oracle's IEEE division and round-half-even."""
     from hashed_sparse_table_b200 import binding
-    C, D = 512, 64
+    C = 512
     tbl = binding.MpzchTable(C, D, 4)
     orc = oracle.OracleTable(C, D, 4)
     rng = np.random.default_rng(11)
