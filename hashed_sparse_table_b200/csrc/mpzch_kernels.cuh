@@ -745,7 +745,20 @@ constexpr int kClusterMax = 4096;
 constexpr int kClusterBuckets = 4096;
 constexpr size_t kClusterSmem = (size_t)kClusterMax * (4 + 8 + 4) + (kClusterBuckets + 1) * 4;
 
-__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, long long& evicted);
+// Scratch of one thread running place_cluster_serial (slot heads, keys and
+// their distinct-id indices, the span's steps).
+struct SerialScratch {
+  unsigned long long heads[32];
+  long long ck[32];
+  long long sl[96];
+  int32_t cu[32];
+};
+constexpr int kSerialThreads = 32;  // threads of k_insert_finish that place listed clusters
+static_assert(sizeof(SerialScratch) * kSerialThreads <= kClusterSmem,
+              "serial scratch must fit the finisher's dynamic shared memory");
+
+__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, SerialScratch& w,
+                                     long long& evicted);
 
 __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
   pdl_enter();
@@ -762,8 +775,11 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
     const int32_t S = p.ctr->n_serial;
     if (S == 0) return;  // block-uniform
     long long ev_serial = 0;
-    for (int32_t i = threadIdx.x; i < S; i += blockDim.x)
-      place_cluster_serial(p, __ldcg(p.lidx[2] + i), ncur, ev_serial);
+    // one warp, each thread with its scratch in the dynamic shared memory
+    SerialScratch* scratch = reinterpret_cast<SerialScratch*>(dsm);
+    if (threadIdx.x < kSerialThreads)
+      for (int32_t i = threadIdx.x; i < S; i += kSerialThreads)
+        place_cluster_serial(p, __ldcg(p.lidx[2] + i), ncur, scratch[threadIdx.x], ev_serial);
     const long long evs = block_sum_ll(ev_serial, sm);
     if (threadIdx.x == 0 && evs) atomic_add_ll(&p.stats->n_evicted, evs);
     return;
@@ -975,9 +991,10 @@ __device__ int32_t cluster_min_unplaced(const WbParams& p, int64_t h, int64_t L,
 // heads per batch, collect and sort the keys, copy the span's steps and decide
 // every placement on the copy; clusters beyond the local limits place key by
 // key in global memory.  Used where the warp path does not apply.
-__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, long long& evicted) {
+__device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, SerialScratch& w,
+                                     long long& evicted) {
   const Geo& g = p.g;
-  unsigned long long heads[kClusterLocal];
+  unsigned long long* heads = w.heads;
   int nh = 0;
   bool overflow = false;
   heads[nh++] = ld_cg(p.shead + h);
@@ -1002,8 +1019,8 @@ __device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, lo
     off += q;
     if (q < 8) break;
   }
-  long long ck[kClusterLocal];
-  int32_t cu[kClusterLocal];
+  long long* ck = w.ck;
+  int32_t* cu = w.cu;
   int n = 0;
   for (int i = 0; i < nh && !overflow; ++i)
     for (int32_t x = (int32_t)(uint32_t)heads[i], hops = 0; x >= 0 && hops <= N && !overflow;
@@ -1011,7 +1028,7 @@ __device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, lo
       overflow |= !sorted_add(ck, cu, n, __ldcg(p.lkey[0] + x), __ldcg(p.lidx[0] + x));
   const int64_t span = L + g.P;
   if (!overflow && span <= kSpanLocal) {
-    long long sl[kSpanLocal];
+    long long* sl = w.sl;
     for (int64_t o0 = 0; o0 < span; o0 += 16) {
       long long v[16];
 #pragma unroll
@@ -1126,6 +1143,8 @@ __device__ bool place_cluster_warp(const WbParams& p, int64_t h, int32_t N, Warp
     sw.us[r] = sw.u[j];
   }
   __syncwarp();
+  int span_pow2 = 1;
+  while (span_pow2 < g.P) span_pow2 <<= 1;
   for (int j = 0; j < n; ++j) {
     const long long k = sw.ks[j];
     int64_t off = home_slot(k, g) - h;
@@ -1140,7 +1159,10 @@ __device__ bool place_cluster_warp(const WbParams& p, int64_t h, int32_t N, Warp
       cl = 0x7FFFFFFFFFFFFFFFll;
       cs = 0x7FFFFFFFFFFFFFFFll;
     }
-    for (int d = 16; d > 0; d >>= 1) {
+    // argmin over lanes 0..P-1 (lanes >= P hold +inf): the xor rounds below
+    // the next power of two >= P reduce every aligned group of that width, so
+    // lane 0 holds the window's minimum; it is then broadcast
+    for (int d = span_pow2 >> 1; d > 0; d >>= 1) {
       const long long ol = __shfl_xor_sync(0xFFFFFFFFu, cl, d);
       const long long os = __shfl_xor_sync(0xFFFFFFFFu, cs, d);
       const int oo = __shfl_xor_sync(0xFFFFFFFFu, co, d);
@@ -1150,6 +1172,9 @@ __device__ bool place_cluster_warp(const WbParams& p, int64_t h, int32_t N, Warp
         co = oo;
       }
     }
+    cl = __shfl_sync(0xFFFFFFFFu, cl, 0);
+    cs = __shfl_sync(0xFFFFFFFFu, cs, 0);
+    co = __shfl_sync(0xFFFFFFFFu, co, 0);
     if (co < 32) {
       if (lane == co) l0 = p.step;
     } else if (lane == co - 32) {

@@ -220,3 +220,66 @@ def test_sharded_step_matches_sharded_oracle(G):
         assert_bitwise(M, so.values(s), f"G={G} shard {s}: values")
         assert tstatus == 0 and cstatus == 0
     so.close()
+
+
+def test_sharded_step_with_negative_ids():
+    """Negative ids: the owner's lookup reports them as misses (bad-key status
+    on the owner's table), the rank's first dedup skips them (bad-key status on
+    the rank's own table), and every other output matches the sharded oracle."""
+    from hashed_sparse_table_b200 import sharded
+    w = SHARD_W.scaled(steps=3, labeled=300, pool=900)
+    G = 2
+    group = sharded.LocalExchangeGroup(G)
+    ao = inputs.author_table(w)
+    got = [[None] * w.steps for _ in range(G)]
+    status = [None] * G
+    errors = []
+
+    def batch(t, r):
+        ids, e, aor = _rank_inputs(w, t, r)
+        ids = ids.copy()
+        ids[5::97] = -1 - np.arange(ids[5::97].size)  # negative ids in both parts
+        return ids, e, inputs.author_rows(w, np.maximum(ids[:w.labeled], 0))
+
+    def rank_main(r):
+        try:
+            shard = sharded.ShardedMpzch(w.capacity, w.dim, w.probes, group.member(r))
+            dev = shard.device
+            ao_d = torch.from_numpy(ao).to(dev)
+            for t in range(w.steps):
+                ids, e, aor = batch(t, r)
+                rows, hit, out, st = shard.train_step(
+                    torch.from_numpy(ids).to(dev), w.labeled, torch.from_numpy(e).to(dev), t,
+                    ao_d, torch.from_numpy(aor).to(dev))
+                got[r][t] = (rows.cpu().numpy(), hit.cpu().numpy(), out.cpu().numpy(),
+                             stats_dict(st))
+            status[r] = shard.table.status()
+            shard.close()
+        except BaseException as ex:  # noqa: BLE001
+            errors.append(ex)
+            group.abort()
+
+    threads = [threading.Thread(target=rank_main, args=(r,)) for r in range(G)]
+    for th in threads:
+        th.start()
+    for th in threads:
+        th.join()
+    if errors:
+        raise errors[0]
+    so = oracle.ShardedOracle(G, w.capacity, w.dim, w.probes)
+    for t in range(w.steps):
+        batches = [batch(t, r) for r in range(G)]
+        for r, (ids, e, aor) in enumerate(batches):
+            _, orows, ohit, oout = so.lookup_gather(ids[:w.labeled], ao, aor)
+            rows, hit, out, _ = got[r][t]
+            assert_bitwise(rows, orows, f"step {t} rank {r}: rows")
+            assert_bitwise(hit, ohit, f"step {t} rank {r}: hit")
+            assert_bitwise(out, oout, f"step {t} rank {r}: features")
+        res = so.writeback([b[0] for b in batches], [b[1] for b in batches], t)
+        for s, (rc, ost) in enumerate(res):
+            assert rc == 0
+            for k in ("n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped"):
+                assert got[s][t][3][k] == ost[k], (t, s, k)
+    from hashed_sparse_table_b200 import binding
+    assert all(st_ & binding.MPZCH_STATUS_BADKEY for st_ in status)
+    so.close()
