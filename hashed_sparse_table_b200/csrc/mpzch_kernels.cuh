@@ -729,9 +729,13 @@ __device__ __forceinline__ void place_key(const WbParams& p, long long k, int32_
   p.urow[u] = (int32_t)best;
 }
 
-// Keys left after the grid-wide rounds, in one block.
+// One block that places what the grid-wide kernels left.  Claim-round path:
+// the keys left after the grid-wide rounds.  Cluster placement path: the
+// clusters listed by k_place_multi (beyond the warp path), one thread each,
+// or -- when the windows may cover the whole ring -- every missing key, by the
+// sort below.
 //
-// Cluster path (at most kClusterMax keys): every key still unplaced only
+// Sort path (at most kClusterMax keys): every key still unplaced only
 // conflicts with unplaced keys whose windows overlap its own (keys placed in
 // earlier rounds are smaller than every unplaced key overlapping them, so
 // their effect already precedes in the sequential order).  The unplaced keys
@@ -745,13 +749,16 @@ constexpr int kClusterMax = 4096;
 constexpr int kClusterBuckets = 4096;
 constexpr size_t kClusterSmem = (size_t)kClusterMax * (4 + 8 + 4) + (kClusterBuckets + 1) * 4;
 
+constexpr int kClusterLocal = 32;  // cluster keys a serial thread sorts locally (else the slow walk)
+constexpr int kSpanLocal = 96;     // slots of a cluster's windows a serial thread copies locally
+
 // Scratch of one thread running place_cluster_serial (slot heads, keys and
 // their distinct-id indices, the span's steps).
 struct SerialScratch {
-  unsigned long long heads[32];
-  long long ck[32];
-  long long sl[96];
-  int32_t cu[32];
+  unsigned long long heads[kClusterLocal];
+  long long ck[kClusterLocal];
+  long long sl[kSpanLocal];
+  int32_t cu[kClusterLocal];
 };
 constexpr int kSerialThreads = 32;  // threads of k_insert_finish that place listed clusters
 static_assert(sizeof(SerialScratch) * kSerialThreads <= kClusterSmem,
@@ -923,21 +930,21 @@ __global__ void __launch_bounds__(1024) k_insert_finish(WbParams p, int r0) {
 // slots no other cluster touches, so placing each cluster's keys in ascending
 // key order, clusters independently, gives the state of the sequential insert
 // of all missing keys in ascending order.  The re-probe linked every missing
-// key into the list of its home slot; here the key whose index heads its slot's
-// list is the slot's representative, a representative with no occupied slot
-// among the P-1 slots before its own heads its cluster, and that thread walks
-// forward (the next occupied slot within P-1 of the last one found), collects
-// the cluster's keys from the slot lists and places them one after another
-// (victim = smallest (last, row) of the window, reading its own earlier
-// writes).  The common case -- a lone key with no neighbour within P-1 slots
-// -- is decided from one batch of loads issued together.
-//
-// Such a cut exists when the windows do not cover the whole ring, which is
-// certain when N * P < C (N missing keys).  Otherwise this kernel places
-// nothing and k_insert_finish places every key.
+// key into the list of its home slot.  The key whose index heads its slot's
+// list represents the slot; a representative with no occupied slot among the
+// P-1 slots before its own heads its cluster.  Three places do the work:
+//   k_place_clusters  one thread per missing key; a lone key (no other key
+//                     within P-1 slots, none sharing its slot) is decided and
+//                     placed from one batch of loads; heads of larger
+//                     clusters are listed;
+//   k_place_multi     one warp per listed cluster (place_cluster_warp);
+//   k_insert_finish   clusters beyond the warp path's limits, one thread each
+//                     (place_cluster_serial), and every key when the windows
+//                     may cover the whole ring.
+// A cut exists when the windows do not cover the whole ring, which is certain
+// when N * P < C (N missing keys); otherwise the grid-wide passes place
+// nothing.
 // ---------------------------------------------------------------------------
-constexpr int kClusterLocal = 32;  // cluster keys sorted locally; larger clusters take the slow walk
-constexpr int kSpanLocal = 96;     // slots of a cluster's windows copied locally
 
 __device__ __forceinline__ bool slot_used(unsigned long long v, uint32_t tag) {
   return (uint32_t)(v >> 32) == tag;
