@@ -143,7 +143,8 @@ def snapshot_from_export(capacity: int, dim: int, rows: np.ndarray, q: np.ndarra
     return snap_keys, snap_q, snap_s
 
 
-def run_pipelined(w: inputs.Workload, steps: Optional[int] = None, flags: int = 0):
+def run_pipelined(w: inputs.Workload, steps: Optional[int] = None, flags: int = 0,
+                  cluster: Optional[int] = None):
     """All steps' inputs uploaded first, then every step issued back to back as
     a pipelined mpzch_train_step (inputs_ready = one event after the uploads),
     each step with its own output buffers; then every output and the final
@@ -151,6 +152,8 @@ def run_pipelined(w: inputs.Workload, steps: Optional[int] = None, flags: int = 
     from hashed_sparse_table_b200 import binding
     T = w.steps if steps is None else steps
     tbl, orc = make_pair(w, flags=flags)
+    if cluster is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT, cluster)
     dev = tbl.device
     ao = inputs.author_table(w)
     ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None

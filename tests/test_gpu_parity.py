@@ -66,6 +66,19 @@ def test_pipelined_train_steps_bit_exact(name):
     run_pipelined(SCALED[name])
 
 
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress"])
+def test_pipelined_train_steps_with_claim_rounds_bit_exact(name):
+    from gpu_harness import run_pipelined
+    run_pipelined(SCALED[name], cluster=0)
+
+
+def test_pipelined_cluster_placement_on_the_grid_bit_exact():
+    """Pipelined steps where the grid-wide placement passes (not the whole-ring
+    fallback) do the inserts."""
+    from gpu_harness import run_pipelined
+    run_pipelined(CLUSTERED["clus_p8"])
+
+
 def test_pipelined_steps_then_other_calls_are_ordered():
     """Calls on the caller's stream after pipelined steps see the final table."""
     from gpu_harness import run_pipelined
