@@ -42,11 +42,14 @@ W = inputs.CFG3_MULTI
 METRIC = "unique rows/s through lookup+gather+writeback"
 UNIT = "unique rows/s"
 PREFILL = 20  # untimed steps that bring the table to its steady state
-# DRAM bytes (read + write) of one k_writeback launch of this workload, from
-# one ncu capture of the current kernel (profiles/k_writeback_multitable_c1m_d512.md)
-WB_TRAFFIC_BYTES = 550.74e6
-WB_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
-                     "(23rd step of the multi-table workload)")
+# DRAM bytes (read + write) of one row-update launch of this workload, per
+# kernel, each from one ncu capture of that kernel as it stands in this source
+# (dram__bytes_read.sum + dram__bytes_write.sum of a steady-state launch).  A
+# kernel missing here reports traffic null.
+ROW_UPDATE_TRAFFIC = {
+    "k_writeback": (550.74e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
+                              "(23rd step of the multi-table workload)"),
+}
 REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
 
 
@@ -90,7 +93,51 @@ def parse():
     ap.add_argument("--e-pool", type=int, default=inputs.E_POOL,
                     help="distinct item-tower target batches cycled through (memory bound for "
                          "profiling runs)")
+    ap.add_argument("--sharding-kernels", type=int, default=0, metavar="G",
+                    help="after the timed region, time the owner partition / combine kernels of "
+                         "hash-owner sharding for G owners on one step of the workload (no "
+                         "exchange: every owner's answer comes from this table)")
+    ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
+                    help="row kernels through registers or through shared memory with bulk "
+                         "copies (default: the library's)")
+    ap.add_argument("--bulk-warps", type=int, default=None)
+    ap.add_argument("--bulk-blocks", type=int, default=None)
+    ap.add_argument("--l2-hint", type=int, default=None, choices=[0, 1, 2],
+                    help="bulk row kernels: L2 policy of table rows (0 evict-first, 1 normal, "
+                         "2 evict-last)")
     return ap.parse_args()
+
+
+def apply_row_options(binding, tbl, args):
+    if args.row_kernel is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_ROW_KERNEL,
+                                 1 if args.row_kernel == "bulk" else 0)
+    if args.bulk_warps is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_BULK_WARPS, args.bulk_warps)
+    if args.bulk_blocks is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_BULK_BLOCKS, args.bulk_blocks)
+    if args.l2_hint is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_L2_HINT_ROWS, args.l2_hint)
+
+
+def row_update_kernel(binding, tbl) -> str:
+    """Name of the row-update kernel the table launches for this workload."""
+    bulk = binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_ROW_KERNEL) == 1
+    return "k_writeback_bulk" if bulk else "k_writeback"
+
+
+def host_cpu():
+    """(logical cores, model name) of the host."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return os.cpu_count(), model
 
 
 def config_dict(extra=None):
@@ -231,14 +278,17 @@ def run_reference(args):
     # bounded sample: at most 20 timed oracle steps, so the run ends within minutes
     k = max(1, min(steps, 20))
     v, tot, el = oracle_sample(k, prefill + args.warmup)
+    ncpu, model = host_cpu()
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
             "n_gpus": args.gpus, "steps": k, "warmup": args.warmup,
             "ms_per_step": el / k * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": config_dict({"prefill_steps": prefill}),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "host_cores": ncpu,
+                             "cpu_model": model, "kind": "oracle",
                              "sample": f"{k} steps of the multi-table workload after "
-                                       f"{prefill + args.warmup} untimed steps, one host thread"},
+                                       f"{prefill + args.warmup} untimed steps, one host thread "
+                                       f"of {ncpu}"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -294,6 +344,7 @@ def run_ours(args):
     if args.insert is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT,
                                  1 if args.insert == "cluster" else 0)
+    apply_row_options(binding, tbl, args)
 
     def step(t, i=None):
         # step t of the stream reads the resident inputs of slot i (default t)
@@ -353,7 +404,14 @@ def run_ours(args):
     wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
     gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
 
+    wb_kernel = row_update_kernel(binding, tbl)
+    wb_traffic = ROW_UPDATE_TRAFFIC.get(wb_kernel, (None, None))
     serving = None if args.no_serving else run_export_and_serve(tbl, binding, torch, dev, peak)
+
+    shard_k = None
+    if args.sharding_kernels > 0:
+        shard_k = run_sharding_kernels(tbl, binding, torch, dev, peak, args.sharding_kernels,
+                                       e_d[0], ao_d)
 
     res_info = None
     if args.res_every > 0:
@@ -370,9 +428,12 @@ def run_ours(args):
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             v, tot, el = oracle_sample(10, args.prefill)
-            cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            ncpu, model = host_cpu()
+            cpu = {"value": v, "unit": UNIT, "cores": 1, "host_cores": ncpu, "cpu_model": model,
+                   "kind": "oracle",
                    "sample": f"10 steps of the same workload after {args.prefill} untimed "
-                             f"steps ({tot} unique rows, {el:.1f} s), one host thread"}
+                             f"steps ({tot} unique rows, {el:.1f} s), one host thread of "
+                             f"{ncpu}"}
         result = {
             "metric": METRIC, "value": tot_units / (max_ms * 1e-3), "unit": UNIT,
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": max_ms / K,
@@ -380,10 +441,10 @@ def run_ours(args):
             "data": "synthetic (seeded Zipf id streams, N(0,1) item-tower targets)",
             "config": config_dict({"prefill_steps": Pf}),
             "gpu_launches": launches,
-            "roofline": {"bound": "hbm", "kernel": "k_writeback", "achieved": wb_gbs,
+            "roofline": {"bound": "hbm", "kernel": wb_kernel, "achieved": wb_gbs,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": wb_gbs / peak, "traffic": WB_TRAFFIC_BYTES,
-                         "traffic_source": WB_TRAFFIC_SOURCE,
+                         "frac": wb_gbs / peak, "traffic": wb_traffic[0],
+                         "traffic_source": wb_traffic[1],
                          "bytes_per_launch": wb_bytes / max(1, wb_launches),
                          "avg_launch_us": wb_ms * 1e3 / max(1, wb_launches)},
             "gather_writeback_gbs": gw_gbs,
@@ -411,6 +472,8 @@ def run_ours(args):
             result["config"]["values"] = "pinned host memory, mapped (host-memory tier)"
         if res_info is not None:
             result["res"] = res_info
+        if shard_k is not None:
+            result["sharding_kernels"] = shard_k
     tbl.close()
     if world > 1:
         dist.barrier()
@@ -525,6 +588,62 @@ def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):
     }
 
 
+def run_sharding_kernels(tbl, binding, torch, dev, peak, G, e_d, ao_d, reps: int = 5):
+    """The data-movement kernels of one sharded step for G owners on one step's
+    batch: the partition of the labeled ids, the partition of the distinct ids
+    with their e rows packed into the send buffer, and the combine of the
+    owners' answers (here: this table's lookup + gather of the partitioned ids)
+    with the always-on concat.  CUDA events on the current stream."""
+    D, A, lab = W.dim, W.ao_dim, W.labeled
+    ids = torch.from_numpy(host_step(10_000, 0)[0]).to(dev)
+    aor = torch.from_numpy(inputs.author_rows(W, host_step(10_000, 0)[0][:lab])).to(dev)
+    n = ids.numel()
+    ws = torch.empty(binding.mpzch_owner_partition_workspace(n, G), dtype=torch.uint8,
+                     device=dev)
+    counts = torch.empty((2, G), dtype=torch.int64, device=dev)
+    l_ids = torch.empty(lab, dtype=torch.int64, device=dev)
+    l_pos = torch.empty(lab, dtype=torch.int32, device=dev)
+    w_ids = torch.empty(n, dtype=torch.int64, device=dev)
+    w_pos = torch.empty(n, dtype=torch.int32, device=dev)
+    w_e = torch.empty((n, D), dtype=torch.float32, device=dev)
+    rows = torch.empty(lab, dtype=torch.int32, device=dev)
+    hit = torch.empty(lab, dtype=torch.uint8, device=dev)
+    out = torch.empty((lab, D + A), dtype=torch.float32, device=dev)
+    uniq, upos, ucnt = tbl.dedup(ids)
+    r_rows, r_hit = tbl.lookup(ids[:lab])
+    r_feat = tbl.gather_fused(r_rows, r_hit)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    t = {"partition_labeled": 0.0, "partition_distinct_e": 0.0, "combine": 0.0}
+    for rep in range(reps + 1):
+        torch.cuda.synchronize()
+        ev[0].record()
+        binding.mpzch_owner_partition(ids[:lab], G, l_ids, l_pos, counts[0], ws)
+        ev[1].record()
+        binding.mpzch_owner_partition(uniq, G, w_ids, w_pos, counts[1], ws, src_pos=upos,
+                                      dev_n=ucnt, e=e_d, e_out=w_e)
+        ev[2].record()
+        binding.mpzch_owner_combine(l_ids, l_pos, G, W.capacity, r_rows, r_feat, rows, hit, out,
+                                    ao_d, aor)
+        ev[3].record()
+        torch.cuda.synchronize()
+        if rep:  # the first pass is a warm-up
+            t["partition_labeled"] += ev[0].elapsed_time(ev[1]) / reps
+            t["partition_distinct_e"] += ev[1].elapsed_time(ev[2]) / reps
+            t["combine"] += ev[2].elapsed_time(ev[3]) / reps
+    U = int(ucnt.item())
+    # algorithmic bytes: ids + source positions in and out; e rows read and written;
+    # combine: send id + position + answer row + row index, author row, fused row written
+    b_scatter_e = U * (8 + 4 + 8 + 4 + 8 * D)
+    b_combine = lab * (8 + 4 + 4 + 4 * D + 4 * A + 4 * (D + A) + 5)
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    return {"owners": G, "distinct_ids": U, "ms": t,
+            "k_owner_scatter_with_e": {"bytes": b_scatter_e,
+                                       "gbs": gbs(b_scatter_e, t["partition_distinct_e"]),
+                                       "frac": gbs(b_scatter_e, t["partition_distinct_e"]) / peak},
+            "k_owner_combine": {"bytes": b_combine, "gbs": gbs(b_combine, t["combine"]),
+                                "frac": gbs(b_combine, t["combine"]) / peak}}
+
+
 def run_res(tbl, binding, torch, args, step_fn, first_step, n_inputs):
     """Training continues (cycling through the resident id batches with new step
     numbers) while every --res-every steps the rows written since the last
@@ -565,46 +684,86 @@ def run_res(tbl, binding, torch, args, step_fn, first_step, n_inputs):
 
 
 def run_e2e(tbl, binding, torch, dev, rank, world, total, K, e_host, E):
-    """Same steps (continuing the stream) with host inputs copied in every step."""
+    """Same steps (continuing the stream) through the public call with host
+    buffers: every step copies its ids, author rows and e from pinned host
+    memory to the device, runs mpzch_train_step, and copies its result back to
+    pinned host memory: the labeled rows, hit mask, fused features (the
+    32,768 x 640 fp32 the loss reads) and the step's counters.  Two device
+    slots alternate; uploads run on a copy stream one step ahead and downloads
+    on another, so step t+1's upload overlaps step t's compute and download.
+    Timed with CUDA events on the caller's stream, which at the end waits for
+    the last download."""
     import torch.distributed as dist
     lab = W.labeled
+    width = W.dim + W.ao_dim
     n0 = max(total, binding.mpzch_get_last_step(tbl.h) + 1)  # continue the step sequence
     host = [host_step(t, rank) for t in range(total, total + K)]
     ids_h = [torch.from_numpy(h[0]).pin_memory() for h in host]
     aor_h = [torch.from_numpy(h[1]).pin_memory() for h in host]
     e_h = [x.pin_memory() for x in e_host]
-    ids_d = torch.empty(W.batch, dtype=torch.int64, device=dev)
-    aor_d = torch.empty(lab, dtype=torch.int32, device=dev)
-    e_d = torch.empty((W.batch, W.dim), dtype=torch.float32, device=dev)
-    rows = torch.empty(lab, dtype=torch.int32, device=dev)
-    hit = torch.empty(lab, dtype=torch.uint8, device=dev)
-    out = torch.empty((lab, W.dim + W.ao_dim), dtype=torch.float32, device=dev)
-    ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
-    st_d = torch.zeros(7, dtype=torch.int64, device=dev)
+    slots = []
+    for _ in range(2):
+        slots.append({
+            "ids": torch.empty(W.batch, dtype=torch.int64, device=dev),
+            "aor": torch.empty(lab, dtype=torch.int32, device=dev),
+            "e": torch.empty((W.batch, W.dim), dtype=torch.float32, device=dev),
+            "rows": torch.empty(lab, dtype=torch.int32, device=dev),
+            "hit": torch.empty(lab, dtype=torch.uint8, device=dev),
+            "out": torch.empty((lab, width), dtype=torch.float32, device=dev),
+            "st": torch.zeros(7, dtype=torch.int64, device=dev),
+            "in_ready": torch.cuda.Event(), "done": torch.cuda.Event(),
+            "down": torch.cuda.Event(),
+            "rows_h": torch.empty(lab, dtype=torch.int32).pin_memory(),
+            "hit_h": torch.empty(lab, dtype=torch.uint8).pin_memory(),
+            "out_h": torch.empty((lab, width), dtype=torch.float32).pin_memory(),
+        })
     st_h = torch.zeros((K, 7), dtype=torch.int64).pin_memory()
+    ao_d = torch.from_numpy(inputs.author_table(W)).to(dev)
+    main = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    t0 = time.perf_counter()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record()
+    ev0.record(main)
+    up.wait_stream(main)
+    down.wait_stream(main)
+
+    def upload(j):
+        b = slots[j % 2]
+        with torch.cuda.stream(up):
+            if j >= 2:  # the slot's previous outputs have been read back
+                up.wait_event(b["down"])
+            b["ids"].copy_(ids_h[j], non_blocking=True)
+            b["aor"].copy_(aor_h[j], non_blocking=True)
+            b["e"].copy_(e_h[(n0 + j) % E], non_blocking=True)
+            b["in_ready"].record(up)
+
+    upload(0)
     for j in range(K):
-        t = n0 + j
-        ids_d.copy_(ids_h[j], non_blocking=True)
-        aor_d.copy_(aor_h[j], non_blocking=True)
-        e_d.copy_(e_h[t % E], non_blocking=True)
-        ev_in = torch.cuda.Event()
-        ev_in.record()
-        binding.mpzch_train_step(tbl.h, ids_d, lab, e_d, t, rows, hit, out, ao_d, aor_d, st_d,
-                                 inputs_ready=ev_in)
-        st_h[j].copy_(st_d, non_blocking=True)
-    ev1.record()
+        b = slots[j % 2]
+        if j + 1 < K:
+            upload(j + 1)
+        binding.mpzch_train_step(tbl.h, b["ids"], lab, b["e"], n0 + j, b["rows"], b["hit"],
+                                 b["out"], ao_d, b["aor"], b["st"], inputs_ready=b["in_ready"])
+        b["done"].record(main)
+        with torch.cuda.stream(down):
+            down.wait_event(b["done"])
+            b["rows_h"].copy_(b["rows"], non_blocking=True)
+            b["hit_h"].copy_(b["hit"], non_blocking=True)
+            b["out_h"].copy_(b["out"], non_blocking=True)
+            st_h[j].copy_(b["st"], non_blocking=True)
+            b["down"].record(down)
+    main.wait_stream(down)
+    ev1.record(main)
     torch.cuda.synchronize()
     ms = ev0.elapsed_time(ev1)
     units, ms = reduce_over_ranks(float(st_h[:, 1].sum().item()), ms, dev)
     h2d = W.batch * 8 + lab * 4 + W.batch * W.dim * 4
+    d2h = lab * 4 + lab + lab * width * 4 + 7 * 8
     return {"value": units / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": 7 * 8, "ms_per_step": ms / K}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / K,
+            "copied_back": "labeled rows, hit mask, fused features, counters"}
 
 
 def run_sharded(args):
@@ -648,6 +807,7 @@ def run_sharded(args):
     stats = torch.zeros((total, 7), dtype=torch.int64, device=dev)
     shard = sharded.ShardedMpzch(W.capacity, W.dim, W.probes, sharded.DistExchange())
     binding.mpzch_reserve(shard.table.h, W.batch * world)
+    apply_row_options(binding, shard.table, args)
     sent = {"lookup": 0, "writeback": 0}
 
     def step(t):

@@ -30,12 +30,18 @@ MPZCH_STATUS_BADKEY = 1
 MPZCH_STATUS_BADROW = 2
 MPZCH_STATUS_BADAO = 4
 MPZCH_STATUS_INTERNAL = 8
+MPZCH_STATUS_TIMEOUT = 16
 MPZCH_NPHASES = 7
 MPZCH_OPT_WIDE_ROUNDS = 1
 MPZCH_VALUES_IN_HOST_MEMORY = 1
 MPZCH_OPT_SIDE_PRIORITY = 2
 MPZCH_OPT_ROW_GRID = 3
 MPZCH_OPT_CLUSTER_INSERT = 4
+MPZCH_OPT_ROW_KERNEL = 5
+MPZCH_OPT_BULK_WARPS = 6
+MPZCH_OPT_BULK_BLOCKS = 7
+MPZCH_OPT_L2_HINT_ROWS = 8
+MPZCH_OPT_WRITE_LIST = 9
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")
@@ -67,6 +73,7 @@ _SIGS = {
     "mpzch_trace_enable": [_p, _i32],
     "mpzch_trace_read": [_p, C.POINTER(C.c_double), C.POINTER(_i64), _i32],
     "mpzch_set_option": [_p, _i32, _i64],
+    "mpzch_get_option": [_p, _i32, C.POINTER(_i64)],
     "mpzch_debug_fail_allocs": [_i32],
     "mpzch_set_learning_rate": [_p, C.c_float],
     "mpzch_res_create": [_p, _i64, _i32, _i32, C.POINTER(_p)],
@@ -291,6 +298,12 @@ def mpzch_set_option(h, option: int, value: int) -> None:
     _check("mpzch_set_option", _lib.mpzch_set_option(h, option, value))
 
 
+def mpzch_get_option(h, option: int) -> int:
+    v = _i64(0)
+    _check("mpzch_get_option", _lib.mpzch_get_option(h, option, C.byref(v)))
+    return int(v.value)
+
+
 def mpzch_set_learning_rate(h, eta: float) -> None:
     _check("mpzch_set_learning_rate", _lib.mpzch_set_learning_rate(h, float(eta)))
 
@@ -485,12 +498,12 @@ class MpzchTable:
         mpzch_writeback(self.h, ids, e, step, stats, stream)
 
     def train_step(self, ids, n_labeled, e, step, ao_table=None, ao_rows=None, stats=None,
-                   inputs_ready=None, stream=None):
+                   inputs_ready=None, stream=None, rows=None, hit=None, out=None):
         dev = ids.device
         w = self.dim + (0 if ao_table is None else ao_table.shape[1])
-        rows = torch.empty(n_labeled, dtype=torch.int32, device=dev)
-        hit = torch.empty(n_labeled, dtype=torch.uint8, device=dev)
-        out = torch.empty((n_labeled, w), dtype=torch.float32, device=dev)
+        rows = torch.empty(n_labeled, dtype=torch.int32, device=dev) if rows is None else rows
+        hit = torch.empty(n_labeled, dtype=torch.uint8, device=dev) if hit is None else hit
+        out = torch.empty((n_labeled, w), dtype=torch.float32, device=dev) if out is None else out
         mpzch_train_step(self.h, ids, n_labeled, e, step, rows, hit, out, ao_table, ao_rows, stats,
                          inputs_ready, stream)
         return rows, hit, out

@@ -87,6 +87,32 @@ unsigned grid_for(int64_t work_threads, int block, int per_sm = 8) {
   return (unsigned)g;
 }
 
+// Blocks of `kern` (with `block` threads, `smem` dynamic bytes) resident on
+// one SM, looked up once per kernel and device; at least 1.
+int resident_blocks(const void* kern, int block, size_t smem) {
+  struct Entry {
+    const void* kern;
+    int device, block;
+    size_t smem;
+    int blocks;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : done)
+    if (e.kern == kern && e.device == dev && e.block == block && e.smem == smem) return e.blocks;
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, block, smem) != cudaSuccess) {
+    cudaGetLastError();
+    b = 1;
+  }
+  if (b < 1) b = 1;
+  done.push_back({kern, dev, block, smem, b});
+  return b;
+}
+
 int after_launch() {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return cudaGetLastError() == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
@@ -214,6 +240,8 @@ struct mpzch_table {
   // cluster placement path: tagged per-slot list heads (C slots) and the tag
   // of the last call (0 is never a call's tag; shead starts all zero)
   unsigned long long* shead = nullptr;
+  int32_t* wentry = nullptr;  // write-list entry of each row's owner in the current step
+  int emit_list = 1;          // cluster path: write list emitted at re-probe and placement
   uint32_t tag = 0;
   bool tag_wrapped = false;
   int cluster_insert = 1;
@@ -233,25 +261,36 @@ struct mpzch_table {
   // write lists (row, position of e), two buffers used by alternate Writebacks
   int32_t* wrow[2] = {nullptr, nullptr};
   int32_t* wpos[2] = {nullptr, nullptr};
-  int32_t* wcnt = nullptr;  // device int32[2]
+  int32_t* wcnt = nullptr;  // device int32[4]: list lengths [0..1], entries taken [2..3]
   int wset = 0;             // buffer of the next Writeback
   // small device words
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
   int32_t* status = nullptr;
-  int32_t* sel_bcount = nullptr;
+  // select: per-tile look-back words, the tile ticket counter, the call epoch
+  // and the ticket count issued so far
+  unsigned long long* sel_tstat = nullptr;
+  unsigned long long* sel_ticket = nullptr;
+  uint32_t sel_epoch = 0;
+  unsigned long long sel_tickets = 0;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
   int side_high_priority = 1;  // priority of the side stream (set before its first use)
   float eta = 1.0f;            // learning rate of the Writeback step
   int row_blocks_per_sm = 8;   // row kernels: 0 = one row per warp, else grid-stride cap
+  int row_kernel = 0;          // 0 = register-staged row kernels, 1 = bulk-copy (shared memory)
+  int bulk_warps = 8;          // bulk row kernels: warps per block
+  int bulk_blocks = 1;         // bulk row kernels: blocks per SM (persistent grid)
+  int l2_hint_rows = 0;        // bulk row kernels: L2 policy of table-row accesses (L2Hint)
   // mpzch_train_step: the row map runs on a second (high-priority) stream
   cudaStream_t side = nullptr;
   cudaStream_t look = nullptr;  // the train step's lookup: highest stream priority
   cudaEvent_t ev_fork = nullptr, ev_lookup = nullptr, ev_map = nullptr;
   cudaEvent_t ev_update[2] = {nullptr, nullptr};  // row update that read write list b
-  cudaEvent_t ev_user = nullptr;    // end of the last other call on a caller stream
+  cudaEvent_t ev_user = nullptr;    // end of every other call so far (created with the table)
+  cudaStream_t user_stream = nullptr;  // stream ev_user was last recorded on
+  bool user_marked = false;
   cudaEvent_t ev_gather = nullptr;  // end of the last train step's gather
   // tracing
   bool trace = false;
@@ -299,11 +338,13 @@ void free_all(mpzch_table* t) {
     dev_free(t->M);
   for (auto& c : t->claims) dev_free(c), c = nullptr;
   dev_free(t->shead);
+  dev_free(t->wentry);
   dev_free(t->ctr);
   dev_free(t->wcnt);
   dev_free(t->stats);
   dev_free(t->status);
-  dev_free(t->sel_bcount);
+  dev_free(t->sel_tstat);
+  dev_free(t->sel_ticket);
   if (t->h_status) cudaFreeHost(t->h_status);
   for (auto& r : t->pending) {
     cudaEventDestroy(r.a);
@@ -333,7 +374,6 @@ int ensure_side_stream(mpzch_table* t) {
       cudaEventCreateWithFlags(&t->ev_map, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_update[0], cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_update[1], cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&t->ev_user, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_gather, cudaEventDisableTiming) != cudaSuccess) {
     cudaGetLastError();
     return MPZCH_ECUDA;
@@ -370,9 +410,14 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
     free_batch_scratch(t);
     return rc;
   }
-  // Scratch hash: empty key (-1) and empty position (all ones).
+  // Scratch hash: empty key (-1) and empty position (all ones).  The fill is
+  // waited for here: the helper streams of mpzch_train_step are not ordered
+  // after `st` when the caller passes an inputs-ready event, so they must not
+  // find the fill still queued (growth is rare and already synchronises).
   if (cudaMemsetAsync(t->hkey, 0xFF, H * sizeof(unsigned long long), st) != cudaSuccess ||
-      cudaMemsetAsync(t->hpos, 0xFF, H * sizeof(uint32_t), st) != cudaSuccess) {
+      cudaMemsetAsync(t->hpos, 0xFF, H * sizeof(uint32_t), st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
     free_batch_scratch(t);
     return MPZCH_ECUDA;
   }
@@ -427,7 +472,7 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
-                                           stats, t->status, nullptr);
+                                           stats, t->status, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -439,6 +484,23 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
 }  // namespace
 
 namespace {
+
+// The single-pass select: one block per tile, tickets continuing from the
+// previous call, a fresh epoch (never 0, the value of the cleared words).
+int launch_select(mpzch_table* t, int64_t since, int32_t* rows_out, int64_t* dev_count,
+                  cudaStream_t st) {
+  const unsigned long long tiles = (unsigned long long)((t->C + kScanTile - 1) / kScanTile);
+  uint32_t epoch = (t->sel_epoch + 1) & ((1u << 30) - 1);
+  if (epoch == 0) epoch = 1;
+  const int rc = launch(k_select_scan, (unsigned)tiles, kScanThreads, st, false,
+                        (const long long*)t->keys, (const long long*)t->last, t->C,
+                        (long long)since, t->sel_tstat, t->sel_ticket, t->sel_tickets, epoch,
+                        rows_out, reinterpret_cast<long long*>(dev_count), t->status);
+  if (rc) return rc;
+  t->sel_epoch = epoch;
+  t->sel_tickets += tiles;
+  return MPZCH_OK;
+}
 
 int enqueue_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit,
                    cudaStream_t st, bool pdl) {
@@ -465,11 +527,42 @@ int check_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_
   return MPZCH_OK;
 }
 
+// Launch shape of a bulk row kernel with `stage_bytes` per stage: warps per
+// block (halved until the block's shared memory fits kBulkSmemMax) and its
+// shared memory; false when even one warp does not fit (the register kernel
+// runs instead), or when the values live in host memory.
+constexpr size_t kBulkSmemMax = 112 * 1024;
+
+bool bulk_shape(const mpzch_table* t, size_t stage_bytes, int* warps, size_t* smem) {
+  if (t->row_kernel != 1 || t->values_on_host) return false;
+  for (int w = t->bulk_warps; w >= 1; w >>= 1) {
+    const size_t b = bulk_smem_bytes(w, stage_bytes);
+    if (b <= kBulkSmemMax) {
+      *warps = w;
+      *smem = b;
+      return true;
+    }
+  }
+  return false;
+}
+
 int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int64_t n,
                    const float* ao_table, int64_t ao_nrows, int32_t ao_dim,
                    const int32_t* ao_rows, float* out, cudaStream_t st, bool pdl) {
   PhaseScope ps(t, PH_GATHER, st);
   const bool has_ao = ao_table != nullptr;
+  int warps = 0;
+  size_t smem = 0;
+  if (bulk_shape(t, (size_t)(t->D + (has_ao ? ao_dim : 0)) * 4, &warps, &smem)) {
+    int64_t g = (int64_t)sm_count() * t->bulk_blocks;
+    const int64_t need = (n + warps - 1) / warps;
+    if (g > need) g = need;
+    return launch_smem(k_gather_bulk, (unsigned)g, (unsigned)(warps * 32), smem, st, pdl, rows,
+                       hit, n, reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
+                       reinterpret_cast<const float4*>(ao_table), ao_nrows,
+                       has_ao ? ao_dim / 4 : 0, ao_rows, reinterpret_cast<float4*>(out),
+                       t->l2_hint_rows, t->status);
+  }
   return launch(k_gather_fused, row_grid(n, t->row_blocks_per_sm), kBlock, st, pdl, rows, hit, n,
                 reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
                 reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
@@ -524,6 +617,9 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.wrow = t->wrow[t->wset];
   p.wpos = t->wpos[t->wset];
   p.wcount = t->wcnt + t->wset;
+  p.wtake = t->wcnt + 2 + t->wset;
+  p.emit = (t->cluster_insert && t->emit_list) ? 1 : 0;
+  p.wentry = t->wentry;
   return p;
 }
 
@@ -543,7 +639,7 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     PhaseScope ps(t, PH_DEDUP, st);
     rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false,
                 p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status,
-                p.wcount);
+                p.wcount, p.wtake);
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
   }
@@ -553,9 +649,12 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     // windows may cover the whole ring
     PhaseScope ps(t, PH_INSERT, st);
     rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !keys_free, p);
-    if (!rc) rc = launch(k_place_multi, grid_for(n * 32, kBlock, 4), kBlock, st, true, p);
+    // one warp per multi-key cluster, as many resident warps as the SMs hold
+    const int multi_per_sm = resident_blocks(reinterpret_cast<const void*>(k_place_multi), kBlock, 0);
+    if (!rc)
+      rc = launch(k_place_multi, grid_for(n * 32, kBlock, multi_per_sm), kBlock, st, true, p);
     if (!rc) rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, 0);
-    if (!rc) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
+    if (!rc && !p.emit) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
     return rc;
   }
   {
@@ -573,9 +672,21 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
 int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool pdl) {
   {
     PhaseScope ps(t, PH_WRITEBACK, st);
-    const int rc = launch(k_writeback, row_grid(p.n, t->row_blocks_per_sm), kBlock, st, pdl,
-                          (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount,
-                          p.M, p.e, p.D4, t->eta);
+    int warps = 0;
+    size_t smem = 0;
+    int rc;
+    if (bulk_shape(t, (size_t)t->D * 8, &warps, &smem)) {
+      int64_t g = (int64_t)sm_count() * t->bulk_blocks;
+      const int64_t need = (p.n + 32 * warps - 1) / (32 * warps);
+      if (g > need) g = need;
+      rc = launch_smem(k_writeback_bulk, (unsigned)g, (unsigned)(warps * 32), smem, st, pdl,
+                       (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount,
+                       p.wtake, p.M, p.e, p.D4, t->eta, t->l2_hint_rows, t->status);
+    } else {
+      rc = launch(k_writeback, row_grid(p.n, t->row_blocks_per_sm), kBlock, st, pdl,
+                  (const int32_t*)p.wrow, (const int32_t*)p.wpos, (const int32_t*)p.wcount, p.M,
+                  p.e, p.D4, t->eta);
+    }
     if (rc) return rc;
   }
   if (t->side && cudaEventRecord(t->ev_update[t->wset], st) != cudaSuccess) return MPZCH_ECUDA;
@@ -584,16 +695,25 @@ int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool 
 }
 
 // Calls other than mpzch_train_step run on the caller's stream: they first
-// wait for the side stream's work, and the next train step's side-stream work
-// waits for them (ev_user).
+// wait for the side stream's work, and the next train step's helper streams
+// wait for them (ev_user).
 int join_side(mpzch_table* t, cudaStream_t st) {
   if (!t->side) return MPZCH_OK;
   return cudaStreamWaitEvent(st, t->ev_map, 0) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
 }
 
+// ev_user marks the end of every call made so far outside mpzch_train_step.
+// A call on a stream other than the previous one first makes that stream wait
+// for the old mark, so the new mark also covers the calls on the old stream.
 int mark_user(mpzch_table* t, cudaStream_t st, int rc) {
-  if (rc || !t->side) return rc;
-  return cudaEventRecord(t->ev_user, st) == cudaSuccess ? MPZCH_OK : MPZCH_ECUDA;
+  if (rc) return rc;
+  if (t->user_marked && st != t->user_stream &&
+      cudaStreamWaitEvent(st, t->ev_user, 0) != cudaSuccess)
+    return MPZCH_ECUDA;
+  if (cudaEventRecord(t->ev_user, st) != cudaSuccess) return MPZCH_ECUDA;
+  t->user_marked = true;
+  t->user_stream = st;
+  return MPZCH_OK;
 }
 
 }  // namespace
@@ -678,7 +798,7 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
-                                           dev_status, nullptr);
+                                           dev_status, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -720,17 +840,21 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   for (int i = 0; i < 3 && !rc; ++i)
     rc = dev_alloc((void**)&t->claims[i], capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->shead, capacity * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->wentry, capacity * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
-  if (!rc) rc = dev_alloc((void**)&t->wcnt, 2 * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->wcnt, 4 * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
   if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
-  if (!rc)
-    rc = dev_alloc((void**)&t->sel_bcount, ((capacity + kSelTile - 1) / kSelTile) * sizeof(int32_t));
+  const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
+  if (!rc) rc = dev_alloc((void**)&t->sel_tstat, sel_tiles * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->sel_ticket, sizeof(unsigned long long));
   if (!rc && cudaHostAlloc((void**)&t->h_status, sizeof(int32_t), cudaHostAllocDefault) != cudaSuccess) {
     t->h_status = nullptr;
     rc = MPZCH_ENOMEM;
   }
   if (!rc && cudaGetDevice(&t->device) != cudaSuccess) rc = MPZCH_ECUDA;
+  if (!rc && cudaEventCreateWithFlags(&t->ev_user, cudaEventDisableTiming) != cudaSuccess)
+    rc = MPZCH_ECUDA;
   if (!rc) {
     bool ok = cudaMemsetAsync(t->keys, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
               cudaMemsetAsync(t->last, 0xFF, capacity * sizeof(long long), st) == cudaSuccess &&
@@ -738,13 +862,21 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
                cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) ==
                    cudaSuccess) &&
               cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
+              cudaMemsetAsync(t->wcnt, 0, 4 * sizeof(int32_t), st) == cudaSuccess &&
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
-              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
+              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->sel_tstat, 0, sel_tiles * sizeof(unsigned long long), st) ==
+                  cudaSuccess &&
+              cudaMemsetAsync(t->sel_ticket, 0, sizeof(unsigned long long), st) == cudaSuccess;
     for (int i = 0; i < 3 && ok; ++i)
       ok = cudaMemsetAsync(t->claims[i], 0xFF, capacity * sizeof(unsigned long long), st) ==
            cudaSuccess;
+    // the table is complete when the call returns: later calls on other
+    // streams (the helper streams of a pipelined train step) need no order
+    // after `stream`
+    if (ok) ok = cudaStreamSynchronize(st) == cudaSuccess;
     if (!ok) rc = MPZCH_ECUDA;
   }
   if (rc) {
@@ -801,8 +933,9 @@ int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t* uniq, in
   if (!on_device(t)) return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
   if (n == 0)
-    return cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess ? MPZCH_OK
-                                                                              : MPZCH_ECUDA;
+    return mark_user(t, st, cudaMemsetAsync(dev_count, 0, sizeof(int64_t), st) == cudaSuccess
+                                ? MPZCH_OK
+                                : MPZCH_ECUDA);
   int rc = join_side(t, st);
   if (!rc) rc = ensure_batch(t, n, st);
   if (rc) return rc;
@@ -886,7 +1019,9 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
       return MPZCH_ECUDA;
   } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
              cudaStreamWaitEvent(t->look, t->ev_fork, 0) != cudaSuccess ||
-             cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess) {
+             cudaStreamWaitEvent(t->look, t->ev_user, 0) != cudaSuccess ||
+             cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess ||
+             cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess) {
     return MPZCH_ECUDA;
   }
   if (n_labeled > 0) {
@@ -922,16 +1057,7 @@ int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows
   if (rc) return rc;
   {
     PhaseScope ps(t, PH_SELECT, st);
-    const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
-    k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
-                                             t->sel_bcount);
-    rc = after_launch();
-    if (!rc) {
-      k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since_step,
-                                                 t->sel_bcount, rows_out,
-                                                 reinterpret_cast<long long*>(dev_count));
-      rc = after_launch();
-    }
+    rc = launch_select(t, since_step, rows_out, dev_count, st);
   }
   return mark_user(t, st, rc);
 }
@@ -945,17 +1071,22 @@ int launch_export(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t*
   const float4* M = reinterpret_cast<const float4*>(t->M);
   long long* ko = reinterpret_cast<long long*>(keys_out);
   long long* lo = reinterpret_cast<long long*>(last_out);
-  const bool q16 = (reinterpret_cast<uintptr_t>(q) & 15) == 0;
-  uint4* q4 = reinterpret_cast<uint4*>(q);
-  const unsigned grid = grid_for(n * 32, kBlock, 4);
-  if (q16 && t->D == 512)
-    return launch_smem(k_export_int8_staged<1>, grid, kBlock, export_stage_smem(1), st, false,
-                       rows, n, dn, M, t->keys, t->C, q4, scale, ko, t->status,
-                       static_cast<const long long*>(t->last), lo);
-  if (q16 && t->D == 1024)
-    return launch_smem(k_export_int8_staged<2>, grid, kBlock, export_stage_smem(2), st, false,
-                       rows, n, dn, M, t->keys, t->C, q4, scale, ko, t->status,
-                       static_cast<const long long*>(t->last), lo);
+  uint32_t* qw = reinterpret_cast<uint32_t*>(q);  // 4-byte aligned (checked by the callers)
+  const long long* lst = static_cast<const long long*>(t->last);
+  const long long* kk = static_cast<const long long*>(t->keys);
+  // one resident wave of the register-heavy row exporter, grid-stride over rows
+  auto go = [&](auto kern) {
+    const int per_sm = resident_blocks(reinterpret_cast<const void*>(kern), kBlock, 0);
+    return launch(kern, grid_for(n * 32, kBlock, per_sm), kBlock, st, false, rows, n, dn, M, kk,
+                  t->C, qw, scale, ko, t->status, lst, lo);
+  };
+  switch (t->D) {
+    case 128: return go(k_export_rows<1>);
+    case 256: return go(k_export_rows<2>);
+    case 512: return go(k_export_rows<4>);
+    case 1024: return go(k_export_rows<8>);
+    default: break;
+  }
   k_export_int8<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
       rows, n, dn, M, t->keys, t->C, t->D / 4, reinterpret_cast<char4*>(q), scale, ko, t->status,
       t->last, lo);
@@ -1143,7 +1274,49 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     t->cluster_insert = (int)value;
     return MPZCH_OK;
   }
+  if (option == MPZCH_OPT_ROW_KERNEL) {
+    if (value != 0 && value != 1) return MPZCH_EINVAL;
+    t->row_kernel = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_BULK_WARPS) {
+    if (value != 1 && value != 2 && value != 4 && value != 8 && value != 16) return MPZCH_EINVAL;
+    t->bulk_warps = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_BULK_BLOCKS) {
+    if (value < 1 || value > 8) return MPZCH_EINVAL;
+    t->bulk_blocks = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_WRITE_LIST) {
+    if (value != 0 && value != 1) return MPZCH_EINVAL;
+    t->emit_list = (int)value;
+    return MPZCH_OK;
+  }
+  if (option == MPZCH_OPT_L2_HINT_ROWS) {
+    if (value < 0 || value > 2) return MPZCH_EINVAL;
+    t->l2_hint_rows = (int)value;
+    return MPZCH_OK;
+  }
   return MPZCH_EINVAL;
+}
+
+int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
+  if (!t || !value) return MPZCH_EINVAL;
+  switch (option) {
+    case MPZCH_OPT_WIDE_ROUNDS: *value = t->wide_rounds; break;
+    case MPZCH_OPT_SIDE_PRIORITY: *value = t->side_high_priority; break;
+    case MPZCH_OPT_ROW_GRID: *value = t->row_blocks_per_sm; break;
+    case MPZCH_OPT_CLUSTER_INSERT: *value = t->cluster_insert; break;
+    case MPZCH_OPT_ROW_KERNEL: *value = t->row_kernel; break;
+    case MPZCH_OPT_BULK_WARPS: *value = t->bulk_warps; break;
+    case MPZCH_OPT_BULK_BLOCKS: *value = t->bulk_blocks; break;
+    case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
+    case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
+    default: return MPZCH_EINVAL;
+  }
+  return MPZCH_OK;
 }
 
 int mpzch_set_learning_rate(mpzch_table* t, float eta) {
@@ -1179,16 +1352,7 @@ int export_since(mpzch_table* t, int64_t since, int32_t* rows, int64_t* dev_coun
   if (rc) return rc;
   {
     PhaseScope ps(t, PH_SELECT, st);
-    const unsigned tiles = (unsigned)((t->C + kSelTile - 1) / kSelTile);
-    k_select_count<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since,
-                                             t->sel_bcount);
-    rc = after_launch();
-    if (!rc) {
-      k_select_scatter<<<tiles, kBlock, 0, st>>>(t->keys, t->last, t->C, (long long)since,
-                                                 t->sel_bcount, rows,
-                                                 reinterpret_cast<long long*>(dev_count));
-      rc = after_launch();
-    }
+    rc = launch_select(t, since, rows, dev_count, st);
   }
   if (!rc) {
     PhaseScope ps(t, PH_EXPORT, st);

@@ -19,7 +19,6 @@ constexpr unsigned long long kNoClaim = 0xFFFFFFFFFFFFFFFFull;   // larger than 
 constexpr uint32_t kNoPos = 0xFFFFFFFFu;
 constexpr int kBlock = 256;
 constexpr int kTile = 1024;  // ids per block in the ordered compactions (4 per thread)
-constexpr int kSelTile = 4096;  // rows per block in select (16 per thread)
 
 // Status bits (mirror of the MPZCH_STATUS_* values of the public header).
 constexpr int kStBadKey = 1, kStBadRow = 2, kStBadAo = 4, kStInternal = 8;
@@ -79,13 +78,24 @@ __device__ __forceinline__ void set_status(int32_t* st, int bits) {
   if (st) atomicOr(st, bits);
 }
 
-// Programmatic dependent launch: let the next kernel of the stream start its
-// launch now, then wait until every earlier grid of the stream has completed
-// and its memory is visible.  Both are no-ops for a kernel launched without
-// the programmatic-serialisation attribute.  Every kernel calls this first,
-// so nothing is read before the producer has finished.
-__device__ __forceinline__ void pdl_enter() {
+// Programmatic dependent launch.  pdl_enter waits until every earlier grid of
+// the stream has completed and its memory is visible; every kernel calls it
+// first, so nothing is read before the producer has finished.  pdl_trigger
+// lets the next kernel of the stream launch; kernels of the row-map chain call
+// it once their main work is done, so the next kernel's blocks are scheduled
+// during this kernel's tail rather than parked on the SMs (holding warps and
+// shared memory that the concurrently running row kernels need) for its whole
+// run.  A kernel that never calls it triggers when its blocks exit.  Both are
+// no-ops for a kernel launched without the programmatic-serialisation
+// attribute.
+__device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_enter() {
+#if defined(MPZCH_PDL_EARLY_TRIGGER) && MPZCH_PDL_EARLY_TRIGGER
+  pdl_trigger();
+#endif
   asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
@@ -255,7 +265,7 @@ constexpr int kDedupThreads = kTile;  // one tile position per thread
 __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status, int32_t* wcount) {
+    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake) {
   pdl_enter();
   __shared__ unsigned long long s_key[kTileHash];
   __shared__ uint32_t s_pos[kTileHash];
@@ -267,6 +277,7 @@ __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
   if (stats && blockIdx.x == 0 && threadIdx.x < 7)
     reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
   if (wcount && blockIdx.x == 0 && threadIdx.x == 0) *wcount = 0;
+  if (wtake && blockIdx.x == 0 && threadIdx.x == 0) *wtake = 0;
   for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
     s_key[j] = kEmptyKey;
     s_pos[j] = kNoPos;
@@ -321,6 +332,7 @@ __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
       s_gslot[jj] = (int32_t)sl;
     }
   }
+  pdl_trigger();
   __syncthreads();
   // 3. every position learns the global slot of its id
   if (i < n && lslot >= 0) slot_of[i] = s_gslot[lslot];
@@ -443,7 +455,11 @@ __device__ __forceinline__ void clear_window(unsigned long long* claims, long lo
 // an array for two purposes.  The (key, distinct-id index) lists rotate the
 // same way.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ bool try_commit(long long k, int32_t uidx,
+struct WbParams;
+__device__ __forceinline__ void emit_placement(const WbParams& p, int64_t row,
+                                               long long victim_last, int32_t uidx);
+
+__device__ __forceinline__ bool try_commit(const WbParams& p, long long k, int32_t uidx,
                                            const unsigned long long* claims,
                                            long long* __restrict__ keys,
                                            long long* __restrict__ last, const Geo& g,
@@ -480,6 +496,7 @@ __device__ __forceinline__ bool try_commit(long long k, int32_t uidx,
   // A row is empty exactly when its last-write step is -1 (key and step are
   // always set together), so a victim with a step is a live key.
   if (best_last != -1) ++evicted;
+  emit_placement(p, best, best_last, uidx);
   keys[best] = k;
   last[best] = step;
   urow[uidx] = (int32_t)best;
@@ -525,10 +542,65 @@ struct WbParams {
   int32_t* wrow;
   int32_t* wpos;
   int32_t* wcount;
+  int32_t* wtake;  // entries of the list already taken by the bulk row update
+  // emit = 1 (cluster path): the re-probe appends the write-list entry of every
+  // resident id and each placement the entry of the id it places, and
+  // wentry[row] holds the entry of the row's current owner in this step; a
+  // placement that evicts an id written earlier in this step turns that id's
+  // entry into a tombstone (row -1), which the row update skips.  emit = 0:
+  // k_write_list builds the list after all placements.
+  int emit;
+  int32_t* wentry;
 };
+
+// Write-list entry m: `row` now belongs to distinct id uidx, whose e row is
+// the one at its first batch position.
+__device__ __forceinline__ void emit_entry(const WbParams& p, int m, int64_t row, int32_t uidx) {
+  p.wrow[m] = (int32_t)row;
+  p.wpos[m] = p.upos[uidx];
+  p.wentry[row] = m;
+}
+
+// A placement into `row` whose previous owner was written in this step (its
+// last-write step is this step: a resident id refreshed by the re-probe, or an
+// id placed earlier in the step): that owner gets no write (n_dropped).
+__device__ __forceinline__ void drop_victim(const WbParams& p, int64_t row, long long victim_last) {
+  if (victim_last == p.step) {
+    p.wrow[p.wentry[row]] = -1;
+    atomic_add_ll(&p.stats->n_dropped, 1LL);
+  }
+}
+
+// Both, for a placement made by one thread.
+__device__ __forceinline__ void emit_placement(const WbParams& p, int64_t row,
+                                               long long victim_last, int32_t uidx) {
+  if (!p.emit) return;
+  drop_victim(p, row, victim_last);
+  emit_entry(p, atomicAdd(p.wcount, 1), row, uidx);
+}
 
 // Two per-thread counts packed as 16-bit halves (each <= the block size).
 __device__ __forceinline__ int pack2(int a, int b) { return a | (b << 16); }
+
+// Block-aggregated append to three lists (counts packed in 10-bit fields, so
+// blocks of at most 1023 threads).  All threads of the block must call it.
+__device__ __forceinline__ void block_append3(int wa, int wb, int wc, int32_t* ca, int32_t* cb,
+                                              int32_t* cc, int& ia, int& ib, int& ic, int* smi) {
+  int total = 0;
+  const int before = block_excl_scan(wa | (wb << 10) | (wc << 20), smi, total);
+  __shared__ int s_base3[3];
+  if (threadIdx.x == 0) {
+    const int ta = total & 1023, tb = (total >> 10) & 1023, tc = total >> 20;
+    s_base3[0] = ta ? atomicAdd(ca, ta) : 0;
+    s_base3[1] = tb ? atomicAdd(cb, tb) : 0;
+    s_base3[2] = tc ? atomicAdd(cc, tc) : 0;
+  }
+  __syncthreads();
+  ia = s_base3[0] + (before & 1023);
+  ib = s_base3[1] + ((before >> 10) & 1023);
+  ic = s_base3[2] + (before >> 20);
+  __syncthreads();
+}
 
 // Block-aggregated append: every thread with want != 0 gets a distinct slot of
 // the list whose length counter is `counter`; one global atomic per block.
@@ -582,8 +654,12 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
         }
       }
     }
-    int u = 0, m = 0;
-    block_append2(first, first && r < 0, &p.ctr->n_unique, &p.ctr->cnt[0], u, m, smi);
+    int u = 0, m = 0, wi = 0;
+    if (p.emit)
+      block_append3(first, first && r < 0, first && r >= 0, &p.ctr->n_unique, &p.ctr->cnt[0],
+                    p.wcount, u, m, wi, smi);
+    else
+      block_append2(first, first && r < 0, &p.ctr->n_unique, &p.ctr->cnt[0], u, m, smi);
     if (first) {
       p.ukey[u] = k;
       p.upos[u] = (int32_t)i;
@@ -591,6 +667,11 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
       if (r >= 0) {
         p.last[r] = p.step;
         ++hits;
+        if (p.emit) {
+          p.wrow[wi] = (int32_t)r;
+          p.wpos[wi] = (int32_t)i;
+          p.wentry[r] = wi;
+        }
       } else {
         p.lkey[0][m] = k;
         p.lidx[0][m] = u;
@@ -604,6 +685,7 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
       }
     }
   }
+  pdl_trigger();
   const long long bh = block_sum_ll(hits, sm);
   const long long bv = block_sum_ll(nvalid, sm);
   if (threadIdx.x == 0) {
@@ -642,7 +724,7 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
     if (i < ncur) {
       k = p.lkey[rc][i];
       u = p.lidx[rc][i];
-      defer = !try_commit(k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted);
+      defer = !try_commit(p, k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted);
     }
     int m = 0, unused = 0;
     block_append2(defer, 0, &p.ctr->cnt[(r + 1) & 3], &p.ctr->cnt[(r + 1) & 3], m, unused, smi);
@@ -653,6 +735,7 @@ __global__ void __launch_bounds__(kBlock) k_insert_round(WbParams p, int r) {
       if (r + 1 < p.wide_rounds) claim_window(p.claims[rn], k, g);
     }
   }
+  pdl_trigger();
   const long long ev = block_sum_ll(evicted, sm);
   if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
   if (blockIdx.x == 0 && threadIdx.x == 0 && ncur > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
@@ -680,7 +763,7 @@ __device__ void finish_by_rounds(const WbParams& p, int r0, int32_t nprev, int32
       if (i < ncur) {
         const long long k = __ldcg(p.lkey[rc] + i);
         const int32_t u = __ldcg(p.lidx[rc] + i);
-        if (!try_commit(k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted)) {
+        if (!try_commit(p, k, u, p.claims[rc], p.keys, p.last, g, p.step, p.urow, evicted)) {
           const int m = atomicAdd(s_next, 1);
           p.lkey[rn][m] = k;
           p.lidx[rn][m] = u;
@@ -724,6 +807,7 @@ __device__ __forceinline__ void place_key(const WbParams& p, long long k, int32_
     }
   }
   if (best_last != -1) ++evicted;
+  emit_placement(p, best, best_last, u);
   p.keys[best] = k;
   p.last[best] = p.step;
   p.urow[u] = (int32_t)best;
@@ -1061,6 +1145,7 @@ __device__ void place_cluster_serial(const WbParams& p, int64_t h, int32_t N, Se
         }
       }
       if (best_last != -1) ++evicted;
+      emit_placement(p, best, best_last, cu[j]);
       sl[best_o] = p.step;
       p.keys[best] = kk;
       p.last[best] = p.step;
@@ -1189,6 +1274,7 @@ __device__ bool place_cluster_warp(const WbParams& p, int64_t h, int32_t N, Warp
     }
     if (lane == 0) {
       if (cl != -1) ++evicted;
+      emit_placement(p, cs, cl, sw.us[j]);
       p.keys[cs] = k;
       p.last[cs] = p.step;
       p.urow[sw.us[j]] = (int32_t)cs;
@@ -1251,9 +1337,14 @@ __device__ int place_lone(const WbParams& p, int32_t m, long long& evicted, int6
     }
   }
   if (best_last != -1) ++evicted;
+  const int32_t u = __ldcg(p.lidx[0] + m);
+  if (p.emit) {
+    drop_victim(p, best, best_last);
+    emit_entry(p, warp_append(p.wcount), best, u);
+  }
   p.keys[best] = k;
   p.last[best] = p.step;
-  p.urow[__ldcg(p.lidx[0] + m)] = (int32_t)best;
+  p.urow[u] = (int32_t)best;
   return 0;
 }
 
@@ -1266,6 +1357,7 @@ __global__ void __launch_bounds__(kBlock) k_place_clusters(WbParams p) {
   const bool ring_may_be_covered = (int64_t)N * p.g.P >= p.g.C;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     p.stats->n_inserted = N;
+    if (p.emit) p.stats->n_unique = p.ctr->n_unique;  // no k_write_list on this path
     if (N > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
   }
   long long evicted = 0;
@@ -1276,6 +1368,7 @@ __global__ void __launch_bounds__(kBlock) k_place_clusters(WbParams p) {
       if (place_lone(p, (int32_t)m, evicted, h)) p.lidx[1][warp_append(&p.ctr->n_multi)] = (int32_t)h;
     }
   }
+  pdl_trigger();
   const long long ev = block_sum_ll(evicted, sm);
   if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
 }
@@ -1298,6 +1391,7 @@ __global__ void __launch_bounds__(kBlock) k_place_multi(WbParams p) {
       p.lidx[2][atomicAdd(&p.ctr->n_serial, 1)] = (int32_t)h;
     __syncwarp();
   }
+  pdl_trigger();
   const long long ev = block_sum_ll(evicted, sm);
   if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
 }
@@ -1340,6 +1434,7 @@ __global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
       p.wpos[m] = p.upos[u];
     }
   }
+  pdl_trigger();
   const long long d = block_sum_ll(dropped, sm);
   if (threadIdx.x == 0 && d) atomic_add_ll(&p.stats->n_dropped, d);
 }
@@ -1363,7 +1458,9 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
   const int32_t W = *wcount;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < W; w += warps) {
-    float4* m = M + (int64_t)wrow[w] * D4;
+    const int32_t r = wrow[w];
+    if (r < 0) continue;  // tombstone: the id lost its row later in the step
+    float4* m = M + (int64_t)r * D4;
     const float4* ev = e + (int64_t)wpos[w] * D4;
     for (int base = 0; base < D4; base += 4 * 32) {
       float4 a[4], b[4];
@@ -1395,45 +1492,453 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Select rows written at or after `since`, ascending (ordered compaction).
+// Bulk-copy row kernels.  A warp keeps kBulkStages rows in flight: one lane
+// issues 1-D bulk copies (cp.async.bulk, global -> shared, no multicast) of
+// each row into the warp's own shared-memory stage, completed on that stage's
+// mbarrier; the lanes read the stage as 16-byte vectors and store the result
+// with coalesced 512 B requests.  The rows in flight live in shared memory, not
+// in registers, so far fewer warps keep HBM busy than in the register path,
+// which leaves warp slots to the latency-bound row-map kernels running
+// alongside.  Every wait on an mbarrier has a time limit; past it the kernel
+// sets MPZCH_STATUS_TIMEOUT, waits (again with a limit) for its copies still
+// in flight and returns.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kBlock) k_select_count(const long long* __restrict__ keys,
-                                                         const long long* __restrict__ last,
-                                                         int64_t C, long long since,
-                                                         int32_t* __restrict__ bcount) {
-  pdl_enter();
-  __shared__ long long sm[33];
-  const int64_t base = (int64_t)blockIdx.x * kSelTile + threadIdx.x;
-  int c = 0;
-#pragma unroll 4
-  for (int u = 0; u < kSelTile / kBlock; ++u) {
-    const int64_t r = base + (int64_t)u * kBlock;
-    if (r < C) c += keys[r] != -1 && last[r] >= since;
-  }
-  const long long t = block_sum_ll(c, sm);
-  if (threadIdx.x == 0) bcount[blockIdx.x] = (int32_t)t;
+constexpr int kStTimeout = 16;
+constexpr int kBulkStages = 3;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any row copy
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
 }
 
-__global__ void __launch_bounds__(kBlock) k_select_scatter(const long long* __restrict__ keys,
-                                                           const long long* __restrict__ last,
-                                                           int64_t C, long long since,
-                                                           const int32_t* __restrict__ bcount,
-                                                           int32_t* __restrict__ rows_out,
-                                                           long long* dev_count) {
-  pdl_enter();
-  __shared__ long long sm[33];
-  __shared__ int smi[33];
-  long long offset = block_prefix_of_counts(bcount, blockIdx.x, sm);
-  // kSelTile rows in kSelTile/kBlock passes of kBlock consecutive rows (coalesced).
-  for (int u = 0; u < kSelTile / kBlock; ++u) {
-    const int64_t r = (int64_t)blockIdx.x * kSelTile + (int64_t)u * kBlock + threadIdx.x;
-    const int f = (r < C) && keys[r] != -1 && last[r] >= since;
-    int total = 0;
-    const int before = block_excl_scan(f, smi, total);
-    if (f) rows_out[offset + before] = (int32_t)r;
-    offset += total;
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// L2 eviction-priority policies for the cache-hinted accesses.
+enum L2Hint { kL2EvictFirst = 0, kL2Normal = 1, kL2EvictLast = 2 };
+
+__device__ __forceinline__ uint64_t l2_policy(int hint) {
+  uint64_t pol;
+  if (hint == kL2EvictFirst)
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  else if (hint == kL2EvictLast)
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// One arrival that also announces `bytes` of bulk-copy data for this phase.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for phase `parity` of the mbarrier to complete, for at most
+// kWaitLimitNs; false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
   }
-  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) *dev_count = offset;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing `bytes` of
+// transaction count on the mbarrier (16-byte aligned addresses, bytes % 16 == 0).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void stg4_hint(float4* p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
+}
+
+// Shared memory of a bulk row kernel: per warp kBulkStages stages of
+// `stage_bytes`, then one 8-byte mbarrier per (warp, stage).
+__host__ __device__ constexpr size_t bulk_smem_bytes(int warps, size_t stage_bytes) {
+  return (size_t)warps * kBulkStages * stage_bytes + (size_t)warps * kBulkStages * 8;
+}
+
+// Per-warp stream of work items taken in chunks of 32 from a shared counter
+// (dynamic, so a warp that starts late takes less); lane l caches item
+// base + l of the current chunk.  Warp-collective.
+struct ChunkCursor {
+  int32_t base, pos, end;
+  bool done;
+};
+
+// Row update through shared memory (same result as k_writeback): for every
+// write-list entry, M[r] <- fl(e_hat - fl(eta * fl(e_hat - e))).  Entries are
+// taken from *wtake in chunks of 32 per warp.
+__global__ void k_writeback_bulk(const int32_t* __restrict__ wrow, const int32_t* __restrict__ wpos,
+                                 const int32_t* wcount, int32_t* wtake, float4* __restrict__ M,
+                                 const float4* __restrict__ e, int D4, float eta, int hint_m,
+                                 int32_t* status) {
+  pdl_enter();
+  extern __shared__ __align__(128) unsigned char bsm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const uint32_t RB = (uint32_t)D4 * 16u;  // bytes of one row
+  const size_t stage_bytes = 2 * (size_t)RB;
+  const uint32_t stage0 = smem_addr(bsm + (size_t)warp * kBulkStages * stage_bytes);
+  const uint32_t bar0 =
+      smem_addr(bsm + (size_t)nwarps * kBulkStages * stage_bytes) + warp * kBulkStages * 8;
+  if (lane == 0)
+    for (int s = 0; s < kBulkStages; ++s) mbar_init(bar0 + 8 * s, 1);
+  mbar_init_fence();
+  __syncwarp();
+  const uint64_t pol_e = l2_policy(kL2EvictFirst);
+  const uint64_t pol_m = l2_policy(hint_m);
+  const int32_t W = *wcount;
+  ChunkCursor cur{0, 0, 0, false};
+  int32_t c_row = 0, c_pos = 0;
+  int32_t srow[kBulkStages];
+  // warp-collective: next entry into stage s (srow[s] = -1 when none is left);
+  // tombstones (row -1) are skipped, across chunk boundaries
+  auto issue = [&](int s) {
+    int32_t r = -1, q = 0;
+    while (r < 0 && !cur.done) {
+      if (cur.pos == cur.end) {
+        int32_t b = 0;
+        if (lane == 0) b = atomicAdd(wtake, 32);
+        b = __shfl_sync(0xFFFFFFFFu, b, 0);
+        if (b >= W) {
+          cur.done = true;
+        } else {
+          cur.base = cur.pos = b;
+          cur.end = b + 32 < W ? b + 32 : W;
+          if (lane < cur.end - b) {
+            c_row = wrow[b + lane];
+            c_pos = wpos[b + lane];
+          }
+        }
+        continue;
+      }
+      const int src = cur.pos - cur.base;
+      r = __shfl_sync(0xFFFFFFFFu, c_row, src);
+      q = __shfl_sync(0xFFFFFFFFu, c_pos, src);
+      ++cur.pos;
+    }
+    if (r >= 0 && lane == 0) {
+      const uint32_t st = stage0 + (uint32_t)(s * stage_bytes);
+      mbar_expect_tx(bar0 + 8 * s, 2 * RB);
+      bulk_load(st, M + (int64_t)r * D4, RB, bar0 + 8 * s, pol_m);
+      bulk_load(st + RB, e + (int64_t)q * D4, RB, bar0 + 8 * s, pol_e);
+    }
+    srow[s] = r;
+  };
+#pragma unroll
+  for (int s = 0; s < kBulkStages; ++s) issue(s);
+  uint32_t pbits = 0;  // bit s: parity of the phase stage s's copies complete
+  bool failed = false;
+  while (!failed) {
+    bool any = false;
+#pragma unroll
+    for (int s = 0; s < kBulkStages; ++s) {
+      if (srow[s] < 0 || failed) continue;
+      any = true;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, (pbits >> s) & 1u))) {
+        failed = true;
+        continue;
+      }
+      pbits ^= 1u << s;
+      const uint32_t st = stage0 + (uint32_t)(s * stage_bytes);
+      float4* m = M + (int64_t)srow[s] * D4;
+      for (int c = lane; c < D4; c += 32) {
+        const float4 a = lds4(st + 16u * c);
+        const float4 b = lds4(st + RB + 16u * c);
+        float4 o;
+        o.x = __fsub_rn(a.x, __fmul_rn(eta, __fsub_rn(a.x, b.x)));
+        o.y = __fsub_rn(a.y, __fmul_rn(eta, __fsub_rn(a.y, b.y)));
+        o.z = __fsub_rn(a.z, __fmul_rn(eta, __fsub_rn(a.z, b.z)));
+        o.w = __fsub_rn(a.w, __fmul_rn(eta, __fsub_rn(a.w, b.w)));
+        stg4_hint(m + c, o, pol_m);
+      }
+      __syncwarp();  // every lane has read the stage before it is refilled
+      issue(s);
+    }
+    if (!any) break;
+  }
+  if (failed) {
+    if (lane == 0) set_status(status, kStTimeout);
+    // copies still in flight must land before the block's shared memory goes
+    for (int s = 0; s < kBulkStages; ++s)
+      if (srow[s] >= 0) mbar_wait(bar0 + 8 * s, (pbits >> s) & 1u);
+  }
+}
+
+// Fused gather through shared memory (same result as k_gather_fused): per
+// output row one bulk copy of the cached row (hits) and one of the always-on
+// row, then the lanes write the row (zeros for a miss) with coalesced 16-byte
+// stores.  Items i = warp, warp + warps, ... in chunks of 32 per warp.
+__global__ void k_gather_bulk(const int32_t* __restrict__ rows, const uint8_t* __restrict__ hit,
+                              int64_t n, const float4* __restrict__ M, int64_t C, int D4,
+                              const float4* __restrict__ ao, int64_t ao_n, int A4,
+                              const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
+                              int hint_m, int32_t* status) {
+  pdl_enter();
+  extern __shared__ __align__(128) unsigned char bsm[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const uint32_t RB = (uint32_t)D4 * 16u, AB = (uint32_t)A4 * 16u;
+  const size_t stage_bytes = (size_t)RB + AB;
+  const uint32_t stage0 = smem_addr(bsm + (size_t)warp * kBulkStages * stage_bytes);
+  const uint32_t bar0 =
+      smem_addr(bsm + (size_t)nwarps * kBulkStages * stage_bytes) + warp * kBulkStages * 8;
+  if (lane == 0)
+    for (int s = 0; s < kBulkStages; ++s) mbar_init(bar0 + 8 * s, 1);
+  mbar_init_fence();
+  __syncwarp();
+  const uint64_t pol_m = l2_policy(hint_m);
+  const uint64_t pol_a = l2_policy(kL2EvictFirst);
+  const int64_t G = (int64_t)gridDim.x * nwarps;
+  const int64_t g = (int64_t)blockIdx.x * nwarps + warp;
+  const int W4 = D4 + A4;
+  // this warp's items: g + k * G for k = 0, 1, ...; lane l caches item k0 + l
+  int64_t k_next = 0;  // next item (as k) to issue
+  int64_t k_base = -32;
+  int32_t c_r = 0, c_a = 0;
+  int c_flags = 0;  // bit 0 hit (in range), bit 1 always-on row in range
+  int64_t sidx[kBulkStages];
+  int sflags[kBulkStages];
+  auto issue = [&](int s) {
+    const int64_t i = g + k_next * G;
+    if (i >= n) {
+      sidx[s] = -1;
+      return;
+    }
+    if (k_next >= k_base + 32) {
+      k_base = k_next;
+      const int64_t li = g + (k_base + lane) * G;
+      c_flags = 0;
+      if (li < n) {
+        const int32_t r = rows[li];
+        if (hit[li]) {
+          if (r >= 0 && (int64_t)r < C)
+            c_flags |= 1;
+          else
+            set_status(status, kStBadRow);
+        }
+        c_r = r;
+        if (A4 > 0) {
+          c_a = ao_rows[li];
+          if (c_a >= 0 && (int64_t)c_a < ao_n)
+            c_flags |= 2;
+          else
+            set_status(status, kStBadAo);
+        }
+      }
+    }
+    const int src = (int)(k_next - k_base);
+    const int32_t r = __shfl_sync(0xFFFFFFFFu, c_r, src);
+    const int32_t a = __shfl_sync(0xFFFFFFFFu, c_a, src);
+    const int f = __shfl_sync(0xFFFFFFFFu, c_flags, src);
+    ++k_next;
+    if (lane == 0) {
+      const uint32_t st = stage0 + (uint32_t)(s * stage_bytes);
+      const uint32_t bytes = ((f & 1) ? RB : 0u) + ((f & 2) ? AB : 0u);
+      mbar_expect_tx(bar0 + 8 * s, bytes);
+      if (f & 1) bulk_load(st, M + (int64_t)r * D4, RB, bar0 + 8 * s, pol_m);
+      if (f & 2) bulk_load(st + RB, ao + (int64_t)a * A4, AB, bar0 + 8 * s, pol_a);
+    }
+    sidx[s] = i;
+    sflags[s] = f;
+  };
+#pragma unroll
+  for (int s = 0; s < kBulkStages; ++s) issue(s);
+  uint32_t pbits = 0;  // bit s: parity of the phase stage s's copies complete
+  bool failed = false;
+  while (!failed) {
+    bool any = false;
+#pragma unroll
+    for (int s = 0; s < kBulkStages; ++s) {
+      if (sidx[s] < 0 || failed) continue;
+      any = true;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(bar0 + 8 * s, (pbits >> s) & 1u))) {
+        failed = true;
+        continue;
+      }
+      pbits ^= 1u << s;
+      const uint32_t st = stage0 + (uint32_t)(s * stage_bytes);
+      float4* dst = out + sidx[s] * (int64_t)W4;
+      const int f = sflags[s];
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = lane; c < W4; c += 32) {
+        float4 v = z;
+        if (c < D4) {
+          if (f & 1) v = lds4(st + 16u * c);
+        } else if (f & 2) {
+          v = lds4(st + 16u * c);
+        }
+        __stcs(dst + c, v);
+      }
+      __syncwarp();
+      issue(s);
+    }
+    if (!any) break;
+  }
+  if (failed) {
+    if (lane == 0) set_status(status, kStTimeout);
+    for (int s = 0; s < kBulkStages; ++s)
+      if (sidx[s] >= 0) mbar_wait(bar0 + 8 * s, (pbits >> s) & 1u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Select rows written at or after `since`, ascending: one pass, one launch.
+// Tiles of kScanTile rows; a block takes the next tile index from a ticket
+// counter (so every tile it waits for belongs to a block that is already
+// running), counts its selected rows and publishes that count; then one warp
+// sums the counts of all earlier tiles -- up to 256 words in flight at once,
+// none of them waiting on another tile's sum -- and the block scatters its
+// rows at that offset.
+//
+// Tile word (64 bits): epoch (bits 63..34, the call's number, so words of
+// earlier calls read as not yet published and nothing is cleared), flag
+// (bit 32), count (31..0).  Thread t of a block reads rows t + 256k (k < 8)
+// of its tile, so every load instruction covers 256 contiguous bytes; the
+// rows' order inside the tile comes from per-warp ballots and a 64-entry
+// scan.  A wait for an earlier tile's word has a time limit
+// (MPZCH_STATUS_TIMEOUT when it runs out).
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 256;
+constexpr int kScanPer = 8;
+constexpr int kScanTile = kScanThreads * kScanPer;
+constexpr unsigned long long kTileAgg = 1ull << 32;
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_select_scan(
+    const long long* __restrict__ keys, const long long* __restrict__ last, int64_t C,
+    long long since, unsigned long long* tstat, unsigned long long* ticket,
+    unsigned long long ticket_base, uint32_t epoch, int32_t* __restrict__ rows_out,
+    long long* dev_count, int32_t* status) {
+  pdl_enter();
+  __shared__ int s_tile;
+  __shared__ int s_off[kScanPer * (kScanThreads / 32) + 1];
+  __shared__ long long s_excl;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) s_tile = (int)(atomicAdd(ticket, 1ull) - ticket_base);
+  __syncthreads();
+  const int tile = s_tile;
+  const int64_t base = (int64_t)tile * kScanTile + threadIdx.x;
+  long long kv[kScanPer], lv[kScanPer];
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    const int64_t r = base + k * kScanThreads;
+    kv[k] = r < C ? __ldcs(keys + r) : -1;
+    lv[k] = r < C ? __ldcs(last + r) : -1;
+  }
+  unsigned ball[kScanPer];
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k) {
+    ball[k] = __ballot_sync(0xFFFFFFFFu, kv[k] != -1 && lv[k] >= since);
+    if (lane == 0) s_off[k * (kScanThreads / 32) + warp] = __popc(ball[k]);
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive scan of the 64 (sub-tile, warp) counts, in row order
+    constexpr int kN = kScanPer * (kScanThreads / 32);
+    const int a = s_off[2 * lane], b = s_off[2 * lane + 1];
+    int x = a + b;
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
+      if (lane >= off) x += y;
+    }
+    const int before = x - a - b;
+    s_off[2 * lane] = before;
+    s_off[2 * lane + 1] = before + a;
+    if (lane == 31) s_off[kN] = x;
+    static_assert(kN == 64, "one warp scans two counts per lane");
+  }
+  __syncthreads();
+  const int total = s_off[kScanPer * (kScanThreads / 32)];
+  if (warp == 0) {
+    const unsigned long long ep = (unsigned long long)epoch << 34;
+    if (lane == 0) st_relaxed_u64(tstat + tile, ep | kTileAgg | (uint32_t)total);
+    long long excl = 0;
+    bool timed_out = false;
+    const uint64_t t0 = global_ns();
+    constexpr int kBatch = 8;  // words per lane in flight
+    for (int q0 = 0; q0 < tile && !timed_out; q0 += 32 * kBatch) {
+      unsigned long long w[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + lane + 32 * u;
+        w[u] = q < tile ? ld_relaxed_u64(tstat + q) : (ep | kTileAgg);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int q = q0 + lane + 32 * u;
+        while ((w[u] >> 34) != epoch || !(w[u] & kTileAgg)) {  // not yet published
+          if (global_ns() - t0 > kWaitLimitNs) {
+            timed_out = true;
+            break;
+          }
+          w[u] = ld_relaxed_u64(tstat + q);
+        }
+        excl += (long long)(uint32_t)w[u];
+      }
+    }
+    for (int off = 16; off > 0; off >>= 1) excl += __shfl_xor_sync(0xFFFFFFFFu, excl, off);
+    if (__any_sync(0xFFFFFFFFu, timed_out) && lane == 0) set_status(status, kStTimeout);
+    if (lane == 0) s_excl = excl;
+  }
+  __syncthreads();
+  const long long excl = s_excl;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int k = 0; k < kScanPer; ++k)
+    if (ball[k] >> lane & 1u)
+      rows_out[excl + s_off[k * (kScanThreads / 32) + warp] + __popc(ball[k] & lt)] =
+          (int32_t)(base + k * kScanThreads);
+  if ((int64_t)(tile + 1) * kScanTile >= C && threadIdx.x == 0) *dev_count = excl + total;
 }
 
 // ---------------------------------------------------------------------------
@@ -1488,61 +1993,6 @@ __device__ __forceinline__ uint32_t pack4(int a, int b, int c, int d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-// Quantise and store one row held by a warp: lane l holds the 16-byte
-// vectors 4l..4l+3 of each 2 KiB chunk (64 contiguous input bytes) as v and
-// writes their 16 int8 values with one 16-byte store per chunk.
-template <int kChunks>
-__device__ __forceinline__ void export_values(const float (&v)[kChunks * 16], uint4* qo, float* sc,
-                                              long long* ko, long long* lo, long long key,
-                                              long long lastv, int lane) {
-  float a = 0.f;
-#pragma unroll
-  for (int e = 0; e < kChunks * 16; ++e) a = fmaxf(a, fabsf(v[e]));
-  for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
-  const float s = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
-  const float rcp = a == 0.f ? 0.f : __frcp_rn(s);
-  const bool fast = a != 0.f && isfinite(rcp);
-#pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch) {
-    float vc[16];
-    int c[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      vc[e] = v[ch * 16 + e];
-      c[e] = 0;
-    }
-    if (a != 0.f) quant_lane<16>(vc, s, rcp, fast, c);
-    __stcs(qo + ch * 32 + lane, make_uint4(pack4(c[0], c[1], c[2], c[3]), pack4(c[4], c[5], c[6], c[7]),
-                                           pack4(c[8], c[9], c[10], c[11]),
-                                           pack4(c[12], c[13], c[14], c[15])));
-  }
-  if (lane == 0) {
-    *sc = s;
-    *ko = key;
-    if (lo) *lo = lastv;
-  }
-}
-
-// Export of one row by one warp, the row loaded into registers.  kChunks
-// chunks of 128 vectors cover dim = 512 * kChunks.
-template <int kChunks>
-__device__ __forceinline__ void export_row_regs(const float4* __restrict__ x, uint4* qo, float* sc,
-                                                long long* ko, long long* lo, long long key,
-                                                long long lastv, int lane) {
-  float v[kChunks * 16];
-#pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 f = __ldcs(x + ch * 128 + 4 * lane + j);
-      v[ch * 16 + 4 * j] = f.x;
-      v[ch * 16 + 4 * j + 1] = f.y;
-      v[ch * 16 + 4 * j + 2] = f.z;
-      v[ch * 16 + 4 * j + 3] = f.w;
-    }
-  export_values<kChunks>(v, qo, sc, ko, lo, key, lastv, lane);
-}
-
 // Any dim (multiple of 4): two passes over the row (max, then quantise) with
 // 4-byte stores.
 __device__ __forceinline__ void export_row_generic(const float4* __restrict__ x, char4* qo, int D4,
@@ -1583,8 +2033,6 @@ __global__ void __launch_bounds__(kBlock, 4) k_export_int8(
     const long long d = *dev_n;
     nn = d < nn ? d : nn;
   }
-  // 16-byte output rows need dim % 16 == 0 and an aligned q
-  const bool vec16 = (D4 % 128 == 0) && ((reinterpret_cast<uintptr_t>(q) & 15) == 0);
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < nn; i += warps) {
     const int32_t r = rows[i];
@@ -1603,108 +2051,94 @@ __global__ void __launch_bounds__(kBlock, 4) k_export_int8(
     const float4* x = M + (int64_t)r * D4;
     const long long key = keys[r];
     const long long lastv = last_out ? last[r] : 0;
-    if (vec16 && D4 == 128)
-      export_row_regs<1>(x, reinterpret_cast<uint4*>(qo), scale + i, keys_out + i, lo, key, lastv,
-                         lane);
-    else if (vec16 && D4 == 256)
-      export_row_regs<2>(x, reinterpret_cast<uint4*>(qo), scale + i, keys_out + i, lo, key, lastv,
-                         lane);
-    else
-      export_row_generic(x, qo, D4, scale + i, keys_out + i, lo, key, lastv, lane);
+    export_row_generic(x, qo, D4, scale + i, keys_out + i, lo, key, lastv, lane);
   }
 }
 
-// Asynchronous 16-byte global -> shared copy (L2 only) and its groups.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
-// Export with the rows staged through shared memory (dim = 512 * kChunks,
-// 16-byte aligned q): each warp owns two row buffers and copies the next row
-// (cp.async) while it quantises the current one, so a row's load latency
-// overlaps the previous row's reduction, rounding and stores.  Lane l stages
-// exactly the vectors it later reads (4l..4l+3 of each chunk), so it waits only
-// for its own copies and no warp barrier is needed.  Same results as
-// k_export_int8.
-template <int kChunks>
-__global__ void __launch_bounds__(kBlock, 4) k_export_int8_staged(
+// Export of rows of D = 128 * kPer values, one warp per row, through
+// registers: lane l holds the 16-byte vectors l + 32 j (j < kPer) of the row,
+// so every load instruction of the warp reads 512 contiguous bytes, and writes
+// their codes as the 4-byte words l + 32 j of the int8 row, so every store
+// instruction writes 128 contiguous bytes.  The next row's values are loaded
+// before the current row is reduced and quantised (two rows in flight per
+// warp).  Same results as k_export_int8.
+template <int kPer>
+__global__ void __launch_bounds__(kBlock) k_export_rows(
     const int32_t* __restrict__ rows, int64_t n, const long long* dev_n,
     const float4* __restrict__ M, const long long* __restrict__ keys, int64_t C,
-    uint4* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
+    uint32_t* __restrict__ q, float* __restrict__ scale, long long* __restrict__ keys_out,
     int32_t* status, const long long* __restrict__ last, long long* __restrict__ last_out) {
   pdl_enter();
-  extern __shared__ __align__(16) float4 s_stage[];
-  constexpr int kVec = kChunks * 128;  // 16-byte vectors per row
+  constexpr int D4 = 32 * kPer;
   const int lane = threadIdx.x & 31;
-  float4* buf = s_stage + (size_t)(threadIdx.x >> 5) * 2 * kVec;
   int64_t nn = n;
   if (dev_n) {
     const long long d = *dev_n;
     nn = d < nn ? d : nn;
   }
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const int64_t first = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  auto issue = [&](int64_t i, int stage) {
-    if (i < nn) {
-      const int32_t r = rows[i];
+  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  float4 cur[kPer];
+  int32_t rc = -1;
+  auto fetch = [&](int64_t k, float4 (&v)[kPer], int32_t& r) {
+    r = -1;
+    if (k < nn) {
+      r = rows[k];
       if (r >= 0 && (int64_t)r < C) {
-        const float4* src = M + (int64_t)r * kVec + 4 * lane;
-        float4* dst = buf + stage * kVec + 4 * lane;
+        const float4* x = M + (int64_t)r * D4 + lane;
 #pragma unroll
-        for (int ch = 0; ch < kChunks; ++ch)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) cp_async16(dst + ch * 128 + j, src + ch * 128 + j);
+        for (int j = 0; j < kPer; ++j) v[j] = __ldcs(x + 32 * j);
       }
     }
-    cp_async_commit();  // one group per issue, empty or not, so the counts stay in step
   };
-  issue(first, 0);
-  int stage = 0;
-  for (int64_t i = first; i < nn; i += warps, stage ^= 1) {
-    issue(i + warps, stage ^ 1);
-    cp_async_wait<1>();  // this lane's copies of row i have landed
-    const int32_t r = rows[i];
-    uint4* qo = q + i * (int64_t)(kChunks * 32);
-    long long* lo = last_out ? last_out + i : nullptr;
-    if (r < 0 || (int64_t)r >= C) {
+  fetch(i, cur, rc);
+  for (; i < nn; i += warps) {
+    float4 nxt[kPer];
+    int32_t rn;
+    fetch(i + warps, nxt, rn);
+    uint32_t* qo = q + i * (int64_t)D4;
+    if (rc < 0 || (int64_t)rc >= C) {
       if (lane == 0) {
         set_status(status, kStBadRow);
         scale[i] = 0.f;
         keys_out[i] = -1;
-        if (lo) *lo = -1;
+        if (last_out) last_out[i] = -1;
       }
 #pragma unroll
-      for (int ch = 0; ch < kChunks; ++ch) qo[ch * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
-      continue;
+      for (int j = 0; j < kPer; ++j) qo[32 * j + lane] = 0u;
+    } else {
+      float x[4 * kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) {
+        x[4 * j] = cur[j].x;
+        x[4 * j + 1] = cur[j].y;
+        x[4 * j + 2] = cur[j].z;
+        x[4 * j + 3] = cur[j].w;
+      }
+      float a = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4 * kPer; ++e) a = fmaxf(a, fabsf(x[e]));
+      for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, off));
+      const float sc = a == 0.f ? 0.f : __fdiv_rn(a, 127.0f);
+      const float rcp = a == 0.f ? 0.f : __frcp_rn(sc);
+      const bool fast = a != 0.f && isfinite(rcp);
+      int c[4 * kPer];
+#pragma unroll
+      for (int e = 0; e < 4 * kPer; ++e) c[e] = 0;
+      if (a != 0.f) quant_lane<4 * kPer>(x, sc, rcp, fast, c);
+#pragma unroll
+      for (int j = 0; j < kPer; ++j)
+        __stcs(qo + 32 * j + lane, pack4(c[4 * j], c[4 * j + 1], c[4 * j + 2], c[4 * j + 3]));
+      if (lane == 0) {
+        scale[i] = sc;
+        keys_out[i] = keys[rc];
+        if (last_out) last_out[i] = last[rc];
+      }
     }
-    const float4* mine = buf + stage * kVec + 4 * lane;
-    float v[kChunks * 16];
 #pragma unroll
-    for (int ch = 0; ch < kChunks; ++ch)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float4 f = mine[ch * 128 + j];
-        v[ch * 16 + 4 * j] = f.x;
-        v[ch * 16 + 4 * j + 1] = f.y;
-        v[ch * 16 + 4 * j + 2] = f.z;
-        v[ch * 16 + 4 * j + 3] = f.w;
-      }
-    export_values<kChunks>(v, qo, scale + i, keys_out + i, lo, keys[r], last_out ? last[r] : 0,
-                           lane);
+    for (int j = 0; j < kPer; ++j) cur[j] = nxt[j];
+    rc = rn;
   }
-  cp_async_wait<0>();
-}
-
-constexpr size_t export_stage_smem(int kChunks) {
-  return (size_t)(kBlock / 32) * 2 * kChunks * 128 * sizeof(float4);
 }
 
 // ---------------------------------------------------------------------------

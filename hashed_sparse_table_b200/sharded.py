@@ -141,9 +141,23 @@ class ShardedMpzch:
                    ao_table: Optional[torch.Tensor] = None, ao_rows: Optional[torch.Tensor] = None,
                    rows=None, hit=None, out=None, stats=None, trace: Optional[dict] = None):
         """Rows (global), hit and fused features of the labeled ids (read
-        before this step's Writeback), and this shard's Writeback counters."""
+        before this step's Writeback), and this shard's Writeback counters.
+
+        With one shard every id is owned here and global rows are local rows,
+        so the step is the table's own train step: no partition, exchange or
+        combine, and no host read of segment sizes.  The counters are then
+        those of that step; they differ from a multi-shard step's only in
+        n_ids, which counts the batch's valid ids (no first dedup ran)."""
         binding = self.binding
         G, dev, D = self.G, self.device, self.dim
+        if G == 1:
+            if stats is None:
+                stats = torch.empty(7, dtype=torch.int64, device=dev)
+            rows, hit, out = self.table.train_step(ids, n_labeled, e, step, ao_table, ao_rows,
+                                                   stats, rows=rows, hit=hit, out=out)
+            if trace is not None:
+                trace["sent_lookup"] = trace["sent_writeback"] = trace["recv_writeback"] = 0
+            return rows, hit, out, stats
         n = ids.numel()
         lab = ids[:n_labeled]
         width = D + (0 if ao_table is None else ao_table.shape[1])

@@ -37,7 +37,11 @@
  *    device sees (bad ids, rows out of range) set bits of a sticky device status
  *    word, read and cleared by mpzch_get_status.  No kernel traps or spins.
  *  - Calls must be issued with the table's device current.  A handle is not
- *    thread-safe; calls on one handle must be ordered on one stream.
+ *    thread-safe: issue its calls from one host thread at a time.  Issue them
+ *    on one stream.  (A call on a different stream than the previous call
+ *    makes its stream wait for the earlier calls, so results stay correct,
+ *    but the two streams are then serialised.)  mpzch_create and a growth of
+ *    the per-batch scratch complete before they return.
  */
 #ifndef MPZCH_H
 #define MPZCH_H
@@ -67,6 +71,7 @@ extern "C" {
 #define MPZCH_STATUS_BADROW 2   /* a row index outside [0, C) was given to gather/export */
 #define MPZCH_STATUS_BADAO 4    /* an always-on row outside [0, ao_nrows) was given */
 #define MPZCH_STATUS_INTERNAL 8 /* an internal bound was hit (never expected) */
+#define MPZCH_STATUS_TIMEOUT 16 /* a bulk row copy did not complete within its time limit */
 
 typedef struct mpzch_table mpzch_table;
 
@@ -160,7 +165,9 @@ MPZCH_API int mpzch_dedup(mpzch_table* t, const int64_t* ids, int64_t n, int64_t
  * at most MPZCH_DEDUP_STATIC_MAX_IDS; larger n returns MPZCH_ERANGE and
  * launches nothing.  The first call on a device looks up the array's device
  * address (cudaGetSymbolAddress) with that device current; make that first
- * call before any stream capture.  Every call uses the same array and each
+ * call before any stream capture.  The address is kept for the life of the
+ * process: after a cudaDeviceReset of that device (or any other teardown of
+ * its primary context) do not call this function again in the same process.  Every call uses the same array and each
  * call clears the part of it that must start empty, so the contents left by
  * the previous call do not matter -- but calls that can overlap on the GPU
  * (different streams, or several host threads) race with each other and give
@@ -206,11 +213,12 @@ MPZCH_API int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e
  * inputs_ready: NULL, or a cudaEvent_t (as void*) recorded after ids, e and
  * ao_rows of this step were written.  With NULL the step starts after all
  * earlier work on `stream`.  With an event the step's row map starts as soon
- * as that event, the previous step's gather and the previous calls on the
- * table allow -- so it overlaps the previous step's row update (pipelined
- * steps, identical results).  Then the caller must also order every read of
- * the previous step's rows, hit and stats buffers, if they are reused for
- * this step, before inputs_ready. */
+ * as that event, the previous step's gather and the table's earlier calls
+ * allow -- so it overlaps the previous step's row update (pipelined steps,
+ * identical results).  Then the caller must also order before inputs_ready
+ * every read of the previous step's rows, hit and stats buffers that are
+ * reused for this step, and every write it made to the table's state itself
+ * (a restore through mpzch_state_views). */
 MPZCH_API int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_labeled,
                                const float* e, int64_t step, const float* ao_table,
                                int64_t ao_nrows, int32_t ao_dim, const int32_t* ao_rows,
@@ -399,7 +407,31 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * 0 = one row per warp, short-lived blocks; k > 0 = at most k blocks of 256
  * threads per SM, each striding over many rows (default 8). */
 #define MPZCH_OPT_ROW_GRID 3
+/* MPZCH_OPT_ROW_KERNEL: how the row kernels (fused gather, row update) move
+ * rows.  0 (default) = through registers: every lane loads its 16-byte
+ * vectors of a row, then stores them.  1 = through shared memory: one lane
+ * per warp issues 1-D bulk copies (cp.async.bulk, completed on an mbarrier)
+ * of the next rows into the warp's stages while the lanes finish the current
+ * one; persistent grid of MPZCH_OPT_BULK_BLOCKS blocks per SM with
+ * MPZCH_OPT_BULK_WARPS warps each (halved until the block's shared memory
+ * fits 112 KiB; the register path runs for rows too large for one warp's
+ * stages, and for values in host memory).  A row copy that has not completed
+ * after one second sets MPZCH_STATUS_TIMEOUT and the kernel returns.
+ * MPZCH_OPT_L2_HINT_ROWS: L2 eviction priority of the bulk kernels' table-row
+ * loads and stores: 0 (default) evict-first, 1 normal, 2 evict-last. */
+#define MPZCH_OPT_ROW_KERNEL 5
+#define MPZCH_OPT_BULK_WARPS 6
+#define MPZCH_OPT_BULK_BLOCKS 7
+#define MPZCH_OPT_L2_HINT_ROWS 8
+/* MPZCH_OPT_WRITE_LIST (cluster placement path): 1 (default) = the list of
+ * rows the Writeback writes is built as ownership is decided -- the re-probe
+ * adds every resident id, each placement the id it places, and a placement
+ * that evicts an id written earlier in the same step cancels that id's entry;
+ * 0 = one more kernel builds the list after all placements. */
+#define MPZCH_OPT_WRITE_LIST 9
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
+/* Current value of an option (MPZCH_EINVAL for an unknown option). */
+MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);
 
 /* Learning rate of the Writeback step for the following calls (Memory Layer
  * section 2, Writeback paragraph: the exact step is SGD at rate 1 on

@@ -71,7 +71,8 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
              state_every: int = 1, values_every: int = 1, value_rows=None, gather_rows: int = -1,
              ids_fn=None, e_fn=None, wide_rounds: Optional[int] = None,
              fused_step: bool = False, eta: Optional[float] = None,
-             flags: int = 0, cluster: Optional[int] = None) -> RunResult:
+             flags: int = 0, cluster: Optional[int] = None,
+             options: Optional[dict] = None) -> RunResult:
     """Runs steps [start, start+steps) of workload w on both sides.
 
     Per step: lookup of the labeled ids, fused gather (with the always-on concat
@@ -85,6 +86,8 @@ def run_pair(w: inputs.Workload, steps: Optional[int] = None, tbl=None, orc=None
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WIDE_ROUNDS, wide_rounds)
     if cluster is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT, cluster)
+    for opt, val in (options or {}).items():
+        binding.mpzch_set_option(tbl.h, opt, val)
     if eta is not None:
         binding.mpzch_set_learning_rate(tbl.h, eta)
         orc.set_learning_rate(eta)
@@ -144,16 +147,20 @@ def snapshot_from_export(capacity: int, dim: int, rows: np.ndarray, q: np.ndarra
 
 
 def run_pipelined(w: inputs.Workload, steps: Optional[int] = None, flags: int = 0,
-                  cluster: Optional[int] = None):
+                  cluster: Optional[int] = None, options: Optional[dict] = None):
     """All steps' inputs uploaded first, then every step issued back to back as
     a pipelined mpzch_train_step (inputs_ready = one event after the uploads),
     each step with its own output buffers; then every output and the final
-    table are compared with the oracle run step by step."""
+    table are compared with the oracle run step by step.  The table is not
+    reserved, so the first step grows the per-batch scratch after the event was
+    recorded (the growth must complete before the helper streams use it)."""
     from hashed_sparse_table_b200 import binding
     T = w.steps if steps is None else steps
     tbl, orc = make_pair(w, flags=flags)
     if cluster is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT, cluster)
+    for opt, val in (options or {}).items():
+        binding.mpzch_set_option(tbl.h, opt, val)
     dev = tbl.device
     ao = inputs.author_table(w)
     ao_d = torch.from_numpy(ao).to(dev) if ao is not None else None

@@ -310,10 +310,11 @@ def test_select_export_and_serve_match_oracle():
     assert 0 < ohit.mean() < 1
 
 
-@pytest.mark.parametrize("D", [16, 512, 1024])
+@pytest.mark.parametrize("D", [16, 128, 256, 512, 1024])
 def test_export_edge_rows(D):
     """All-zero rows (scale 0), rows with a single large element, negative absmax
-    (dims 512 and 1024 take the staged export kernel, others the register one)."""
+    (dims 128, 256, 512 and 1024 take the interleaved row exporter, others the
+    generic one)."""
     from hashed_sparse_table_b200 import binding
     C = 64
     tbl = binding.MpzchTable(C, D, 4)
@@ -347,7 +348,7 @@ def test_export_edge_rows(D):
         assert not q[i].any() and s[i].item() == 0.0 and k[i].item() == -1
 
 
-@pytest.mark.parametrize("D", [64, 512, 1024])
+@pytest.mark.parametrize("D", [64, 128, 256, 512, 1024])
 def test_export_near_half_integer_quotients(D):
     """Rows built so that x/scale lands on or within a few ulps of k + 1/2 (the
     rounding boundary), plus subnormal-scale rows: every int8 byte must match
@@ -463,3 +464,63 @@ def test_launch_counter_and_trace():
     for ph in ("lookup", "gather", "dedup", "insert", "writeback"):
         ms, launches = tr[ph]
         assert launches > 0 and ms > 0, (ph, tr[ph])
+
+
+@pytest.mark.parametrize("C", [1, 7, 2048, 2049, 6000, 100_003, 1 << 20])
+def test_select_tiles_ragged_tails_and_repeated_calls(C):
+    """The single-pass select over one tile, exactly one, one plus one row, many
+    with a ragged tail, and the 1M-row table; several calls in a row on the same
+    table (the look-back words and tile tickets carry over between calls); rows
+    chosen by every threshold from none to all.  Compared with the oracle and
+    with the definition (ascending rows with a live key and last >= since)."""
+    from hashed_sparse_table_b200 import binding
+    tbl = binding.MpzchTable(C, 4, 1)
+    orc = oracle.OracleTable(C, 4, 1, track_all=False)
+    rng = np.random.default_rng(C)
+    keys = rng.integers(0, 1 << 40, C, dtype=np.int64)
+    last = rng.integers(-1, 100, C, dtype=np.int64)
+    empty = rng.random(C) < 0.3
+    keys[empty] = -1
+    last[empty] = -1
+    k_d, l_d, _ = tbl.state()
+    k_d.copy_(torch.from_numpy(keys))
+    l_d.copy_(torch.from_numpy(last))
+    orc.set_state(keys, last, 99)
+    for since in (-5, 0, 37, 99, 100, 37):
+        rows_d, cnt_d = tbl.select_written_since(since)
+        n = int(cnt_d.item())
+        want = np.nonzero((keys != -1) & (last >= since))[0].astype(np.int32)
+        assert n == want.size, (since, n, want.size)
+        assert_bitwise(rows_d[:n].cpu().numpy(), want, f"select since {since}")
+        assert_bitwise(rows_d[:n].cpu().numpy(), orc.select_written_since(since),
+                       f"select since {since} vs oracle")
+    assert tbl.status() == 0
+
+
+# a table with room (missing ids x P < C, so the grid-wide placement passes run)
+# whose flat id stream touches a large share of the rows every step: the whole
+# window of some missing ids was written in the same step, so an id written
+# earlier in the step is evicted again (its write-list entry is cancelled)
+DROPS = W("drops_p2", 14, capacity=4096, dim=16, probes=2, steps=14, labeled=1500, pool=0,
+          zipf_alpha=0.6, zipf_keys=5_000, fresh_frac=0.05)
+
+
+@pytest.mark.parametrize("write_list", [1, 0])
+@pytest.mark.parametrize("fused", [False, True])
+def test_cluster_path_drops_with_both_write_list_builders(write_list, fused):
+    """Evictions of ids written earlier in the same step on the grid-wide
+    cluster path, with the write list emitted at re-probe and placement
+    (cancelled entries) and with the separate list kernel: identical counters,
+    rows, features and state, every step."""
+    from hashed_sparse_table_b200 import binding
+    r = run_pair(DROPS, fused_step=fused,
+                 options={binding.MPZCH_OPT_WRITE_LIST: write_list})
+    assert sum(s["n_dropped"] for s in r.stats) > 0
+    assert max(s["n_inserted"] for s in r.stats) * DROPS.probes < DROPS.capacity
+
+
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress"])
+def test_pipelined_steps_with_the_separate_write_list_kernel(name):
+    from gpu_harness import run_pipelined
+    from hashed_sparse_table_b200 import binding
+    run_pipelined(SCALED[name], options={binding.MPZCH_OPT_WRITE_LIST: 0})

@@ -209,6 +209,10 @@ def test_sharded_step_matches_sharded_oracle(G):
             assert rc == 0
             gst = results[s][t][3]
             for k in STATS_KEYS:
+                if k == "n_ids" and G == 1:
+                    # one shard: no first dedup, the table's Writeback sees the batch itself
+                    assert gst[k] == int((batches[0][0] >= 0).sum()), (t, gst)
+                    continue
                 assert gst[k] == ost[k], (G, t, s, k, gst, ost)
             evicted += ost["n_evicted"]
     assert evicted > 0  # the workload fills the shards
