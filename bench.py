@@ -100,6 +100,9 @@ def parse():
     ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
                     help="row kernels through registers or through shared memory with bulk "
                          "copies (default: the library's)")
+    ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
+                    help="cluster path: write list emitted at re-probe and placement, or built "
+                         "by a separate kernel (default: the library's)")
     ap.add_argument("--bulk-warps", type=int, default=None)
     ap.add_argument("--bulk-blocks", type=int, default=None)
     ap.add_argument("--l2-hint", type=int, default=None, choices=[0, 1, 2],
@@ -109,6 +112,9 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
+    if args.write_list is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WRITE_LIST,
+                                 1 if args.write_list == "emit" else 0)
     if args.row_kernel is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_ROW_KERNEL,
                                  1 if args.row_kernel == "bulk" else 0)
@@ -575,7 +581,7 @@ def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):
     return {
         "export": {"rows": n, "since_step": since, "ms": export_ms,
                    "rows_per_s": n / (export_ms * 1e-3),
-                   "roofline": {"bound": "hbm", "kernel": "k_export_int8", "achieved": exp_gbs,
+                   "roofline": {"bound": "hbm", "kernel": "k_export_rows", "achieved": exp_gbs,
                                 "peak": peak, "unit": "GB/s", "frac": exp_gbs / peak,
                                 "bytes_per_launch": exp_bytes,
                                 "avg_launch_us": exp_ms / reps * 1e3},

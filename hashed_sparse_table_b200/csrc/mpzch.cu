@@ -253,8 +253,10 @@ struct mpzch_table {
   int32_t* slot_of = nullptr;
   int32_t* bcount = nullptr;
   long long* ukey = nullptr;
-  int32_t* upos = nullptr;
-  int32_t* urow = nullptr;
+  // first positions and rows of the distinct ids, two sets used by alternate
+  // Writebacks (on the cluster path they are the write list the row update reads)
+  int32_t* upos[2] = {nullptr, nullptr};
+  int32_t* urow[2] = {nullptr, nullptr};
   int32_t* snext = nullptr;  // next key of the same home slot (cluster path)
   long long* lkey[3] = {nullptr, nullptr, nullptr};  // insert round lists: keys
   int32_t* lidx[3] = {nullptr, nullptr, nullptr};    // and their distinct-id index
@@ -267,12 +269,9 @@ struct mpzch_table {
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
   int32_t* status = nullptr;
-  // select: per-tile look-back words, the tile ticket counter, the call epoch
-  // and the ticket count issued so far
-  unsigned long long* sel_tstat = nullptr;
-  unsigned long long* sel_ticket = nullptr;
-  uint32_t sel_epoch = 0;
-  unsigned long long sel_tickets = 0;
+  // select: per-tile ballot words and row counts
+  uint32_t* sel_masks = nullptr;
+  int32_t* sel_tcount = nullptr;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
@@ -312,8 +311,8 @@ void free_batch_scratch(mpzch_table* t) {
   dev_free(t->slot_of);
   dev_free(t->bcount);
   dev_free(t->ukey);
-  dev_free(t->upos);
-  dev_free(t->urow);
+  for (auto& l : t->upos) dev_free(l), l = nullptr;
+  for (auto& l : t->urow) dev_free(l), l = nullptr;
   dev_free(t->snext);
   t->snext = nullptr;
   for (auto& l : t->lkey) dev_free(l), l = nullptr;
@@ -322,7 +321,7 @@ void free_batch_scratch(mpzch_table* t) {
   for (auto& l : t->wpos) dev_free(l), l = nullptr;
   t->hkey = nullptr;
   t->hpos = nullptr;
-  t->slot_of = t->bcount = t->upos = t->urow = nullptr;
+  t->slot_of = t->bcount = nullptr;
   t->ukey = nullptr;
   t->cap = 0;
   t->hmask = 0;
@@ -343,8 +342,8 @@ void free_all(mpzch_table* t) {
   dev_free(t->wcnt);
   dev_free(t->stats);
   dev_free(t->status);
-  dev_free(t->sel_tstat);
-  dev_free(t->sel_ticket);
+  dev_free(t->sel_masks);
+  dev_free(t->sel_tcount);
   if (t->h_status) cudaFreeHost(t->h_status);
   for (auto& r : t->pending) {
     cudaEventDestroy(r.a);
@@ -399,8 +398,8 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   if (!rc) rc = dev_alloc((void**)&t->slot_of, cap * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->bcount, tiles * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
-  if (!rc) rc = dev_alloc((void**)&t->upos, cap * sizeof(int32_t));
-  if (!rc) rc = dev_alloc((void**)&t->urow, cap * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->upos[i], cap * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->urow[i], cap * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->snext, cap * sizeof(int32_t));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lkey[i], cap * sizeof(long long));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lidx[i], cap * sizeof(int32_t));
@@ -485,21 +484,19 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
 
 namespace {
 
-// The single-pass select: one block per tile, tickets continuing from the
-// previous call, a fresh epoch (never 0, the value of the cleared words).
+// Select in two launches (marks + counts, then offsets + scatter), the second
+// with programmatic dependent launch.
 int launch_select(mpzch_table* t, int64_t since, int32_t* rows_out, int64_t* dev_count,
                   cudaStream_t st) {
-  const unsigned long long tiles = (unsigned long long)((t->C + kScanTile - 1) / kScanTile);
-  uint32_t epoch = (t->sel_epoch + 1) & ((1u << 30) - 1);
-  if (epoch == 0) epoch = 1;
-  const int rc = launch(k_select_scan, (unsigned)tiles, kScanThreads, st, false,
-                        (const long long*)t->keys, (const long long*)t->last, t->C,
-                        (long long)since, t->sel_tstat, t->sel_ticket, t->sel_tickets, epoch,
-                        rows_out, reinterpret_cast<long long*>(dev_count), t->status);
-  if (rc) return rc;
-  t->sel_epoch = epoch;
-  t->sel_tickets += tiles;
-  return MPZCH_OK;
+  const unsigned tiles = (unsigned)((t->C + kScanTile - 1) / kScanTile);
+  int rc = launch(k_select_mark, tiles, kScanThreads, st, false, (const long long*)t->keys,
+                  (const long long*)t->last, t->C, (long long)since, t->sel_masks,
+                  t->sel_tcount);
+  if (!rc)
+    rc = launch(k_select_scatter, tiles, kScanThreads, st, true, (const uint32_t*)t->sel_masks,
+                (const int32_t*)t->sel_tcount, t->C, rows_out,
+                reinterpret_cast<long long*>(dev_count));
+  return rc;
 }
 
 int enqueue_lookup(mpzch_table* t, const int64_t* ids, int64_t n, int32_t* rows, uint8_t* hit,
@@ -590,8 +587,8 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.hmask = t->hmask;
   p.slot_of = t->slot_of;
   p.ukey = t->ukey;
-  p.upos = t->upos;
-  p.urow = t->urow;
+  p.upos = t->upos[t->wset];
+  p.urow = t->urow[t->wset];
   p.keys = t->keys;
   p.last = t->last;
   p.M = reinterpret_cast<float4*>(t->M);
@@ -614,12 +611,14 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.tag = t->tag;
   p.shead = t->shead;
   p.snext = t->snext;
-  p.wrow = t->wrow[t->wset];
-  p.wpos = t->wpos[t->wset];
   p.wcount = t->wcnt + t->wset;
   p.wtake = t->wcnt + 2 + t->wset;
   p.emit = (t->cluster_insert && t->emit_list) ? 1 : 0;
   p.wentry = t->wentry;
+  // emit: the distinct-id arrays are the list; otherwise k_write_list fills
+  // the compacted buffers
+  p.wrow = p.emit ? p.urow : t->wrow[t->wset];
+  p.wpos = p.emit ? p.upos : t->wpos[t->wset];
   return p;
 }
 
@@ -846,8 +845,8 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
   if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
   const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
-  if (!rc) rc = dev_alloc((void**)&t->sel_tstat, sel_tiles * sizeof(unsigned long long));
-  if (!rc) rc = dev_alloc((void**)&t->sel_ticket, sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->sel_masks, sel_tiles * kScanWords * sizeof(uint32_t));
+  if (!rc) rc = dev_alloc((void**)&t->sel_tcount, sel_tiles * sizeof(int32_t));
   if (!rc && cudaHostAlloc((void**)&t->h_status, sizeof(int32_t), cudaHostAllocDefault) != cudaSuccess) {
     t->h_status = nullptr;
     rc = MPZCH_ENOMEM;
@@ -866,10 +865,7 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
-              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess &&
-              cudaMemsetAsync(t->sel_tstat, 0, sel_tiles * sizeof(unsigned long long), st) ==
-                  cudaSuccess &&
-              cudaMemsetAsync(t->sel_ticket, 0, sizeof(unsigned long long), st) == cudaSuccess;
+              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
     for (int i = 0; i < 3 && ok; ++i)
       ok = cudaMemsetAsync(t->claims[i], 0xFF, capacity * sizeof(unsigned long long), st) ==
            cudaSuccess;

@@ -543,64 +543,56 @@ struct WbParams {
   int32_t* wpos;
   int32_t* wcount;
   int32_t* wtake;  // entries of the list already taken by the bulk row update
-  // emit = 1 (cluster path): the re-probe appends the write-list entry of every
-  // resident id and each placement the entry of the id it places, and
-  // wentry[row] holds the entry of the row's current owner in this step; a
-  // placement that evicts an id written earlier in this step turns that id's
-  // entry into a tombstone (row -1), which the row update skips.  emit = 0:
-  // k_write_list builds the list after all placements.
+  // emit = 1 (cluster path): the write list is the distinct-id arrays of this
+  // call themselves -- entry u = (urow[u], upos[u]), wrow/wpos point at them
+  // and *wcount is set to the number of distinct ids -- so nothing is
+  // appended.  wentry[row] holds the distinct-id index of the row's owner in
+  // this step (set by the re-probe for resident ids and by each placement); a
+  // placement that evicts an id written earlier in this step marks that id's
+  // urow as kDroppedRow, which the row update skips.  emit = 0: k_write_list
+  // builds a compacted list in separate buffers after all placements.
   int emit;
   int32_t* wentry;
+  // lookup of the first n_fill batch positions (the labeled ids of a train
+  // step) taken from the re-probe: the re-probe stores, per scratch-hash slot,
+  // the row its id held before this step's inserts (hrow), and the fill pass
+  // gives every position its id's row (rows, hit); n_fill = 0: no fill
+  int32_t* hrow;
+  int64_t n_fill;
+  int32_t* fill_rows;
+  uint8_t* fill_hit;
 };
 
-// Write-list entry m: `row` now belongs to distinct id uidx, whose e row is
-// the one at its first batch position.
-__device__ __forceinline__ void emit_entry(const WbParams& p, int m, int64_t row, int32_t uidx) {
-  p.wrow[m] = (int32_t)row;
-  p.wpos[m] = p.upos[uidx];
-  p.wentry[row] = m;
+// Lookup result of batch position i < n_fill: the row its id held before the
+// step's inserts (-1: missing; negative ids have no scratch slot and were
+// flagged by the dedup).  Reads only what the dedup and the re-probe wrote.
+__device__ __forceinline__ void fill_lookup(const WbParams& p, int64_t i) {
+  const int32_t s = p.slot_of[i];
+  const int32_t r = s >= 0 ? __ldcg(p.hrow + s) : -1;
+  p.fill_rows[i] = r;
+  p.fill_hit[i] = r >= 0 ? 1 : 0;
 }
 
-// A placement into `row` whose previous owner was written in this step (its
-// last-write step is this step: a resident id refreshed by the re-probe, or an
-// id placed earlier in the step): that owner gets no write (n_dropped).
-__device__ __forceinline__ void drop_victim(const WbParams& p, int64_t row, long long victim_last) {
-  if (victim_last == p.step) {
-    p.wrow[p.wentry[row]] = -1;
-    atomic_add_ll(&p.stats->n_dropped, 1LL);
-  }
-}
+// urow value of a distinct id that was placed and then evicted again later in
+// the same step (it gets no write); -1 still means "not placed yet".
+constexpr int32_t kDroppedRow = -2;
 
-// Both, for a placement made by one thread.
+// Bookkeeping of a placement into `row` for distinct id uidx (emit mode): a
+// previous owner written in this step (its last-write step is this step: a
+// resident id refreshed by the re-probe, or an id placed earlier in the
+// step) loses its write (n_dropped), and uidx becomes the row's owner.
 __device__ __forceinline__ void emit_placement(const WbParams& p, int64_t row,
                                                long long victim_last, int32_t uidx) {
   if (!p.emit) return;
-  drop_victim(p, row, victim_last);
-  emit_entry(p, atomicAdd(p.wcount, 1), row, uidx);
+  if (victim_last == p.step) {
+    p.urow[p.wentry[row]] = kDroppedRow;
+    atomic_add_ll(&p.stats->n_dropped, 1LL);
+  }
+  p.wentry[row] = uidx;
 }
 
 // Two per-thread counts packed as 16-bit halves (each <= the block size).
 __device__ __forceinline__ int pack2(int a, int b) { return a | (b << 16); }
-
-// Block-aggregated append to three lists (counts packed in 10-bit fields, so
-// blocks of at most 1023 threads).  All threads of the block must call it.
-__device__ __forceinline__ void block_append3(int wa, int wb, int wc, int32_t* ca, int32_t* cb,
-                                              int32_t* cc, int& ia, int& ib, int& ic, int* smi) {
-  int total = 0;
-  const int before = block_excl_scan(wa | (wb << 10) | (wc << 20), smi, total);
-  __shared__ int s_base3[3];
-  if (threadIdx.x == 0) {
-    const int ta = total & 1023, tb = (total >> 10) & 1023, tc = total >> 20;
-    s_base3[0] = ta ? atomicAdd(ca, ta) : 0;
-    s_base3[1] = tb ? atomicAdd(cb, tb) : 0;
-    s_base3[2] = tc ? atomicAdd(cc, tc) : 0;
-  }
-  __syncthreads();
-  ia = s_base3[0] + (before & 1023);
-  ib = s_base3[1] + ((before >> 10) & 1023);
-  ic = s_base3[2] + (before >> 20);
-  __syncthreads();
-}
 
 // Block-aggregated append: every thread with want != 0 gets a distinct slot of
 // the list whose length counter is `counter`; one global atomic per block.
@@ -651,15 +643,12 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
           p.hpos[s] = kNoPos;
           h = home_slot(k, g);
           r = find_row_thread(p.keys, k, h, g);
+          if (p.n_fill) p.hrow[s] = (int32_t)r;
         }
       }
     }
-    int u = 0, m = 0, wi = 0;
-    if (p.emit)
-      block_append3(first, first && r < 0, first && r >= 0, &p.ctr->n_unique, &p.ctr->cnt[0],
-                    p.wcount, u, m, wi, smi);
-    else
-      block_append2(first, first && r < 0, &p.ctr->n_unique, &p.ctr->cnt[0], u, m, smi);
+    int u = 0, m = 0;
+    block_append2(first, first && r < 0, &p.ctr->n_unique, &p.ctr->cnt[0], u, m, smi);
     if (first) {
       p.ukey[u] = k;
       p.upos[u] = (int32_t)i;
@@ -667,11 +656,7 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
       if (r >= 0) {
         p.last[r] = p.step;
         ++hits;
-        if (p.emit) {
-          p.wrow[wi] = (int32_t)r;
-          p.wpos[wi] = (int32_t)i;
-          p.wentry[r] = wi;
-        }
+        if (p.emit) p.wentry[r] = u;
       } else {
         p.lkey[0][m] = k;
         p.lidx[0][m] = u;
@@ -692,6 +677,15 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
     if (bh) atomic_add_ll(&p.stats->n_hit_unique, bh);
     if (bv) atomic_add_ll(&p.stats->n_ids, bv);
   }
+}
+
+// The lookup fill as a kernel of its own (claim-round insert path, where no
+// placement pass follows the re-probe).
+__global__ void __launch_bounds__(kBlock) k_lookup_fill(WbParams p) {
+  pdl_enter();
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_fill; i += stride)
+    fill_lookup(p, i);
 }
 
 // Grid-wide insert round r (see the insert comment above): clears the claims
@@ -1069,7 +1063,7 @@ __device__ int32_t cluster_min_unplaced(const WbParams& p, int64_t h, int64_t L,
     for (int32_t x = (int32_t)(uint32_t)v, hops = 0; x >= 0 && hops <= N;
          x = __ldcg(p.snext + x), ++hops) {
       const long long k = __ldcg(p.lkey[0] + x);
-      if (__ldcg(p.urow + __ldcg(p.lidx[0] + x)) < 0 && (arg < 0 || k < kmin)) {
+      if (__ldcg(p.urow + __ldcg(p.lidx[0] + x)) == -1 && (arg < 0 || k < kmin)) {
         arg = x;
         kmin = k;
       }
@@ -1338,10 +1332,7 @@ __device__ int place_lone(const WbParams& p, int32_t m, long long& evicted, int6
   }
   if (best_last != -1) ++evicted;
   const int32_t u = __ldcg(p.lidx[0] + m);
-  if (p.emit) {
-    drop_victim(p, best, best_last);
-    emit_entry(p, warp_append(p.wcount), best, u);
-  }
+  emit_placement(p, best, best_last, u);
   p.keys[best] = k;
   p.last[best] = p.step;
   p.urow[u] = (int32_t)best;
@@ -1357,12 +1348,17 @@ __global__ void __launch_bounds__(kBlock) k_place_clusters(WbParams p) {
   const bool ring_may_be_covered = (int64_t)N * p.g.P >= p.g.C;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     p.stats->n_inserted = N;
-    if (p.emit) p.stats->n_unique = p.ctr->n_unique;  // no k_write_list on this path
+    if (p.emit) {  // no k_write_list on this path: the list is the distinct-id arrays
+      p.stats->n_unique = p.ctr->n_unique;
+      *p.wcount = p.ctr->n_unique;
+    }
     if (N > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
   }
   long long evicted = 0;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_fill; i += stride)
+    fill_lookup(p, i);
   if (!ring_may_be_covered) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t m = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; m < N; m += stride) {
       int64_t h = 0;
       if (place_lone(p, (int32_t)m, evicted, h)) p.lidx[1][warp_append(&p.ctr->n_multi)] = (int32_t)h;
@@ -1824,51 +1820,32 @@ __global__ void k_gather_bulk(const int32_t* __restrict__ rows, const uint8_t* _
 }
 
 // ---------------------------------------------------------------------------
-// Select rows written at or after `since`, ascending: one pass, one launch.
-// Tiles of kScanTile rows; a block takes the next tile index from a ticket
-// counter (so every tile it waits for belongs to a block that is already
-// running), counts its selected rows and publishes that count; then one warp
-// sums the counts of all earlier tiles -- up to 256 words in flight at once,
-// none of them waiting on another tile's sum -- and the block scatters its
-// rows at that offset.
-//
-// Tile word (64 bits): epoch (bits 63..34, the call's number, so words of
-// earlier calls read as not yet published and nothing is cleared), flag
-// (bit 32), count (31..0).  Thread t of a block reads rows t + 256k (k < 8)
-// of its tile, so every load instruction covers 256 contiguous bytes; the
-// rows' order inside the tile comes from per-warp ballots and a 64-entry
-// scan.  A wait for an earlier tile's word has a time limit
-// (MPZCH_STATUS_TIMEOUT when it runs out).
+// Select rows written at or after `since`, ascending, in two launches over
+// tiles of kScanTile rows.  Thread t of a block reads rows t + 256k (k < 8) of
+// its tile, so every load instruction covers 256 contiguous bytes.
+//   k_select_mark     per tile, the 64 ballot words of its (sub-tile, warp)
+//                     groups and its row count (the only pass over the table);
+//   k_select_scatter  per tile, the sum of the earlier tiles' counts (a block
+//                     reduction over at most a few thousand ints, L2-resident),
+//                     then every selected row written at that offset plus its
+//                     rank inside the tile, from the ballot words.
+// The second kernel is launched with programmatic dependent launch, so its
+// blocks start while the first drains.  No block waits on another.
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 256;
 constexpr int kScanPer = 8;
 constexpr int kScanTile = kScanThreads * kScanPer;
-constexpr unsigned long long kTileAgg = 1ull << 32;
+constexpr int kScanWords = kScanPer * (kScanThreads / 32);  // ballot words per tile
 
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-__global__ void __launch_bounds__(kScanThreads) k_select_scan(
-    const long long* __restrict__ keys, const long long* __restrict__ last, int64_t C,
-    long long since, unsigned long long* tstat, unsigned long long* ticket,
-    unsigned long long ticket_base, uint32_t epoch, int32_t* __restrict__ rows_out,
-    long long* dev_count, int32_t* status) {
+__global__ void __launch_bounds__(kScanThreads) k_select_mark(const long long* __restrict__ keys,
+                                                              const long long* __restrict__ last,
+                                                              int64_t C, long long since,
+                                                              uint32_t* __restrict__ masks,
+                                                              int32_t* __restrict__ tcount) {
   pdl_enter();
-  __shared__ int s_tile;
-  __shared__ int s_off[kScanPer * (kScanThreads / 32) + 1];
-  __shared__ long long s_excl;
+  __shared__ int s_cnt[kScanThreads / 32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) s_tile = (int)(atomicAdd(ticket, 1ull) - ticket_base);
-  __syncthreads();
-  const int tile = s_tile;
-  const int64_t base = (int64_t)tile * kScanTile + threadIdx.x;
+  const int64_t base = (int64_t)blockIdx.x * kScanTile + threadIdx.x;
   long long kv[kScanPer], lv[kScanPer];
 #pragma unroll
   for (int k = 0; k < kScanPer; ++k) {
@@ -1876,69 +1853,59 @@ __global__ void __launch_bounds__(kScanThreads) k_select_scan(
     kv[k] = r < C ? __ldcs(keys + r) : -1;
     lv[k] = r < C ? __ldcs(last + r) : -1;
   }
-  unsigned ball[kScanPer];
+  int c = 0;
 #pragma unroll
   for (int k = 0; k < kScanPer; ++k) {
-    ball[k] = __ballot_sync(0xFFFFFFFFu, kv[k] != -1 && lv[k] >= since);
-    if (lane == 0) s_off[k * (kScanThreads / 32) + warp] = __popc(ball[k]);
+    const unsigned b = __ballot_sync(0xFFFFFFFFu, kv[k] != -1 && lv[k] >= since);
+    if (lane == 0) masks[(int64_t)blockIdx.x * kScanWords + k * (kScanThreads / 32) + warp] = b;
+    c += __popc(b);
   }
+  pdl_trigger();
+  if (lane == 0) s_cnt[warp] = c;
   __syncthreads();
-  if (warp == 0) {  // exclusive scan of the 64 (sub-tile, warp) counts, in row order
-    constexpr int kN = kScanPer * (kScanThreads / 32);
-    const int a = s_off[2 * lane], b = s_off[2 * lane + 1];
-    int x = a + b;
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < kScanThreads / 32; ++w) t += s_cnt[w];
+    tcount[blockIdx.x] = t;
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_select_scatter(
+    const uint32_t* __restrict__ masks, const int32_t* __restrict__ tcount, int64_t C,
+    int32_t* __restrict__ rows_out, long long* dev_count) {
+  pdl_enter();
+  __shared__ long long sm[33];
+  __shared__ int s_off[kScanWords + 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tile = blockIdx.x;
+  // offset of this tile: counts of tiles 0 .. tile-1
+  long long acc = 0;
+  for (int q = threadIdx.x; q < tile; q += kScanThreads) acc += tcount[q];
+  const long long excl = block_sum_ll(acc, sm);
+  if (warp == 0) {  // exclusive scan of the 64 group counts, in row order
+    const uint32_t a = masks[(int64_t)tile * kScanWords + 2 * lane];
+    const uint32_t b = masks[(int64_t)tile * kScanWords + 2 * lane + 1];
+    const int ca = __popc(a), cb = __popc(b);
+    int x = ca + cb;
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
       if (lane >= off) x += y;
     }
-    const int before = x - a - b;
-    s_off[2 * lane] = before;
-    s_off[2 * lane + 1] = before + a;
-    if (lane == 31) s_off[kN] = x;
-    static_assert(kN == 64, "one warp scans two counts per lane");
+    s_off[2 * lane] = x - ca - cb;
+    s_off[2 * lane + 1] = x - cb;
+    if (lane == 31) s_off[kScanWords] = x;
+    static_assert(kScanWords == 64, "one warp scans two counts per lane");
   }
   __syncthreads();
-  const int total = s_off[kScanPer * (kScanThreads / 32)];
-  if (warp == 0) {
-    const unsigned long long ep = (unsigned long long)epoch << 34;
-    if (lane == 0) st_relaxed_u64(tstat + tile, ep | kTileAgg | (uint32_t)total);
-    long long excl = 0;
-    bool timed_out = false;
-    const uint64_t t0 = global_ns();
-    constexpr int kBatch = 8;  // words per lane in flight
-    for (int q0 = 0; q0 < tile && !timed_out; q0 += 32 * kBatch) {
-      unsigned long long w[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int q = q0 + lane + 32 * u;
-        w[u] = q < tile ? ld_relaxed_u64(tstat + q) : (ep | kTileAgg);
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int q = q0 + lane + 32 * u;
-        while ((w[u] >> 34) != epoch || !(w[u] & kTileAgg)) {  // not yet published
-          if (global_ns() - t0 > kWaitLimitNs) {
-            timed_out = true;
-            break;
-          }
-          w[u] = ld_relaxed_u64(tstat + q);
-        }
-        excl += (long long)(uint32_t)w[u];
-      }
-    }
-    for (int off = 16; off > 0; off >>= 1) excl += __shfl_xor_sync(0xFFFFFFFFu, excl, off);
-    if (__any_sync(0xFFFFFFFFu, timed_out) && lane == 0) set_status(status, kStTimeout);
-    if (lane == 0) s_excl = excl;
-  }
-  __syncthreads();
-  const long long excl = s_excl;
+  const int64_t base = (int64_t)tile * kScanTile + threadIdx.x;
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int k = 0; k < kScanPer; ++k)
-    if (ball[k] >> lane & 1u)
-      rows_out[excl + s_off[k * (kScanThreads / 32) + warp] + __popc(ball[k] & lt)] =
-          (int32_t)(base + k * kScanThreads);
-  if ((int64_t)(tile + 1) * kScanTile >= C && threadIdx.x == 0) *dev_count = excl + total;
+  for (int k = 0; k < kScanPer; ++k) {
+    const int g = k * (kScanThreads / 32) + warp;
+    const uint32_t b = masks[(int64_t)tile * kScanWords + g];
+    if (b >> lane & 1u) rows_out[excl + s_off[g] + __popc(b & lt)] = (int32_t)(base + k * kScanThreads);
+  }
+  if (tile == gridDim.x - 1 && threadIdx.x == 0) *dev_count = excl + s_off[kScanWords];
 }
 
 // ---------------------------------------------------------------------------
