@@ -75,6 +75,9 @@ def parse():
                     help="table values in pinned host memory (host-memory tier): the row "
                          "kernels move them over the host link; reports the link's copy "
                          "bandwidth as 'host_link'")
+    ap.add_argument("--hbm-cache-rows", type=int, default=0,
+                    help="with --host-values: an HBM cache of this many rows (power of two) in "
+                         "front of the host-memory values (hot/cold tier)")
     ap.add_argument("--row-grid", type=int, default=None,
                     help="row kernels: 0 = one row per warp, k = k blocks per SM grid-stride")
     ap.add_argument("--side-priority", type=int, default=None, choices=[0, 1],
@@ -341,6 +344,8 @@ def run_ours(args):
     tbl = binding.MpzchTable(W.capacity, W.dim, W.probes,
                              flags=binding.MPZCH_VALUES_IN_HOST_MEMORY if args.host_values else 0)
     binding.mpzch_reserve(tbl.h, W.batch)
+    if args.hbm_cache_rows:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_HBM_CACHE_ROWS, args.hbm_cache_rows)
     if args.row_grid is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_ROW_GRID, args.row_grid)
     if args.side_priority is not None:
@@ -476,6 +481,11 @@ def run_ours(args):
             link["row_update_frac_of_bidirectional"] = link_gbs / link["bidirectional_gbs"]
             result["host_link"] = link
             result["config"]["values"] = "pinned host memory, mapped (host-memory tier)"
+            if args.hbm_cache_rows:
+                result["config"]["hbm_cache_rows"] = args.hbm_cache_rows
+                result["config"]["values"] += (f", HBM cache of {args.hbm_cache_rows} rows "
+                                               f"({args.hbm_cache_rows / W.capacity:.0%} of the "
+                                               "table) in front")
         if res_info is not None:
             result["res"] = res_info
         if shard_k is not None:

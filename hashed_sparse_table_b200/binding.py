@@ -42,6 +42,7 @@ MPZCH_OPT_BULK_WARPS = 6
 MPZCH_OPT_BULK_BLOCKS = 7
 MPZCH_OPT_L2_HINT_ROWS = 8
 MPZCH_OPT_WRITE_LIST = 9
+MPZCH_OPT_HBM_CACHE_ROWS = 10
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")
@@ -74,6 +75,7 @@ _SIGS = {
     "mpzch_trace_read": [_p, C.POINTER(C.c_double), C.POINTER(_i64), _i32],
     "mpzch_set_option": [_p, _i32, _i64],
     "mpzch_get_option": [_p, _i32, C.POINTER(_i64)],
+    "mpzch_tier_sync": [_p, _i32, _p],
     "mpzch_debug_fail_allocs": [_i32],
     "mpzch_set_learning_rate": [_p, C.c_float],
     "mpzch_res_create": [_p, _i64, _i32, _i32, C.POINTER(_p)],
@@ -302,6 +304,10 @@ def mpzch_get_option(h, option: int) -> int:
     v = _i64(0)
     _check("mpzch_get_option", _lib.mpzch_get_option(h, option, C.byref(v)))
     return int(v.value)
+
+
+def mpzch_tier_sync(h, discard: bool = False, stream=None) -> None:
+    _check("mpzch_tier_sync", _lib.mpzch_tier_sync(h, 1 if discard else 0, _stream(stream)))
 
 
 def mpzch_set_learning_rate(h, eta: float) -> None:

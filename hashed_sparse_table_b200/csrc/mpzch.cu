@@ -3,6 +3,7 @@
 #include "mpzch.h"
 #include "mpzch_internal.h"
 #include "mpzch_kernels.cuh"
+#include "mpzch_tier.cuh"
 
 #include <cuda_runtime.h>
 
@@ -250,6 +251,7 @@ struct mpzch_table {
   uint64_t hmask = 0;
   unsigned long long* hkey = nullptr;
   uint32_t* hpos = nullptr;
+  int32_t* hrow = nullptr;  // pre-insert row of each scratch-hash slot's id (train-step lookup)
   int32_t* slot_of = nullptr;
   int32_t* bcount = nullptr;
   long long* ukey = nullptr;
@@ -282,9 +284,11 @@ struct mpzch_table {
   int bulk_warps = 8;          // bulk row kernels: warps per block
   int bulk_blocks = 1;         // bulk row kernels: blocks per SM (persistent grid)
   int l2_hint_rows = 0;        // bulk row kernels: L2 policy of table-row accesses (L2Hint)
+  // hot/cold tier (values in host memory): HBM cache of tier_rows rows, 0 = none
+  int64_t tier_rows = 0;
+  Tier tier{};
   // mpzch_train_step: the row map runs on a second (high-priority) stream
   cudaStream_t side = nullptr;
-  cudaStream_t look = nullptr;  // the train step's lookup: highest stream priority
   cudaEvent_t ev_fork = nullptr, ev_lookup = nullptr, ev_map = nullptr;
   cudaEvent_t ev_update[2] = {nullptr, nullptr};  // row update that read write list b
   cudaEvent_t ev_user = nullptr;    // end of every other call so far (created with the table)
@@ -308,6 +312,8 @@ namespace {
 void free_batch_scratch(mpzch_table* t) {
   dev_free(t->hkey);
   dev_free(t->hpos);
+  dev_free(t->hrow);
+  t->hrow = nullptr;
   dev_free(t->slot_of);
   dev_free(t->bcount);
   dev_free(t->ukey);
@@ -338,6 +344,10 @@ void free_all(mpzch_table* t) {
   for (auto& c : t->claims) dev_free(c), c = nullptr;
   dev_free(t->shead);
   dev_free(t->wentry);
+  dev_free(t->tier.cache);
+  dev_free(t->tier.owner);
+  dev_free(t->tier.won);
+  dev_free(t->tier.claim);
   dev_free(t->ctr);
   dev_free(t->wcnt);
   dev_free(t->stats);
@@ -358,7 +368,6 @@ void free_all(mpzch_table* t) {
   if (t->ev_user) cudaEventDestroy(t->ev_user);
   if (t->ev_gather) cudaEventDestroy(t->ev_gather);
   if (t->side) cudaStreamDestroy(t->side);
-  if (t->look) cudaStreamDestroy(t->look);
 }
 
 int ensure_side_stream(mpzch_table* t) {
@@ -367,7 +376,6 @@ int ensure_side_stream(mpzch_table* t) {
   if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
       cudaStreamCreateWithPriority(&t->side, cudaStreamNonBlocking,
                                    t->side_high_priority ? greatest : least) != cudaSuccess ||
-      cudaStreamCreateWithPriority(&t->look, cudaStreamNonBlocking, greatest) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_lookup, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&t->ev_map, cudaEventDisableTiming) != cudaSuccess ||
@@ -395,6 +403,7 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   int rc = MPZCH_OK;
   if (!rc) rc = dev_alloc((void**)&t->hkey, H * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->hpos, H * sizeof(uint32_t));
+  if (!rc) rc = dev_alloc((void**)&t->hrow, H * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->slot_of, cap * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->bcount, tiles * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
@@ -548,6 +557,11 @@ int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int6
                    const int32_t* ao_rows, float* out, cudaStream_t st, bool pdl) {
   PhaseScope ps(t, PH_GATHER, st);
   const bool has_ao = ao_table != nullptr;
+  if (t->tier_rows > 0)
+    return launch(k_tier_gather, row_grid(n, t->row_blocks_per_sm), kBlock, st, pdl, rows, hit, n,
+                  t->tier, reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
+                  reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
+                  ao_rows, reinterpret_cast<float4*>(out), t->status);
   int warps = 0;
   size_t smem = 0;
   if (bulk_shape(t, (size_t)(t->D + (has_ao ? ao_dim : 0)) * 4, &warps, &smem)) {
@@ -569,6 +583,7 @@ int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int6
 int check_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t n, int64_t step) {
   if (!t || n < 0 || n > 0x7FFFFFFFLL) return MPZCH_EINVAL;
   if (step <= t->last_step) return MPZCH_EINVAL;
+  if (t->tier_rows > 0 && step >= (int64_t)1 << 31) return MPZCH_EINVAL;  // claim words hold 31 bits
   if (n > 0 && (!ids || !e)) return MPZCH_EINVAL;
   if (!on_device(t)) return MPZCH_EINVAL;
   if (reinterpret_cast<uintptr_t>(e) & 15) return MPZCH_EINVAL;
@@ -584,6 +599,10 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.D4 = t->D / 4;
   p.hkey = t->hkey;
   p.hpos = t->hpos;
+  p.hrow = t->hrow;
+  p.n_fill = 0;
+  p.fill_rows = nullptr;
+  p.fill_hit = nullptr;
   p.hmask = t->hmask;
   p.slot_of = t->slot_of;
   p.ukey = t->ukey;
@@ -623,10 +642,13 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
 }
 
 // Row map of one Writeback on stream `st`: dedup + re-probe + refresh, then
-// the insert rounds and the write list.  With `keys_free` the inserts (the
-// first writes to the key array in the step) wait for that event: a lookup of
-// this step on another stream must read the keys first.
-int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEvent_t keys_free) {
+// the inserts (and, on the claim-round path or without emitted lists, the
+// write list).  With p.n_fill > 0 (train step) the first n_fill positions'
+// lookup results are filled from the re-probe, after `fill_after` (the
+// previous gather, which may still read the same rows/hit buffers), and
+// `fill_done` is recorded once they are written.
+int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEvent_t fill_after,
+                    cudaEvent_t fill_done) {
   const int64_t n = p.n;
   int rc;
   if (t->tag_wrapped) {
@@ -642,27 +664,37 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
   }
-  if (keys_free && cudaStreamWaitEvent(st, keys_free, 0) != cudaSuccess) return MPZCH_ECUDA;
+  const bool wait = p.n_fill > 0 && fill_after;
+  if (wait && cudaStreamWaitEvent(st, fill_after, 0) != cudaSuccess) return MPZCH_ECUDA;
   if (p.cluster) {
-    // cluster placement; the single-block finisher only acts when the
-    // windows may cover the whole ring
+    // cluster placement (its first pass also fills the lookup); the
+    // single-block finisher only acts when the windows may cover the whole
+    // ring or a cluster exceeds the warp path
     PhaseScope ps(t, PH_INSERT, st);
-    rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !keys_free, p);
+    rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !wait, p);
+    if (!rc && p.n_fill > 0 && fill_done && cudaEventRecord(fill_done, st) != cudaSuccess)
+      rc = MPZCH_ECUDA;
     // one warp per multi-key cluster, as many resident warps as the SMs hold
     const int multi_per_sm = resident_blocks(reinterpret_cast<const void*>(k_place_multi), kBlock, 0);
     if (!rc)
-      rc = launch(k_place_multi, grid_for(n * 32, kBlock, multi_per_sm), kBlock, st, true, p);
+      rc = launch(k_place_multi, grid_for(n * 32, kBlock, multi_per_sm), kBlock, st,
+                  !(p.n_fill > 0 && fill_done), p);
     if (!rc) rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, 0);
     if (!rc && !p.emit) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
     return rc;
   }
   {
     PhaseScope ps(t, PH_INSERT, st);
+    if (p.n_fill > 0) {
+      rc = launch(k_lookup_fill, grid_for(p.n_fill, kBlock), kBlock, st, !wait, p);
+      if (!rc && fill_done && cudaEventRecord(fill_done, st) != cudaSuccess) rc = MPZCH_ECUDA;
+    }
     const unsigned grid = grid_for(n, kBlock, 4);
     for (int r = 0; r < t->wide_rounds && !rc; ++r)
-      rc = launch(k_insert_round, grid, kBlock, st, !keys_free || r > 0, p, r);
+      rc = launch(k_insert_round, grid, kBlock, st, r > 0 || (!wait && p.n_fill == 0), p, r);
     if (!rc)
-      rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, t->wide_rounds);
+      rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st,
+                       t->wide_rounds > 0 || p.n_fill == 0, p, t->wide_rounds);
     if (!rc) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
   }
   return rc;
@@ -674,7 +706,20 @@ int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool 
     int warps = 0;
     size_t smem = 0;
     int rc;
-    if (bulk_shape(t, (size_t)t->D * 8, &warps, &smem)) {
+    if (t->tier_rows > 0) {
+      // claims, evictions, then the update (three passes over the write list)
+      const unsigned g = row_grid(p.n, t->row_blocks_per_sm);
+      float4* host = p.M;
+      rc = launch(k_tier_claim, grid_for(p.n, kBlock), kBlock, st, pdl, (const int32_t*)p.wrow,
+                  (const int32_t*)p.wcount, t->tier, (long long)p.step);
+      if (!rc)
+        rc = launch(k_tier_evict, g, kBlock, st, true, (const int32_t*)p.wrow,
+                    (const int32_t*)p.wcount, t->tier, host, p.D4, (long long)p.step);
+      if (!rc)
+        rc = launch(k_tier_update, g, kBlock, st, true, (const int32_t*)p.wrow,
+                    (const int32_t*)p.wpos, (const int32_t*)p.wcount, t->tier, host, p.e, p.D4,
+                    t->eta, (long long)p.step);
+    } else if (bulk_shape(t, (size_t)t->D * 8, &warps, &smem)) {
       int64_t g = (int64_t)sm_count() * t->bulk_blocks;
       const int64_t need = (p.n + 32 * warps - 1) / (32 * warps);
       if (g > need) g = need;
@@ -959,7 +1004,7 @@ int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e, int64_t 
   rc = ensure_batch(t, n, st);
   if (rc) return rc;
   const WbParams p = make_params(t, ids, e, n, step, stats);
-  rc = enqueue_row_map(t, p, st, nullptr);
+  rc = enqueue_row_map(t, p, st, nullptr, nullptr);
   if (!rc) rc = enqueue_row_update(t, p, st, true);
   if (rc) return rc;
   t->last_step = step;
@@ -990,46 +1035,40 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
     t->last_step = step;
     return mark_user(t, st, MPZCH_OK);
   }
-  const WbParams p = make_params(t, ids, e, n, step, stats);
-  // Three streams.  Lookup stream (highest priority): the lookup, once the
-  // keys hold the previous step's inserts.  Side stream (low priority):
-  // dedup + refresh, then -- after the lookup has read the keys -- inserts and
-  // the write list.  Caller's stream: gather, then the row update.  Without
-  // inputs_ready both helper streams start after everything earlier on the
-  // caller's stream.  With it (pipelined) they wait only for what they need:
-  // the inputs and the last other call on the table; the lookup also for the
-  // previous gather (which read rows/hit) and the previous row map (final
-  // keys); the side stream for the row update that last read this write-list
-  // buffer (the row map touches nothing a gather reads: keys, steps, scratch
-  // and the write list, never the values) -- so they overlap the previous
-  // step's gather and row update.
+  WbParams p = make_params(t, ids, e, n, step, stats);
+  p.n_fill = n_labeled;
+  p.fill_rows = rows;
+  p.fill_hit = hit;
+  // Two streams.  Side stream (high priority): the row map -- dedup, re-probe
+  // (which also gives the labeled ids' lookup: the rows their ids held before
+  // this step's inserts), placement with the lookup fill, write list.
+  // Caller's stream: the gather once the fill is done, then the row update
+  // once the row map is done.  Without inputs_ready the side stream starts
+  // after everything earlier on the caller's stream.  With it (pipelined) the
+  // side stream waits only for the inputs, the table's other calls and the row
+  // update that last read this step's write-list buffers -- so the row map
+  // overlaps the previous step's gather and row update -- and its fill waits
+  // for the previous gather (which may read the same rows/hit buffers).  The
+  // row map touches nothing a gather reads except rows/hit: keys, steps,
+  // scratch and the write list, never the values.
+  cudaEvent_t fill_after = nullptr;
   if (inputs_ready) {
     cudaEvent_t in = reinterpret_cast<cudaEvent_t>(inputs_ready);
-    if (cudaStreamWaitEvent(t->look, in, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->look, t->ev_user, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->look, t->ev_gather, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->look, t->ev_map, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(t->side, in, 0) != cudaSuccess ||
+    if (cudaStreamWaitEvent(t->side, in, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess)
       return MPZCH_ECUDA;
+    fill_after = t->ev_gather;
   } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
-             cudaStreamWaitEvent(t->look, t->ev_fork, 0) != cudaSuccess ||
-             cudaStreamWaitEvent(t->look, t->ev_user, 0) != cudaSuccess ||
              cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess ||
              cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess) {
     return MPZCH_ECUDA;
   }
-  if (n_labeled > 0) {
-    rc = enqueue_lookup(t, ids, n_labeled, rows, hit, t->look, false);
-    if (rc) return rc;
-  }
-  if (cudaEventRecord(t->ev_lookup, t->look) != cudaSuccess) return MPZCH_ECUDA;
-  rc = enqueue_row_map(t, p, t->side, t->ev_lookup);
+  rc = enqueue_row_map(t, p, t->side, fill_after, t->ev_lookup);
   if (rc) return rc;
   if (cudaEventRecord(t->ev_map, t->side) != cudaSuccess) return MPZCH_ECUDA;
-  // Caller's stream: gather once the lookup is done, then the row update once
-  // the row map is done (and after the gather has read the values).
+  // Caller's stream: gather once the lookup fill is done, then the row update
+  // once the row map is done (and after the gather has read the values).
   if (n_labeled > 0) {
     if (cudaStreamWaitEvent(st, t->ev_lookup, 0) != cudaSuccess) return MPZCH_ECUDA;
     rc = enqueue_gather(t, rows, hit, n_labeled, ao_table, ao_nrows, ao_dim, ao_rows, out, st,
@@ -1061,8 +1100,16 @@ int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows
 namespace {
 // Row export: the staged kernel (shared-memory double buffering) for dim 512
 // or 1024 with a 16-byte aligned q, the register kernel for every other shape.
+int tier_flush(mpzch_table* t, cudaStream_t st) {
+  if (t->tier_rows <= 0) return MPZCH_OK;
+  return launch(k_tier_flush, row_grid(t->tier_rows, t->row_blocks_per_sm), kBlock, st, false,
+                t->tier, t->tier_rows, reinterpret_cast<float4*>(t->M), t->D / 4);
+}
+
 int launch_export(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n, int8_t* q,
                   float* scale, int64_t* keys_out, int64_t* last_out, cudaStream_t st) {
+  // a tiered table's export reads host rows: cached rows are written back first
+  if (int rc = tier_flush(t, st)) return rc;
   const long long* dn = reinterpret_cast<const long long*>(dev_n);
   const float4* M = reinterpret_cast<const float4*>(t->M);
   long long* ko = reinterpret_cast<long long*>(keys_out);
@@ -1248,6 +1295,67 @@ int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, int32_t npha
   return MPZCH_OK;
 }
 
+namespace {
+// Replaces the tier by one of `rows` slots (0 = none), after writing every
+// cached row back; the device is synchronised around the change.
+int set_tier_rows(mpzch_table* t, int64_t rows) {
+  if (rows < 0 || rows > t->C || (rows & (rows - 1)) != 0 || (rows > 0 && !t->values_on_host) ||
+      !on_device(t))
+    return MPZCH_EINVAL;
+  if (t->tier_rows > 0) {
+    if (tier_flush(t, nullptr) != MPZCH_OK || cudaDeviceSynchronize() != cudaSuccess)
+      return MPZCH_ECUDA;
+  } else if (cudaDeviceSynchronize() != cudaSuccess) {
+    return MPZCH_ECUDA;
+  }
+  dev_free(t->tier.cache);
+  dev_free(t->tier.owner);
+  dev_free(t->tier.won);
+  dev_free(t->tier.claim);
+  t->tier = Tier{};
+  t->tier_rows = 0;
+  if (rows == 0) return MPZCH_OK;
+  Tier tr{};
+  int rc = dev_alloc((void**)&tr.cache, (size_t)rows * t->D * sizeof(float));
+  if (!rc) rc = dev_alloc((void**)&tr.owner, rows * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&tr.won, rows * sizeof(long long));
+  if (!rc) rc = dev_alloc((void**)&tr.claim, rows * sizeof(unsigned long long));
+  if (!rc && (cudaMemset(tr.owner, 0xFF, rows * sizeof(int32_t)) != cudaSuccess ||
+              cudaMemset(tr.won, 0xFF, rows * sizeof(long long)) != cudaSuccess ||
+              cudaMemset(tr.claim, 0, rows * sizeof(unsigned long long)) != cudaSuccess ||
+              cudaDeviceSynchronize() != cudaSuccess))
+    rc = MPZCH_ECUDA;
+  if (rc) {
+    cudaGetLastError();
+    dev_free(tr.cache);
+    dev_free(tr.owner);
+    dev_free(tr.won);
+    dev_free(tr.claim);
+    return rc;
+  }
+  tr.mask = (uint32_t)(rows - 1);
+  t->tier = tr;
+  t->tier_rows = rows;
+  return MPZCH_OK;
+}
+}  // namespace
+
+int mpzch_tier_sync(mpzch_table* t, int32_t discard, void* stream) {
+  if (!t || (discard != 0 && discard != 1) || !on_device(t)) return MPZCH_EINVAL;
+  if (t->tier_rows <= 0) return MPZCH_OK;
+  cudaStream_t st = S(stream);
+  int rc = join_side(t, st);
+  if (rc) return rc;
+  if (discard) {
+    rc = cudaMemsetAsync(t->tier.owner, 0xFF, t->tier_rows * sizeof(int32_t), st) == cudaSuccess
+             ? MPZCH_OK
+             : MPZCH_ECUDA;
+  } else {
+    rc = tier_flush(t, st);
+  }
+  return mark_user(t, st, rc);
+}
+
 int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
   if (!t) return MPZCH_EINVAL;
   if (option == MPZCH_OPT_SIDE_PRIORITY) {
@@ -1285,6 +1393,7 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     t->bulk_blocks = (int)value;
     return MPZCH_OK;
   }
+  if (option == MPZCH_OPT_HBM_CACHE_ROWS) return set_tier_rows(t, value);
   if (option == MPZCH_OPT_WRITE_LIST) {
     if (value != 0 && value != 1) return MPZCH_EINVAL;
     t->emit_list = (int)value;
@@ -1310,6 +1419,7 @@ int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
     case MPZCH_OPT_BULK_BLOCKS: *value = t->bulk_blocks; break;
     case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
     case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
+    case MPZCH_OPT_HBM_CACHE_ROWS: *value = t->tier_rows; break;
     default: return MPZCH_EINVAL;
   }
   return MPZCH_OK;

@@ -203,12 +203,14 @@ MPZCH_API int mpzch_writeback(mpzch_table* t, const int64_t* ids, const float* e
  *   mpzch_writeback(ids, e, n, step, dev_stats);
  * rows/hit/out/ao_* as in those calls (may be NULL when n_labeled == 0).
  *
- * Inside, the lookup runs on a highest-priority stream of the table and the
- * rest of the row map (dedup, refresh, inserts) on a second stream
- * (MPZCH_OPT_SIDE_PRIORITY); the gather and the row update run on `stream`,
- * the gather once the lookup is done and the row update once the row map is
- * done.  Later work on `stream` is ordered after all of it (rows,
- * hit, out, stats and the table are complete there).
+ * Inside, the row map (dedup, refresh, inserts) runs on a second stream of
+ * the table (MPZCH_OPT_SIDE_PRIORITY).  Its re-probe of the distinct ids also
+ * gives the lookup: rows/hit of the labeled positions are the rows their ids
+ * held before this step's inserts, filled in by the first placement pass.
+ * The gather and the row update run on `stream`, the gather once the lookup
+ * fill is done and the row update once the row map is done.  Later work on
+ * `stream` is ordered after all of it (rows, hit, out, stats and the table are
+ * complete there).
  *
  * inputs_ready: NULL, or a cudaEvent_t (as void*) recorded after ids, e and
  * ao_rows of this step were written.  With NULL the step starts after all
@@ -429,9 +431,30 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * that evicts an id written earlier in the same step cancels that id's entry;
  * 0 = one more kernel builds the list after all placements. */
 #define MPZCH_OPT_WRITE_LIST 9
+/* MPZCH_OPT_HBM_CACHE_ROWS (tables with MPZCH_VALUES_IN_HOST_MEMORY only):
+ * keep an HBM cache of this many rows (a power of two <= capacity; 0 = none,
+ * the default) in front of the host-memory values -- the hot/cold tier (Memory
+ * Layer section 2: the 512-d table is sharded across GPU and CPU).  Row r can
+ * live in cache slot r mod H; the cache is write-back.  In each Writeback a
+ * written row keeps its slot, or the smallest written row whose slot's owner
+ * was not written takes it (the old owner's value is written back to the host
+ * first); reads take a row from the cache when it holds it.  Every value read
+ * or written is exactly that of a table without the cache.  Changing the size
+ * writes every cached row back and synchronises the device.  Values read
+ * through mpzch_state_views are the host rows: call mpzch_tier_sync first.
+ * Steps of a tiered table must stay below 2^31. */
+#define MPZCH_OPT_HBM_CACHE_ROWS 10
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 /* Current value of an option (MPZCH_EINVAL for an unknown option). */
 MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);
+
+/* Hot/cold tier (MPZCH_OPT_HBM_CACHE_ROWS), on `stream`: discard = 0 writes
+ * every cached row back to its host row (the cache stays valid; do this
+ * before reading values through mpzch_state_views); discard = 1 empties the
+ * cache without writing back (after the caller replaced the host values, e.g.
+ * a restore).  A table without a cache: no-op.  The int8 export writes the
+ * cache back by itself. */
+MPZCH_API int mpzch_tier_sync(mpzch_table* t, int32_t discard, void* stream);
 
 /* Learning rate of the Writeback step for the following calls (Memory Layer
  * section 2, Writeback paragraph: the exact step is SGD at rate 1 on

@@ -54,6 +54,8 @@ def make_pair(w: inputs.Workload, track_all: bool = True, track_rows: Optional[n
 
 
 def compare_state(tbl, orc, what: str, value_rows: Optional[np.ndarray] = None, values=True):
+    from hashed_sparse_table_b200 import binding
+    binding.mpzch_tier_sync(tbl.h)  # an HBM row cache writes its rows back (no-op without one)
     keys, last, M = tbl.state()
     ok, ol, _ = orc.state()
     assert_bitwise(keys.cpu().numpy(), ok, f"{what}: keys")

@@ -524,3 +524,39 @@ def test_pipelined_steps_with_the_separate_write_list_kernel(name):
     from gpu_harness import run_pipelined
     from hashed_sparse_table_b200 import binding
     run_pipelined(SCALED[name], options={binding.MPZCH_OPT_WRITE_LIST: 0})
+
+
+@pytest.mark.parametrize("wide", [0, 2])
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress"])
+def test_fused_step_claim_rounds_lookup_fill(name, wide):
+    """The train step's lookup comes from the re-probe; on the claim-round
+    insert path a kernel of its own fills it, followed by 0 or 2 grid-wide
+    rounds: rows, hit, features and state bit-exact every step."""
+    run_pair(SCALED[name].scaled(steps=8), fused_step=True, cluster=0, wide_rounds=wide)
+
+
+def test_fused_step_labeled_negative_ids():
+    """Negative ids among the labeled positions of a train step: rows -1, hit 0,
+    zero cached branch, the bad-key status, and the rest bit-exact."""
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c3_small"].scaled(steps=4)
+    tbl, orc = make_pair(w)
+    ao = inputs.author_table(w)
+    ao_d = torch.from_numpy(ao).cuda()
+    for t in range(w.steps):
+        ids = inputs.step_ids(w, t).copy()
+        ids[3::41] = -7
+        e = inputs.step_e(w, t, rows=ids.size)
+        lab = w.labeled
+        aor = inputs.author_rows(w, np.maximum(ids[:lab], 0))
+        st = torch.zeros(7, dtype=torch.int64, device="cuda")
+        rows, hit, out = tbl.train_step(torch.from_numpy(ids).cuda(), lab, torch.from_numpy(e).cuda(),
+                                        t, ao_d, torch.from_numpy(aor).cuda(), st)
+        _, orows, ohit = orc.lookup(ids[:lab])
+        oout = orc.gather_fused(orows, ohit, ao, aor)
+        orc.writeback(ids, e, t)
+        assert_bitwise(rows.cpu().numpy(), orows, f"step {t}: rows")
+        assert_bitwise(hit.cpu().numpy(), ohit, f"step {t}: hit")
+        assert_bitwise(out.cpu().numpy(), oout, f"step {t}: features")
+        assert tbl.status() & binding.MPZCH_STATUS_BADKEY
+    compare_state(tbl, orc, "after negative labeled ids")
