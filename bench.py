@@ -826,10 +826,15 @@ def run_sharded(args):
     apply_row_options(binding, shard.table, args)
     sent = {"lookup": 0, "writeback": 0}
 
+    # step t+1 is prepared (partitions, segment-size exchange) before step t
+    # finishes, so the sizes reach the host while step t runs
+    pending = {0: shard.prepare(ids_d[0], lab, e_d[0])}
+
     def step(t):
         tr = {}
-        shard.train_step(ids_d[t], lab, e_d[t % E], t, ao_d, aor_d[t], rows, hit, out, stats[t],
-                         trace=tr)
+        if t + 1 < total:
+            pending[t + 1] = shard.prepare(ids_d[t + 1], lab, e_d[(t + 1) % E])
+        shard.finish(pending.pop(t), t, ao_d, aor_d[t], rows, hit, out, stats[t], trace=tr)
         return tr
 
     for t in range(Pf + Wm):
@@ -880,7 +885,8 @@ def run_sharded(args):
             "config": config_dict({
                 "prefill_steps": Pf, "shards": world,
                 "parallelism": f"hash-owner sharding: one {W.capacity}-row shard per GPU, ids, "
-                               "e rows and lookup answers exchanged all-to-all (NCCL)"}),
+                               "e rows and lookup answers exchanged all-to-all (NCCL), segment "
+                               "sizes exchanged one step ahead"}),
             "gpu_launches": launches,
             "roofline": {"bound": "hbm", "kernel": "k_writeback", "achieved": wb_gbs,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",

@@ -18,6 +18,13 @@ order):
   4. send the lookup answers back all-to-all and combine them at their batch
      positions with the rank's always-on rows (kernel).
 
+prepare() does step 1 and starts the exchange of segment sizes (an
+all-to-all whose result is copied to pinned host memory asynchronously);
+finish() reads the sizes on the host and does the rest.  A caller that
+issues step t+1's prepare before step t's finish (every rank in the same
+order) never makes the host wait for the GPU in the middle of a step;
+train_step() is prepare + finish.
+
 Every step of the path runs in the library's kernels; this module only moves
 segments between ranks: torch.distributed ``all_to_all_single`` (NCCL on the
 GPUs), or ``LocalExchangeGroup`` for G shards on one GPU in one process.
@@ -43,9 +50,28 @@ class DistExchange:
     def sizes(self, send: torch.Tensor) -> torch.Tensor:
         """send: int64 [G, k] on this rank's device, row g for rank g.  Returns,
         on the host, [2, G, k]: what this rank sends and what it receives."""
+        return self.sizes_wait(self.sizes_async(send))
+
+    def sizes_async(self, send: torch.Tensor):
+        """Starts the exchange of `send` and its copy to pinned host memory;
+        sizes_wait returns the host tensor once the copy has landed."""
         recv = torch.empty_like(send)
         self.dist.all_to_all_single(recv, send, group=self.group)
-        return torch.stack([send, recv]).cpu()
+        both = torch.stack([send, recv])
+        if not both.is_cuda:
+            return both, None
+        host = torch.empty(both.shape, dtype=both.dtype, pin_memory=True)
+        host.copy_(both, non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        return host, ev
+
+    @staticmethod
+    def sizes_wait(handle) -> torch.Tensor:
+        host, ev = handle
+        if ev is not None:
+            ev.synchronize()
+        return host
 
     def all_to_all(self, send: torch.Tensor, send_splits: List[int],
                    recv_splits: List[int]) -> torch.Tensor:
@@ -99,6 +125,13 @@ class LocalExchange:
         self._done()
         return out
 
+    def sizes_async(self, send: torch.Tensor):
+        return self.sizes(send), None
+
+    @staticmethod
+    def sizes_wait(handle) -> torch.Tensor:
+        return handle[0]
+
     def all_to_all(self, send: torch.Tensor, send_splits: List[int],
                    recv_splits: List[int]) -> torch.Tensor:
         got = self._swap((send, send_splits))
@@ -148,24 +181,22 @@ class ShardedMpzch:
         combine, and no host read of segment sizes.  The counters are then
         those of that step; they differ from a multi-shard step's only in
         n_ids, which counts the batch's valid ids (no first dedup ran)."""
+        return self.finish(self.prepare(ids, n_labeled, e), step, ao_table, ao_rows, rows, hit,
+                           out, stats, trace)
+
+    def prepare(self, ids: torch.Tensor, n_labeled: int, e: torch.Tensor) -> "Prepared":
+        """Steps 1-2a of a sharded step: the partitions by owner (labeled ids;
+        distinct ids with their e rows packed) and the start of the segment-
+        size exchange.  Issuing the next step's prepare before this step's
+        finish lets the sizes reach the host while this step runs, so the host
+        never waits for the GPU in the middle of a step.  Every rank must issue
+        prepares and finishes in the same order (they are collectives)."""
+        if self.G == 1:
+            return Prepared(ids=ids, n_labeled=n_labeled, e=e)
         binding = self.binding
         G, dev, D = self.G, self.device, self.dim
-        if G == 1:
-            if stats is None:
-                stats = torch.empty(7, dtype=torch.int64, device=dev)
-            rows, hit, out = self.table.train_step(ids, n_labeled, e, step, ao_table, ao_rows,
-                                                   stats, rows=rows, hit=hit, out=out)
-            if trace is not None:
-                trace["sent_lookup"] = trace["sent_writeback"] = trace["recv_writeback"] = 0
-            return rows, hit, out, stats
         n = ids.numel()
         lab = ids[:n_labeled]
-        width = D + (0 if ao_table is None else ao_table.shape[1])
-        rows = torch.empty(n_labeled, dtype=torch.int32, device=dev) if rows is None else rows
-        hit = torch.empty(n_labeled, dtype=torch.uint8, device=dev) if hit is None else hit
-        out = torch.empty((n_labeled, width), dtype=torch.float32, device=dev) if out is None else out
-        stats = torch.empty(7, dtype=torch.int64, device=dev) if stats is None else stats
-        # 1. partitions by owner: labeled ids; distinct ids with their e rows
         counts = torch.empty((2, G), dtype=torch.int64, device=dev)
         ws = self._workspace(max(n, n_labeled))  # both partitions run in order on one stream
         l_ids = torch.empty(n_labeled, dtype=torch.int64, device=dev)
@@ -177,15 +208,36 @@ class ShardedMpzch:
         w_e = torch.empty((n, D), dtype=torch.float32, device=dev)
         binding.mpzch_owner_partition(uniq, G, w_ids, w_pos, counts[1], ws, src_pos=upos,
                                       dev_n=ucnt, e=e, e_out=w_e)
-        # 2. segment sizes, then ids and e rows
-        sz = self.ex.sizes(counts.t().contiguous()).tolist()  # [send|recv][peer][lookup|wb]
+        return Prepared(ids=ids, n_labeled=n_labeled, e=e, l_ids=l_ids, l_pos=l_pos, w_ids=w_ids,
+                        w_e=w_e, sizes=self.ex.sizes_async(counts.t().contiguous()))
+
+    def finish(self, prep: "Prepared", step: int, ao_table: Optional[torch.Tensor] = None,
+               ao_rows: Optional[torch.Tensor] = None, rows=None, hit=None, out=None, stats=None,
+               trace: Optional[dict] = None):
+        """Steps 2b-4 of a sharded step prepared by prepare()."""
+        binding = self.binding
+        G, dev, D = self.G, self.device, self.dim
+        n_labeled = prep.n_labeled
+        width = D + (0 if ao_table is None else ao_table.shape[1])
+        rows = torch.empty(n_labeled, dtype=torch.int32, device=dev) if rows is None else rows
+        hit = torch.empty(n_labeled, dtype=torch.uint8, device=dev) if hit is None else hit
+        out = torch.empty((n_labeled, width), dtype=torch.float32, device=dev) if out is None else out
+        stats = torch.empty(7, dtype=torch.int64, device=dev) if stats is None else stats
+        if G == 1:
+            self.table.train_step(prep.ids, n_labeled, prep.e, step, ao_table, ao_rows, stats,
+                                  rows=rows, hit=hit, out=out)
+            if trace is not None:
+                trace["sent_lookup"] = trace["sent_writeback"] = trace["recv_writeback"] = 0
+            return rows, hit, out, stats
+        # 2b. segment sizes on the host, then ids and e rows
+        sz = self.ex.sizes_wait(prep.sizes).tolist()  # [send|recv][peer][lookup|wb]
         s_l = [sz[0][g][0] for g in range(G)]
         r_l = [sz[1][g][0] for g in range(G)]
         s_w = [sz[0][g][1] for g in range(G)]
         r_w = [sz[1][g][1] for g in range(G)]
-        r_lids = self.ex.all_to_all(l_ids, s_l, r_l)
-        r_wids = self.ex.all_to_all(w_ids, s_w, r_w)
-        r_we = self.ex.all_to_all(w_e, s_w, r_w)
+        r_lids = self.ex.all_to_all(prep.l_ids, s_l, r_l)
+        r_wids = self.ex.all_to_all(prep.w_ids, s_w, r_w)
+        r_we = self.ex.all_to_all(prep.w_e, s_w, r_w)
         # 3. owner: lookup + gather before the Writeback
         r_rows, r_hit = self.table.lookup(r_lids)
         r_feat = self.table.gather_fused(r_rows, r_hit)
@@ -193,10 +245,20 @@ class ShardedMpzch:
         # 4. answers back in send order, placed at their batch positions
         b_rows = self.ex.all_to_all(r_rows, r_l, s_l)
         b_feat = self.ex.all_to_all(r_feat, r_l, s_l)
-        binding.mpzch_owner_combine(l_ids, l_pos, G, self.capacity, b_rows, b_feat, rows, hit, out,
-                                    ao_table, ao_rows, self.status)
+        binding.mpzch_owner_combine(prep.l_ids, prep.l_pos, G, self.capacity, b_rows, b_feat, rows,
+                                    hit, out, ao_table, ao_rows, self.status)
         if trace is not None:
             trace["sent_lookup"] = sum(s_l)
             trace["sent_writeback"] = sum(s_w)
             trace["recv_writeback"] = sum(r_w)
         return rows, hit, out, stats
+
+
+class Prepared:
+    """The partitioned buffers and the pending segment sizes of one sharded step."""
+
+    def __init__(self, ids, n_labeled, e, l_ids=None, l_pos=None, w_ids=None, w_e=None,
+                 sizes=None):
+        self.ids, self.n_labeled, self.e = ids, n_labeled, e
+        self.l_ids, self.l_pos, self.w_ids, self.w_e = l_ids, l_pos, w_ids, w_e
+        self.sizes = sizes

@@ -14,6 +14,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -104,7 +105,7 @@ class FakeTable:
         stats[:6] = torch.tensor([st[k] for k in keys], dtype=torch.int64)
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, lookahead=False):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
@@ -122,10 +123,22 @@ def _worker(rank, world, port, out):
         sh._ws = torch.empty(0, dtype=torch.uint8)
         ao = torch.from_numpy(ao_table())
         res = []
+
+        def prep(t):
+            ids, e, _ = rank_batch(t, rank)
+            return sh.prepare(torch.from_numpy(ids), LABELED, torch.from_numpy(e))
+
+        nxt = prep(0) if lookahead else None
         for t in range(STEPS):
             ids, e, aor = rank_batch(t, rank)
-            rows, hit, feats, st = sh.train_step(torch.from_numpy(ids), LABELED, torch.from_numpy(e),
-                                                 t, ao, torch.from_numpy(aor))
+            if lookahead:  # step t+1 is prepared (sizes exchanged) before step t finishes
+                cur = nxt
+                nxt = prep(t + 1) if t + 1 < STEPS else None
+                rows, hit, feats, st = sh.finish(cur, t, ao, torch.from_numpy(aor))
+            else:
+                rows, hit, feats, st = sh.train_step(torch.from_numpy(ids), LABELED,
+                                                     torch.from_numpy(e), t, ao,
+                                                     torch.from_numpy(aor))
             res.append((rows.numpy().copy(), hit.numpy().copy(), feats.numpy().copy(),
                         st.numpy().copy()))
         out[rank] = (res, sh.table.orc.state()[0], sh.table.orc.values())
@@ -140,11 +153,13 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_sharded_step_over_two_gloo_ranks_matches_the_sharded_oracle():
+@pytest.mark.parametrize("lookahead", [False, True])
+def test_sharded_step_over_two_gloo_ranks_matches_the_sharded_oracle(lookahead):
+    """train_step per step, and prepare(t+1) issued before finish(t)."""
     mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
-    mp.start_processes(_worker, args=(G, _free_port(), out), nprocs=G, start_method="spawn",
-                       join=True)
+    mp.start_processes(_worker, args=(G, _free_port(), out, lookahead), nprocs=G,
+                       start_method="spawn", join=True)
     so = oracle.ShardedOracle(G, C_S, D, P)
     ao = ao_table()
     evicted = 0
