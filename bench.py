@@ -103,6 +103,9 @@ def parse():
     ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
                     help="row kernels through registers or through shared memory with bulk "
                          "copies (default: the library's)")
+    ap.add_argument("--fused-step", type=int, default=None, choices=[0, 1],
+                    help="gather and row update of a train step as one kernel (1) or two (0) "
+                         "(default: the library's)")
     ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
                     help="cluster path: write list emitted at re-probe and placement, or built "
                          "by a separate kernel (default: the library's)")
@@ -115,6 +118,8 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
+    if args.fused_step is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP, args.fused_step)
     if args.write_list is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WRITE_LIST,
                                  1 if args.write_list == "emit" else 0)
@@ -129,10 +134,17 @@ def apply_row_options(binding, tbl, args):
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_L2_HINT_ROWS, args.l2_hint)
 
 
-def row_update_kernel(binding, tbl) -> str:
+def row_update_kernel(binding, tbl, args) -> str:
     """Name of the row-update kernel the table launches for this workload."""
+    if args.host_values and args.hbm_cache_rows:
+        return "k_tier_update"
     bulk = binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_ROW_KERNEL) == 1
-    return "k_writeback_bulk" if bulk else "k_writeback"
+    if bulk:
+        return "k_writeback_bulk"
+    fused = binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP) == 1
+    if fused and not args.host_values and not args.separate_calls:
+        return "k_gather_update"
+    return "k_writeback"
 
 
 def host_cpu():
@@ -412,11 +424,15 @@ def run_ours(args):
     g_ms, _ = trace["gather"]
     g_bytes = n_hit_lab * 4 * D + K * lab * (4 * A + 4 * (D + A) + 9)
     peak, peak_kind = load_peaks()
+    wb_kernel = row_update_kernel(binding, tbl, args)
+    wb_traffic = ROW_UPDATE_TRAFFIC.get(wb_kernel, (None, None))
+    if wb_kernel == "k_gather_update":
+        # one kernel does the gather and the row update (traced as the row update):
+        # its algorithmic bytes are both
+        wb_bytes += g_bytes
+        g_bytes, g_ms = 0, 0.0
     wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
     gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
-
-    wb_kernel = row_update_kernel(binding, tbl)
-    wb_traffic = ROW_UPDATE_TRAFFIC.get(wb_kernel, (None, None))
     serving = None if args.no_serving else run_export_and_serve(tbl, binding, torch, dev, peak)
 
     shard_k = None

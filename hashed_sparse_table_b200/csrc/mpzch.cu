@@ -265,7 +265,12 @@ struct mpzch_table {
   // write lists (row, position of e), two buffers used by alternate Writebacks
   int32_t* wrow[2] = {nullptr, nullptr};
   int32_t* wpos[2] = {nullptr, nullptr};
-  int32_t* wcnt = nullptr;  // device int32[4]: list lengths [0..1], entries taken [2..3]
+  int32_t* wcnt = nullptr;  // device int32[6]: list lengths [0..1], entries taken [2..3],
+                            // gather items finished [4..5] (per write-list buffer)
+  uint32_t* gmark[2] = {nullptr, nullptr};  // rows a step's gather reads (fused kernel)
+  int fuse_gather_update = 1;  // train step: gather and row update as one kernel
+  const void* prev_rows = nullptr;  // rows/hit buffers of the previous train step
+  const void* prev_hit = nullptr;
   int wset = 0;             // buffer of the next Writeback
   // small device words
   StepCtr* ctr = nullptr;
@@ -350,6 +355,7 @@ void free_all(mpzch_table* t) {
   dev_free(t->tier.claim);
   dev_free(t->ctr);
   dev_free(t->wcnt);
+  for (auto& g : t->gmark) dev_free(g), g = nullptr;
   dev_free(t->stats);
   dev_free(t->status);
   dev_free(t->sel_masks);
@@ -480,7 +486,7 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
-                                           stats, t->status, nullptr, nullptr);
+                                           stats, t->status, nullptr, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -632,6 +638,9 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.snext = t->snext;
   p.wcount = t->wcnt + t->wset;
   p.wtake = t->wcnt + 2 + t->wset;
+  p.gdone = t->wcnt + 4 + t->wset;
+  p.gmark = nullptr;  // set by a fused train step
+  p.gtag = (uint32_t)(step + 1);
   p.emit = (t->cluster_insert && t->emit_list) ? 1 : 0;
   p.wentry = t->wentry;
   // emit: the distinct-id arrays are the list; otherwise k_write_list fills
@@ -660,7 +669,7 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     PhaseScope ps(t, PH_DEDUP, st);
     rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false,
                 p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status,
-                p.wcount, p.wtake);
+                p.wcount, p.wtake, p.gdone);
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
   }
@@ -842,7 +851,7 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
-                                           dev_status, nullptr, nullptr);
+                                           dev_status, nullptr, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -886,7 +895,8 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   if (!rc) rc = dev_alloc((void**)&t->shead, capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->wentry, capacity * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
-  if (!rc) rc = dev_alloc((void**)&t->wcnt, 4 * sizeof(int32_t));
+  if (!rc) rc = dev_alloc((void**)&t->wcnt, 6 * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->gmark[i], capacity * sizeof(uint32_t));
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
   if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
   const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
@@ -906,7 +916,9 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
                cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) ==
                    cudaSuccess) &&
               cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
-              cudaMemsetAsync(t->wcnt, 0, 4 * sizeof(int32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->wcnt, 0, 6 * sizeof(int32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->gmark[0], 0, capacity * sizeof(uint32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->gmark[1], 0, capacity * sizeof(uint32_t), st) == cudaSuccess &&
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
@@ -1039,17 +1051,23 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
   p.n_fill = n_labeled;
   p.fill_rows = rows;
   p.fill_hit = hit;
+  // The gather and the row update run as one kernel (register row kernels,
+  // values in device memory): the fill marks the rows the gather reads.
+  const bool fused = t->fuse_gather_update && n_labeled > 0 && t->row_kernel == 0 &&
+                     t->tier_rows == 0 && !t->values_on_host;
+  if (fused) p.gmark = t->gmark[t->wset];
   // Two streams.  Side stream (high priority): the row map -- dedup, re-probe
   // (which also gives the labeled ids' lookup: the rows their ids held before
   // this step's inserts), placement with the lookup fill, write list.
   // Caller's stream: the gather once the fill is done, then the row update
-  // once the row map is done.  Without inputs_ready the side stream starts
-  // after everything earlier on the caller's stream.  With it (pipelined) the
-  // side stream waits only for the inputs, the table's other calls and the row
-  // update that last read this step's write-list buffers -- so the row map
-  // overlaps the previous step's gather and row update -- and its fill waits
-  // for the previous gather (which may read the same rows/hit buffers).  The
-  // row map touches nothing a gather reads except rows/hit: keys, steps,
+  // once the row map is done (fused: one kernel once the row map is done).
+  // Without inputs_ready the side stream starts after everything earlier on
+  // the caller's stream.  With it (pipelined) the side stream waits only for
+  // the inputs, the table's other calls and the row update that last read this
+  // step's write-list buffers -- so the row map overlaps the previous step's
+  // gather and row update -- and, when this step reuses the previous step's
+  // rows/hit buffers, its fill waits for the previous gather, which reads them.
+  // The row map touches nothing a gather reads except rows/hit: keys, steps,
   // scratch and the write list, never the values.
   cudaEvent_t fill_after = nullptr;
   if (inputs_ready) {
@@ -1058,7 +1076,7 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
         cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess ||
         cudaStreamWaitEvent(t->side, t->ev_update[t->wset], 0) != cudaSuccess)
       return MPZCH_ECUDA;
-    fill_after = t->ev_gather;
+    if (rows == t->prev_rows || hit == t->prev_hit) fill_after = t->ev_gather;
   } else if (cudaEventRecord(t->ev_fork, st) != cudaSuccess ||
              cudaStreamWaitEvent(t->side, t->ev_fork, 0) != cudaSuccess ||
              cudaStreamWaitEvent(t->side, t->ev_user, 0) != cudaSuccess) {
@@ -1067,6 +1085,29 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
   rc = enqueue_row_map(t, p, t->side, fill_after, t->ev_lookup);
   if (rc) return rc;
   if (cudaEventRecord(t->ev_map, t->side) != cudaSuccess) return MPZCH_ECUDA;
+  t->prev_rows = rows;
+  t->prev_hit = hit;
+  if (fused) {
+    if (cudaStreamWaitEvent(st, t->ev_map, 0) != cudaSuccess) return MPZCH_ECUDA;
+    {
+      PhaseScope ps(t, PH_WRITEBACK, st);
+      const bool has_ao = ao_table != nullptr;
+      rc = launch(k_gather_update, row_grid(n, t->row_blocks_per_sm), kBlock, st, false,
+                  (const int32_t*)rows, (const uint8_t*)hit, (int32_t)n_labeled,
+                  reinterpret_cast<float4*>(t->M), t->C, t->D / 4,
+                  reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
+                  ao_rows, reinterpret_cast<float4*>(out), (const int32_t*)p.wrow,
+                  (const int32_t*)p.wpos, (const int32_t*)p.wcount, p.e, t->eta,
+                  (const uint32_t*)p.gmark, p.gtag, p.wtake, p.gdone, t->status);
+      if (rc) return rc;
+    }
+    if (cudaEventRecord(t->ev_gather, st) != cudaSuccess ||
+        cudaEventRecord(t->ev_update[t->wset], st) != cudaSuccess)
+      return MPZCH_ECUDA;
+    t->wset ^= 1;
+    t->last_step = step;
+    return MPZCH_OK;
+  }
   // Caller's stream: gather once the lookup fill is done, then the row update
   // once the row map is done (and after the gather has read the values).
   if (n_labeled > 0) {
@@ -1394,6 +1435,11 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     return MPZCH_OK;
   }
   if (option == MPZCH_OPT_HBM_CACHE_ROWS) return set_tier_rows(t, value);
+  if (option == MPZCH_OPT_FUSED_STEP) {
+    if (value != 0 && value != 1) return MPZCH_EINVAL;
+    t->fuse_gather_update = (int)value;
+    return MPZCH_OK;
+  }
   if (option == MPZCH_OPT_WRITE_LIST) {
     if (value != 0 && value != 1) return MPZCH_EINVAL;
     t->emit_list = (int)value;
@@ -1420,6 +1466,7 @@ int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
     case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
     case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
     case MPZCH_OPT_HBM_CACHE_ROWS: *value = t->tier_rows; break;
+    case MPZCH_OPT_FUSED_STEP: *value = t->fuse_gather_update; break;
     default: return MPZCH_EINVAL;
   }
   return MPZCH_OK;

@@ -78,6 +78,17 @@ __device__ __forceinline__ void set_status(int32_t* st, int bits) {
   if (st) atomicOr(st, bits);
 }
 
+// Waits on other warps or on copies in flight give up after this long and set
+// MPZCH_STATUS_TIMEOUT (far beyond any legitimate wait).
+constexpr int kStTimeout = 16;
+constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Programmatic dependent launch.  pdl_enter waits until every earlier grid of
 // the stream has completed and its memory is visible; every kernel calls it
 // first, so nothing is read before the producer has finished.  pdl_trigger
@@ -265,7 +276,7 @@ constexpr int kDedupThreads = kTile;  // one tile position per thread
 __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake) {
+    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake, int32_t* gdone) {
   pdl_enter();
   __shared__ unsigned long long s_key[kTileHash];
   __shared__ uint32_t s_pos[kTileHash];
@@ -278,6 +289,7 @@ __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
   if (wcount && blockIdx.x == 0 && threadIdx.x == 0) *wcount = 0;
   if (wtake && blockIdx.x == 0 && threadIdx.x == 0) *wtake = 0;
+  if (gdone && blockIdx.x == 0 && threadIdx.x == 0) *gdone = 0;
   for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
     s_key[j] = kEmptyKey;
     s_pos[j] = kNoPos;
@@ -542,7 +554,8 @@ struct WbParams {
   int32_t* wrow;
   int32_t* wpos;
   int32_t* wcount;
-  int32_t* wtake;  // entries of the list already taken by the bulk row update
+  int32_t* wtake;  // entries of the list already taken by the bulk row update / fused kernel
+  int32_t* gdone;  // gather items finished (fused gather + row update)
   // emit = 1 (cluster path): the write list is the distinct-id arrays of this
   // call themselves -- entry u = (urow[u], upos[u]), wrow/wpos point at them
   // and *wcount is set to the number of distinct ids -- so nothing is
@@ -561,6 +574,10 @@ struct WbParams {
   int64_t n_fill;
   int32_t* fill_rows;
   uint8_t* fill_hit;
+  // rows the step's gather reads (hit rows of the filled positions) get
+  // gmark[row] = gtag when gmark is set (fused gather + row update)
+  uint32_t* gmark;
+  uint32_t gtag;
 };
 
 // Lookup result of batch position i < n_fill: the row its id held before the
@@ -571,6 +588,7 @@ __device__ __forceinline__ void fill_lookup(const WbParams& p, int64_t i) {
   const int32_t r = s >= 0 ? __ldcg(p.hrow + s) : -1;
   p.fill_rows[i] = r;
   p.fill_hit[i] = r >= 0 ? 1 : 0;
+  if (p.gmark && r >= 0) p.gmark[r] = p.gtag;
 }
 
 // urow value of a distinct id that was placed and then evicted again later in
@@ -1488,6 +1506,148 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
+// Fused gather + row update of a train step, one launch.  Work items: the
+// n_gather gather positions first, then the write list in reverse order (so
+// the rows of the labeled ids, listed first, come last).  Warps take 32 items
+// at a time from a counter.  A warp publishes each chunk's finished gather
+// items (release add); a row-update item whose row this step's gather reads
+// (gmark[row] == gtag) first waits until all gather items are published
+// (acquire poll) -- the gather reads e_hat before the row update overwrites
+// it.  Every gather item is taken before any row-update item, by warps that
+// are running, so the wait ends; it has a time limit all the same
+// (MPZCH_STATUS_TIMEOUT, and the kernel returns).  Same results as
+// k_gather_fused followed by k_writeback.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void atom_add_release(int32_t* p, int32_t v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int32_t ld_acquire(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(kBlock, 4) k_gather_update(
+    const int32_t* __restrict__ rows, const uint8_t* __restrict__ hit, int32_t n_gather,
+    float4* __restrict__ M, int64_t C, int D4, const float4* __restrict__ ao, int64_t ao_n, int A4,
+    const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
+    const int32_t* __restrict__ wrow, const int32_t* __restrict__ wpos, const int32_t* wcount,
+    const float4* __restrict__ e, float eta, const uint32_t* __restrict__ gmark, uint32_t gtag,
+    int32_t* take, int32_t* gdone, int32_t* status) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int32_t W = *wcount;
+  const int32_t total = n_gather + W;
+  const int W4 = D4 + A4;
+  bool gather_done = false;  // this warp has seen every gather item published
+  for (;;) {
+    int32_t base = 0;
+    if (lane == 0) base = atomicAdd(take, 32);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (base >= total) break;
+    const int32_t end = base + 32 < total ? base + 32 : total;
+    // gather items of the chunk
+    const int32_t gend = end < n_gather ? end : n_gather;
+    for (int32_t i = base; i < gend; ++i) {
+      const int32_t r = rows[i];
+      bool h = hit[i] != 0;
+      if (h && (r < 0 || (int64_t)r >= C)) {
+        if (lane == 0) set_status(status, kStBadRow);
+        h = false;
+      }
+      int32_t a = 0;
+      bool has_a = A4 > 0;
+      if (has_a) {
+        a = ao_rows[i];
+        if (a < 0 || (int64_t)a >= ao_n) {
+          if (lane == 0) set_status(status, kStBadAo);
+          has_a = false;
+        }
+      }
+      const float4* src = M + (int64_t)(h ? r : 0) * D4;
+      const float4* asrc = ao + (int64_t)a * A4;
+      float4* dst = out + (int64_t)i * W4;
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int cb = 0; cb < W4; cb += 4 * 32) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = cb + u * 32 + lane;
+          v[u] = z;
+          if (c < D4) {
+            if (h) v[u] = __ldcs(src + c);
+          } else if (c < W4 && has_a) {
+            v[u] = __ldcs(asrc + (c - D4));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = cb + u * 32 + lane;
+          if (c < W4) __stcs(dst + c, v[u]);
+        }
+      }
+    }
+    if (gend > base) {
+      __syncwarp();  // every lane's loads of the chunk have returned
+      if (lane == 0) atom_add_release(gdone, gend - base);
+    }
+    // row-update items of the chunk (write list in reverse)
+    for (int32_t j = (base > n_gather ? base : n_gather); j < end; ++j) {
+      const int32_t w = W - 1 - (j - n_gather);
+      const int32_t r = wrow[w];
+      if (r < 0) continue;  // tombstone
+      if (!gather_done && gmark[r] == gtag) {
+        bool ok = true;
+        if (lane == 0) {
+          if (ld_acquire(gdone) < n_gather) {
+            const uint64_t t0 = global_ns();
+            while (ld_acquire(gdone) < n_gather) {
+              if (global_ns() - t0 > kWaitLimitNs) {
+                ok = false;
+                break;
+              }
+            }
+          }
+        }
+        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+        if (!ok) {
+          if (lane == 0) set_status(status, kStTimeout);
+          return;
+        }
+        __syncwarp();
+        gather_done = true;
+      }
+      float4* m = M + (int64_t)r * D4;
+      const float4* ev = e + (int64_t)wpos[w] * D4;
+      for (int cb = 0; cb < D4; cb += 4 * 32) {
+        float4 a4[4], b4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = cb + q * 32 + lane;
+          if (c < D4) {
+            a4[q] = __ldcs(m + c);
+            b4[q] = __ldcs(ev + c);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = cb + q * 32 + lane;
+          if (c < D4) {
+            float4 o;
+            o.x = __fsub_rn(a4[q].x, __fmul_rn(eta, __fsub_rn(a4[q].x, b4[q].x)));
+            o.y = __fsub_rn(a4[q].y, __fmul_rn(eta, __fsub_rn(a4[q].y, b4[q].y)));
+            o.z = __fsub_rn(a4[q].z, __fmul_rn(eta, __fsub_rn(a4[q].z, b4[q].z)));
+            o.w = __fsub_rn(a4[q].w, __fmul_rn(eta, __fsub_rn(a4[q].w, b4[q].w)));
+            __stcs(m + c, o);
+          }
+        }
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Bulk-copy row kernels.  A warp keeps kBulkStages rows in flight: one lane
 // issues 1-D bulk copies (cp.async.bulk, global -> shared, no multicast) of
 // each row into the warp's own shared-memory stage, completed on that stage's
@@ -1499,18 +1659,10 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
 // sets MPZCH_STATUS_TIMEOUT, waits (again with a limit) for its copies still
 // in flight and returns.
 // ---------------------------------------------------------------------------
-constexpr int kStTimeout = 16;
 constexpr int kBulkStages = 3;
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s: far beyond any row copy
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 // L2 eviction-priority policies for the cache-hinted accesses.

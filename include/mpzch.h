@@ -444,6 +444,12 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * through mpzch_state_views are the host rows: call mpzch_tier_sync first.
  * Steps of a tiered table must stay below 2^31. */
 #define MPZCH_OPT_HBM_CACHE_ROWS 10
+/* MPZCH_OPT_FUSED_STEP: 1 (default) = mpzch_train_step runs its gather and
+ * its row update as one kernel (when the values are in device memory and the
+ * register row kernels are selected): warps take the gather positions first,
+ * then the write list; the update of a row the step's gather reads waits until
+ * every gather position is done.  0 = two kernels.  Results are identical. */
+#define MPZCH_OPT_FUSED_STEP 11
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 /* Current value of an option (MPZCH_EINVAL for an unknown option). */
 MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);

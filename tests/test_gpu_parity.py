@@ -560,3 +560,57 @@ def test_fused_step_labeled_negative_ids():
         assert_bitwise(out.cpu().numpy(), oout, f"step {t}: features")
         assert tbl.status() & binding.MPZCH_STATUS_BADKEY
     compare_state(tbl, orc, "after negative labeled ids")
+
+
+@pytest.mark.parametrize("name", ["c3_small", "c4_stress", "nonpow2"])
+def test_two_kernel_step_bit_exact(name):
+    """MPZCH_OPT_FUSED_STEP = 0: gather and row update as two kernels, with
+    separate and pipelined steps."""
+    from gpu_harness import run_pipelined
+    from hashed_sparse_table_b200 import binding
+    opts = {binding.MPZCH_OPT_FUSED_STEP: 0}
+    run_pair(SCALED[name], fused_step=True, options=opts)
+    run_pipelined(SCALED[name], options=opts)
+
+
+@pytest.mark.parametrize("fused", [1, 0])
+def test_pipelined_steps_sharing_rows_and_hit_buffers(fused):
+    """Pipelined steps that reuse one rows/hit pair (each with its own fused
+    output): a step's lookup fill must wait for the previous step's gather,
+    which reads those buffers.  Every step's features and the final rows/hit
+    and state match the oracle."""
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c3_small"].scaled(steps=10)
+    tbl, orc = make_pair(w)
+    binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP, fused)
+    dev = tbl.device
+    ao = inputs.author_table(w)
+    ao_d = torch.from_numpy(ao).to(dev)
+    lab = w.labeled
+    host = [(inputs.step_ids(w, t), inputs.step_e(w, t)) for t in range(w.steps)]
+    aor = [inputs.author_rows(w, h[0][:lab]) for h in host]
+    dev_in = [(torch.from_numpy(i).to(dev), torch.from_numpy(e).to(dev),
+               torch.from_numpy(a).to(dev)) for (i, e), a in zip(host, aor)]
+    rows = torch.empty(lab, dtype=torch.int32, device=dev)
+    hit = torch.empty(lab, dtype=torch.uint8, device=dev)
+    outs = [torch.empty((lab, w.dim + ao.shape[1]), dtype=torch.float32, device=dev)
+            for _ in range(w.steps)]
+    stats = [torch.empty(7, dtype=torch.int64, device=dev) for _ in range(w.steps)]
+    ready = torch.cuda.Event()
+    ready.record()
+    for t in range(w.steps):
+        ids_d, e_d, aor_d = dev_in[t]
+        binding.mpzch_train_step(tbl.h, ids_d, lab, e_d, t, rows, hit, outs[t], ao_d, aor_d,
+                                 stats[t], inputs_ready=ready)
+    torch.cuda.synchronize()
+    for t in range(w.steps):
+        ids, e = host[t]
+        _, orows, ohit = orc.lookup(ids[:lab])
+        oout = orc.gather_fused(orows, ohit, ao, aor[t])
+        orc.writeback(ids, e, t)
+        assert_bitwise(outs[t].cpu().numpy(), oout, f"step {t}: features")
+        if t == w.steps - 1:
+            assert_bitwise(rows.cpu().numpy(), orows, "last rows")
+            assert_bitwise(hit.cpu().numpy(), ohit, "last hit")
+    compare_state(tbl, orc, "shared rows/hit buffers")
+    assert tbl.status() == 0
