@@ -106,6 +106,8 @@ def parse():
     ap.add_argument("--fused-step", type=int, default=None, choices=[0, 1],
                     help="gather and row update of a train step as one kernel (1) or two (0) "
                          "(default: the library's)")
+    ap.add_argument("--place-merged", type=int, default=None, choices=[0, 1],
+                    help="cluster path: lone ids and clusters placed by one kernel (1) or two (0)")
     ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
                     help="cluster path: write list emitted at re-probe and placement, or built "
                          "by a separate kernel (default: the library's)")
@@ -118,6 +120,8 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
+    if args.place_merged is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_PLACE_MERGED, args.place_merged)
     if args.fused_step is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP, args.fused_step)
     if args.write_list is not None:

@@ -276,7 +276,8 @@ constexpr int kDedupThreads = kTile;  // one tile position per thread
 __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake, int32_t* gdone) {
+    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake, int32_t* gdone,
+    int32_t* gtake) {
   pdl_enter();
   __shared__ unsigned long long s_key[kTileHash];
   __shared__ uint32_t s_pos[kTileHash];
@@ -290,6 +291,7 @@ __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
   if (wcount && blockIdx.x == 0 && threadIdx.x == 0) *wcount = 0;
   if (wtake && blockIdx.x == 0 && threadIdx.x == 0) *wtake = 0;
   if (gdone && blockIdx.x == 0 && threadIdx.x == 0) *gdone = 0;
+  if (gtake && blockIdx.x == 0 && threadIdx.x == 0) *gtake = 0;
   for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
     s_key[j] = kEmptyKey;
     s_pos[j] = kNoPos;
@@ -556,6 +558,7 @@ struct WbParams {
   int32_t* wcount;
   int32_t* wtake;  // entries of the list already taken by the bulk row update / fused kernel
   int32_t* gdone;  // gather items finished (fused gather + row update)
+  int32_t* gtake;  // gather items taken (fused gather + row update)
   // emit = 1 (cluster path): the write list is the distinct-id arrays of this
   // call themselves -- entry u = (urow[u], upos[u]), wrow/wpos point at them
   // and *wcount is set to the number of distinct ids -- so nothing is
@@ -1410,6 +1413,58 @@ __global__ void __launch_bounds__(kBlock) k_place_multi(WbParams p) {
   if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
 }
 
+// Both placement passes in one launch (and the lookup fill): each warp takes
+// kPlaceKeys missing keys, lanes 0..kPlaceKeys-1 run the lone-key check of one
+// key each (placing lone keys), and then the whole warp places, one after
+// another, the clusters whose heads it found.  A lone key's window touches no
+// slot of any cluster and the clusters' slot sets are disjoint, so the two
+// kinds of placement run side by side without ordering.  Clusters beyond the
+// warp path are listed for k_insert_finish, as with k_place_multi.
+constexpr int kPlaceKeys = 8;
+
+__global__ void __launch_bounds__(kBlock) k_place_all(WbParams p) {
+  pdl_enter();
+  __shared__ long long sm[33];
+  __shared__ WarpCluster s_warp[kBlock / 32];
+  const int32_t N = p.ctr->cnt[0];
+  const bool ring_may_be_covered = (int64_t)N * p.g.P >= p.g.C;
+  const int lane = threadIdx.x & 31;
+  WarpCluster& sw = s_warp[threadIdx.x >> 5];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.stats->n_inserted = N;
+    if (p.emit) {  // no k_write_list on this path: the list is the distinct-id arrays
+      p.stats->n_unique = p.ctr->n_unique;
+      *p.wcount = p.ctr->n_unique;
+    }
+    if (N > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
+  }
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_fill; i += stride)
+    fill_lookup(p, i);
+  long long evicted = 0;
+  if (!ring_may_be_covered) {
+    const int64_t warps = stride >> 5;
+    for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+         w * kPlaceKeys < N; w += warps) {
+      const int64_t m = w * kPlaceKeys + lane;
+      int64_t h = 0;
+      const bool head = lane < kPlaceKeys && m < N && place_lone(p, (int32_t)m, evicted, h);
+      unsigned heads = __ballot_sync(0xFFFFFFFFu, head);
+      while (heads) {
+        const int src = __ffs(heads) - 1;
+        heads &= heads - 1;
+        const int64_t hh = __shfl_sync(0xFFFFFFFFu, h, src);
+        if (!place_cluster_warp(p, hh, N, sw, evicted) && lane == 0)
+          p.lidx[2][atomicAdd(&p.ctr->n_serial, 1)] = (int32_t)hh;
+        __syncwarp();
+      }
+    }
+  }
+  pdl_trigger();
+  const long long ev = block_sum_ll(evicted, sm);
+  if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
+}
+
 // ---------------------------------------------------------------------------
 // End of the row map: the write list holds (row, position of e) for every
 // distinct id that still owns its row after all inserts (a distinct id evicted
@@ -1506,17 +1561,17 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Fused gather + row update of a train step, one launch.  Work items: the
-// n_gather gather positions first, then the write list in reverse order (so
-// the rows of the labeled ids, listed first, come last).  Warps take 32 items
-// at a time from a counter.  A warp publishes each chunk's finished gather
-// items (release add); a row-update item whose row this step's gather reads
-// (gmark[row] == gtag) first waits until all gather items are published
-// (acquire poll) -- the gather reads e_hat before the row update overwrites
-// it.  Every gather item is taken before any row-update item, by warps that
-// are running, so the wait ends; it has a time limit all the same
-// (MPZCH_STATUS_TIMEOUT, and the kernel returns).  Same results as
-// k_gather_fused followed by k_writeback.
+// Fused gather + row update of a train step, one launch.  Each warp first
+// takes gather positions two at a time from one counter until none is left,
+// then publishes how many it finished (one release add per warp), then takes
+// row-update items 32 at a time from a second counter: the write list in
+// reverse order, so the rows of the labeled ids, listed first, come last.  A
+// row-update item whose row this step's gather reads (gmark[row] == gtag)
+// first waits until every gather position is published (acquire poll with
+// backoff) -- the gather reads e_hat before the row update overwrites it.
+// Gather positions are only ever held by warps that are running, so the wait
+// ends; it has a time limit all the same (MPZCH_STATUS_TIMEOUT, and the kernel
+// returns).  Same results as k_gather_fused followed by k_writeback.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void atom_add_release(int32_t* p, int32_t v) {
   asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
@@ -1534,21 +1589,19 @@ __global__ void __launch_bounds__(kBlock, 4) k_gather_update(
     const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
     const int32_t* __restrict__ wrow, const int32_t* __restrict__ wpos, const int32_t* wcount,
     const float4* __restrict__ e, float eta, const uint32_t* __restrict__ gmark, uint32_t gtag,
-    int32_t* take, int32_t* gdone, int32_t* status) {
+    int32_t* gtake, int32_t* wtake, int32_t* gdone, int32_t* status) {
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int32_t W = *wcount;
-  const int32_t total = n_gather + W;
   const int W4 = D4 + A4;
-  bool gather_done = false;  // this warp has seen every gather item published
+  // 1. gather positions, two per claim
+  int32_t mine = 0;
   for (;;) {
     int32_t base = 0;
-    if (lane == 0) base = atomicAdd(take, 32);
+    if (lane == 0) base = atomicAdd(gtake, 2);
     base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    if (base >= total) break;
-    const int32_t end = base + 32 < total ? base + 32 : total;
-    // gather items of the chunk
-    const int32_t gend = end < n_gather ? end : n_gather;
+    if (base >= n_gather) break;
+    const int32_t gend = base + 2 < n_gather ? base + 2 : n_gather;
     for (int32_t i = base; i < gend; ++i) {
       const int32_t r = rows[i];
       bool h = hit[i] != 0;
@@ -1588,25 +1641,33 @@ __global__ void __launch_bounds__(kBlock, 4) k_gather_update(
         }
       }
     }
-    if (gend > base) {
-      __syncwarp();  // every lane's loads of the chunk have returned
-      if (lane == 0) atom_add_release(gdone, gend - base);
-    }
-    // row-update items of the chunk (write list in reverse)
-    for (int32_t j = (base > n_gather ? base : n_gather); j < end; ++j) {
-      const int32_t w = W - 1 - (j - n_gather);
+    mine += gend - base;
+  }
+  if (mine) {
+    __syncwarp();  // every lane's loads have returned (their values were stored)
+    if (lane == 0) atom_add_release(gdone, mine);
+  }
+  // 2. row-update items, 32 per claim, the write list in reverse
+  bool gather_done = false;  // this warp has seen every gather position published
+  for (;;) {
+    int32_t base = 0;
+    if (lane == 0) base = atomicAdd(wtake, 32);
+    base = __shfl_sync(0xFFFFFFFFu, base, 0);
+    if (base >= W) break;
+    const int32_t end = base + 32 < W ? base + 32 : W;
+    for (int32_t j = base; j < end; ++j) {
+      const int32_t w = W - 1 - j;
       const int32_t r = wrow[w];
       if (r < 0) continue;  // tombstone
       if (!gather_done && gmark[r] == gtag) {
         bool ok = true;
-        if (lane == 0) {
-          if (ld_acquire(gdone) < n_gather) {
-            const uint64_t t0 = global_ns();
-            while (ld_acquire(gdone) < n_gather) {
-              if (global_ns() - t0 > kWaitLimitNs) {
-                ok = false;
-                break;
-              }
+        if (lane == 0 && ld_acquire(gdone) < n_gather) {
+          const uint64_t t0 = global_ns();
+          while (ld_acquire(gdone) < n_gather) {
+            __nanosleep(256);
+            if (global_ns() - t0 > kWaitLimitNs) {
+              ok = false;
+              break;
             }
           }
         }
