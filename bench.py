@@ -103,11 +103,6 @@ def parse():
     ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
                     help="row kernels through registers or through shared memory with bulk "
                          "copies (default: the library's)")
-    ap.add_argument("--fused-step", type=int, default=None, choices=[0, 1],
-                    help="gather and row update of a train step as one kernel (1) or two (0) "
-                         "(default: the library's)")
-    ap.add_argument("--place-merged", type=int, default=None, choices=[0, 1],
-                    help="cluster path: lone ids and clusters placed by one kernel (1) or two (0)")
     ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
                     help="cluster path: write list emitted at re-probe and placement, or built "
                          "by a separate kernel (default: the library's)")
@@ -120,10 +115,6 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
-    if args.place_merged is not None:
-        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_PLACE_MERGED, args.place_merged)
-    if args.fused_step is not None:
-        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP, args.fused_step)
     if args.write_list is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WRITE_LIST,
                                  1 if args.write_list == "emit" else 0)
@@ -143,12 +134,7 @@ def row_update_kernel(binding, tbl, args) -> str:
     if args.host_values and args.hbm_cache_rows:
         return "k_tier_update"
     bulk = binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_ROW_KERNEL) == 1
-    if bulk:
-        return "k_writeback_bulk"
-    fused = binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP) == 1
-    if fused and not args.host_values and not args.separate_calls:
-        return "k_gather_update"
-    return "k_writeback"
+    return "k_writeback_bulk" if bulk and not args.host_values else "k_writeback"
 
 
 def host_cpu():
@@ -430,11 +416,6 @@ def run_ours(args):
     peak, peak_kind = load_peaks()
     wb_kernel = row_update_kernel(binding, tbl, args)
     wb_traffic = ROW_UPDATE_TRAFFIC.get(wb_kernel, (None, None))
-    if wb_kernel == "k_gather_update":
-        # one kernel does the gather and the row update (traced as the row update):
-        # its algorithmic bytes are both
-        wb_bytes += g_bytes
-        g_bytes, g_ms = 0, 0.0
     wb_gbs = wb_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
     gw_gbs = (wb_bytes + g_bytes) / ((wb_ms + g_ms) * 1e-3) / 1e9 if wb_ms + g_ms > 0 else 0.0
     serving = None if args.no_serving else run_export_and_serve(tbl, binding, torch, dev, peak)

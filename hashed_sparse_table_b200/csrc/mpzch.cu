@@ -265,11 +265,7 @@ struct mpzch_table {
   // write lists (row, position of e), two buffers used by alternate Writebacks
   int32_t* wrow[2] = {nullptr, nullptr};
   int32_t* wpos[2] = {nullptr, nullptr};
-  int32_t* wcnt = nullptr;  // device int32[8]: list lengths [0..1], entries taken [2..3],
-                            // gather items finished [4..5] and taken [6..7] (per buffer)
-  uint32_t* gmark[2] = {nullptr, nullptr};  // rows a step's gather reads (fused kernel)
-  int fuse_gather_update = 0;  // train step: gather and row update as one kernel
-  int place_merged = 0;        // cluster path: both placement passes as one kernel
+  int32_t* wcnt = nullptr;  // device int32[4]: list lengths [0..1], entries taken [2..3]
   const void* prev_rows = nullptr;  // rows/hit buffers of the previous train step
   const void* prev_hit = nullptr;
   int wset = 0;             // buffer of the next Writeback
@@ -356,7 +352,6 @@ void free_all(mpzch_table* t) {
   dev_free(t->tier.claim);
   dev_free(t->ctr);
   dev_free(t->wcnt);
-  for (auto& g : t->gmark) dev_free(g), g = nullptr;
   dev_free(t->stats);
   dev_free(t->status);
   dev_free(t->sel_masks);
@@ -487,7 +482,7 @@ int run_dedup(mpzch_table* t, const int64_t* ids, int64_t n, long long* uniq, in
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr,
-                                           stats, t->status, nullptr, nullptr, nullptr, nullptr);
+                                           stats, t->status, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(t->slot_of, t->hpos, n, t->bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -639,10 +634,6 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   p.snext = t->snext;
   p.wcount = t->wcnt + t->wset;
   p.wtake = t->wcnt + 2 + t->wset;
-  p.gdone = t->wcnt + 4 + t->wset;
-  p.gtake = t->wcnt + 6 + t->wset;
-  p.gmark = nullptr;  // set by a fused train step
-  p.gtag = (uint32_t)(step + 1);
   p.emit = (t->cluster_insert && t->emit_list) ? 1 : 0;
   p.wentry = t->wentry;
   // emit: the distinct-id arrays are the list; otherwise k_write_list fills
@@ -671,7 +662,7 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     PhaseScope ps(t, PH_DEDUP, st);
     rc = launch(k_dedup_insert, (unsigned)((n + kTile - 1) / kTile), kDedupThreads, st, false,
                 p.ids, n, t->hkey, t->hpos, t->hmask, t->slot_of, t->ctr, p.stats, t->status,
-                p.wcount, p.wtake, p.gdone, p.gtake);
+                p.wcount, p.wtake);
     if (!rc) rc = launch(k_first_reprobe, grid_for(n, kBlock), kBlock, st, true, p);
     if (rc) return rc;
   }
@@ -683,26 +674,13 @@ int enqueue_row_map(mpzch_table* t, const WbParams& p, cudaStream_t st, cudaEven
     // ring or a cluster exceeds the warp path
     PhaseScope ps(t, PH_INSERT, st);
     const bool recorded = p.n_fill > 0 && fill_done;
-    if (t->place_merged) {
-      // lone keys and clusters in one launch: kPlaceKeys keys per warp
-      const int per_sm = resident_blocks(reinterpret_cast<const void*>(k_place_all), kBlock, 0);
-      int64_t work = (n + kPlaceKeys - 1) / kPlaceKeys * 32;
-      if (work < p.n_fill) work = p.n_fill;
-      rc = launch(k_place_all, grid_for(work, kBlock, per_sm), kBlock, st, !wait, p);
-      if (!rc && recorded && cudaEventRecord(fill_done, st) != cudaSuccess) rc = MPZCH_ECUDA;
-    } else {
-      rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !wait, p);
-      if (!rc && recorded && cudaEventRecord(fill_done, st) != cudaSuccess) rc = MPZCH_ECUDA;
-      // one warp per multi-key cluster, as many resident warps as the SMs hold
-      const int multi_per_sm =
-          resident_blocks(reinterpret_cast<const void*>(k_place_multi), kBlock, 0);
-      if (!rc)
-        rc = launch(k_place_multi, grid_for(n * 32, kBlock, multi_per_sm), kBlock, st, !recorded,
-                    p);
-    }
+    rc = launch(k_place_clusters, grid_for(n, kBlock, 4), kBlock, st, !wait, p);
+    if (!rc && recorded && cudaEventRecord(fill_done, st) != cudaSuccess) rc = MPZCH_ECUDA;
+    // one warp per multi-key cluster, as many resident warps as the SMs hold
+    const int multi_per_sm = resident_blocks(reinterpret_cast<const void*>(k_place_multi), kBlock, 0);
     if (!rc)
-      rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st,
-                       !(t->place_merged && recorded), p, 0);
+      rc = launch(k_place_multi, grid_for(n * 32, kBlock, multi_per_sm), kBlock, st, !recorded, p);
+    if (!rc) rc = launch_smem(k_insert_finish, 1, 1024, kClusterSmem, st, true, p, 0);
     if (!rc && !p.emit) rc = launch(k_write_list, grid_for(n, kBlock, 4), kBlock, st, true, p);
     return rc;
   }
@@ -865,7 +843,7 @@ int mpzch_dedup_static(const int64_t* ids, int64_t n, int64_t* uniq, int32_t* po
   const long long* id = reinterpret_cast<const long long*>(ids);
   const unsigned tiles = (unsigned)((n + kTile - 1) / kTile);
   k_dedup_insert<<<tiles, kDedupThreads, 0, st>>>(id, n, hkey, hpos, H - 1, slot_of, ctr, nullptr,
-                                           dev_status, nullptr, nullptr, nullptr, nullptr);
+                                           dev_status, nullptr, nullptr);
   if (after_launch()) return MPZCH_ECUDA;
   k_dedup_count<<<tiles, kBlock, 0, st>>>(slot_of, hpos, n, bcount);
   if (after_launch()) return MPZCH_ECUDA;
@@ -909,8 +887,7 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   if (!rc) rc = dev_alloc((void**)&t->shead, capacity * sizeof(unsigned long long));
   if (!rc) rc = dev_alloc((void**)&t->wentry, capacity * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->ctr, sizeof(StepCtr));
-  if (!rc) rc = dev_alloc((void**)&t->wcnt, 8 * sizeof(int32_t));
-  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->gmark[i], capacity * sizeof(uint32_t));
+  if (!rc) rc = dev_alloc((void**)&t->wcnt, 4 * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&t->stats, sizeof(WbStats));
   if (!rc) rc = dev_alloc((void**)&t->status, sizeof(int32_t));
   const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
@@ -930,9 +907,7 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
                cudaMemsetAsync(t->M, 0, (size_t)capacity * dim * sizeof(float), st) ==
                    cudaSuccess) &&
               cudaMemsetAsync(t->ctr, 0, sizeof(StepCtr), st) == cudaSuccess &&
-              cudaMemsetAsync(t->wcnt, 0, 8 * sizeof(int32_t), st) == cudaSuccess &&
-              cudaMemsetAsync(t->gmark[0], 0, capacity * sizeof(uint32_t), st) == cudaSuccess &&
-              cudaMemsetAsync(t->gmark[1], 0, capacity * sizeof(uint32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->wcnt, 0, 4 * sizeof(int32_t), st) == cudaSuccess &&
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
@@ -1065,16 +1040,11 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
   p.n_fill = n_labeled;
   p.fill_rows = rows;
   p.fill_hit = hit;
-  // The gather and the row update run as one kernel (register row kernels,
-  // values in device memory): the fill marks the rows the gather reads.
-  const bool fused = t->fuse_gather_update && n_labeled > 0 && t->row_kernel == 0 &&
-                     t->tier_rows == 0 && !t->values_on_host;
-  if (fused) p.gmark = t->gmark[t->wset];
   // Two streams.  Side stream (high priority): the row map -- dedup, re-probe
   // (which also gives the labeled ids' lookup: the rows their ids held before
   // this step's inserts), placement with the lookup fill, write list.
   // Caller's stream: the gather once the fill is done, then the row update
-  // once the row map is done (fused: one kernel once the row map is done).
+  // once the row map is done.
   // Without inputs_ready the side stream starts after everything earlier on
   // the caller's stream.  With it (pipelined) the side stream waits only for
   // the inputs, the table's other calls and the row update that last read this
@@ -1101,27 +1071,6 @@ int mpzch_train_step(mpzch_table* t, const int64_t* ids, int64_t n, int64_t n_la
   if (cudaEventRecord(t->ev_map, t->side) != cudaSuccess) return MPZCH_ECUDA;
   t->prev_rows = rows;
   t->prev_hit = hit;
-  if (fused) {
-    if (cudaStreamWaitEvent(st, t->ev_map, 0) != cudaSuccess) return MPZCH_ECUDA;
-    {
-      PhaseScope ps(t, PH_WRITEBACK, st);
-      const bool has_ao = ao_table != nullptr;
-      rc = launch(k_gather_update, row_grid(n, t->row_blocks_per_sm), kBlock, st, false,
-                  (const int32_t*)rows, (const uint8_t*)hit, (int32_t)n_labeled,
-                  reinterpret_cast<float4*>(t->M), t->C, t->D / 4,
-                  reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
-                  ao_rows, reinterpret_cast<float4*>(out), (const int32_t*)p.wrow,
-                  (const int32_t*)p.wpos, (const int32_t*)p.wcount, p.e, t->eta,
-                  (const uint32_t*)p.gmark, p.gtag, p.gtake, p.wtake, p.gdone, t->status);
-      if (rc) return rc;
-    }
-    if (cudaEventRecord(t->ev_gather, st) != cudaSuccess ||
-        cudaEventRecord(t->ev_update[t->wset], st) != cudaSuccess)
-      return MPZCH_ECUDA;
-    t->wset ^= 1;
-    t->last_step = step;
-    return MPZCH_OK;
-  }
   // Caller's stream: gather once the lookup fill is done, then the row update
   // once the row map is done (and after the gather has read the values).
   if (n_labeled > 0) {
@@ -1449,16 +1398,6 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     return MPZCH_OK;
   }
   if (option == MPZCH_OPT_HBM_CACHE_ROWS) return set_tier_rows(t, value);
-  if (option == MPZCH_OPT_PLACE_MERGED) {
-    if (value != 0 && value != 1) return MPZCH_EINVAL;
-    t->place_merged = (int)value;
-    return MPZCH_OK;
-  }
-  if (option == MPZCH_OPT_FUSED_STEP) {
-    if (value != 0 && value != 1) return MPZCH_EINVAL;
-    t->fuse_gather_update = (int)value;
-    return MPZCH_OK;
-  }
   if (option == MPZCH_OPT_WRITE_LIST) {
     if (value != 0 && value != 1) return MPZCH_EINVAL;
     t->emit_list = (int)value;
@@ -1485,8 +1424,6 @@ int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
     case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
     case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
     case MPZCH_OPT_HBM_CACHE_ROWS: *value = t->tier_rows; break;
-    case MPZCH_OPT_FUSED_STEP: *value = t->fuse_gather_update; break;
-    case MPZCH_OPT_PLACE_MERGED: *value = t->place_merged; break;
     default: return MPZCH_EINVAL;
   }
   return MPZCH_OK;

@@ -276,8 +276,7 @@ constexpr int kDedupThreads = kTile;  // one tile position per thread
 __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     const long long* __restrict__ ids, int64_t n, unsigned long long* __restrict__ hkey,
     uint32_t* __restrict__ hpos, uint64_t hmask, int32_t* __restrict__ slot_of, StepCtr* ctr,
-    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake, int32_t* gdone,
-    int32_t* gtake) {
+    WbStats* stats, int32_t* status, int32_t* wcount, int32_t* wtake) {
   pdl_enter();
   __shared__ unsigned long long s_key[kTileHash];
   __shared__ uint32_t s_pos[kTileHash];
@@ -290,8 +289,6 @@ __global__ void __launch_bounds__(kDedupThreads) k_dedup_insert(
     reinterpret_cast<long long*>(stats)[threadIdx.x] = 0;
   if (wcount && blockIdx.x == 0 && threadIdx.x == 0) *wcount = 0;
   if (wtake && blockIdx.x == 0 && threadIdx.x == 0) *wtake = 0;
-  if (gdone && blockIdx.x == 0 && threadIdx.x == 0) *gdone = 0;
-  if (gtake && blockIdx.x == 0 && threadIdx.x == 0) *gtake = 0;
   for (int j = threadIdx.x; j < kTileHash; j += blockDim.x) {
     s_key[j] = kEmptyKey;
     s_pos[j] = kNoPos;
@@ -556,9 +553,7 @@ struct WbParams {
   int32_t* wrow;
   int32_t* wpos;
   int32_t* wcount;
-  int32_t* wtake;  // entries of the list already taken by the bulk row update / fused kernel
-  int32_t* gdone;  // gather items finished (fused gather + row update)
-  int32_t* gtake;  // gather items taken (fused gather + row update)
+  int32_t* wtake;  // entries of the list already taken by the bulk row update
   // emit = 1 (cluster path): the write list is the distinct-id arrays of this
   // call themselves -- entry u = (urow[u], upos[u]), wrow/wpos point at them
   // and *wcount is set to the number of distinct ids -- so nothing is
@@ -577,10 +572,6 @@ struct WbParams {
   int64_t n_fill;
   int32_t* fill_rows;
   uint8_t* fill_hit;
-  // rows the step's gather reads (hit rows of the filled positions) get
-  // gmark[row] = gtag when gmark is set (fused gather + row update)
-  uint32_t* gmark;
-  uint32_t gtag;
 };
 
 // Lookup result of batch position i < n_fill: the row its id held before the
@@ -591,7 +582,6 @@ __device__ __forceinline__ void fill_lookup(const WbParams& p, int64_t i) {
   const int32_t r = s >= 0 ? __ldcg(p.hrow + s) : -1;
   p.fill_rows[i] = r;
   p.fill_hit[i] = r >= 0 ? 1 : 0;
-  if (p.gmark && r >= 0) p.gmark[r] = p.gtag;
 }
 
 // urow value of a distinct id that was placed and then evicted again later in
@@ -1413,58 +1403,6 @@ __global__ void __launch_bounds__(kBlock) k_place_multi(WbParams p) {
   if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
 }
 
-// Both placement passes in one launch (and the lookup fill): each warp takes
-// kPlaceKeys missing keys, lanes 0..kPlaceKeys-1 run the lone-key check of one
-// key each (placing lone keys), and then the whole warp places, one after
-// another, the clusters whose heads it found.  A lone key's window touches no
-// slot of any cluster and the clusters' slot sets are disjoint, so the two
-// kinds of placement run side by side without ordering.  Clusters beyond the
-// warp path are listed for k_insert_finish, as with k_place_multi.
-constexpr int kPlaceKeys = 8;
-
-__global__ void __launch_bounds__(kBlock) k_place_all(WbParams p) {
-  pdl_enter();
-  __shared__ long long sm[33];
-  __shared__ WarpCluster s_warp[kBlock / 32];
-  const int32_t N = p.ctr->cnt[0];
-  const bool ring_may_be_covered = (int64_t)N * p.g.P >= p.g.C;
-  const int lane = threadIdx.x & 31;
-  WarpCluster& sw = s_warp[threadIdx.x >> 5];
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    p.stats->n_inserted = N;
-    if (p.emit) {  // no k_write_list on this path: the list is the distinct-id arrays
-      p.stats->n_unique = p.ctr->n_unique;
-      *p.wcount = p.ctr->n_unique;
-    }
-    if (N > 0) atomic_add_ll(&p.stats->n_rounds, 1LL);
-  }
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < p.n_fill; i += stride)
-    fill_lookup(p, i);
-  long long evicted = 0;
-  if (!ring_may_be_covered) {
-    const int64_t warps = stride >> 5;
-    for (int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-         w * kPlaceKeys < N; w += warps) {
-      const int64_t m = w * kPlaceKeys + lane;
-      int64_t h = 0;
-      const bool head = lane < kPlaceKeys && m < N && place_lone(p, (int32_t)m, evicted, h);
-      unsigned heads = __ballot_sync(0xFFFFFFFFu, head);
-      while (heads) {
-        const int src = __ffs(heads) - 1;
-        heads &= heads - 1;
-        const int64_t hh = __shfl_sync(0xFFFFFFFFu, h, src);
-        if (!place_cluster_warp(p, hh, N, sw, evicted) && lane == 0)
-          p.lidx[2][atomicAdd(&p.ctr->n_serial, 1)] = (int32_t)hh;
-        __syncwarp();
-      }
-    }
-  }
-  pdl_trigger();
-  const long long ev = block_sum_ll(evicted, sm);
-  if (threadIdx.x == 0 && ev) atomic_add_ll(&p.stats->n_evicted, ev);
-}
-
 // ---------------------------------------------------------------------------
 // End of the row map: the write list holds (row, position of e) for every
 // distinct id that still owns its row after all inserts (a distinct id evicted
@@ -1554,154 +1492,6 @@ __global__ void __launch_bounds__(kBlock) k_writeback(const int32_t* __restrict_
           o.z = __fsub_rn(a[q].z, __fmul_rn(eta, __fsub_rn(a[q].z, b[q].z)));
           o.w = __fsub_rn(a[q].w, __fmul_rn(eta, __fsub_rn(a[q].w, b[q].w)));
           __stcs(m + c, o);
-        }
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Fused gather + row update of a train step, one launch.  Each warp first
-// takes gather positions two at a time from one counter until none is left,
-// then publishes how many it finished (one release add per warp), then takes
-// row-update items 32 at a time from a second counter: the write list in
-// reverse order, so the rows of the labeled ids, listed first, come last.  A
-// row-update item whose row this step's gather reads (gmark[row] == gtag)
-// first waits until every gather position is published (acquire poll with
-// backoff) -- the gather reads e_hat before the row update overwrites it.
-// Gather positions are only ever held by warps that are running, so the wait
-// ends; it has a time limit all the same (MPZCH_STATUS_TIMEOUT, and the kernel
-// returns).  Same results as k_gather_fused followed by k_writeback.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void atom_add_release(int32_t* p, int32_t v) {
-  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-__device__ __forceinline__ int32_t ld_acquire(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__global__ void __launch_bounds__(kBlock, 4) k_gather_update(
-    const int32_t* __restrict__ rows, const uint8_t* __restrict__ hit, int32_t n_gather,
-    float4* __restrict__ M, int64_t C, int D4, const float4* __restrict__ ao, int64_t ao_n, int A4,
-    const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
-    const int32_t* __restrict__ wrow, const int32_t* __restrict__ wpos, const int32_t* wcount,
-    const float4* __restrict__ e, float eta, const uint32_t* __restrict__ gmark, uint32_t gtag,
-    int32_t* gtake, int32_t* wtake, int32_t* gdone, int32_t* status) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int32_t W = *wcount;
-  const int W4 = D4 + A4;
-  // 1. gather positions, two per claim
-  int32_t mine = 0;
-  for (;;) {
-    int32_t base = 0;
-    if (lane == 0) base = atomicAdd(gtake, 2);
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    if (base >= n_gather) break;
-    const int32_t gend = base + 2 < n_gather ? base + 2 : n_gather;
-    for (int32_t i = base; i < gend; ++i) {
-      const int32_t r = rows[i];
-      bool h = hit[i] != 0;
-      if (h && (r < 0 || (int64_t)r >= C)) {
-        if (lane == 0) set_status(status, kStBadRow);
-        h = false;
-      }
-      int32_t a = 0;
-      bool has_a = A4 > 0;
-      if (has_a) {
-        a = ao_rows[i];
-        if (a < 0 || (int64_t)a >= ao_n) {
-          if (lane == 0) set_status(status, kStBadAo);
-          has_a = false;
-        }
-      }
-      const float4* src = M + (int64_t)(h ? r : 0) * D4;
-      const float4* asrc = ao + (int64_t)a * A4;
-      float4* dst = out + (int64_t)i * W4;
-      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int cb = 0; cb < W4; cb += 4 * 32) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = cb + u * 32 + lane;
-          v[u] = z;
-          if (c < D4) {
-            if (h) v[u] = __ldcs(src + c);
-          } else if (c < W4 && has_a) {
-            v[u] = __ldcs(asrc + (c - D4));
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int c = cb + u * 32 + lane;
-          if (c < W4) __stcs(dst + c, v[u]);
-        }
-      }
-    }
-    mine += gend - base;
-  }
-  if (mine) {
-    __syncwarp();  // every lane's loads have returned (their values were stored)
-    if (lane == 0) atom_add_release(gdone, mine);
-  }
-  // 2. row-update items, 32 per claim, the write list in reverse
-  bool gather_done = false;  // this warp has seen every gather position published
-  for (;;) {
-    int32_t base = 0;
-    if (lane == 0) base = atomicAdd(wtake, 32);
-    base = __shfl_sync(0xFFFFFFFFu, base, 0);
-    if (base >= W) break;
-    const int32_t end = base + 32 < W ? base + 32 : W;
-    for (int32_t j = base; j < end; ++j) {
-      const int32_t w = W - 1 - j;
-      const int32_t r = wrow[w];
-      if (r < 0) continue;  // tombstone
-      if (!gather_done && gmark[r] == gtag) {
-        bool ok = true;
-        if (lane == 0 && ld_acquire(gdone) < n_gather) {
-          const uint64_t t0 = global_ns();
-          while (ld_acquire(gdone) < n_gather) {
-            __nanosleep(256);
-            if (global_ns() - t0 > kWaitLimitNs) {
-              ok = false;
-              break;
-            }
-          }
-        }
-        ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-        if (!ok) {
-          if (lane == 0) set_status(status, kStTimeout);
-          return;
-        }
-        __syncwarp();
-        gather_done = true;
-      }
-      float4* m = M + (int64_t)r * D4;
-      const float4* ev = e + (int64_t)wpos[w] * D4;
-      for (int cb = 0; cb < D4; cb += 4 * 32) {
-        float4 a4[4], b4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = cb + q * 32 + lane;
-          if (c < D4) {
-            a4[q] = __ldcs(m + c);
-            b4[q] = __ldcs(ev + c);
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = cb + q * 32 + lane;
-          if (c < D4) {
-            float4 o;
-            o.x = __fsub_rn(a4[q].x, __fmul_rn(eta, __fsub_rn(a4[q].x, b4[q].x)));
-            o.y = __fsub_rn(a4[q].y, __fmul_rn(eta, __fsub_rn(a4[q].y, b4[q].y)));
-            o.z = __fsub_rn(a4[q].z, __fmul_rn(eta, __fsub_rn(a4[q].z, b4[q].z)));
-            o.w = __fsub_rn(a4[q].w, __fmul_rn(eta, __fsub_rn(a4[q].w, b4[q].w)));
-            __stcs(m + c, o);
-          }
         }
       }
     }

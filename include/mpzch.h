@@ -444,18 +444,6 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * through mpzch_state_views are the host rows: call mpzch_tier_sync first.
  * Steps of a tiered table must stay below 2^31. */
 #define MPZCH_OPT_HBM_CACHE_ROWS 10
-/* MPZCH_OPT_FUSED_STEP: 1 = mpzch_train_step runs its gather and
- * its row update as one kernel (when the values are in device memory and the
- * register row kernels are selected): warps take the gather positions first,
- * then the write list; the update of a row the step's gather reads waits until
- * every gather position is done.  0 (default) = two kernels.  Results are
- * identical. */
-#define MPZCH_OPT_FUSED_STEP 11
-/* MPZCH_OPT_PLACE_MERGED (cluster placement path): 1 = lone missing
- * ids and multi-id clusters are placed by one kernel (a warp checks 8 ids and
- * places the clusters it heads); 0 (default) = two kernels (a thread per id,
- * then a warp per listed cluster).  Results are identical. */
-#define MPZCH_OPT_PLACE_MERGED 12
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 /* Current value of an option (MPZCH_EINVAL for an unknown option). */
 MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);

@@ -149,8 +149,7 @@ def _keys_with_home(C, slots, count_per_slot, start):
 
 
 @pytest.mark.parametrize("fused", [False, True])
-@pytest.mark.parametrize("merged", [0, 1])
-def test_cluster_placement_long_chains_and_shared_slots(fused, merged):
+def test_cluster_placement_long_chains_and_shared_slots(fused):
     """Clusters beyond the 32 keys sorted in registers: a chain of 40 keys with
     start slots 2 apart that wraps past the last row, and 36 keys sharing one
     start slot (28 of them are evicted again in the same step)."""
@@ -167,9 +166,7 @@ def test_cluster_placement_long_chains_and_shared_slots(fused, merged):
         repeat = batches[-1][:50] if batches else np.empty(0, np.int64)
         ids = np.concatenate([chain, shared, other, repeat])
         batches.append(ids[rng.permutation(ids.size)])
-    from hashed_sparse_table_b200 import binding
-    r = run_pair(w, steps=4, ids_fn=lambda t: batches[t], fused_step=fused,
-                 options={binding.MPZCH_OPT_PLACE_MERGED: merged})
+    r = run_pair(w, steps=4, ids_fn=lambda t: batches[t], fused_step=fused)
     for s in r.stats:
         assert s["n_inserted"] * P < C  # the grid-wide cluster path
     assert sum(s["n_dropped"] for s in r.stats) >= 4 * 28
@@ -565,40 +562,7 @@ def test_fused_step_labeled_negative_ids():
     compare_state(tbl, orc, "after negative labeled ids")
 
 
-@pytest.mark.parametrize("fused", [0, 1])
-@pytest.mark.parametrize("name", ["c3_small", "c4_stress", "nonpow2", "p_eq_c"])
-def test_fused_and_two_kernel_step_bit_exact(name, fused):
-    """MPZCH_OPT_FUSED_STEP: gather and row update as one kernel or two, with
-    train steps one at a time and pipelined."""
-    from gpu_harness import run_pipelined
-    from hashed_sparse_table_b200 import binding
-    opts = {binding.MPZCH_OPT_FUSED_STEP: fused}
-    run_pair(SCALED[name], fused_step=True, options=opts)
-    run_pipelined(SCALED[name], options=opts)
-
-
-@pytest.mark.parametrize("merged", [0, 1])
-@pytest.mark.parametrize("name", list(CLUSTERED) + ["c2_small"])
-def test_placement_one_or_two_kernels_bit_exact(name, merged):
-    """MPZCH_OPT_PLACE_MERGED: lone ids and clusters placed by one kernel or
-    two; separate calls and pipelined train steps (with the fused step)."""
-    from gpu_harness import run_pipelined
-    from hashed_sparse_table_b200 import binding
-    w = CLUSTERED.get(name) or SCALED[name]
-    opts = {binding.MPZCH_OPT_PLACE_MERGED: merged}
-    run_pair(w, options=opts)
-    run_pipelined(w, options={**opts, binding.MPZCH_OPT_FUSED_STEP: 1})
-
-
-def test_placement_merged_long_chains_and_drops():
-    from hashed_sparse_table_b200 import binding
-    r = run_pair(DROPS, fused_step=True, options={binding.MPZCH_OPT_PLACE_MERGED: 1,
-                                                  binding.MPZCH_OPT_FUSED_STEP: 1})
-    assert sum(s["n_dropped"] for s in r.stats) > 0
-
-
-@pytest.mark.parametrize("fused", [1, 0])
-def test_pipelined_steps_sharing_rows_and_hit_buffers(fused):
+def test_pipelined_steps_sharing_rows_and_hit_buffers():
     """Pipelined steps that reuse one rows/hit pair (each with its own fused
     output): a step's lookup fill must wait for the previous step's gather,
     which reads those buffers.  Every step's features and the final rows/hit
@@ -606,7 +570,6 @@ def test_pipelined_steps_sharing_rows_and_hit_buffers(fused):
     from hashed_sparse_table_b200 import binding
     w = SCALED["c3_small"].scaled(steps=10)
     tbl, orc = make_pair(w)
-    binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_FUSED_STEP, fused)
     dev = tbl.device
     ao = inputs.author_table(w)
     ao_d = torch.from_numpy(ao).to(dev)
