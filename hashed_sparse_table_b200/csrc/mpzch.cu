@@ -259,6 +259,8 @@ struct mpzch_table {
   // Writebacks (on the cluster path they are the write list the row update reads)
   int32_t* upos[2] = {nullptr, nullptr};
   int32_t* urow[2] = {nullptr, nullptr};
+  uint8_t* uhit[2] = {nullptr, nullptr};  // resident before the step, per distinct id
+  uint8_t* whit[2] = {nullptr, nullptr};  // the same, aligned with the compacted write lists
   int32_t* snext = nullptr;  // next key of the same home slot (cluster path)
   long long* lkey[3] = {nullptr, nullptr, nullptr};  // insert round lists: keys
   int32_t* lidx[3] = {nullptr, nullptr, nullptr};    // and their distinct-id index
@@ -321,6 +323,8 @@ void free_batch_scratch(mpzch_table* t) {
   dev_free(t->ukey);
   for (auto& l : t->upos) dev_free(l), l = nullptr;
   for (auto& l : t->urow) dev_free(l), l = nullptr;
+  for (auto& l : t->uhit) dev_free(l), l = nullptr;
+  for (auto& l : t->whit) dev_free(l), l = nullptr;
   dev_free(t->snext);
   t->snext = nullptr;
   for (auto& l : t->lkey) dev_free(l), l = nullptr;
@@ -411,6 +415,8 @@ int ensure_batch(mpzch_table* t, int64_t n, cudaStream_t st) {
   if (!rc) rc = dev_alloc((void**)&t->ukey, cap * sizeof(long long));
   for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->upos[i], cap * sizeof(int32_t));
   for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->urow[i], cap * sizeof(int32_t));
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->uhit[i], cap);
+  for (int i = 0; i < 2 && !rc; ++i) rc = dev_alloc((void**)&t->whit[i], cap);
   if (!rc) rc = dev_alloc((void**)&t->snext, cap * sizeof(int32_t));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lkey[i], cap * sizeof(long long));
   for (int i = 0; i < 3 && !rc; ++i) rc = dev_alloc((void**)&t->lidx[i], cap * sizeof(int32_t));
@@ -640,6 +646,8 @@ WbParams make_params(mpzch_table* t, const int64_t* ids, const float* e, int64_t
   // the compacted buffers
   p.wrow = p.emit ? p.urow : t->wrow[t->wset];
   p.wpos = p.emit ? p.upos : t->wpos[t->wset];
+  p.uhit = t->uhit[t->wset];
+  p.whit = p.emit ? p.uhit : t->whit[t->wset];
   return p;
 }
 
@@ -712,7 +720,7 @@ int enqueue_row_update(mpzch_table* t, const WbParams& p, cudaStream_t st, bool 
       const unsigned g = row_grid(p.n, t->row_blocks_per_sm);
       float4* host = p.M;
       rc = launch(k_tier_claim, grid_for(p.n, kBlock), kBlock, st, pdl, (const int32_t*)p.wrow,
-                  (const int32_t*)p.wcount, t->tier, (long long)p.step);
+                  (const uint8_t*)p.whit, (const int32_t*)p.wcount, t->tier, (long long)p.step);
       if (!rc)
         rc = launch(k_tier_evict, g, kBlock, st, true, (const int32_t*)p.wrow,
                     (const int32_t*)p.wcount, t->tier, host, p.D4, (long long)p.step);

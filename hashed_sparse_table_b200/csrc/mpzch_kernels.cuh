@@ -553,6 +553,11 @@ struct WbParams {
   int32_t* wrow;
   int32_t* wpos;
   int32_t* wcount;
+  // per distinct id: 1 when it was resident before the step (set by the
+  // re-probe), and the same flag aligned with the write list (uhit itself on
+  // the cluster path, a compacted copy written by k_write_list otherwise)
+  uint8_t* uhit;
+  uint8_t* whit;
   int32_t* wtake;  // entries of the list already taken by the bulk row update
   // emit = 1 (cluster path): the write list is the distinct-id arrays of this
   // call themselves -- entry u = (urow[u], upos[u]), wrow/wpos point at them
@@ -664,6 +669,7 @@ __global__ void __launch_bounds__(kBlock) k_first_reprobe(WbParams p) {
       p.ukey[u] = k;
       p.upos[u] = (int32_t)i;
       p.urow[u] = (int32_t)r;
+      p.uhit[u] = r >= 0 ? 1 : 0;
       if (r >= 0) {
         p.last[r] = p.step;
         ++hits;
@@ -1439,6 +1445,7 @@ __global__ void __launch_bounds__(kBlock) k_write_list(WbParams p) {
     if (owned) {
       p.wrow[m] = r;
       p.wpos[m] = p.upos[u];
+      p.whit[m] = p.uhit[u];
     }
   }
   pdl_trigger();

@@ -13,7 +13,11 @@
 //                  (step, current owner?, ~row); the largest word wins, so a
 //                  slot's current owner keeps it when it is written in this
 //                  step, and otherwise the smallest written row takes it (the
-//                  step in the high bits makes words of earlier steps lose);
+//                  step in the high bits makes words of earlier steps lose).
+//                  Admission: a row that was not resident before the step (a
+//                  freshly inserted id, likelier to be cold) only claims an
+//                  empty slot, so it does not push out a row kept from earlier
+//                  steps;
 //   k_tier_evict   the winner of each slot it does not own yet writes the old
 //                  owner's cached value back to the host row and takes the
 //                  slot (owner = row, won = step: its value is still on the host);
@@ -50,6 +54,7 @@ __device__ __forceinline__ unsigned long long tier_claim_word(long long step, bo
 
 // Pass 1: claims (one thread per write-list entry; tombstones skipped).
 __global__ void __launch_bounds__(kBlock) k_tier_claim(const int32_t* __restrict__ wrow,
+                                                       const uint8_t* __restrict__ whit,
                                                        const int32_t* wcount, Tier tr,
                                                        long long step) {
   pdl_enter();
@@ -59,7 +64,9 @@ __global__ void __launch_bounds__(kBlock) k_tier_claim(const int32_t* __restrict
     const int32_t r = wrow[w];
     if (r < 0) continue;
     const uint32_t s = (uint32_t)r & tr.mask;
-    atomicMax(tr.claim + s, tier_claim_word(step, tr.owner[s] == r, r));
+    const int32_t o = tr.owner[s];
+    if (o != r && o >= 0 && !whit[w]) continue;  // admission: see the header
+    atomicMax(tr.claim + s, tier_claim_word(step, o == r, r));
   }
   pdl_trigger();
 }

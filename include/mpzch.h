@@ -436,9 +436,10 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * the default) in front of the host-memory values -- the hot/cold tier (Memory
  * Layer section 2: the 512-d table is sharded across GPU and CPU).  Row r can
  * live in cache slot r mod H; the cache is write-back.  In each Writeback a
- * written row keeps its slot, or the smallest written row whose slot's owner
- * was not written takes it (the old owner's value is written back to the host
- * first); reads take a row from the cache when it holds it.  Every value read
+ * written row keeps its slot; a slot whose owner was not written goes to the
+ * smallest written row that was resident before the step (a freshly inserted
+ * id only takes an empty slot), and the old owner's value is written back to
+ * the host first; reads take a row from the cache when it holds it.  Every value read
  * or written is exactly that of a table without the cache.  Changing the size
  * writes every cached row back and synchronises the device.  Values read
  * through mpzch_state_views are the host rows: call mpzch_tier_sync first.
