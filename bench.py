@@ -47,7 +47,7 @@ PREFILL = 20  # untimed steps that bring the table to its steady state
 # (dram__bytes_read.sum + dram__bytes_write.sum of a steady-state launch).  A
 # kernel missing here reports traffic null.
 ROW_UPDATE_TRAFFIC = {
-    "k_writeback": (550.74e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
+    "k_writeback": (551.65e6, "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch "
                               "(23rd step of the multi-table workload)"),
 }
 REPLICA_STRIDE = 1_000_000  # id-stream offset between replicas (ranks)
@@ -103,6 +103,8 @@ def parse():
     ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
                     help="row kernels through registers or through shared memory with bulk "
                          "copies (default: the library's)")
+    ap.add_argument("--select-passes", type=int, default=None, choices=[1, 2],
+                    help="select in two launches or one (default: the library's)")
     ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
                     help="cluster path: write list emitted at re-probe and placement, or built "
                          "by a separate kernel (default: the library's)")
@@ -115,6 +117,8 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
+    if args.select_passes is not None:
+        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SELECT_PASSES, args.select_passes)
     if args.write_list is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WRITE_LIST,
                                  1 if args.write_list == "emit" else 0)
@@ -828,14 +832,21 @@ def run_sharded(args):
     sent = {"lookup": 0, "writeback": 0}
 
     # step t+1 is prepared (partitions, segment-size exchange) before step t
-    # finishes, so the sizes reach the host while step t runs
-    pending = {0: shard.prepare(ids_d[0], lab, e_d[0])}
+    # finishes, so the sizes reach the host while step t runs; with one shard
+    # the step is the table's own train step, pipelined like the local bench
+    # (inputs resident from `ready` on, rows/hit buffers alternating)
+    ready = torch.cuda.Event()
+    ready.record()
+    rows_t = [rows, torch.empty_like(rows)]
+    hit_t = [hit, torch.empty_like(hit)]
+    pending = {0: shard.prepare(ids_d[0], lab, e_d[0], inputs_ready=ready)}
 
     def step(t):
         tr = {}
         if t + 1 < total:
-            pending[t + 1] = shard.prepare(ids_d[t + 1], lab, e_d[(t + 1) % E])
-        shard.finish(pending.pop(t), t, ao_d, aor_d[t], rows, hit, out, stats[t], trace=tr)
+            pending[t + 1] = shard.prepare(ids_d[t + 1], lab, e_d[(t + 1) % E], inputs_ready=ready)
+        shard.finish(pending.pop(t), t, ao_d, aor_d[t], rows_t[t % 2], hit_t[t % 2], out, stats[t],
+                     trace=tr)
         return tr
 
     for t in range(Pf + Wm):

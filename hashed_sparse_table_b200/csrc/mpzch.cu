@@ -275,16 +275,23 @@ struct mpzch_table {
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
   int32_t* status = nullptr;
-  // select: per-tile ballot words and row counts
+  // select: per-tile ballot words and row counts (two launches); per-tile
+  // published counts, the tile ticket counter, the call epoch and the tickets
+  // issued so far (one launch)
   uint32_t* sel_masks = nullptr;
   int32_t* sel_tcount = nullptr;
+  unsigned long long* sel_tword = nullptr;
+  unsigned long long* sel_ticket = nullptr;
+  uint32_t sel_epoch = 0;
+  unsigned long long sel_tickets = 0;
+  int select_passes = 2;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
   int side_high_priority = 1;  // priority of the side stream (set before its first use)
   float eta = 1.0f;            // learning rate of the Writeback step
   int row_blocks_per_sm = 8;   // row kernels: 0 = one row per warp, else grid-stride cap
-  int row_kernel = 0;          // 0 = register-staged row kernels, 1 = bulk-copy (shared memory)
+  int row_kernel = 0;          // 0 = rows through registers, 1 = bulk copies into shared memory
   int bulk_warps = 8;          // bulk row kernels: warps per block
   int bulk_blocks = 1;         // bulk row kernels: blocks per SM (persistent grid)
   int l2_hint_rows = 0;        // bulk row kernels: L2 policy of table-row accesses (L2Hint)
@@ -360,6 +367,8 @@ void free_all(mpzch_table* t) {
   dev_free(t->status);
   dev_free(t->sel_masks);
   dev_free(t->sel_tcount);
+  dev_free(t->sel_tword);
+  dev_free(t->sel_ticket);
   if (t->h_status) cudaFreeHost(t->h_status);
   for (auto& r : t->pending) {
     cudaEventDestroy(r.a);
@@ -505,6 +514,19 @@ namespace {
 // with programmatic dependent launch.
 int launch_select(mpzch_table* t, int64_t since, int32_t* rows_out, int64_t* dev_count,
                   cudaStream_t st) {
+  if (t->select_passes == 1) {
+    const unsigned long long tiles = (unsigned long long)((t->C + kSelBigTile - 1) / kSelBigTile);
+    uint32_t epoch = t->sel_epoch + 1;
+    if (epoch == 0) epoch = 1;  // 0 is the value of the cleared words
+    const int rc = launch(k_select_one, (unsigned)tiles, kSelBigThreads, st, false,
+                          (const long long*)t->keys, (const long long*)t->last, t->C,
+                          (long long)since, t->sel_tword, t->sel_ticket, t->sel_tickets, epoch,
+                          rows_out, reinterpret_cast<long long*>(dev_count), t->status);
+    if (rc) return rc;
+    t->sel_epoch = epoch;
+    t->sel_tickets += tiles;
+    return MPZCH_OK;
+  }
   const unsigned tiles = (unsigned)((t->C + kScanTile - 1) / kScanTile);
   int rc = launch(k_select_mark, tiles, kScanThreads, st, false, (const long long*)t->keys,
                   (const long long*)t->last, t->C, (long long)since, t->sel_masks,
@@ -901,6 +923,9 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
   if (!rc) rc = dev_alloc((void**)&t->sel_masks, sel_tiles * kScanWords * sizeof(uint32_t));
   if (!rc) rc = dev_alloc((void**)&t->sel_tcount, sel_tiles * sizeof(int32_t));
+  const int64_t sel_big = (capacity + kSelBigTile - 1) / kSelBigTile;
+  if (!rc) rc = dev_alloc((void**)&t->sel_tword, sel_big * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&t->sel_ticket, sizeof(unsigned long long));
   if (!rc && cudaHostAlloc((void**)&t->h_status, sizeof(int32_t), cudaHostAllocDefault) != cudaSuccess) {
     t->h_status = nullptr;
     rc = MPZCH_ENOMEM;
@@ -919,7 +944,10 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
-              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
+              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess &&
+              cudaMemsetAsync(t->sel_tword, 0, sel_big * sizeof(unsigned long long), st) ==
+                  cudaSuccess &&
+              cudaMemsetAsync(t->sel_ticket, 0, sizeof(unsigned long long), st) == cudaSuccess;
     for (int i = 0; i < 3 && ok; ++i)
       ok = cudaMemsetAsync(t->claims[i], 0xFF, capacity * sizeof(unsigned long long), st) ==
            cudaSuccess;
@@ -1110,14 +1138,15 @@ int mpzch_select_written_since(mpzch_table* t, int64_t since_step, int32_t* rows
 }
 
 namespace {
-// Row export: the staged kernel (shared-memory double buffering) for dim 512
-// or 1024 with a 16-byte aligned q, the register kernel for every other shape.
+// Writes every row the hot/cold tier's HBM cache holds back to its host row.
 int tier_flush(mpzch_table* t, cudaStream_t st) {
   if (t->tier_rows <= 0) return MPZCH_OK;
   return launch(k_tier_flush, row_grid(t->tier_rows, t->row_blocks_per_sm), kBlock, st, false,
                 t->tier, t->tier_rows, reinterpret_cast<float4*>(t->M), t->D / 4);
 }
 
+// Row export: the interleaved register kernel for D = 128, 256, 512, 1024 (one
+// resident wave, grid-stride), the generic kernel for every other dim.
 int launch_export(mpzch_table* t, const int32_t* rows, int64_t n, const int64_t* dev_n, int8_t* q,
                   float* scale, int64_t* keys_out, int64_t* last_out, cudaStream_t st) {
   // a tiered table's export reads host rows: cached rows are written back first
@@ -1406,6 +1435,11 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     return MPZCH_OK;
   }
   if (option == MPZCH_OPT_HBM_CACHE_ROWS) return set_tier_rows(t, value);
+  if (option == MPZCH_OPT_SELECT_PASSES) {
+    if (value != 1 && value != 2) return MPZCH_EINVAL;
+    t->select_passes = (int)value;
+    return MPZCH_OK;
+  }
   if (option == MPZCH_OPT_WRITE_LIST) {
     if (value != 0 && value != 1) return MPZCH_EINVAL;
     t->emit_list = (int)value;
@@ -1432,6 +1466,7 @@ int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
     case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
     case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
     case MPZCH_OPT_HBM_CACHE_ROWS: *value = t->tier_rows; break;
+    case MPZCH_OPT_SELECT_PASSES: *value = t->select_passes; break;
     default: return MPZCH_EINVAL;
   }
   return MPZCH_OK;

@@ -184,15 +184,18 @@ class ShardedMpzch:
         return self.finish(self.prepare(ids, n_labeled, e), step, ao_table, ao_rows, rows, hit,
                            out, stats, trace)
 
-    def prepare(self, ids: torch.Tensor, n_labeled: int, e: torch.Tensor) -> "Prepared":
+    def prepare(self, ids: torch.Tensor, n_labeled: int, e: torch.Tensor,
+                inputs_ready=None) -> "Prepared":
         """Steps 1-2a of a sharded step: the partitions by owner (labeled ids;
         distinct ids with their e rows packed) and the start of the segment-
         size exchange.  Issuing the next step's prepare before this step's
         finish lets the sizes reach the host while this step runs, so the host
         never waits for the GPU in the middle of a step.  Every rank must issue
-        prepares and finishes in the same order (they are collectives)."""
+        prepares and finishes in the same order (they are collectives).
+        inputs_ready (a CUDA event recorded after ids and e were written) lets a
+        one-shard step run pipelined like the table's own train step."""
         if self.G == 1:
-            return Prepared(ids=ids, n_labeled=n_labeled, e=e)
+            return Prepared(ids=ids, n_labeled=n_labeled, e=e, inputs_ready=inputs_ready)
         binding = self.binding
         G, dev, D = self.G, self.device, self.dim
         n = ids.numel()
@@ -225,7 +228,7 @@ class ShardedMpzch:
         stats = torch.empty(7, dtype=torch.int64, device=dev) if stats is None else stats
         if G == 1:
             self.table.train_step(prep.ids, n_labeled, prep.e, step, ao_table, ao_rows, stats,
-                                  rows=rows, hit=hit, out=out)
+                                  inputs_ready=prep.inputs_ready, rows=rows, hit=hit, out=out)
             if trace is not None:
                 trace["sent_lookup"] = trace["sent_writeback"] = trace["recv_writeback"] = 0
             return rows, hit, out, stats
@@ -258,7 +261,7 @@ class Prepared:
     """The partitioned buffers and the pending segment sizes of one sharded step."""
 
     def __init__(self, ids, n_labeled, e, l_ids=None, l_pos=None, w_ids=None, w_e=None,
-                 sizes=None):
+                 sizes=None, inputs_ready=None):
         self.ids, self.n_labeled, self.e = ids, n_labeled, e
         self.l_ids, self.l_pos, self.w_ids, self.w_e = l_ids, l_pos, w_ids, w_e
-        self.sizes = sizes
+        self.sizes, self.inputs_ready = sizes, inputs_ready
