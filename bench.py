@@ -103,8 +103,6 @@ def parse():
     ap.add_argument("--row-kernel", choices=["reg", "bulk"], default=None,
                     help="row kernels through registers or through shared memory with bulk "
                          "copies (default: the library's)")
-    ap.add_argument("--select-passes", type=int, default=None, choices=[1, 2],
-                    help="select in two launches or one (default: the library's)")
     ap.add_argument("--write-list", choices=["emit", "kernel"], default=None,
                     help="cluster path: write list emitted at re-probe and placement, or built "
                          "by a separate kernel (default: the library's)")
@@ -117,8 +115,6 @@ def parse():
 
 
 def apply_row_options(binding, tbl, args):
-    if args.select_passes is not None:
-        binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SELECT_PASSES, args.select_passes)
     if args.write_list is not None:
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_WRITE_LIST,
                                  1 if args.write_list == "emit" else 0)

@@ -43,7 +43,6 @@ MPZCH_OPT_BULK_BLOCKS = 7
 MPZCH_OPT_L2_HINT_ROWS = 8
 MPZCH_OPT_WRITE_LIST = 9
 MPZCH_OPT_HBM_CACHE_ROWS = 10
-MPZCH_OPT_SELECT_PASSES = 13
 PHASES = ("lookup", "gather", "dedup", "insert", "writeback", "select", "export")
 STATS_FIELDS = ("n_ids", "n_unique", "n_hit_unique", "n_inserted", "n_evicted", "n_dropped",
                 "n_rounds")

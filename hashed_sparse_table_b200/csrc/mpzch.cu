@@ -275,16 +275,9 @@ struct mpzch_table {
   StepCtr* ctr = nullptr;
   WbStats* stats = nullptr;  // used when the caller passes no stats buffer
   int32_t* status = nullptr;
-  // select: per-tile ballot words and row counts (two launches); per-tile
-  // published counts, the tile ticket counter, the call epoch and the tickets
-  // issued so far (one launch)
+  // select: per-tile ballot words and row counts
   uint32_t* sel_masks = nullptr;
   int32_t* sel_tcount = nullptr;
-  unsigned long long* sel_tword = nullptr;
-  unsigned long long* sel_ticket = nullptr;
-  uint32_t sel_epoch = 0;
-  unsigned long long sel_tickets = 0;
-  int select_passes = 2;
   int32_t* h_status = nullptr;  // pinned host word for mpzch_get_status
   int64_t last_step = -1;
   int wide_rounds = 3;  // grid-wide insert rounds before the single-block finisher
@@ -367,8 +360,6 @@ void free_all(mpzch_table* t) {
   dev_free(t->status);
   dev_free(t->sel_masks);
   dev_free(t->sel_tcount);
-  dev_free(t->sel_tword);
-  dev_free(t->sel_ticket);
   if (t->h_status) cudaFreeHost(t->h_status);
   for (auto& r : t->pending) {
     cudaEventDestroy(r.a);
@@ -514,19 +505,6 @@ namespace {
 // with programmatic dependent launch.
 int launch_select(mpzch_table* t, int64_t since, int32_t* rows_out, int64_t* dev_count,
                   cudaStream_t st) {
-  if (t->select_passes == 1) {
-    const unsigned long long tiles = (unsigned long long)((t->C + kSelBigTile - 1) / kSelBigTile);
-    uint32_t epoch = t->sel_epoch + 1;
-    if (epoch == 0) epoch = 1;  // 0 is the value of the cleared words
-    const int rc = launch(k_select_one, (unsigned)tiles, kSelBigThreads, st, false,
-                          (const long long*)t->keys, (const long long*)t->last, t->C,
-                          (long long)since, t->sel_tword, t->sel_ticket, t->sel_tickets, epoch,
-                          rows_out, reinterpret_cast<long long*>(dev_count), t->status);
-    if (rc) return rc;
-    t->sel_epoch = epoch;
-    t->sel_tickets += tiles;
-    return MPZCH_OK;
-  }
   const unsigned tiles = (unsigned)((t->C + kScanTile - 1) / kScanTile);
   int rc = launch(k_select_mark, tiles, kScanThreads, st, false, (const long long*)t->keys,
                   (const long long*)t->last, t->C, (long long)since, t->sel_masks,
@@ -923,9 +901,6 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
   const int64_t sel_tiles = (capacity + kScanTile - 1) / kScanTile;
   if (!rc) rc = dev_alloc((void**)&t->sel_masks, sel_tiles * kScanWords * sizeof(uint32_t));
   if (!rc) rc = dev_alloc((void**)&t->sel_tcount, sel_tiles * sizeof(int32_t));
-  const int64_t sel_big = (capacity + kSelBigTile - 1) / kSelBigTile;
-  if (!rc) rc = dev_alloc((void**)&t->sel_tword, sel_big * sizeof(unsigned long long));
-  if (!rc) rc = dev_alloc((void**)&t->sel_ticket, sizeof(unsigned long long));
   if (!rc && cudaHostAlloc((void**)&t->h_status, sizeof(int32_t), cudaHostAllocDefault) != cudaSuccess) {
     t->h_status = nullptr;
     rc = MPZCH_ENOMEM;
@@ -944,10 +919,7 @@ int mpzch_create_ex(int64_t capacity, int32_t dim, int32_t probes, uint32_t flag
               cudaMemsetAsync(t->shead, 0, capacity * sizeof(unsigned long long), st) ==
                   cudaSuccess &&
               cudaMemsetAsync(t->stats, 0, sizeof(WbStats), st) == cudaSuccess &&
-              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess &&
-              cudaMemsetAsync(t->sel_tword, 0, sel_big * sizeof(unsigned long long), st) ==
-                  cudaSuccess &&
-              cudaMemsetAsync(t->sel_ticket, 0, sizeof(unsigned long long), st) == cudaSuccess;
+              cudaMemsetAsync(t->status, 0, sizeof(int32_t), st) == cudaSuccess;
     for (int i = 0; i < 3 && ok; ++i)
       ok = cudaMemsetAsync(t->claims[i], 0xFF, capacity * sizeof(unsigned long long), st) ==
            cudaSuccess;
@@ -1435,11 +1407,6 @@ int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {
     return MPZCH_OK;
   }
   if (option == MPZCH_OPT_HBM_CACHE_ROWS) return set_tier_rows(t, value);
-  if (option == MPZCH_OPT_SELECT_PASSES) {
-    if (value != 1 && value != 2) return MPZCH_EINVAL;
-    t->select_passes = (int)value;
-    return MPZCH_OK;
-  }
   if (option == MPZCH_OPT_WRITE_LIST) {
     if (value != 0 && value != 1) return MPZCH_EINVAL;
     t->emit_list = (int)value;
@@ -1466,7 +1433,6 @@ int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value) {
     case MPZCH_OPT_L2_HINT_ROWS: *value = t->l2_hint_rows; break;
     case MPZCH_OPT_WRITE_LIST: *value = t->emit_list; break;
     case MPZCH_OPT_HBM_CACHE_ROWS: *value = t->tier_rows; break;
-    case MPZCH_OPT_SELECT_PASSES: *value = t->select_passes; break;
     default: return MPZCH_EINVAL;
   }
   return MPZCH_OK;

@@ -1918,103 +1918,6 @@ __global__ void __launch_bounds__(kScanThreads) k_select_scatter(
   if (tile == gridDim.x - 1 && threadIdx.x == 0) *dev_count = excl + s_off[kScanWords];
 }
 
-// Select in one launch (MPZCH_OPT_SELECT_PASSES = 1): tiles of kSelBigTile rows
-// (1024 threads x 8 rows, rows t + 1024k per thread), so a 2^20-row table has
-// 128 tiles.  A block takes its tile from a ticket counter (every tile it waits
-// for then belongs to a block that is already running), publishes the tile's
-// count in a 64-bit word (call epoch in bits 63..32, count below; the epoch
-// makes words of earlier calls read as unpublished, so nothing is cleared),
-// and one warp sums the counts of all earlier tiles, polling an unpublished
-// word with a short sleep between reads and a time limit
-// (MPZCH_STATUS_TIMEOUT).  The rows are then written at that offset plus their
-// rank in the tile from 256 ballot words.
-constexpr int kSelBigThreads = 1024;
-constexpr int kSelBigTile = kSelBigThreads * kScanPer;
-constexpr int kSelBigWords = kScanPer * (kSelBigThreads / 32);  // 256
-
-__global__ void __launch_bounds__(kSelBigThreads) k_select_one(
-    const long long* __restrict__ keys, const long long* __restrict__ last, int64_t C,
-    long long since, unsigned long long* tword, unsigned long long* ticket,
-    unsigned long long ticket_base, uint32_t epoch, int32_t* __restrict__ rows_out,
-    long long* dev_count, int32_t* status) {
-  pdl_enter();
-  __shared__ int s_tile;
-  __shared__ int s_off[kSelBigWords + 1];
-  __shared__ long long s_excl;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (threadIdx.x == 0) s_tile = (int)(atomicAdd(ticket, 1ull) - ticket_base);
-  __syncthreads();
-  const int tile = s_tile;
-  const int64_t base = (int64_t)tile * kSelBigTile + threadIdx.x;
-  long long kv[kScanPer], lv[kScanPer];
-#pragma unroll
-  for (int k = 0; k < kScanPer; ++k) {
-    const int64_t r = base + (int64_t)k * kSelBigThreads;
-    kv[k] = r < C ? __ldcs(keys + r) : -1;
-    lv[k] = r < C ? __ldcs(last + r) : -1;
-  }
-  unsigned ball[kScanPer];
-#pragma unroll
-  for (int k = 0; k < kScanPer; ++k) {
-    ball[k] = __ballot_sync(0xFFFFFFFFu, kv[k] != -1 && lv[k] >= since);
-    if (lane == 0) s_off[k * 32 + warp] = __popc(ball[k]);
-  }
-  __syncthreads();
-  if (warp == 0) {  // exclusive scan of the 256 group counts (8 per lane), in row order
-    int c[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      c[q] = s_off[lane * 8 + q];
-      sum += c[q];
-    }
-    int x = sum;
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xFFFFFFFFu, x, off);
-      if (lane >= off) x += y;
-    }
-    int run = x - sum;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      s_off[lane * 8 + q] = run;
-      run += c[q];
-    }
-    if (lane == 31) s_off[kSelBigWords] = x;
-  }
-  __syncthreads();
-  const int total = s_off[kSelBigWords];
-  if (warp == 0) {
-    const unsigned long long ep = (unsigned long long)epoch << 32;
-    if (lane == 0) atomicExch(tword + tile, ep | (uint32_t)total);
-    long long excl = 0;
-    bool timed_out = false;
-    const uint64_t t0 = global_ns();
-    for (int q = lane; q < tile && !timed_out; q += 32) {
-      unsigned long long w = atomicAdd(tword + q, 0ull);
-      while ((w >> 32) != epoch) {  // not yet published in this call
-        __nanosleep(128);
-        if (global_ns() - t0 > kWaitLimitNs) {
-          timed_out = true;
-          break;
-        }
-        w = atomicAdd(tword + q, 0ull);
-      }
-      excl += (long long)(uint32_t)w;
-    }
-    for (int off = 16; off > 0; off >>= 1) excl += __shfl_xor_sync(0xFFFFFFFFu, excl, off);
-    if (__any_sync(0xFFFFFFFFu, timed_out) && lane == 0) set_status(status, kStTimeout);
-    if (lane == 0) s_excl = excl;
-  }
-  __syncthreads();
-  const long long excl = s_excl;
-  const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int k = 0; k < kScanPer; ++k)
-    if (ball[k] >> lane & 1u)
-      rows_out[excl + s_off[k * 32 + warp] + __popc(ball[k] & lt)] =
-          (int32_t)(base + (int64_t)k * kSelBigThreads);
-  if ((int64_t)(tile + 1) * kSelBigTile >= C && threadIdx.x == 0) *dev_count = excl + total;
-}
-
 // ---------------------------------------------------------------------------
 // int8 export: one warp per row.  a = max|x| (exact), scale = a/127 and x/scale
 // as IEEE divisions, round-half-even, clamp to +-127.  With last_out, the row's

@@ -445,13 +445,6 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
  * through mpzch_state_views are the host rows: call mpzch_tier_sync first.
  * Steps of a tiered table must stay below 2^31. */
 #define MPZCH_OPT_HBM_CACHE_ROWS 10
-/* MPZCH_OPT_SELECT_PASSES: how mpzch_select_written_since and the streaming
- * exporter find the rows: 2 (default) = two launches (per-tile marks and
- * counts, then offsets and the scatter); 1 = one launch over 8192-row tiles,
- * each tile adding up the counts the earlier tiles published (a tile waits
- * only for tiles already running; a wait has a time limit and sets
- * MPZCH_STATUS_TIMEOUT).  Results are identical. */
-#define MPZCH_OPT_SELECT_PASSES 13
 MPZCH_API int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value);
 /* Current value of an option (MPZCH_EINVAL for an unknown option). */
 MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);

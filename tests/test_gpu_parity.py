@@ -466,18 +466,15 @@ def test_launch_counter_and_trace():
         assert launches > 0 and ms > 0, (ph, tr[ph])
 
 
-@pytest.mark.parametrize("passes", [2, 1])
 @pytest.mark.parametrize("C", [1, 7, 2048, 2049, 6000, 8193, 100_003, 1 << 20])
-def test_select_tiles_ragged_tails_and_repeated_calls(C, passes):
-    """The select in two launches and in one, over one tile, exactly one, one
-    plus one row, many with a ragged tail, and the 1M-row table; several calls
-    in a row on the same table (per-tile words are rewritten, or carry the
-    call's epoch, in every call); rows chosen by every threshold from none to
-    all.  Compared with the oracle and with the definition (ascending rows with
-    a live key and last >= since)."""
+def test_select_tiles_ragged_tails_and_repeated_calls(C):
+    """The select over one tile, exactly one, one plus one row, many with a
+    ragged tail, and the 1M-row table; several calls in a row on the same table
+    (the per-tile marks and counts are rewritten by every call); rows chosen by
+    every threshold from none to all.  Compared with the oracle and with the
+    definition (ascending rows with a live key and last >= since)."""
     from hashed_sparse_table_b200 import binding
     tbl = binding.MpzchTable(C, 4, 1)
-    binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_SELECT_PASSES, passes)
     orc = oracle.OracleTable(C, 4, 1, track_all=False)
     rng = np.random.default_rng(C)
     keys = rng.integers(0, 1 << 40, C, dtype=np.int64)
