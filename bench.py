@@ -532,8 +532,9 @@ def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):
     """Export and serving on the trained table: rows written in the last 50
     steps -> int8 export (select + quantise), the serving snapshot image, and the
     serving gather of 4,096 requests x 1,024 candidates (Zipf 0.9 over 5M) in
-    512-request chunks.  CUDA events on the current stream; L2 is not flushed
-    between repetitions (each pass moves several GB)."""
+    512-request chunks.  Three untimed select + export pairs first; CUDA events
+    on the current stream; L2 is not flushed between repetitions (each pass
+    moves several GB)."""
     D, P, C = W.dim, W.probes, W.capacity
     last_step = binding.mpzch_get_last_step(tbl.h)
     since = last_step - inputs.CFG5_SERVE_SINCE + 1
@@ -542,6 +543,9 @@ def run_export_and_serve(tbl, binding, torch, dev, peak, reps: int = 5):
     q = torch.empty((C, D), dtype=torch.int8, device=dev)
     scale = torch.empty(C, dtype=torch.float32, device=dev)
     keys = torch.empty(C, dtype=torch.int64, device=dev)
+    for _ in range(3):  # warm-up (first launches load the kernels)
+        binding.mpzch_select_written_since(tbl.h, since, rows_d, cnt)
+        binding.mpzch_export_int8(tbl.h, rows_d, q, scale, keys, n=C, dev_n=cnt)
     binding.mpzch_trace_read(tbl.h)
     binding.mpzch_trace_enable(tbl.h, True)
     torch.cuda.synchronize()

@@ -14,7 +14,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmpzch.so")
 SOURCES = [os.path.join(CSRC, "mpzch.cu"), os.path.join(CSRC, "mpzch_res.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, "mpzch_kernels.cuh"), os.path.join(CSRC, "mpzch_internal.h"),
+DEPS = SOURCES + [os.path.join(CSRC, "mpzch_kernels.cuh"), os.path.join(CSRC, "mpzch_tier.cuh"),
+                  os.path.join(CSRC, "mpzch_internal.h"),
                   os.path.join(ROOT, "include", "mpzch.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

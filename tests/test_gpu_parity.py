@@ -466,13 +466,14 @@ def test_launch_counter_and_trace():
         assert launches > 0 and ms > 0, (ph, tr[ph])
 
 
-@pytest.mark.parametrize("C", [1, 7, 2048, 2049, 6000, 8193, 100_003, 1 << 20])
+@pytest.mark.parametrize("C", [1, 7, 2048, 2049, 6000, 8193, 100_003, 1 << 20, (1 << 22) + 5])
 def test_select_tiles_ragged_tails_and_repeated_calls(C):
     """The select over one tile, exactly one, one plus one row, many with a
-    ragged tail, and the 1M-row table; several calls in a row on the same table
-    (the per-tile marks and counts are rewritten by every call); rows chosen by
-    every threshold from none to all.  Compared with the oracle and with the
-    definition (ascending rows with a live key and last >= since)."""
+    ragged tail, the 1M-row table and 4M rows (2049 tiles); several calls in a
+    row on the same table (the per-tile marks and counts are rewritten by every
+    call); rows chosen by every threshold from none to all.  Compared with the
+    oracle and with the definition (ascending rows with a live key and
+    last >= since)."""
     from hashed_sparse_table_b200 import binding
     tbl = binding.MpzchTable(C, 4, 1)
     orc = oracle.OracleTable(C, 4, 1, track_all=False)
