@@ -1178,7 +1178,9 @@ int mpzch_serve_gather(const int64_t* snap_keys, int64_t capacity, int32_t probe
   if ((reinterpret_cast<uintptr_t>(out) & 15) || (reinterpret_cast<uintptr_t>(snap_q) & 3))
     return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  k_serve_gather<<<grid_for(n * 32, kBlock), kBlock, 0, st>>>(
+  // one resident wave, grid-stride over the ids
+  const int per_sm = resident_blocks(reinterpret_cast<const void*>(k_serve_gather), kBlock, 0);
+  k_serve_gather<<<grid_for(n * 32, kBlock, per_sm), kBlock, 0, st>>>(
       reinterpret_cast<const long long*>(snap_keys), make_geo(capacity, probes),
       reinterpret_cast<const char4*>(snap_q), snap_scale, dim / 4,
       reinterpret_cast<const long long*>(ids), n, rows, hit, reinterpret_cast<float4*>(out),

@@ -2122,8 +2122,37 @@ __global__ void __launch_bounds__(kBlock) k_export_rows(
 // Serving gather from an int8 snapshot: one warp per id; lanes j < P probe the
 // window, the first matching probe offset wins; then out = hit ? q*scale : +0.
 // Lane l stores the 16-byte vector l + 32*c, so every store request covers a
-// contiguous 512 B of the output row.
+// contiguous 512 B of the output row.  A warp's ids are i, i + warps, ...,
+// software-pipelined one id deep: while the current id's int8 row and scale
+// load, the next id's window is probed and the id after it is loaded, so an
+// id costs one dependent round trip to memory (three without the pipeline).
 // ---------------------------------------------------------------------------
+constexpr int kServeVec = 4;  // char4 codes per lane in the overlapped round (D <= 512)
+
+// First probe load of key k (k < 0: none): lane j < min(P, 32) loads window
+// slot j; returns that key (-1 when the lane loads nothing) and sets h.
+__device__ __forceinline__ long long serve_probe_issue(const long long* __restrict__ snap_keys,
+                                                       const Geo& g, long long k, int lane,
+                                                       int64_t& h) {
+  h = k >= 0 ? home_slot(k, g) : 0;
+  return (k >= 0 && lane < g.P) ? __ldg(snap_keys + wslot(h, lane, g)) : -1;
+}
+
+// Row of key k from its first probe load w (and the window's slots 32.. when
+// P > 32): the slot of the smallest matching offset, or -1.
+__device__ __forceinline__ int64_t serve_probe_resolve(const long long* __restrict__ snap_keys,
+                                                       const Geo& g, long long k, int lane,
+                                                       int64_t h, long long w) {
+  int32_t best = 0x7FFFFFFF;
+  if (k >= 0) {
+    if (lane < g.P && w == k) best = lane;
+    for (int32_t j = lane + 32; j < g.P; j += 32)
+      if (__ldg(snap_keys + wslot(h, j, g)) == k && j < best) best = j;
+  }
+  for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xFFFFFFFFu, best, off));
+  return (k >= 0 && best != 0x7FFFFFFF) ? wslot(h, best, g) : -1;
+}
+
 __global__ void __launch_bounds__(kBlock) k_serve_gather(
     const long long* __restrict__ snap_keys, Geo g, const char4* __restrict__ q,
     const float* __restrict__ scale, int D4, const long long* __restrict__ ids, int64_t n,
@@ -2132,34 +2161,58 @@ __global__ void __launch_bounds__(kBlock) k_serve_gather(
   pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += warps) {
-    const long long k = ids[i];
-    int32_t best = 0x7FFFFFFF;
-    int64_t h = 0;
-    if (k >= 0) {
-      h = home_slot(k, g);
-      for (int32_t j = lane; j < g.P; j += 32)
-        if (__ldg(snap_keys + wslot(h, j, g)) == k && j < best) best = j;
+  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (i >= n) return;  // warp-uniform
+  // prologue: the first id's row, the second id
+  long long k = ids[i];
+  long long kn = i + warps < n ? ids[i + warps] : -1;
+  int64_t h = 0;
+  const long long w0 = serve_probe_issue(snap_keys, g, k, lane, h);
+  int64_t r = serve_probe_resolve(snap_keys, g, k, lane, h, w0);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  while (true) {
+    const int64_t nx = i + warps;
+    // issue: the next id's first probe load, the id after it, this id's row
+    int64_t hn = 0;
+    const long long wn = nx < n ? serve_probe_issue(snap_keys, g, kn, lane, hn) : -1;
+    const long long kn2 = nx + warps < n ? ids[nx + warps] : -1;
+    const char4* qr = q + (r >= 0 ? r : 0) * (int64_t)D4;
+    const float sc = r >= 0 ? __ldg(scale + r) : 0.f;
+    char4 v[kServeVec];
+#pragma unroll
+    for (int u = 0; u < kServeVec; ++u) {
+      const int c = u * 32 + lane;
+      v[u] = make_char4(0, 0, 0, 0);
+      if (r >= 0 && c < D4) v[u] = __ldg(qr + c);
     }
-    for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xFFFFFFFFu, best, off));
-    const int64_t r = (k >= 0 && best != 0x7FFFFFFF) ? wslot(h, best, g) : -1;
     if (lane == 0) {
       if (k < 0) set_status(status, kStBadKey);
       rows[i] = (int32_t)r;
       hit[i] = r >= 0;
     }
     float4* o = out + i * (int64_t)D4;
-    if (r >= 0) {
-      const float s = __ldg(scale + r);
-      const char4* qr = q + r * (int64_t)D4;
-      for (int c = lane; c < D4; c += 32) {
-        const char4 v = __ldg(qr + c);
-        __stcs(o + c, make_float4(__fmul_rn((float)v.x, s), __fmul_rn((float)v.y, s),
-                                  __fmul_rn((float)v.z, s), __fmul_rn((float)v.w, s)));
-      }
-    } else {
-      for (int c = lane; c < D4; c += 32) __stcs(o + c, make_float4(0.f, 0.f, 0.f, 0.f));
+#pragma unroll
+    for (int u = 0; u < kServeVec; ++u) {
+      const int c = u * 32 + lane;
+      if (c < D4)
+        __stcs(o + c, r >= 0 ? make_float4(__fmul_rn((float)v[u].x, sc), __fmul_rn((float)v[u].y, sc),
+                                           __fmul_rn((float)v[u].z, sc), __fmul_rn((float)v[u].w, sc))
+                             : z);
     }
+    for (int c = kServeVec * 32 + lane; c < D4; c += 32) {  // rows wider than 512
+      if (r >= 0) {
+        const char4 x = __ldg(qr + c);
+        __stcs(o + c, make_float4(__fmul_rn((float)x.x, sc), __fmul_rn((float)x.y, sc),
+                                  __fmul_rn((float)x.z, sc), __fmul_rn((float)x.w, sc)));
+      } else {
+        __stcs(o + c, z);
+      }
+    }
+    if (nx >= n) break;  // warp-uniform
+    r = serve_probe_resolve(snap_keys, g, kn, lane, hn, wn);
+    i = nx;
+    k = kn;
+    kn = kn2;
   }
 }
 

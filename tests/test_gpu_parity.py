@@ -602,3 +602,45 @@ def test_pipelined_steps_sharing_rows_and_hit_buffers():
             assert_bitwise(hit.cpu().numpy(), ohit, "last hit")
     compare_state(tbl, orc, "shared rows/hit buffers")
     assert tbl.status() == 0
+
+
+@pytest.mark.parametrize("P,D,n", [(1, 16, 1), (8, 512, 7), (8, 512, 100_003), (40, 1024, 20_000),
+                                   (8, 132, 50_001)])
+def test_serve_gather_windows_widths_and_lengths(P, D, n):
+    """Serving gather against the oracle on a snapshot whose keys sit in their
+    windows (an oracle table filled by Writebacks) with arbitrary int8 codes
+    and scales: one id, fewer ids than warps, many ids per warp (the
+    one-id-deep pipeline), windows wider than a warp (P = 40), rows of 16, 132
+    (33 vectors), 512 and 1024 (beyond the overlapped round) values; the
+    candidates mix resident ids, never-seen ids and negative ids."""
+    from hashed_sparse_table_b200 import binding
+    C = 4096
+    orc = oracle.OracleTable(C, 4, P, track_all=False)
+    rng = np.random.default_rng(P * 1000 + D)
+    seen = rng.choice(1 << 40, 6000, replace=False).astype(np.int64)
+    for t in range(3):
+        ids = seen[t * 2000:(t + 1) * 2000]
+        orc.writeback(ids, rng.standard_normal((ids.size, 4)).astype(np.float32), t)
+    keys, _, _ = orc.state()
+    q = rng.integers(-127, 128, (C, D), dtype=np.int64).astype(np.int8)
+    scale = (rng.random(C) * 0.02).astype(np.float32)
+    scale[::17] = 0.0
+    cand = seen[rng.integers(0, seen.size, n)]
+    fresh = rng.random(n) < 0.2
+    cand[fresh] = (1 << 41) + np.arange(int(fresh.sum()))  # never seen
+    cand[6::13] = -3
+    rc, orow, ohit, oout = oracle.serve_gather(keys, C, P, q, scale, D, cand)
+    dev = torch.device("cuda", 0)
+    rows = torch.empty(n, dtype=torch.int32, device=dev)
+    hit = torch.empty(n, dtype=torch.uint8, device=dev)
+    out = torch.empty((n, D), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    binding.mpzch_serve_gather(torch.from_numpy(keys).to(dev), P, torch.from_numpy(q).to(dev),
+                               torch.from_numpy(scale).to(dev), torch.from_numpy(cand).to(dev),
+                               rows, hit, out, status=status)
+    assert_bitwise(rows.cpu().numpy(), orow, "serve rows")
+    assert_bitwise(hit.cpu().numpy(), ohit, "serve hit")
+    assert_bitwise(out.cpu().numpy(), oout, "serve features")
+    assert int(status.item()) == (binding.MPZCH_STATUS_BADKEY if n > 6 else 0)
+    if n > 100:
+        assert 0 < ohit.mean() < 1
