@@ -382,6 +382,8 @@ def run_ours(args):
         step(t)
     binding.mpzch_trace_read(tbl.h)  # drop warm-up records
     binding.mpzch_trace_enable(tbl.h, True)
+    if args.hbm_cache_rows:
+        binding.mpzch_tier_stats(tbl.h, reset=True)  # count the timed steps only
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -393,6 +395,7 @@ def run_ours(args):
     ev1.record(stream)
     torch.cuda.synchronize()
     launches = binding.mpzch_launch_count() - l0
+    tier_st = binding.mpzch_tier_stats(tbl.h) if args.hbm_cache_rows else None
     if world > 1:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
@@ -475,8 +478,20 @@ def run_ours(args):
             result.update(serving)
         if args.host_values:
             link = host_link_bandwidth(torch, dev)
-            # the row update moves each written row over the link twice (read + write)
-            link_bytes = n_written * 2 * 4 * D
+            # the row update moves each uncached written row over the link twice (read +
+            # write) and each evicted cached row once; without a cache every written row
+            if tier_st is not None:
+                link_rows = (tier_st["update_read_host"] + tier_st["update_write_host"]
+                             + tier_st["write_back"])
+                result["tier"] = dict(tier_st)
+                result["tier"]["update_read_cache_frac"] = tier_st["update_read_cache"] / max(
+                    1, tier_st["update_read_cache"] + tier_st["update_read_host"])
+                result["tier"]["gather_cache_frac"] = tier_st["gather_cache"] / max(
+                    1, tier_st["gather_cache"] + tier_st["gather_host"])
+                result["tier"]["link_mb_per_step"] = link_rows * 4 * D / K / 1e6
+            else:
+                link_rows = n_written * 2
+            link_bytes = link_rows * 4 * D
             link_gbs = link_bytes / (wb_ms * 1e-3) / 1e9 if wb_ms > 0 else 0.0
             link["row_update_link_gbs"] = link_gbs
             link["row_update_frac_of_bidirectional"] = link_gbs / link["bidirectional_gbs"]

@@ -76,6 +76,7 @@ _SIGS = {
     "mpzch_set_option": [_p, _i32, _i64],
     "mpzch_get_option": [_p, _i32, C.POINTER(_i64)],
     "mpzch_tier_sync": [_p, _i32, _p],
+    "mpzch_tier_stats": [_p, _p, _i32, _p],
     "mpzch_debug_fail_allocs": [_i32],
     "mpzch_set_learning_rate": [_p, C.c_float],
     "mpzch_res_create": [_p, _i64, _i32, _i32, C.POINTER(_p)],
@@ -308,6 +309,17 @@ def mpzch_get_option(h, option: int) -> int:
 
 def mpzch_tier_sync(h, discard: bool = False, stream=None) -> None:
     _check("mpzch_tier_sync", _lib.mpzch_tier_sync(h, 1 if discard else 0, _stream(stream)))
+
+
+TIER_STAT_NAMES = ("update_read_cache", "update_read_host", "update_write_cache",
+                   "update_write_host", "write_back", "gather_cache", "gather_host")
+
+
+def mpzch_tier_stats(h, reset: bool = False, stream=None) -> dict:
+    """Hot/cold tier counters (see include/mpzch.h), as a dict of ints."""
+    out = (C.c_int64 * len(TIER_STAT_NAMES))()
+    _check("mpzch_tier_stats", _lib.mpzch_tier_stats(h, out, 1 if reset else 0, _stream(stream)))
+    return dict(zip(TIER_STAT_NAMES, (int(x) for x in out)))
 
 
 def mpzch_set_learning_rate(h, eta: float) -> None:

@@ -354,6 +354,7 @@ void free_all(mpzch_table* t) {
   dev_free(t->tier.owner);
   dev_free(t->tier.won);
   dev_free(t->tier.claim);
+  dev_free(t->tier.stats);
   dev_free(t->ctr);
   dev_free(t->wcnt);
   dev_free(t->stats);
@@ -1327,6 +1328,7 @@ int set_tier_rows(mpzch_table* t, int64_t rows) {
   dev_free(t->tier.owner);
   dev_free(t->tier.won);
   dev_free(t->tier.claim);
+  dev_free(t->tier.stats);
   t->tier = Tier{};
   t->tier_rows = 0;
   if (rows == 0) return MPZCH_OK;
@@ -1335,7 +1337,9 @@ int set_tier_rows(mpzch_table* t, int64_t rows) {
   if (!rc) rc = dev_alloc((void**)&tr.owner, rows * sizeof(int32_t));
   if (!rc) rc = dev_alloc((void**)&tr.won, rows * sizeof(long long));
   if (!rc) rc = dev_alloc((void**)&tr.claim, rows * sizeof(unsigned long long));
+  if (!rc) rc = dev_alloc((void**)&tr.stats, kTierStats * sizeof(unsigned long long));
   if (!rc && (cudaMemset(tr.owner, 0xFF, rows * sizeof(int32_t)) != cudaSuccess ||
+              cudaMemset(tr.stats, 0, kTierStats * sizeof(unsigned long long)) != cudaSuccess ||
               cudaMemset(tr.won, 0xFF, rows * sizeof(long long)) != cudaSuccess ||
               cudaMemset(tr.claim, 0, rows * sizeof(unsigned long long)) != cudaSuccess ||
               cudaDeviceSynchronize() != cudaSuccess))
@@ -1346,6 +1350,7 @@ int set_tier_rows(mpzch_table* t, int64_t rows) {
     dev_free(tr.owner);
     dev_free(tr.won);
     dev_free(tr.claim);
+    dev_free(tr.stats);
     return rc;
   }
   tr.mask = (uint32_t)(rows - 1);
@@ -1369,6 +1374,22 @@ int mpzch_tier_sync(mpzch_table* t, int32_t discard, void* stream) {
     rc = tier_flush(t, st);
   }
   return mark_user(t, st, rc);
+}
+
+int mpzch_tier_stats(mpzch_table* t, int64_t* counts, int32_t reset, void* stream) {
+  if (!t || !counts || (reset != 0 && reset != 1) || !on_device(t)) return MPZCH_EINVAL;
+  for (int i = 0; i < kTierStats; ++i) counts[i] = 0;
+  if (t->tier_rows <= 0) return MPZCH_OK;
+  cudaStream_t st = S(stream);
+  int rc = join_side(t, st);
+  if (rc) return rc;
+  unsigned long long h[kTierStats];
+  if (cudaMemcpyAsync(h, t->tier.stats, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      (reset && cudaMemsetAsync(t->tier.stats, 0, sizeof(h), st) != cudaSuccess) ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    return MPZCH_ECUDA;
+  for (int i = 0; i < kTierStats; ++i) counts[i] = (int64_t)h[i];
+  return mark_user(t, st, MPZCH_OK);
 }
 
 int mpzch_set_option(mpzch_table* t, int32_t option, int64_t value) {

@@ -26,7 +26,10 @@
 //                  to the cache when the row owns its slot now, else to the host.
 // The values every read sees are therefore exactly those of one plain table,
 // whatever the placement.  Gathers and exports read a row from the cache when
-// owner[slot] is that row, else from the host.
+// owner[slot] is that row, else from the host.  Counters (kTierStat*) record
+// where each row update and gathered row was read and written, and the
+// write-backs of evicted rows; each block sums its own in shared memory and
+// adds them once.
 #pragma once
 #include "mpzch_kernels.cuh"
 
@@ -37,8 +40,24 @@ struct Tier {
   int32_t* owner;        // [H] table row held in the slot, -1 none
   long long* won;        // [H] step in which the current owner took the slot
   unsigned long long* claim;  // [H] claim words (never cleared)
+  unsigned long long* stats;  // [kTierStats] counters
   uint32_t mask;         // H - 1
 };
+
+// Counters: row updates whose e_hat came from the cache / the host, whose
+// result went to the cache / the host; cached rows written back on eviction;
+// gathered rows read from the cache / the host.
+constexpr int kTierStatUpdReadCache = 0, kTierStatUpdReadHost = 1, kTierStatUpdWriteCache = 2,
+              kTierStatUpdWriteHost = 3, kTierStatWriteBack = 4, kTierStatGatherCache = 5,
+              kTierStatGatherHost = 6, kTierStats = 7;
+
+// Block-level counter sums: lane 0 of a warp adds to shared memory; after the
+// block's last row every thread passes tier_stats_flush, whose first threads
+// add the sums to the global counters.
+__device__ __forceinline__ void tier_stats_flush(unsigned* s, unsigned long long* g) {
+  __syncthreads();
+  if (threadIdx.x < kTierStats && s[threadIdx.x]) atomicAdd(g + threadIdx.x, (unsigned long long)s[threadIdx.x]);
+}
 
 __device__ __forceinline__ const float4* tier_row(const Tier& tr, const float4* host, int32_t r,
                                                   int D4) {
@@ -78,6 +97,9 @@ __global__ void __launch_bounds__(kBlock) k_tier_evict(const int32_t* __restrict
                                                        float4* __restrict__ host, int D4,
                                                        long long step) {
   pdl_enter();
+  __shared__ unsigned s_st[kTierStats];
+  if (threadIdx.x < kTierStats) s_st[threadIdx.x] = 0;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int32_t W = *wcount;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -91,6 +113,7 @@ __global__ void __launch_bounds__(kBlock) k_tier_evict(const int32_t* __restrict
       const float4* src = tr.cache + (int64_t)s * D4;
       float4* dst = host + (int64_t)o * D4;
       for (int c = lane; c < D4; c += 32) dst[c] = __ldcg(src + c);
+      if (lane == 0) atomicAdd(s_st + kTierStatWriteBack, 1u);
     }
     __syncwarp();
     if (lane == 0) {
@@ -99,6 +122,7 @@ __global__ void __launch_bounds__(kBlock) k_tier_evict(const int32_t* __restrict
     }
   }
   pdl_trigger();
+  tier_stats_flush(s_st, tr.stats);
 }
 
 // Pass 3: the row update M[r] <- fl(e_hat - fl(eta * fl(e_hat - e))), e_hat
@@ -110,6 +134,9 @@ __global__ void __launch_bounds__(kBlock) k_tier_update(const int32_t* __restric
                                                         const float4* __restrict__ e, int D4,
                                                         float eta, long long step) {
   pdl_enter();
+  __shared__ unsigned s_st[kTierStats];
+  if (threadIdx.x < kTierStats) s_st[threadIdx.x] = 0;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int32_t W = *wcount;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -121,6 +148,10 @@ __global__ void __launch_bounds__(kBlock) k_tier_update(const int32_t* __restric
     const bool fresh = owns && tr.won[s] == step;  // took the slot in this step: value on the host
     const float4* src = (owns && !fresh) ? tr.cache + (int64_t)s * D4 : host + (int64_t)r * D4;
     float4* dst = owns ? tr.cache + (int64_t)s * D4 : host + (int64_t)r * D4;
+    if (lane == 0) {
+      atomicAdd(s_st + ((owns && !fresh) ? kTierStatUpdReadCache : kTierStatUpdReadHost), 1u);
+      atomicAdd(s_st + (owns ? kTierStatUpdWriteCache : kTierStatUpdWriteHost), 1u);
+    }
     const float4* ev = e + (int64_t)wpos[w] * D4;
     for (int base = 0; base < D4; base += 4 * 32) {
       float4 a[4], b[4];
@@ -146,6 +177,7 @@ __global__ void __launch_bounds__(kBlock) k_tier_update(const int32_t* __restric
       }
     }
   }
+  tier_stats_flush(s_st, tr.stats);
 }
 
 // Fused gather over the tier (same result as k_gather_fused on one table).
@@ -155,6 +187,9 @@ __global__ void __launch_bounds__(kBlock) k_tier_gather(
     int64_t ao_n, int A4, const int32_t* __restrict__ ao_rows, float4* __restrict__ out,
     int32_t* status) {
   pdl_enter();
+  __shared__ unsigned s_st[kTierStats];
+  if (threadIdx.x < kTierStats) s_st[threadIdx.x] = 0;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int W4 = D4 + A4;
@@ -175,6 +210,8 @@ __global__ void __launch_bounds__(kBlock) k_tier_gather(
       }
     }
     const float4* src = h ? tier_row(tr, host, r, D4) : host;
+    if (h && lane == 0)
+      atomicAdd(s_st + (src == host + (int64_t)r * D4 ? kTierStatGatherHost : kTierStatGatherCache), 1u);
     const float4* asrc = ao + (int64_t)a * A4;
     float4* dst = out + i * (int64_t)W4;
     for (int c = lane; c < W4; c += 32) {
@@ -187,6 +224,7 @@ __global__ void __launch_bounds__(kBlock) k_tier_gather(
       __stcs(dst + c, v);
     }
   }
+  tier_stats_flush(s_st, tr.stats);
 }
 
 // Writes every cached row back to its host row (the cache stays valid).

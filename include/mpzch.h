@@ -457,6 +457,17 @@ MPZCH_API int mpzch_get_option(mpzch_table* t, int32_t option, int64_t* value);
  * cache back by itself. */
 MPZCH_API int mpzch_tier_sync(mpzch_table* t, int32_t discard, void* stream);
 
+/* Hot/cold tier counters since the cache was created or last reset, read
+ * after the work on `stream` (and the table's side stream) has completed
+ * (the call synchronises `stream`).  counts: host int64[7] =
+ *   [0] row updates whose e_hat was read from the cache, [1] from the host,
+ *   [2] row updates whose result was written to the cache, [3] to the host,
+ *   [4] cached rows written back to the host when another row took their slot,
+ *   [5] gathered rows read from the cache, [6] from the host.
+ * reset = 1 zeroes the counters after reading them.  A table without a cache
+ * gives zeros. */
+MPZCH_API int mpzch_tier_stats(mpzch_table* t, int64_t* counts, int32_t reset, void* stream);
+
 /* Learning rate of the Writeback step for the following calls (Memory Layer
  * section 2, Writeback paragraph: the exact step is SGD at rate 1 on
  * g = e_hat - e; the alternative it is compared with, minimising

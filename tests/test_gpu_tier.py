@@ -99,3 +99,53 @@ def test_tier_option_checks():
     binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_HBM_CACHE_ROWS, 256)
     assert binding.mpzch_get_option(tbl.h, binding.MPZCH_OPT_HBM_CACHE_ROWS) == 256
     binding.mpzch_tier_sync(dev_tbl.h)  # no cache: no-op
+
+
+@pytest.mark.parametrize("rows", [1, 512, 1 << 13])
+def test_tier_counters_account_for_every_row(rows):
+    """The tier counters against the oracle's step counters and lookups: every
+    written row's e_hat is read once (cache or host) and its result written
+    once, every gathered hit is read once, and a row is read from the cache
+    only after it was written there.  With a cache of the whole table (one
+    slot per row) no result goes to the host, nothing is written back, every
+    gathered hit comes from the cache, and a row's e_hat comes from the host
+    exactly once (its first write), so host reads = rows holding a key at the
+    end.  Reset zeroes the counters."""
+    from hashed_sparse_table_b200 import binding
+    w = SCALED["c3_small"].scaled(steps=10)
+    tbl, orc = make_pair(w, flags=_host())
+    binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_HBM_CACHE_ROWS, rows)
+    dev = tbl.device
+    ao = inputs.author_table(w)
+    ao_d = torch.from_numpy(ao).to(dev)
+    stats_d = torch.zeros(7, dtype=torch.int64, device=dev)
+    written = hits = 0
+    for t in range(w.steps):
+        ids = inputs.step_ids(w, t)
+        e = inputs.step_e(w, t, rows=ids.size)
+        lab = min(w.labeled, ids.size)
+        aor = inputs.author_rows(w, ids[:lab])
+        tbl.train_step(torch.from_numpy(ids).to(dev), lab, torch.from_numpy(e).to(dev), t, ao_d,
+                       torch.from_numpy(aor).to(dev), stats_d)
+        rc, _, ohit = orc.lookup(ids[:lab])
+        assert rc == 0
+        hits += int(ohit.sum())
+        rc, ost = orc.writeback(ids, e, t)
+        assert rc == 0
+        written += ost["n_unique"] - ost["n_dropped"]
+    st = binding.mpzch_tier_stats(tbl.h)
+    assert st["update_read_cache"] + st["update_read_host"] == written, st
+    assert st["update_write_cache"] + st["update_write_host"] == written, st
+    assert st["gather_cache"] + st["gather_host"] == hits, st
+    assert st["update_read_cache"] <= st["update_write_cache"], st
+    if rows == w.capacity:
+        keys, _, _ = orc.state()
+        assert st["update_write_host"] == 0 and st["write_back"] == 0, st
+        assert st["gather_host"] == 0, st
+        assert st["update_read_host"] == int((keys != -1).sum()), st
+    elif rows > 1:
+        assert st["write_back"] > 0 and st["update_read_cache"] > 0, st
+    st2 = binding.mpzch_tier_stats(tbl.h, reset=True)
+    assert st2 == st
+    assert set(binding.mpzch_tier_stats(tbl.h).values()) == {0}
+    assert tbl.status() == 0
