@@ -583,7 +583,14 @@ int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int6
                        has_ao ? ao_dim / 4 : 0, ao_rows, reinterpret_cast<float4*>(out),
                        t->l2_hint_rows, t->status);
   }
-  return launch(k_gather_fused, row_grid(n, t->row_blocks_per_sm), kBlock, st, pdl, rows, hit, n,
+  // at most one resident wave: the blocks a second, partial wave would add
+  // only start as the first wave's finish, and the step waits for them
+  int per_sm = t->row_blocks_per_sm;
+  if (per_sm > 0) {
+    const int res = resident_blocks(reinterpret_cast<const void*>(k_gather_fused), kBlock, 0);
+    if (per_sm > res) per_sm = res;
+  }
+  return launch(k_gather_fused, row_grid(n, per_sm), kBlock, st, pdl, rows, hit, n,
                 reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
                 reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
                 ao_rows, reinterpret_cast<float4*>(out), t->status);

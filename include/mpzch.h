@@ -407,7 +407,8 @@ MPZCH_API int mpzch_trace_read(mpzch_table* t, double* ms, int64_t* launches, in
 #define MPZCH_OPT_SIDE_PRIORITY 2
 /* MPZCH_OPT_ROW_GRID: grid of the row kernels (fused gather, row update):
  * 0 = one row per warp, short-lived blocks; k > 0 = at most k blocks of 256
- * threads per SM, each striding over many rows (default 8). */
+ * threads per SM, each striding over many rows (default 8; the fused gather
+ * takes at most the blocks that fit on an SM at once). */
 #define MPZCH_OPT_ROW_GRID 3
 /* MPZCH_OPT_ROW_KERNEL: how the row kernels (fused gather, row update) move
  * rows.  0 (default) = through registers: every lane loads its 16-byte
