@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-serving", action="store_true",
                     help="skip the export + serving measurement after the timed region")
+    ap.add_argument("--eta", type=float, default=None,
+                    help="learning rate of the Writeback step (default 1: the exact step)")
     ap.add_argument("--res-every", type=int, default=0,
                     help="after the timed region, train for --res-seconds more while streaming "
                          "the rows written every N steps to a host int8 snapshot (RES); "
@@ -358,6 +360,8 @@ def run_ours(args):
         binding.mpzch_set_option(tbl.h, binding.MPZCH_OPT_CLUSTER_INSERT,
                                  1 if args.insert == "cluster" else 0)
     apply_row_options(binding, tbl, args)
+    if args.eta is not None:
+        binding.mpzch_set_learning_rate(tbl.h, args.eta)
 
     def step(t, i=None):
         # step t of the stream reads the resident inputs of slot i (default t)
@@ -454,7 +458,8 @@ def run_ours(args):
             "n_gpus": world, "steps": K, "warmup": Wm, "ms_per_step": max_ms / K,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded Zipf id streams, N(0,1) item-tower targets)",
-            "config": config_dict({"prefill_steps": Pf}),
+            "config": config_dict({"prefill_steps": Pf} if args.eta is None
+                                  else {"prefill_steps": Pf, "eta": args.eta}),
             "gpu_launches": launches,
             "roofline": {"bound": "hbm", "kernel": wb_kernel, "achieved": wb_gbs,
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
