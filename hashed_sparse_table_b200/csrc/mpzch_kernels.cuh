@@ -103,12 +103,7 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-__device__ __forceinline__ void pdl_enter() {
-#if defined(MPZCH_PDL_EARLY_TRIGGER) && MPZCH_PDL_EARLY_TRIGGER
-  pdl_trigger();
-#endif
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-}
+__device__ __forceinline__ void pdl_enter() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Row of `k` by one thread scanning the whole window (first match in probe
 // order; the identity map holds at most one).  -1 if absent.  Loads of 8
