@@ -678,7 +678,7 @@ def run_sharding_kernels(tbl, binding, torch, dev, peak, G, e_d, ao_d, reps: int
     b_combine = lab * (8 + 4 + 4 + 4 * D + 4 * A + 4 * (D + A) + 5)
     gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
     return {"owners": G, "distinct_ids": U, "ms": t,
-            "k_owner_scatter_with_e": {"bytes": b_scatter_e,
+            "partition_with_e_rows": {"bytes": b_scatter_e,
                                        "gbs": gbs(b_scatter_e, t["partition_distinct_e"]),
                                        "frac": gbs(b_scatter_e, t["partition_distinct_e"]) / peak},
             "k_owner_combine": {"bytes": b_combine, "gbs": gbs(b_combine, t["combine"]),

@@ -1228,9 +1228,13 @@ int mpzch_owner_partition(const int64_t* ids, const int32_t* src_pos, int64_t n,
   if (!rc) rc = launch(k_owner_offsets, 1, 1024, st, true, blk, nb, (int)n_owners, cnt);
   if (!rc)
     rc = launch(k_owner_scatter, nb, kPartTile, st, true, k, src_pos, n, dn, (int)n_owners,
-                static_cast<const int32_t*>(blk), reinterpret_cast<const float4*>(e),
-                e ? dim / 4 : 0, reinterpret_cast<long long*>(ids_out), pos_out,
-                reinterpret_cast<float4*>(e_out));
+                static_cast<const int32_t*>(blk), reinterpret_cast<long long*>(ids_out), pos_out);
+  if (!rc && e) {
+    const int per_sm = resident_blocks(reinterpret_cast<const void*>(k_owner_pack_rows), kBlock, 0);
+    rc = launch(k_owner_pack_rows, grid_for(n * 32, kBlock, per_sm), kBlock, st, true,
+                static_cast<const int32_t*>(pos_out), n, dn, reinterpret_cast<const float4*>(e),
+                dim / 4, reinterpret_cast<float4*>(e_out));
+  }
   return rc;
 }
 

@@ -2218,15 +2218,16 @@ __global__ void __launch_bounds__(kBlock) k_serve_gather(
 // belongs to shard owner(k) = (splitmix64(k) >> 32) mod G.
 //
 // The partition is a stable counting sort by owner in three launches over
-// tiles of kPartTile ids (one id per thread):
+// tiles of kPartTile ids (one id per thread), and a fourth that packs e rows:
 //   k_owner_count    per tile and owner, the number of ids (owner-major matrix);
 //   k_owner_offsets  one block: exclusive scan of that matrix in owner-major
 //                    order (= each tile's first output slot per owner) and the
 //                    per-owner totals;
 //   k_owner_scatter  each id's slot = its tile's offset for its owner + the ids
 //                    of that owner in earlier warps of the tile + earlier lanes
-//                    of its warp (__match_any_sync groups a warp by owner), then
-//                    each warp copies its ids' e rows to the packed send buffer.
+//                    of its warp (__match_any_sync groups a warp by owner);
+//   k_owner_pack_rows  with e rows: each slot's e row copied from its source
+//                    position into the packed send buffer.
 // Order within an owner is batch order, so the owner sees each rank's ids in
 // the order the rank had them.
 // ---------------------------------------------------------------------------
@@ -2313,9 +2314,8 @@ __global__ void __launch_bounds__(1024) k_owner_offsets(int32_t* __restrict__ bl
 
 __global__ void __launch_bounds__(kPartTile) k_owner_scatter(
     const long long* __restrict__ ids, const int32_t* __restrict__ src_pos, int64_t n,
-    const long long* dev_n, int G, const int32_t* __restrict__ off, const float4* __restrict__ e,
-    int D4, long long* __restrict__ ids_out, int32_t* __restrict__ pos_out,
-    float4* __restrict__ e_out) {
+    const long long* dev_n, int G, const int32_t* __restrict__ off,
+    long long* __restrict__ ids_out, int32_t* __restrict__ pos_out) {
   pdl_enter();
   __shared__ uint16_t wcnt[32 * kMaxOwners];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -2342,14 +2342,27 @@ __global__ void __launch_bounds__(kPartTile) k_owner_scatter(
     ids_out[dst] = key;
     pos_out[dst] = src;
   }
-  if (!e) return;
-  // the warp's rows, one after another; lane l moves 16-byte vectors l + 32c
-  for (int l = 0; l < 32; ++l) {
-    const long long d = __shfl_sync(0xFFFFFFFFu, dst, l);
-    const int32_t sp = __shfl_sync(0xFFFFFFFFu, src, l);
-    if (d < 0) continue;
+}
+
+// Packs the e rows of the partitioned ids into the send buffer, e_out[d] =
+// e[pos_out[d]] for d < n_eff, one warp per row over a grid of every SM (the
+// partition's tiles are too few to keep HBM busy: 96 tiles for 97k distinct
+// ids); the next row's source position is loaded while the current row moves.
+__global__ void __launch_bounds__(kBlock) k_owner_pack_rows(const int32_t* __restrict__ pos_out,
+                                                            int64_t n, const long long* dev_n,
+                                                            const float4* __restrict__ e,
+                                                            int D4,
+                                                            float4* __restrict__ e_out) {
+  pdl_enter();
+  const int lane = threadIdx.x & 31;
+  const int64_t n_eff = part_n(n, dev_n);
+  const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  int64_t d = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int32_t sp = d < n_eff ? pos_out[d] : 0;
+  while (d < n_eff) {
     const float4* srow = e + (int64_t)sp * D4;
     float4* drow = e_out + d * D4;
+    const int64_t nx = d + warps;
     for (int base = 0; base < D4; base += 4 * 32) {
       float4 v[4];
 #pragma unroll
@@ -2357,12 +2370,14 @@ __global__ void __launch_bounds__(kPartTile) k_owner_scatter(
         const int c = base + u * 32 + lane;
         if (c < D4) v[u] = __ldcs(srow + c);
       }
+      if (base == 0 && nx < n_eff) sp = pos_out[nx];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int c = base + u * 32 + lane;
         if (c < D4) __stcs(drow + c, v[u]);
       }
     }
+    d = nx;
   }
 }
 
