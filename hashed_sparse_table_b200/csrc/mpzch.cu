@@ -1254,11 +1254,27 @@ int mpzch_owner_combine(const int64_t* send_ids, const int32_t* pos, int64_t n, 
       (reinterpret_cast<uintptr_t>(ao_table) & 15))
     return MPZCH_EINVAL;
   cudaStream_t st = S(stream);
-  return launch(k_owner_combine, grid_for(n * 32, kBlock), kBlock, st, false,
-                reinterpret_cast<const long long*>(send_ids), pos, n, (int)n_owners,
-                shard_capacity, recv_rows, reinterpret_cast<const float4*>(recv_feat), dim / 4,
-                reinterpret_cast<const float4*>(ao_table), ao_nrows, ao_table ? ao_dim / 4 : 0,
-                ao_rows, rows, hit, reinterpret_cast<float4*>(out), dev_status);
+  const int W4 = dim / 4 + (ao_table ? ao_dim / 4 : 0);
+  const int vec = W4 > 32 * kCombineVecMax ? kCombineVecMax : (W4 + 31) / 32;
+  auto go = [&](auto kern) {
+    // one resident wave, grid-stride over the entries
+    const int per_sm = resident_blocks(reinterpret_cast<const void*>(kern), kBlock, 0);
+    return launch(kern, grid_for(n * 32, kBlock, per_sm), kBlock, st, false,
+                  reinterpret_cast<const long long*>(send_ids), pos, n, (int)n_owners,
+                  shard_capacity, recv_rows, reinterpret_cast<const float4*>(recv_feat), dim / 4,
+                  reinterpret_cast<const float4*>(ao_table), ao_nrows, ao_table ? ao_dim / 4 : 0,
+                  ao_rows, rows, hit, reinterpret_cast<float4*>(out), dev_status);
+  };
+  switch (vec) {
+    case 1: return go(k_owner_combine<1>);
+    case 2: return go(k_owner_combine<2>);
+    case 3: return go(k_owner_combine<3>);
+    case 4: return go(k_owner_combine<4>);
+    case 5: return go(k_owner_combine<5>);
+    case 6: return go(k_owner_combine<6>);
+    case 7: return go(k_owner_combine<7>);
+    default: return go(k_owner_combine<kCombineVecMax>);
+  }
 }
 
 int mpzch_state_views(mpzch_table* t, int64_t** keys, int64_t** last, float** M) {

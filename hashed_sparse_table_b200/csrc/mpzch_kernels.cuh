@@ -2318,7 +2318,7 @@ __global__ void __launch_bounds__(kPartTile) k_owner_scatter(
     long long* __restrict__ ids_out, int32_t* __restrict__ pos_out) {
   pdl_enter();
   __shared__ uint16_t wcnt[32 * kMaxOwners];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5;
   const int64_t n_eff = part_n(n, dev_n);
   const int64_t i = (int64_t)blockIdx.x * kPartTile + threadIdx.x;
   long long key;
@@ -2386,6 +2386,24 @@ __global__ void __launch_bounds__(kBlock) k_owner_pack_rows(const int32_t* __res
 // (-1 = miss) and D gathered values (+0 on a miss).  Writes, at pos[j], the
 // global row owner * Cs + row (or -1), hit, and the fused feature row: the
 // owner's D values, then the always-on row ao[ao_rows[pos[j]]].
+constexpr int kCombineVecMax = 8;  // 16-byte vectors per lane and round (1024 floats per row)
+
+// Indices of send-buffer entry j: its batch position, the owner's answer row
+// and the position's always-on row.
+__device__ __forceinline__ void combine_indices(const int32_t* __restrict__ pos,
+                                                const int32_t* __restrict__ recv_rows,
+                                                const int32_t* __restrict__ ao_rows, int A4,
+                                                int64_t j, int32_t& p, int32_t& r, int32_t& a) {
+  p = pos[j];
+  r = recv_rows[j];
+  a = A4 > 0 ? ao_rows[p] : 0;
+}
+
+// One warp per send-buffer entry, a resident wave grid-striding over them;
+// the next entry's indices are loaded while the current row is in flight and
+// all loads of a round (kVec vectors per lane: the answer and the always-on
+// row together when they fit) are issued before its stores.
+template <int kVec>
 __global__ void __launch_bounds__(kBlock) k_owner_combine(
     const long long* __restrict__ send_ids, const int32_t* __restrict__ pos, int64_t n, int G,
     int64_t Cs, const int32_t* __restrict__ recv_rows, const float4* __restrict__ recv_feat,
@@ -2396,17 +2414,15 @@ __global__ void __launch_bounds__(kBlock) k_owner_combine(
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int W4 = D4 + A4;
-  for (int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; j < n; j += warps) {
-    const int32_t p = pos[j];
-    const int32_t r = recv_rows[j];
-    int32_t a = 0;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int32_t p = 0, r = -1, a = 0;
+  if (j < n) combine_indices(pos, recv_rows, ao_rows, A4, j, p, r, a);
+  while (j < n) {
     bool has_a = A4 > 0;
-    if (has_a) {
-      a = ao_rows[p];
-      if (a < 0 || (int64_t)a >= ao_n) {
-        if (lane == 0) set_status(status, kStBadAo);
-        has_a = false;
-      }
+    if (has_a && (a < 0 || (int64_t)a >= ao_n)) {
+      if (lane == 0) set_status(status, kStBadAo);
+      has_a = false;
     }
     if (lane == 0) {
       const int o = owner_of(send_ids[j], G);
@@ -2414,13 +2430,13 @@ __global__ void __launch_bounds__(kBlock) k_owner_combine(
       hit[p] = r >= 0;
     }
     const float4* src = recv_feat + j * (int64_t)D4;
-    const float4* asrc = ao + (int64_t)a * A4;
+    const float4* asrc = ao + (int64_t)(has_a ? a : 0) * A4;
     float4* dst = out + (int64_t)p * W4;
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int base = 0; base < W4; base += 4 * 32) {
-      float4 v[4];
+    const int64_t nx = j + warps;
+    for (int base = 0; base < W4; base += kVec * 32) {
+      float4 v[kVec];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kVec; ++u) {
         const int c = base + u * 32 + lane;
         v[u] = z;
         if (c < D4)
@@ -2428,12 +2444,14 @@ __global__ void __launch_bounds__(kBlock) k_owner_combine(
         else if (c < W4 && has_a)
           v[u] = __ldg(asrc + (c - D4));
       }
+      if (base == 0 && nx < n) combine_indices(pos, recv_rows, ao_rows, A4, nx, p, r, a);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < kVec; ++u) {
         const int c = base + u * 32 + lane;
         if (c < W4) __stcs(dst + c, v[u]);
       }
     }
+    j = nx;
   }
 }
 
