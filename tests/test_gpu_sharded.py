@@ -49,20 +49,22 @@ def _partition(ids, G, src_pos=None, dev_n=None, e=None):
             None if e_out is None else e_out.cpu().numpy())
 
 
-@pytest.mark.parametrize("n,G,use_src,dev_n,with_e", [
-    (5000, 5, False, None, False),     # ragged last tile
-    (3 * 1024, 8, True, None, True),   # whole tiles, src positions, e rows
-    (7777, 3, True, 4321, True),       # device count below n
-    (2048, 1, False, None, True),      # one owner: order unchanged
-    (20000, 256, False, None, False),  # maximum owners
-    (1, 4, False, None, True),
-    (100, 4, False, 0, True),          # device count 0
+@pytest.mark.parametrize("n,G,use_src,dev_n,with_e,width", [
+    (5000, 5, False, None, False, 16),     # ragged last tile
+    (3 * 1024, 8, True, None, True, 16),   # whole tiles, src positions, e rows
+    (7777, 3, True, 4321, True, 16),       # device count below n
+    (2048, 1, False, None, True, 16),      # one owner: order unchanged
+    (20000, 256, False, None, False, 16),  # maximum owners
+    (1, 4, False, None, True, 16),
+    (100, 4, False, 0, True, 16),          # device count 0
+    (9000, 8, True, 8500, True, 516),      # rows of 129 vectors: a second, one-vector round
+    (4100, 2, False, None, True, 1028),    # rows of 257 vectors
 ])
-def test_partition_is_a_stable_sort_by_owner(n, G, use_src, dev_n, with_e):
+def test_partition_is_a_stable_sort_by_owner(n, G, use_src, dev_n, with_e, width):
     rng = np.random.default_rng(n + G)
     ids = inputs.zipf_keys(rng, 0.9, 50_000, n)
     src = rng.permutation(n).astype(np.int32) if use_src else None
-    e = rng.standard_normal((n, 16)).astype(np.float32) if with_e else None
+    e = rng.standard_normal((n, width)).astype(np.float32) if with_e else None
     got_ids, got_pos, got_cnt, got_e = _partition(ids, G, src, dev_n, e)
     m = n if dev_n is None else min(dev_n, n)
     own = oracle.owners(ids[:m], G)
@@ -101,16 +103,21 @@ def test_partition_rejects_bad_arguments():
         binding.mpzch_owner_partition(ids, 4, out, pos, cnt, ws[:0])
 
 
-def test_combine_places_answers_at_batch_positions():
+@pytest.mark.parametrize("D,A,n", [(32, 8, 3000), (512, 128, 20000), (1024, 288, 5000),
+                                   (4, 0, 777)])
+def test_combine_places_answers_at_batch_positions(D, A, n):
+    """Rows of one round of loads (10 and 160 vectors), of two (328 vectors:
+    answer and always-on parts across the rounds), and without an always-on
+    table; entries far more than warps (one-entry-deep pipeline)."""
     from hashed_sparse_table_b200 import binding
     dev = torch.device("cuda")
-    rng = np.random.default_rng(11)
-    G, Cs, D, A, n = 4, 1000, 32, 8, 3000
+    rng = np.random.default_rng(11 + D)
+    G, Cs = 4, 1000
     ids = rng.integers(0, 1 << 40, size=n, dtype=np.int64)
     got_ids, got_pos, _, _ = _partition(ids, G)
     recv_rows = rng.integers(-1, Cs, size=n).astype(np.int32)
     recv_feat = rng.standard_normal((n, D)).astype(np.float32)
-    ao = rng.standard_normal((50, A)).astype(np.float32)
+    ao = rng.standard_normal((50, A)).astype(np.float32) if A else None
     aor = rng.integers(0, 50, size=n).astype(np.int32)
     aor[17] = 50  # out of range: zeros and BADAO
     rows = torch.full((n,), -9, dtype=torch.int32, device=dev)
@@ -119,7 +126,7 @@ def test_combine_places_answers_at_batch_positions():
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     T = lambda x: torch.from_numpy(x).to(dev)  # noqa: E731
     binding.mpzch_owner_combine(T(got_ids), T(got_pos), G, Cs, T(recv_rows), T(recv_feat), rows,
-                                hit, out, T(ao), T(aor), status)
+                                hit, out, T(ao) if A else None, T(aor) if A else None, status)
     own = oracle.owners(got_ids, G)
     want_rows = np.empty(n, np.int32)
     want_hit = np.empty(n, np.uint8)
@@ -127,12 +134,13 @@ def test_combine_places_answers_at_batch_positions():
     want_rows[got_pos] = np.where(recv_rows >= 0, own * Cs + recv_rows, -1)
     want_hit[got_pos] = recv_rows >= 0
     want_out[got_pos, :D] = recv_feat
-    ok = (aor >= 0) & (aor < 50)
-    want_out[:, D:] = np.where(ok[:, None], ao[np.clip(aor, 0, 49)], 0.0)
+    if A:
+        ok = (aor >= 0) & (aor < 50)
+        want_out[:, D:] = np.where(ok[:, None], ao[np.clip(aor, 0, 49)], 0.0)
     assert_bitwise(rows.cpu().numpy(), want_rows, "rows")
     assert_bitwise(hit.cpu().numpy(), want_hit, "hit")
     assert_bitwise(out.cpu().numpy(), want_out, "out")
-    assert status.item() == 4
+    assert status.item() == (4 if A else 0)
 
 
 def _rank_inputs(w, t, r):
