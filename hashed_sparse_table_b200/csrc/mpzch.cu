@@ -566,11 +566,32 @@ int enqueue_gather(mpzch_table* t, const int32_t* rows, const uint8_t* hit, int6
                    const int32_t* ao_rows, float* out, cudaStream_t st, bool pdl) {
   PhaseScope ps(t, PH_GATHER, st);
   const bool has_ao = ao_table != nullptr;
-  if (t->tier_rows > 0)
-    return launch(k_tier_gather, row_grid(n, t->row_blocks_per_sm), kBlock, st, pdl, rows, hit, n,
-                  t->tier, reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
-                  reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
-                  ao_rows, reinterpret_cast<float4*>(out), t->status);
+  if (t->tier_rows > 0) {
+    const int W4 = t->D / 4 + (has_ao ? ao_dim / 4 : 0);
+    const int vec = W4 > 32 * kTierGatherVecMax ? kTierGatherVecMax : (W4 + 31) / 32;
+    auto go = [&](auto kern) {
+      // one resident wave, grid-stride over the rows
+      int per_sm = t->row_blocks_per_sm;
+      if (per_sm > 0) {
+        const int res = resident_blocks(reinterpret_cast<const void*>(kern), kBlock, 0);
+        if (per_sm > res) per_sm = res;
+      }
+      return launch(kern, row_grid(n, per_sm), kBlock, st, pdl, rows, hit, n, t->tier,
+                    reinterpret_cast<const float4*>(t->M), t->C, t->D / 4,
+                    reinterpret_cast<const float4*>(ao_table), ao_nrows, has_ao ? ao_dim / 4 : 0,
+                    ao_rows, reinterpret_cast<float4*>(out), t->status);
+    };
+    switch (vec) {
+      case 1: return go(k_tier_gather<1>);
+      case 2: return go(k_tier_gather<2>);
+      case 3: return go(k_tier_gather<3>);
+      case 4: return go(k_tier_gather<4>);
+      case 5: return go(k_tier_gather<5>);
+      case 6: return go(k_tier_gather<6>);
+      case 7: return go(k_tier_gather<7>);
+      default: return go(k_tier_gather<kTierGatherVecMax>);
+    }
+  }
   int warps = 0;
   size_t smem = 0;
   if (bulk_shape(t, (size_t)(t->D + (has_ao ? ao_dim : 0)) * 4, &warps, &smem)) {

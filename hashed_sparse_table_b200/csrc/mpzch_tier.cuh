@@ -181,6 +181,13 @@ __global__ void __launch_bounds__(kBlock) k_tier_update(const int32_t* __restric
 }
 
 // Fused gather over the tier (same result as k_gather_fused on one table).
+// A warp's rows are i, i + warps, ...; the next row's indices are loaded
+// while the current row is in flight (host reads are long), and every load of
+// a round (kVec vectors per lane: the table and always-on parts together when
+// they fit) is issued before its stores.
+constexpr int kTierGatherVecMax = 8;
+
+template <int kVec>
 __global__ void __launch_bounds__(kBlock) k_tier_gather(
     const int32_t* __restrict__ rows, const uint8_t* __restrict__ hit, int64_t n, Tier tr,
     const float4* __restrict__ host, int64_t C, int D4, const float4* __restrict__ ao,
@@ -193,36 +200,56 @@ __global__ void __launch_bounds__(kBlock) k_tier_gather(
   const int lane = threadIdx.x & 31;
   const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int W4 = D4 + A4;
-  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += warps) {
-    const int32_t r = rows[i];
-    bool h = hit[i] != 0;
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  int32_t r = 0, a = 0;
+  uint8_t hb = 0;
+  if (i < n) {
+    r = rows[i];
+    hb = hit[i];
+    if (A4 > 0) a = ao_rows[i];
+  }
+  while (i < n) {
+    bool h = hb != 0;
     if (h && (r < 0 || (int64_t)r >= C)) {
       if (lane == 0) set_status(status, kStBadRow);
       h = false;
     }
-    int32_t a = 0;
     bool has_a = A4 > 0;
-    if (has_a) {
-      a = ao_rows[i];
-      if (a < 0 || (int64_t)a >= ao_n) {
-        if (lane == 0) set_status(status, kStBadAo);
-        has_a = false;
-      }
+    if (has_a && (a < 0 || (int64_t)a >= ao_n)) {
+      if (lane == 0) set_status(status, kStBadAo);
+      has_a = false;
     }
     const float4* src = h ? tier_row(tr, host, r, D4) : host;
     if (h && lane == 0)
       atomicAdd(s_st + (src == host + (int64_t)r * D4 ? kTierStatGatherHost : kTierStatGatherCache), 1u);
-    const float4* asrc = ao + (int64_t)a * A4;
+    const float4* asrc = ao + (int64_t)(has_a ? a : 0) * A4;
     float4* dst = out + i * (int64_t)W4;
-    for (int c = lane; c < W4; c += 32) {
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (c < D4) {
-        if (h) v = __ldcg(src + c);
-      } else if (has_a) {
-        v = __ldg(asrc + (c - D4));
+    const int64_t nx = i + warps;
+    for (int base = 0; base < W4; base += kVec * 32) {
+      float4 v[kVec];
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int c = base + u * 32 + lane;
+        v[u] = z;
+        if (c < D4) {
+          if (h) v[u] = __ldcg(src + c);
+        } else if (c < W4 && has_a) {
+          v[u] = __ldg(asrc + (c - D4));
+        }
       }
-      __stcs(dst + c, v);
+      if (base == 0 && nx < n) {
+        r = rows[nx];
+        hb = hit[nx];
+        if (A4 > 0) a = ao_rows[nx];
+      }
+#pragma unroll
+      for (int u = 0; u < kVec; ++u) {
+        const int c = base + u * 32 + lane;
+        if (c < W4) __stcs(dst + c, v[u]);
+      }
     }
+    i = nx;
   }
   tier_stats_flush(s_st, tr.stats);
 }
